@@ -1,0 +1,16 @@
+"""fp64 CPU oracle for exact attention (test infrastructure only).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` use this package. It shares no code with the CUDA library.
+"""
+
+from .attention import (  # noqa: F401
+    attention_bwd,
+    attention_fwd,
+    head_bwd,
+    head_fwd,
+    kvcache_decode,
+    lse_combine,
+    scores,
+    visible_mask,
+)

@@ -1,0 +1,319 @@
+"""Plain fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module. The CUDA library never calls it, and this module imports nothing from
+the CUDA library or its Python binding.
+
+Sources (web pages; cited by title and section):
+
+* "FlashAttention 实战指南:如何把训练内存省 20 倍、速度提 4 倍" (kwkr.cn)
+  - §长序列注意力为什么会爆内存: attention is three steps, QK^T, softmax, then
+    multiply by V; the tiled method is exact, i.e. it equals this plain
+    definition up to floating-point rounding. So the oracle is the plain
+    definition, with the full score matrix materialised and masked explicitly.
+  - §上手…三步走: tensors are (batch, seqlen, nheads, headdim); causal=True for
+    autoregressive use; a varlen family handles unequal lengths in a batch.
+  - §进阶参数: window_size=(left, right), (-1, -1) meaning unbounded; softcap
+    bounds the logits to [-softcap, softcap]; K/V may have fewer heads than Q
+    as long as Hq is an integer multiple of Hkv (MQA/GQA).
+  - §增量解码场景 flash_attn_with_kvcache: the new K, V are appended to the
+    existing cache and attention is then done in place; cache_seqlens marks
+    each sample's valid length; block_table pages the cache; num_splits
+    splits the KV range.
+* "AI模型推理优化 Flash Attention原理" (52runoob.com)
+  - §先搞清楚原理: the standard attention function, scores = Q K^T / sqrt(d),
+    softmax over the last dim, then times V.
+  - §实际怎么用: the KVCache class, whose update writes the new k, v at the
+    current position and returns the prefix up to the new position.
+
+Readings where the pages leave a step open (each one is listed in the design
+notes of the repository):
+
+* softcap is the tanh form ``c * tanh(x / c)``, applied after ``scale`` and
+  before masking; ``softcap == 0`` disables it. It keeps every logit inside
+  (-c, c), which is what the guide's sentence asks for.
+* window bounds are inclusive; causal means ``window_right = 0``.
+* when Sq != Sk the diagonal is aligned bottom-right: query i may see key j iff
+  ``i + (Sk - Sq) - L <= j <= i + (Sk - Sq) + R``.
+* a row with no visible key gets O = 0 and LSE = -inf (and zero gradients).
+* LSE is the natural-log log-sum-exp of the (scaled, softcapped) logits.
+* GQA maps query head h to kv head ``h // (Hq // Hkv)``.
+* ``cache_seqlens[b]`` is the length *before* the append; the new token lands
+  at position ``cache_seqlens[b]`` and attention covers ``cache_seqlens[b]+1``
+  keys.
+
+Every array is float64. 16-bit inputs are converted exactly (every bf16 and
+fp16 value is representable in float64), so the oracle sees the same values
+the GPU sees.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "visible_mask",
+    "scores",
+    "head_fwd",
+    "head_bwd",
+    "attention_fwd",
+    "attention_bwd",
+    "kvcache_decode",
+    "lse_combine",
+]
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast of a numpy array or a CPU torch tensor to float64."""
+    if hasattr(x, "detach"):  # torch tensor (bf16 has no numpy dtype)
+        import torch
+
+        return x.detach().to(torch.float64).cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def visible_mask(sq: int, sk: int, causal: bool, window_left: int, window_right: int,
+                 rows: np.ndarray | None = None) -> np.ndarray:
+    """Boolean [len(rows), sk] matrix: True where query i may attend key j.
+
+    Guide §进阶参数: window (left, right) with -1 meaning unbounded; causal is
+    the window with right = 0. Alignment is bottom-right (delta = sk - sq).
+    """
+    if rows is None:
+        rows = np.arange(sq)
+    i = np.asarray(rows, dtype=np.int64)[:, None]
+    j = np.arange(sk, dtype=np.int64)[None, :]
+    delta = sk - sq
+    right = 0 if causal else window_right
+    ok = np.ones((i.shape[0], sk), dtype=bool)
+    if right >= 0:
+        ok &= j <= i + delta + right
+    if window_left >= 0:
+        ok &= j >= i + delta - window_left
+    return ok
+
+
+def scores(q_h: np.ndarray, k_h: np.ndarray, scale: float, softcap: float):
+    """Logits of one head: returns (X, Y) with Y = scale * q k^T and
+    X = softcap * tanh(Y / softcap) (X = Y when softcap == 0).
+
+    Notes §先搞清楚原理 (scores = Q K^T * scale); guide §进阶参数 (softcap).
+    """
+    y = scale * (_f64(q_h) @ _f64(k_h).T)
+    if softcap > 0.0:
+        x = softcap * np.tanh(y / softcap)
+    else:
+        x = y
+    return x, y
+
+
+def head_fwd(q_h, k_h, v_h, scale: float, causal: bool = False, window_left: int = -1,
+             window_right: int = -1, softcap: float = 0.0, rows=None, _score_hook=None):
+    """One head of the forward pass.
+
+    q_h: [Sq, D]; k_h, v_h: [Sk, D]. ``rows`` optionally selects query rows
+    (indices into 0..Sq-1) so that sampled rows of a long sequence can be
+    checked without the whole matrix. Returns (O [rows, D], LSE [rows]).
+
+    Steps, in the order of the notes' standard attention: logits, mask,
+    softmax along the keys, weighted sum of V. The softmax is evaluated as
+    exp(X - m) / sum(exp(X - m)) with m the row max, which is the same value.
+    """
+    q_h = _f64(q_h)
+    k_h = _f64(k_h)
+    v_h = _f64(v_h)
+    sq, sk = q_h.shape[0], k_h.shape[0]
+    if rows is None:
+        rows = np.arange(sq)
+    rows = np.asarray(rows, dtype=np.int64)
+    x, _ = scores(q_h[rows], k_h, scale, softcap)
+    if _score_hook is not None:
+        x = _score_hook(x)
+    vis = visible_mask(sq, sk, causal, window_left, window_right, rows)
+    x = np.where(vis, x, -np.inf)
+    m = np.max(x, axis=1, initial=-np.inf)
+    has = np.isfinite(m)
+    m_safe = np.where(has, m, 0.0)
+    p = np.exp(x - m_safe[:, None])  # exp(-inf) = 0 on masked entries
+    l = p.sum(axis=1)
+    o = np.zeros((rows.shape[0], v_h.shape[1]))
+    o[has] = (p[has] / l[has, None]) @ v_h
+    lse = np.full(rows.shape[0], -np.inf)
+    lse[has] = m[has] + np.log(l[has])
+    return o, lse
+
+
+def head_bwd(q_h, k_h, v_h, do_h, scale: float, causal: bool = False, window_left: int = -1,
+             window_right: int = -1, softcap: float = 0.0):
+    """One head of the backward pass of ``head_fwd`` (all rows).
+
+    With P the row-normalised softmax probabilities (zero where masked):
+      dV = P^T dO,  dP = dO V^T,  Drow = rowsum(P * dP),  dX = P * (dP - Drow)
+    and through softcap X = c tanh(Y / c): dY = dX * (1 - tanh(Y / c)^2),
+      dQ = scale * dY K,  dK = scale * dY^T Q.
+    This is the chain rule of the definition; the guide (§长序列…) says the
+    tiled backward recomputes these quantities rather than storing P.
+    """
+    q_h = _f64(q_h)
+    k_h = _f64(k_h)
+    v_h = _f64(v_h)
+    do_h = _f64(do_h)
+    sq, sk = q_h.shape[0], k_h.shape[0]
+    x, y = scores(q_h, k_h, scale, softcap)
+    vis = visible_mask(sq, sk, causal, window_left, window_right)
+    x = np.where(vis, x, -np.inf)
+    m = np.max(x, axis=1, initial=-np.inf)
+    has = np.isfinite(m)
+    m_safe = np.where(has, m, 0.0)
+    p = np.exp(x - m_safe[:, None])
+    l = p.sum(axis=1)
+    l_safe = np.where(has, l, 1.0)
+    p = p / l_safe[:, None]
+    dv = p.T @ do_h
+    dp = do_h @ v_h.T
+    drow = np.sum(p * dp, axis=1)
+    dx = p * (dp - drow[:, None])
+    if softcap > 0.0:
+        t = np.tanh(y / softcap)
+        dy = dx * (1.0 - t * t)
+    else:
+        dy = dx
+    dq = scale * (dy @ k_h)
+    dk = scale * (dy.T @ q_h)
+    return dq, dk, dv
+
+
+def _segments(q, cu_seqlens):
+    """Yield (b, q-token slice) for fixed-length (B,S,...) or varlen inputs."""
+    if cu_seqlens is None:
+        for b in range(q.shape[0]):
+            yield b, (b,)
+    else:
+        cu = [int(c) for c in np.asarray(cu_seqlens).tolist()]
+        for b in range(len(cu) - 1):
+            yield b, (slice(cu[b], cu[b + 1]),)
+
+
+def attention_fwd(q, k, v, scale: float, causal: bool = False, window=(-1, -1),
+                  softcap: float = 0.0, cu_seqlens=None):
+    """Full forward over all batches and heads.
+
+    Fixed length: q (B, S, Hq, D), k/v (B, S, Hkv, D) -> O (B, S, Hq, D),
+    LSE (B, Hq, S). Varlen (cu_seqlens given, int prefix sums of length B+1):
+    q (total, Hq, D), k/v (total, Hkv, D) -> O (total, Hq, D), LSE (Hq, total);
+    each segment is an independent sequence with Sq = Sk = its length (guide
+    §上手…三步走, varlen family).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    hq, hkv = q.shape[-2], k.shape[-2]
+    assert hq % hkv == 0, "Hq must be an integer multiple of Hkv"
+    g = hq // hkv
+    o = np.zeros(q.shape)
+    if cu_seqlens is None:
+        lse = np.zeros((q.shape[0], hq, q.shape[1]))
+    else:
+        lse = np.zeros((hq, q.shape[0]))
+    for b, sl in _segments(q, cu_seqlens):
+        qb, kb, vb = q[sl], k[sl], v[sl]
+        for h in range(hq):
+            ob, lb = head_fwd(qb[:, h], kb[:, h // g], vb[:, h // g], scale, causal,
+                              window[0], window[1], softcap)
+            if cu_seqlens is None:
+                o[b, :, h] = ob
+                lse[b, h] = lb
+            else:
+                o[sl[0], h] = ob
+                lse[h, sl[0]] = lb
+    return o, lse
+
+
+def attention_bwd(q, k, v, do, scale: float, causal: bool = False, window=(-1, -1),
+                  softcap: float = 0.0, cu_seqlens=None):
+    """Gradients (dQ, dK, dV) of sum(O * dO); same layouts as attention_fwd.
+    For GQA the per-query-head dK/dV contributions of a group are summed into
+    their shared kv head."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    hq, hkv = q.shape[-2], k.shape[-2]
+    g = hq // hkv
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for b, sl in _segments(q, cu_seqlens):
+        for h in range(hq):
+            a, bb, c = head_bwd(q[sl][:, h], k[sl][:, h // g], v[sl][:, h // g], do[sl][:, h],
+                                scale, causal, window[0], window[1], softcap)
+            if cu_seqlens is None:
+                dq[b, :, h] = a
+                dk[b, :, h // g] += bb
+                dv[b, :, h // g] += c
+            else:
+                dq[sl[0], h] = a
+                dk[sl[0], h // g] += bb
+                dv[sl[0], h // g] += c
+    return dq, dk, dv
+
+
+def kvcache_decode(q, k_new, v_new, k_cache_logical, v_cache_logical, cache_seqlens,
+                   scale: float, causal: bool = True, window=(-1, -1), softcap: float = 0.0,
+                   heads=None):
+    """One decode step against a *logical, contiguous* per-sequence cache.
+
+    q (B, 1, Hq, D); k_new, v_new (B, 1, Hkv, D); k/v_cache_logical: sequence
+    of B arrays, each holding at least cache_seqlens[b] rows of shape
+    (rows, Hkv, D). Following the notes' KVCache.update, the new k, v are
+    written at position L_b = cache_seqlens[b] and the prefix of length L_b+1
+    is returned; attention then runs for the single query at logical position
+    L_b over those L_b+1 keys (bottom-right alignment: causal lets it see all
+    of them). The paged layout and block_table are not used here at all.
+
+    ``heads`` optionally restricts the query heads evaluated (others left 0).
+    Returns (O (B, 1, Hq, D), LSE (B, Hq, 1), appended_k list, appended_v list).
+    """
+    q = _f64(q)
+    k_new = _f64(k_new)
+    v_new = _f64(v_new)
+    bsz, _, hq, d = q.shape
+    hkv = k_new.shape[2]
+    g = hq // hkv
+    o = np.zeros((bsz, 1, hq, d))
+    lse = np.zeros((bsz, hq, 1))
+    ks, vs = [], []
+    for b in range(bsz):
+        n = int(cache_seqlens[b])
+        kb = np.concatenate([_f64(k_cache_logical[b])[:n], k_new[b]], axis=0)
+        vb = np.concatenate([_f64(v_cache_logical[b])[:n], v_new[b]], axis=0)
+        ks.append(kb)
+        vs.append(vb)
+        for h in (range(hq) if heads is None else heads):
+            ob, lb = head_fwd(q[b, :, h], kb[:, h // g], vb[:, h // g], scale, causal,
+                              window[0], window[1], softcap)
+            o[b, 0, h] = ob[0]
+            lse[b, h, 0] = lb[0]
+    return o, lse, ks, vs
+
+
+def lse_combine(o_parts, lse_parts):
+    """Merge attention results computed over disjoint key ranges.
+
+    o_parts: [n, ..., D] each normalised over its own range; lse_parts [n, ...].
+    LSE = log(sum_s exp(LSE_s)); O = sum_s exp(LSE_s - LSE) * O_s. This is the
+    identity that lets num_splits (guide §增量解码场景) split the KV range.
+    Parts with LSE_s = -inf (no visible key) carry zero weight.
+    """
+    o_parts = _f64(o_parts)
+    lse_parts = _f64(lse_parts)
+    m = np.max(lse_parts, axis=0)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse_parts - m_safe[None])
+    s = w.sum(axis=0)
+    has = s > 0
+    lse = np.where(has, m_safe + np.log(np.where(has, s, 1.0)), -np.inf)
+    wn = np.where(has[None], w / np.where(has, s, 1.0)[None], 0.0)
+    o = np.sum(wn[..., None] * o_parts, axis=0)
+    return o, lse
