@@ -1,0 +1,240 @@
+"""Python binding of the exact-attention C ABI (include/fa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libfa.so``. PyTorch provides device memory and the current
+stream; nothing here computes attention, and there is no fallback: if the
+library is missing, importing this package raises.
+
+Low-level names mirror the C ABI (``fa_fwd``, ``fa_bwd``, ``fa_fwd_kvcache``,
+``fa_bwd_workspace_size``, ``fa_kvcache_workspace_size``,
+``fa_get_device_status``, ``fa_last_error``, ``fa_version``) and take torch
+tensors where the C call takes pointers. ``fwd``, ``bwd`` and
+``fwd_kvcache`` additionally allocate outputs and workspaces with torch.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "FaError", "lib",
+    "fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_bwd_workspace_size", "fa_kvcache_workspace_size",
+    "fa_get_device_status", "fa_last_error", "fa_version",
+    "fwd", "bwd", "fwd_kvcache",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+_STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+           4: "FA_ERR_TIMEOUT"}
+_DTYPE = {torch.bfloat16: 0, torch.float16: 1}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m exact_attention_149_b200.build` "
+        "(nvcc, sm_100a). There is no CPU or library fallback.")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_z = ctypes.c_size_t
+
+lib.fa_fwd.restype = _i
+lib.fa_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _p, _i, _i, _p]
+lib.fa_bwd.restype = _i
+lib.fa_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f,
+                       _p, _i, _i, _p, _z, _p]
+lib.fa_fwd_kvcache.restype = _i
+lib.fa_fwd_kvcache.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
+                               _i, _i, _i, _f, _i, _i, _p, _z, _p]
+lib.fa_bwd_workspace_size.restype = _z
+lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+lib.fa_kvcache_workspace_size.restype = _z
+lib.fa_kvcache_workspace_size.argtypes = [_i, _i, _i, _i]
+lib.fa_get_device_status.restype = _i
+lib.fa_get_device_status.argtypes = [ctypes.POINTER(_i)]
+lib.fa_last_error.restype = ctypes.c_char_p
+lib.fa_last_error.argtypes = []
+lib.fa_version.restype = ctypes.c_char_p
+lib.fa_version.argtypes = []
+
+
+def fa_last_error() -> str:
+    return lib.fa_last_error().decode()
+
+
+def fa_version() -> str:
+    return lib.fa_version().decode()
+
+
+def _check(status: int):
+    if status != FA_OK:
+        raise FaError(status, fa_last_error())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dt(t) -> int:
+    if t.dtype not in _DTYPE:
+        raise FaError(FA_ERR_INVALID_ARG, f"dtype {t.dtype} not supported (bf16/fp16)")
+    return _DTYPE[t.dtype]
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not isinstance(t, int):
+            if not t.is_cuda:
+                raise FaError(FA_ERR_INVALID_ARG, "tensors must live on a CUDA device")
+            if not t.is_contiguous():
+                raise FaError(FA_ERR_INVALID_ARG, "tensors must be contiguous")
+
+
+# ---------------------------------------------------------------------------
+# C-ABI mirrors
+# ---------------------------------------------------------------------------
+def fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, scale, causal, window_left, window_right,
+           softcap, cu_seqlens, total_tokens, dtype, stream=None):
+    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, scale,
+                      int(causal), window_left, window_right, softcap, _ptr(cu_seqlens),
+                      total_tokens, dtype, _stream(stream)))
+
+
+def fa_bwd_workspace_size(B, Hq, S, D, total_tokens=0) -> int:
+    return int(lib.fa_bwd_workspace_size(B, Hq, S, D, total_tokens))
+
+
+def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, window_left,
+           window_right, softcap, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes,
+           stream=None):
+    _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                      _ptr(dk), _ptr(dv), B, Hq, Hkv, S, D, scale, int(causal), window_left,
+                      window_right, softcap, _ptr(cu_seqlens), total_tokens, dtype,
+                      _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def fa_kvcache_workspace_size(B, Hq, D, num_splits) -> int:
+    return int(lib.fa_kvcache_workspace_size(B, Hq, D, num_splits))
+
+
+def fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, out, lse, B,
+                   Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
+                   window_left, window_right, softcap, num_splits, dtype, workspace,
+                   workspace_bytes, stream=None):
+    _check(lib.fa_fwd_kvcache(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                              _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse), B, Hq,
+                              Hkv, D, page_size, max_pages_per_seq, num_pages, scale, int(causal),
+                              window_left, window_right, softcap, num_splits, dtype,
+                              _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def fa_get_device_status() -> int:
+    v = ctypes.c_int(0)
+    _check(lib.fa_get_device_status(ctypes.byref(v)))
+    return v.value
+
+
+# ---------------------------------------------------------------------------
+# tensor-level conveniences (allocation through torch only)
+# ---------------------------------------------------------------------------
+def _scale(scale, D):
+    return float(D) ** -0.5 if scale is None else float(scale)
+
+
+def fwd(q, k, v, scale=None, causal=False, window=(-1, -1), softcap=0.0, cu_seqlens=None,
+        max_seqlen=None, out=None, lse=None, stream=None):
+    """q (B,S,Hq,D), k/v (B,S,Hkv,D) -> (out, lse (B,Hq,S)); varlen: q (T,Hq,D),
+    cu_seqlens int32 (B+1) on the device, lse (Hq,T)."""
+    _need_cuda(q, k, v, cu_seqlens)
+    if cu_seqlens is None:
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+        T = 0
+        lse_shape = (B, Hq, S)
+    else:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise FaError(FA_ERR_INVALID_ARG, "max_seqlen is required with cu_seqlens")
+        S = int(max_seqlen)
+        lse_shape = (Hq, T)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, _scale(scale, D), causal, window[0], window[1],
+           softcap, cu_seqlens, T, _dt(q), stream)
+    return out, lse
+
+
+def bwd(q, k, v, out, lse, dout, scale=None, causal=False, window=(-1, -1), softcap=0.0,
+        cu_seqlens=None, max_seqlen=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(out * dout); layouts as in fwd."""
+    _need_cuda(q, k, v, out, lse, dout, cu_seqlens)
+    if cu_seqlens is None:
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+        T = 0
+    else:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        S = int(max_seqlen)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = fa_bwd_workspace_size(B, Hq, S, D, T)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, _scale(scale, D), causal,
+           window[0], window[1], softcap, cu_seqlens, T, _dt(q), workspace, workspace.numel(),
+           stream)
+    return dq, dk, dv
+
+
+def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_new=None,
+                scale=None, causal=True, window=(-1, -1), softcap=0.0, num_splits=1, out=None,
+                lse=None, workspace=None, stream=None):
+    """One decode step: q (B,1,Hq,D); caches (num_pages, page_size, Hkv, D);
+    block_table int32 (B, max_pages); cache_seqlens int32 (B). Appends
+    k_new/v_new (B,1,Hkv,D) in place, then attends. Returns (out, lse)."""
+    _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new)
+    B, _, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_cache.shape
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    nbytes = fa_kvcache_workspace_size(B, Hq, D, num_splits)
+    if workspace is None and nbytes > 0:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, out, lse, B, Hq,
+                   Hkv, D, page_size, block_table.shape[1], num_pages, _scale(scale, D), causal,
+                   window[0], window[1], softcap, num_splits, _dt(q), workspace,
+                   0 if workspace is None else workspace.numel(), stream)
+    return out, lse

@@ -1,0 +1,220 @@
+// Host side of the C ABI declared in include/fa.h: argument validation, TMA
+// descriptor encoding, launch configuration. The whole library is this one
+// translation unit (kernels are included as headers), so the device status
+// word in ptx.cuh is shared by every kernel and read back here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/fa.h"
+#include "ptx.cuh"
+#include "fwd_kernel.cuh"
+#include "bwd_kernel.cuh"
+#include "decode_kernel.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fa_status fail(fa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+fa_status ok() {
+  g_last_error.clear();
+  return FA_OK;
+}
+
+#define FA_CUDA_CHECK(expr)                                                            \
+  do {                                                                                 \
+    cudaError_t e_ = (expr);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(FA_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));       \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// device checks
+// ---------------------------------------------------------------------------
+fa_status check_device() {
+  static std::mutex mu;
+  static int verdict[128] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 128) return fail(FA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (verdict[dev] == 0) {
+    int major = 0, minor = 0;
+    FA_CUDA_CHECK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    FA_CUDA_CHECK(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    if (verdict[dev] == 2)
+      return fail(FA_ERR_UNSUPPORTED, "device %d has compute capability %d.%d; this library is built for sm_100a (10.0)",
+                  dev, major, minor);
+  }
+  if (verdict[dev] != 1) return fail(FA_ERR_UNSUPPORTED, "device %d is not compute capability 10.0", dev);
+  return FA_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a (tokens, heads, D) row-major 16-bit tensor; box = 64 columns
+// (128 B, one swizzle row) x 1 head x `rows` tokens, 128-byte swizzle.
+fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, int H, long long T,
+                       int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(rows)};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, dt == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// common option validation for fwd/bwd
+fa_status check_common(int B, int Hq, int Hkv, int S, int D, float scale, int wl, int wr,
+                       float softcap, fa_dtype dt, const int32_t* cu, int total) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1)
+    return fail(FA_ERR_INVALID_ARG, "B, Hq, Hkv and S must be >= 1 (got %d, %d, %d, %d)", B, Hq, Hkv, S);
+  if (Hq % Hkv != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be an integer multiple of Hkv (%d)", Hq, Hkv);
+  if (D != 64 && D != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+  if (wl < -1 || wr < -1) return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (got %d, %d)", wl, wr);
+  if (!(softcap >= 0.f) || !std::isfinite(softcap))
+    return fail(FA_ERR_INVALID_ARG, "softcap must be finite and >= 0");
+  if (dt != FA_BF16 && dt != FA_FP16) return fail(FA_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dt));
+  if (cu != nullptr && total < 1) return fail(FA_ERR_INVALID_ARG, "total_tokens must be >= 1 with cu_seqlens");
+  if (static_cast<long long>(Hq) * D * 2 % 16 != 0 || static_cast<long long>(Hkv) * D * 2 % 16 != 0)
+    return fail(FA_ERR_INVALID_ARG, "row strides must be multiples of 16 bytes");
+  const long long T = cu ? static_cast<long long>(total) : static_cast<long long>(B) * S;
+  if (T > (1ll << 31) - 1) return fail(FA_ERR_INVALID_ARG, "too many tokens");
+  return FA_OK;
+}
+
+template <typename K>
+fa_status set_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess)
+    return fail(FA_ERR_CUDA, "cudaFuncSetAttribute(smem=%d) failed: %s", bytes, cudaGetErrorString(e));
+  return FA_OK;
+}
+
+template <int kD, bool kBF16>
+fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const fa::FwdParams& p, cudaStream_t st) {
+  using Sh = fa::FwdShape<kD>;
+  auto kern = fa::fwd_kernel<kD, kBF16>;
+  fa_status s = set_smem(kern, Sh::kSmemBytes);
+  if (s != FA_OK) return s;
+  const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "grid too large");
+  kern<<<static_cast<unsigned>(grid), Sh::kThreads, Sh::kSmemBytes, st>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "fwd launch failed: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_last_error(void) { return g_last_error.c_str(); }
+
+const char* fa_version(void) { return "exact-attention-b200 0.1.0 (sm_100a)"; }
+
+fa_status fa_get_device_status(int* status_out) {
+  if (status_out == nullptr) return fail(FA_ERR_INVALID_ARG, "status_out is NULL");
+  int v = 0;
+  const int zero = 0;
+  FA_CUDA_CHECK(cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(int)));
+  FA_CUDA_CHECK(cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(int)));
+  *status_out = v == fa::kDevTimeout ? static_cast<int>(FA_ERR_TIMEOUT) : 0;
+  return ok();
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                 int Hkv, int S, int D, float scale, int causal, int window_left, int window_right,
+                 float softcap, const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype,
+                 void* stream) {
+  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd: null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be 16-byte aligned");
+  fa_status s = check_common(B, Hq, Hkv, S, D, scale, window_left, window_right, softcap, dtype,
+                             cu_seqlens, total_tokens);
+  if (s != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+
+  const long long T = cu_seqlens ? total_tokens : static_cast<long long>(B) * S;
+  CUtensorMap tq, tk, tv;
+  if ((s = make_map_thd(&tq, q, dtype, D, Hq, T, 128)) != FA_OK) return s;
+  if ((s = make_map_thd(&tk, k, dtype, D, Hkv, T, 128)) != FA_OK) return s;
+  if ((s = make_map_thd(&tv, v, dtype, D, Hkv, T, 128)) != FA_OK) return s;
+
+  fa::FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.total = static_cast<int>(T);
+  p.group = Hq / Hkv;
+  p.n_qblocks = (S + 255) / 256;
+  const float log2e = 1.4426950408889634f;
+  p.scale_log2 = scale * log2e;
+  p.softcap = softcap;
+  p.cap_in = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_out_log2 = softcap * log2e;
+  p.wl = window_left;
+  p.wr = causal ? 0 : window_right;
+  p.o = out;
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) {
+    s = dtype == FA_BF16 ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);
+  } else {
+    s = dtype == FA_BF16 ? launch_fwd<64, true>(tq, tk, tv, p, st) : launch_fwd<64, false>(tq, tk, tv, p, st);
+  }
+  if (s != FA_OK) return s;
+  return ok();
+}
+
+}  // extern "C"
+
+#include "bwd_api.inc"
+#include "decode_api.inc"

@@ -1,0 +1,413 @@
+// Forward attention kernel for sm_100a.
+//
+// One CTA computes 256 query rows (two 128-row Q tiles) of one (sequence,
+// query head) against the K/V tiles the mask leaves visible, with an online
+// softmax ("FlashAttention 实战指南" §长序列注意力为什么会爆内存: tile Q, K,
+// V into on-chip memory, update the row max and row sum tile by tile, never
+// materialise the attention matrix).
+//
+// Warp roles (320 threads):
+//   warp 0      TMA producer: Q tiles once, then K_j, V_j into a ring of
+//               shared-memory slots (128-byte swizzle).
+//   warp 1      MMA issuer (one lane): S_t = Q_t K_j^T into TMEM, then
+//               O_t += P_t V_j with P_t read from TMEM. Owns TMEM alloc.
+//   warps 2-5   softmax group 0 (Q tile 0), one thread per query row.
+//   warps 6-9   softmax group 1 (Q tile 1).
+// The two softmax groups alternate with the tensor core: while group 0
+// exponentiates S_0, the tensor core runs group 1's PV and QK, and so on.
+//
+// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 at 256,
+// O_1 at 256 + D. P_t (16-bit, two per 32-bit column) overwrites the upper
+// 64 columns of S_t after the row has been read into registers.
+//
+// The running max is only moved (and O rescaled) when a row max grows by
+// more than 2^8 in the exp2 domain; otherwise the stale max is kept, which
+// is exact after the final division by the row sum and keeps P <= 256.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  int B, Hq, Hkv, S, total;  // S: sequence length (max length when varlen)
+  int group;                 // Hq / Hkv
+  int n_qblocks;             // ceil(S / 256)
+  float scale_log2;          // scale * log2(e)
+  float softcap;             // 0 = off
+  float cap_in;              // scale / softcap
+  float cap_out_log2;        // softcap * log2(e)
+  int wl, wr;                // window, -1 = unbounded (causal already folded into wr)
+  void* o;
+  float* lse;
+  const int* cu_seqlens;     // nullable
+};
+
+template <int kD>
+struct FwdShape {
+  static constexpr int kBM = 128;                    // rows per Q tile
+  static constexpr int kBN = 128;                    // keys per KV tile
+  static constexpr int kChunks = kD / 64;            // 128-byte column chunks
+  static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 B
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = kD == 128 ? 4 : 8;  // K/V ring slots
+  static constexpr int kBarOffset = (2 + kStages) * kTileBytes;
+  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + align slack
+  static constexpr int kThreads = 320;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kColS = 0;      // + 128 * t
+  static constexpr int kColP = 64;     // + 128 * t
+  static constexpr int kColO = 256;    // + kD * t
+};
+
+// Barrier block in shared memory.
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t s_full[2];
+  uint64_t p_ready[2];
+  uint64_t o_final[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool fwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        atomicExch(&g_device_status, kDevTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Logit transform in the exp2 domain: scale (and optional tanh softcap).
+__device__ __forceinline__ float fwd_logit(float s, const FwdParams& p) {
+  if (p.softcap > 0.f) return p.cap_out_log2 * tanhf(s * p.cap_in);
+  return s * p.scale_log2;
+}
+
+template <int kD, bool kBF16>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Sh = FwdShape<kD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;                               // 2 tiles
+  uint8_t* sKV = smem + 2 * Sh::kTileBytes;         // kStages tiles
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + Sh::kBarOffset);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: heaviest query blocks first -------------------------------
+  const int bh = p.B * p.Hq;
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / bh;
+  const int rem = static_cast<int>(blockIdx.x) % bh;
+  const int h = rem % p.Hq;
+  const int b = rem / p.Hq;
+  int seq_start, seq_len;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    seq_len = p.cu_seqlens[b + 1] - seq_start;
+  } else {
+    seq_start = b * p.S;
+    seq_len = p.S;
+  }
+  const int q0 = qb * 256;
+  if (q0 >= seq_len) return;  // uniform across the CTA, before any barrier
+  const int kvh = h / p.group;
+
+  // visible key range of the whole 256-row block (self-attention: Sk = Sq)
+  const int row_hi = min(q0 + 255, seq_len - 1);
+  int key_hi = seq_len - 1;
+  if (p.wr >= 0) key_hi = min(key_hi, row_hi + p.wr);
+  int key_lo = 0;
+  if (p.wl >= 0) key_lo = max(0, q0 - p.wl);
+  const int n_begin = key_lo / Sh::kBN;
+  const int n_end = key_hi >= key_lo ? key_hi / Sh::kBN + 1 : n_begin;
+  const int n_tiles = n_end - n_begin;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < Sh::kStages; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_ready[t], 4);
+      mbar_init(&bars->o_final[t], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, Sh::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bars->q_full, 2 * Sh::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < Sh::kChunks; ++c)
+          tma_load_3d(&tm_q, &bars->q_full, sQ + t * Sh::kTileBytes + c * Sh::kChunkBytes, c * 64,
+                      h, seq_start + q0 + t * 128);
+      int fill = 0;
+      for (int j = 0; j < n_tiles && !*abort; ++j) {
+        const int tok = seq_start + (n_begin + j) * Sh::kBN;
+        for (int kv = 0; kv < 2; ++kv, ++fill) {
+          const int slot = fill % Sh::kStages;
+          const uint32_t ph = static_cast<uint32_t>(fill / Sh::kStages) & 1u;
+          if (!fwd_wait(&bars->kv_empty[slot], ph ^ 1u, abort)) break;
+          mbar_arrive_expect_tx(&bars->kv_full[slot], Sh::kTileBytes);
+          uint8_t* dst = sKV + slot * Sh::kTileBytes;
+          const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+          for (int c = 0; c < Sh::kChunks; ++c)
+            tma_load_3d(tm, &bars->kv_full[slot], dst + c * Sh::kChunkBytes, c * 64, kvh, tok);
+        }
+      }
+      // drain: every issued load must land before the CTA may exit
+      for (int f = max(0, fill - Sh::kStages); f < fill; ++f) {
+        const int slot = f % Sh::kStages;
+        mbar_wait(&bars->kv_full[slot], static_cast<uint32_t>(f / Sh::kStages) & 1u);
+      }
+      mbar_wait(&bars->q_full, 0);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (elect_one()) {
+      constexpr uint32_t id_qk = idesc_f16(kBF16, 128, 128, false, false);
+      constexpr uint32_t id_pv = idesc_f16(kBF16, 128, kD, false, true);
+      const uint32_t sq_addr = smem_u32(sQ);
+      const uint32_t skv_addr = smem_u32(sKV);
+      bool ok = fwd_wait(&bars->q_full, 0, abort);
+      tc_fence_after();
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t a0 = sq_addr + t * Sh::kTileBytes;
+        const uint32_t b0 = skv_addr + slot * Sh::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32;
+          umma_ss(tmem + Sh::kColS + 128 * t, sdesc_sw128(a0 + off, 16, 1024),
+                  sdesc_sw128(b0 + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool first) {
+        const uint32_t b0 = skv_addr + slot * Sh::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          umma_ts(tmem + Sh::kColO + kD * t, tmem + Sh::kColS + 128 * t + Sh::kColP + kk * 8,
+                  sdesc_sw128(b0 + kk * 2048, Sh::kChunkBytes, 1024), id_pv,
+                  (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      for (int it = 0; it < n_tiles && ok; ++it) {
+        const int fk = 2 * it, fv = 2 * it + 1;
+        const int sk = fk % Sh::kStages;
+        if (!(ok = fwd_wait(&bars->kv_full[sk], static_cast<uint32_t>(fk / Sh::kStages) & 1u, abort)))
+          break;
+        tc_fence_after();
+        if (it > 0) {
+          const int fvp = fv - 2, svp = fvp % Sh::kStages;
+          // PV_0 of the previous tile, then QK_0 of this tile
+          if (!(ok = fwd_wait(&bars->p_ready[0], static_cast<uint32_t>(it - 1) & 1u, abort))) break;
+          tc_fence_after();
+          issue_pv(0, svp, it == 1);
+          issue_qk(0, sk);
+          umma_commit(&bars->s_full[0]);
+          if (!(ok = fwd_wait(&bars->p_ready[1], static_cast<uint32_t>(it - 1) & 1u, abort))) break;
+          tc_fence_after();
+          issue_pv(1, svp, it == 1);
+          umma_commit(&bars->kv_empty[svp]);
+          issue_qk(1, sk);
+          umma_commit(&bars->s_full[1]);
+          umma_commit(&bars->kv_empty[sk]);
+        } else {
+          issue_qk(0, sk);
+          umma_commit(&bars->s_full[0]);
+          issue_qk(1, sk);
+          umma_commit(&bars->s_full[1]);
+          umma_commit(&bars->kv_empty[sk]);
+        }
+        // V_it must be resident before next round's PV
+        const int sv = fv % Sh::kStages;
+        if (!(ok = fwd_wait(&bars->kv_full[sv], static_cast<uint32_t>(fv / Sh::kStages) & 1u, abort)))
+          break;
+      }
+      if (ok && n_tiles > 0) {
+        const int fvl = 2 * (n_tiles - 1) + 1, svl = fvl % Sh::kStages;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = fwd_wait(&bars->p_ready[t], static_cast<uint32_t>(n_tiles - 1) & 1u, abort)))
+            break;
+          tc_fence_after();
+          issue_pv(t, svl, n_tiles == 1);
+          umma_commit(&bars->o_final[t]);
+        }
+        umma_commit(&bars->kv_empty[svl]);
+      }
+      // wait for everything this thread issued before TMEM is released
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ======================= softmax groups =======================
+    const int t = (warp - 2) >> 2;            // Q tile of this group
+    const int lane_base = 32 * (warp & 3);    // TMEM lanes this warp may touch
+    const int row = lane_base + lane;         // row within the Q tile
+    const int qrow = q0 + t * 128 + row;      // row within the sequence
+    const uint32_t t_s = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColS + 128 * t;
+    const uint32_t t_p = t_s + Sh::kColP;
+    const uint32_t t_o = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColO + kD * t;
+    // tile-level visibility of this 128-row tile
+    const int r_lo = q0 + t * 128 + lane_base;   // this warp's first row
+    const int r_hi = r_lo + 31;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+      if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it) & 1u, abort))) break;
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(t_s + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+        }
+      }
+      const int k0 = (n_begin + it) * Sh::kBN;
+      // does any (row, key) of this warp's 32 x 128 block need masking?
+      bool need_mask = (k0 + 127 >= seq_len);
+      if (p.wr >= 0) need_mask |= (k0 + 127 > r_lo + p.wr);
+      if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
+      float mt = -INFINITY;
+      if (need_mask) {
+        int jmax = seq_len - 1;
+        if (p.wr >= 0) jmax = min(jmax, qrow + p.wr);
+        int jmin = p.wl >= 0 ? qrow - p.wl : INT32_MIN;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int j = k0 + i;
+          const float v = (j > jmax || j < jmin) ? -INFINITY : fwd_logit(x[i], p);
+          x[i] = v;
+          mt = fmaxf(mt, v);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          x[i] = fwd_logit(x[i], p);
+          mt = fmaxf(mt, x[i]);
+        }
+      }
+      const float m_new = fmaxf(m_run, mt);
+      const bool grow = m_new > m_run + 8.0f;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
+        if (m_new != -INFINITY) m_run = m_new;
+        l_run *= alpha;
+        if (it > 0) {
+          // O_t holds the previous PV results (complete: s_full commit
+          // follows them); rescale it in place
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_o + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(t_o + c * 32, r);
+          }
+        }
+      }
+      const float base = (m_run == -INFINITY) ? 0.f : m_run;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float e0 = ex2_approx(x[c * 64 + 2 * i] - base);
+          const float e1 = ex2_approx(x[c * 64 + 2 * i + 1] - base);
+          lsum += e0 + e1;
+          r[i] = pack2<kBF16>(e0, e1);
+        }
+        tmem_st32(t_p + c * 32, r);
+      }
+      l_run += lsum;
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_ready[t]);
+    }
+    // ---- epilogue: O / l and LSE ----
+    if (ok && n_tiles > 0) ok = fwd_wait(&bars->o_final[t], 0, abort);
+    tc_fence_after();
+    const bool valid_row = qrow < seq_len;
+    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+    typedef uint4 Vec;
+    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
+                    (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD * 2;
+#pragma unroll 1
+    for (int c = 0; c < kD / 32; ++c) {
+      uint32_t r[32];
+      if (ok && n_tiles > 0) {
+        tmem_ld32(t_o + c * 32, r);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        w[i] = pack2<kBF16>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+      if (valid_row) {
+        Vec* dst = reinterpret_cast<Vec*>(orow + c * 64);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    }
+    if (valid_row) {
+      const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      const size_t li = p.cu_seqlens != nullptr
+                            ? static_cast<size_t>(h) * p.total + seq_start + qrow
+                            : (static_cast<size_t>(b) * p.Hq + h) * p.S + qrow;
+      p.lse[li] = lse;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Sh::kTmemCols);
+  }
+}
+
+}  // namespace fa

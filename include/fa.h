@@ -1,0 +1,164 @@
+/*
+ * exact-attention for B200 (sm_100a): C ABI.
+ *
+ * Exact scaled-dot-product attention O = softmax(scale * Q K^T) V computed
+ * tile by tile with an online softmax, so the n x n score matrix never reaches
+ * device memory ("FlashAttention 实战指南:如何把训练内存省 20 倍、速度提 4 倍",
+ * §长序列注意力为什么会爆内存: tiling into on-chip memory, a running row max
+ * and row sum, recomputation in the backward pass; the result equals the
+ * plain three-step definition, "AI模型推理优化 Flash Attention原理",
+ * §先搞清楚原理).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor arguments are DEVICE pointers owned by the caller, contiguous
+ *   with the last dimension at stride 1, 16-byte aligned. The library never
+ *   allocates or frees device memory; scratch space is passed in through a
+ *   caller-owned workspace sized by the matching *_workspace_size() query.
+ * - Layout (guide §上手…三步走): q (B, S, Hq, D); k, v (B, S, Hkv, D);
+ *   out like q; lse float32 (B, Hq, S).
+ *   Varlen (cu_seqlens != NULL): sequences are packed along the token axis,
+ *   q (total, Hq, D), k, v (total, Hkv, D), lse (Hq, total); cu_seqlens is a
+ *   DEVICE int32 array of B + 1 non-decreasing prefix sums with
+ *   cu_seqlens[0] = 0 and cu_seqlens[B] = total; S is then the maximum
+ *   sequence length (an upper bound is fine).
+ * - dtype applies to q, k, v, out, dout, dq, dk, dv, k_new, v_new and the
+ *   caches alike; arithmetic accumulates in float32.
+ * - Options (guide §进阶参数): causal; a sliding window
+ *   (window_left, window_right), -1 meaning unbounded, bounds inclusive,
+ *   causal forcing window_right = 0; softcap > 0 replaces every logit x by
+ *   softcap * tanh(x / softcap) after scaling (0 disables it); GQA: Hq must be
+ *   an integer multiple of Hkv and query head h reads kv head h / (Hq / Hkv).
+ *   When the query and key lengths differ (decode) the causal diagonal is
+ *   aligned to the bottom-right corner.
+ * - LSE is the natural-log log-sum-exp of each row's scaled (and softcapped)
+ *   logits; a row with no visible key gets O = 0 and LSE = -inf.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and returns after the launch. Errors never abort: the
+ *   call returns a status and fa_last_error() describes it. Invalid
+ *   arguments are rejected on the host before anything is launched.
+ * - Head dimension D must be 64 or 128. The device must be compute
+ *   capability 10.0 (B200).
+ */
+#ifndef EXACT_ATTENTION_FA_H_
+#define EXACT_ATTENTION_FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad option, misaligned */
+  FA_ERR_UNSUPPORTED = 2, /* head dim or device not supported */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = 4      /* a kernel gave up on a bounded wait (see fa_get_device_status) */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Forward pass: out = softmax(scale * q k^T [softcap, mask]) v and lse.
+ * Guide §长序列注意力为什么会爆内存 (tiling + online softmax), §进阶参数
+ * (causal, window, softcap, GQA), §上手…三步走 (varlen via cu_seqlens).
+ *   total_tokens: number of packed tokens when cu_seqlens != NULL, else ignored.
+ * Errors: FA_ERR_INVALID_ARG for null q/k/v/out/lse, B/Hq/Hkv/S < 1,
+ *   Hq % Hkv != 0, window < -1, softcap < 0 or not finite, scale not finite,
+ *   misaligned pointers; FA_ERR_UNSUPPORTED for D not in {64, 128} or a
+ *   device other than compute capability 10.0; FA_ERR_CUDA on launch failure.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                 int Hq, int Hkv, int S, int D, float scale, int causal, int window_left,
+                 int window_right, float softcap, const int32_t* cu_seqlens, int total_tokens,
+                 fa_dtype dtype, void* stream);
+
+/*
+ * Workspace bytes needed by fa_bwd for these sizes (float32 dQ accumulator
+ * plus per-row dot(dO, O)); total_tokens as in fa_fwd (ignored if <= 0).
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int Hq, int S, int D, int total_tokens);
+
+/*
+ * Backward pass: gradients of sum(out * dout) with respect to q, k, v, by
+ * recomputing the attention probabilities from q, k and the saved lse
+ * instead of storing them (guide §长序列注意力为什么会爆内存: the backward
+ * pass does not keep the attention matrix and recomputes it when needed).
+ *   out, lse: the results of fa_fwd with the same arguments.
+ *   dq like q; dk, dv like k, v (for GQA the contributions of every query
+ *   head of a group are summed into the shared kv head).
+ *   workspace: device memory of at least fa_bwd_workspace_size() bytes,
+ *   256-byte aligned; its contents on entry do not matter.
+ * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null dout/dq/dk/dv or a
+ *   workspace that is null or too small.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S,
+                 int D, float scale, int causal, int window_left, int window_right, float softcap,
+                 const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/* Workspace bytes needed by fa_fwd_kvcache (float32 per-split partial
+ * outputs and log-sum-exps); 0 when num_splits == 1. */
+FA_API size_t fa_kvcache_workspace_size(int B, int Hq, int D, int num_splits);
+
+/*
+ * One decode step against a paged KV cache (guide §增量解码场景
+ * flash_attn_with_kvcache): the new key/value of each sequence is appended
+ * IN PLACE at logical position cache_seqlens[b], then the single query
+ * attends over the cache_seqlens[b] + 1 keys; the KV range is split into
+ * num_splits parts whose partial results are merged by a log-sum-exp combine.
+ *   q (B, 1, Hq, D); k_new, v_new (B, 1, Hkv, D), or both NULL for no append
+ *     (the query then attends over cache_seqlens[b] keys).
+ *   k_cache, v_cache (num_pages, page_size, Hkv, D): the page pool; logical
+ *     position p of sequence b lives in page block_table[b, p / page_size],
+ *     slot p % page_size ("FlashAttention技术深度解析" §动态缓存架构: a page
+ *     table maps logical blocks to physical ones).
+ *   block_table: DEVICE int32 (B, max_pages_per_seq), every referenced entry
+ *     in [0, num_pages).
+ *   cache_seqlens: DEVICE int32 (B), valid length BEFORE the append; the
+ *     library does not increment it (the caller advances its own position).
+ *   out (B, 1, Hq, D); lse float32 (B, Hq, 1).
+ *   page_size: a multiple of 64.
+ *   workspace: at least fa_kvcache_workspace_size(B, Hq, D, num_splits)
+ *     bytes of device memory (may be NULL when that is 0).
+ * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null cache/table/lengths,
+ *   num_splits < 1, page_size not a positive multiple of 64, or a workspace
+ *   that is too small. Lengths and table entries live on the device and are
+ *   not read by the host; cache_seqlens[b] (+1 with an append) must not
+ *   exceed max_pages_per_seq * page_size.
+ */
+FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                         void* v_cache, const int32_t* block_table, const int32_t* cache_seqlens,
+                         void* out, float* lse, int B, int Hq, int Hkv, int D, int page_size,
+                         int max_pages_per_seq, int num_pages, float scale, int causal,
+                         int window_left, int window_right, float softcap, int num_splits,
+                         fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Reads and clears the library's device status word on the current device
+ * (synchronous). *status_out = 0 if no kernel reported a problem since the
+ * last call, FA_ERR_TIMEOUT if one gave up on a bounded wait. Returns
+ * FA_ERR_CUDA if the word cannot be read.
+ */
+FA_API fa_status fa_get_device_status(int* status_out);
+
+/* Message describing the last error returned on the calling thread. */
+FA_API const char* fa_last_error(void);
+
+/* Library version string. */
+FA_API const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_FA_H_ */

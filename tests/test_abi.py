@@ -1,0 +1,151 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The shared library must load on a machine without a GPU, export every
+function include/fa.h declares, and reject invalid arguments on the host
+with a status code and a message, before anything is launched.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from exact_attention_149_b200 import build
+
+    build.build()
+    import exact_attention_149_b200 as m
+
+    return m
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            src = open(os.path.join(inc, fn), encoding="utf-8").read()
+            names += re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_bwd_workspace_size",
+              "fa_kvcache_workspace_size", "fa_get_device_status", "fa_last_error", "fa_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(fa):
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_version(fa):
+    assert "sm_100a" in fa.fa_version()
+
+
+def test_workspace_sizes(fa):
+    # dQ accumulator (float32 T*Hq*D) + row dots (float32 T*Hq), each padded to 256 B
+    n = fa.fa_bwd_workspace_size(2, 32, 8192, 128)
+    assert n == 2 * 8192 * 32 * 128 * 4 + 2 * 8192 * 32 * 4
+    assert fa.fa_bwd_workspace_size(3, 4, 0, 128, 1000) == 1000 * 4 * 128 * 4 + 16128 + 256 * 0
+    assert fa.fa_kvcache_workspace_size(64, 32, 128, 1) == 0
+    assert fa.fa_kvcache_workspace_size(64, 32, 128, 16) == 16 * 64 * 32 * 129 * 4
+
+
+def _fwd_status(fa, **kw):
+    args = dict(q=16, k=16, v=16, out=16, lse=16, B=1, Hq=2, Hkv=2, S=128, D=64, scale=0.125,
+                causal=0, wl=-1, wr=-1, softcap=0.0, cu=None, total=0, dtype=0)
+    args.update(kw)
+    return fa.lib.fa_fwd(args["q"], args["k"], args["v"], args["out"], args["lse"], args["B"],
+                         args["Hq"], args["Hkv"], args["S"], args["D"], args["scale"],
+                         args["causal"], args["wl"], args["wr"], args["softcap"], args["cu"],
+                         args["total"], args["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1),
+    (dict(out=None), 1),
+    (dict(q=8), 1),                 # misaligned
+    (dict(B=0), 1),
+    (dict(S=0), 1),
+    (dict(Hq=3, Hkv=2), 1),         # Hq not a multiple of Hkv
+    (dict(wl=-2), 1),
+    (dict(softcap=-1.0), 1),
+    (dict(softcap=float("inf")), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(dtype=7), 1),
+    (dict(D=96), 2),                # unsupported head dim
+    (dict(D=256), 2),
+    (dict(cu=16, total=0), 1),
+])
+def test_fwd_rejects_bad_arguments(fa, kw, status):
+    assert _fwd_status(fa, **kw) == status
+    assert fa.fa_last_error() != ""
+
+
+def test_bwd_rejects_bad_arguments(fa):
+    lib = fa.lib
+    base = [16] * 9 + [1, 2, 2, 128, 64, 0.125, 0, -1, -1, 0.0, None, 0, 0]
+    # null dout
+    a = list(base)
+    a[5] = None
+    assert lib.fa_bwd(*a, 16, 1 << 20, None) in (1, 2)
+    # workspace too small
+    assert lib.fa_bwd(*base, 16, 8, None) in (1, 2)
+    # workspace missing
+    assert lib.fa_bwd(*base, None, 1 << 20, None) in (1, 2)
+
+
+def test_kvcache_rejects_bad_arguments(fa):
+    lib = fa.lib
+
+    def call(**kw):
+        a = dict(q=16, kn=16, vn=16, kc=16, vc=16, bt=16, cs=16, out=16, lse=16, B=2, Hq=4,
+                 Hkv=2, D=128, ps=256, mp=4, npg=8, scale=0.1, causal=1, wl=-1, wr=-1,
+                 softcap=0.0, splits=1, dtype=0, ws=None, wsb=0)
+        a.update(kw)
+        return lib.fa_fwd_kvcache(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["bt"], a["cs"],
+                                  a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["D"], a["ps"],
+                                  a["mp"], a["npg"], a["scale"], a["causal"], a["wl"], a["wr"],
+                                  a["softcap"], a["splits"], a["dtype"], a["ws"], a["wsb"], None)
+
+    assert call(kc=None) == 1
+    assert call(bt=None) == 1
+    assert call(cs=None) == 1
+    assert call(splits=0) == 1
+    assert call(ps=100) == 1
+    assert call(Hq=3) == 1
+    assert call(kn=None) == 1 or call(kn=None) == 3  # k_new without v_new is invalid
+    assert call(splits=4, ws=None, wsb=0) == 1        # workspace required
+    assert call(D=80) == 2
+
+
+def test_valid_call_without_gpu_reports_cuda_error(fa):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _fwd_status(fa) == 3  # FA_ERR_CUDA: no device to launch on
+    assert "cuda" in fa.fa_last_error().lower() or "device" in fa.fa_last_error().lower()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """The binding raises on import when libfa.so is absent: no fallback."""
+    import subprocess
+    import sys
+
+    pkg = os.path.join(ROOT, "exact_attention_149_b200")
+    dst = tmp_path / "exact_attention_149_b200"
+    dst.mkdir()
+    (dst / "__init__.py").write_text(open(os.path.join(pkg, "__init__.py"), encoding="utf-8").read())
+    r = subprocess.run([sys.executable, "-c", "import exact_attention_149_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libfa.so" in r.stderr
