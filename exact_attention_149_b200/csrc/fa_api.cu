@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -163,7 +164,12 @@ fa_status fa_get_device_status(int* status_out) {
   const int zero = 0;
   FA_CUDA_CHECK(cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(int)));
   FA_CUDA_CHECK(cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(int)));
-  *status_out = v == fa::kDevTimeout ? static_cast<int>(FA_ERR_TIMEOUT) : 0;
+  if (v == fa::kDevTimeout)
+    *status_out = static_cast<int>(FA_ERR_TIMEOUT);
+  else if (v == fa::kDevBadIndex)
+    *status_out = static_cast<int>(FA_ERR_INVALID_ARG);
+  else
+    *status_out = 0;
   return ok();
 }
 

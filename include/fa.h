@@ -146,8 +146,10 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_
 /*
  * Reads and clears the library's device status word on the current device
  * (synchronous). *status_out = 0 if no kernel reported a problem since the
- * last call, FA_ERR_TIMEOUT if one gave up on a bounded wait. Returns
- * FA_ERR_CUDA if the word cannot be read.
+ * last call, FA_ERR_TIMEOUT if one gave up on a bounded wait, and
+ * FA_ERR_INVALID_ARG if a decode kernel met a cache length or page-table
+ * entry out of range (it then skipped the out-of-range access and its output
+ * is not valid). Returns FA_ERR_CUDA if the word cannot be read.
  */
 FA_API fa_status fa_get_device_status(int* status_out);
 
