@@ -1,0 +1,471 @@
+"""Benchmark of the exact-attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workloads (seeded synthetic N(0,1) bf16 inputs; the pages' own benchmark,
+fp16/bf16 x head dim 64/128 x sequence 512..16k, ships no data):
+
+* headline step: forward + backward of causal attention, B=2, Hq=Hkv=32,
+  S=8192, D=128 (q, k, v, dO resident in HBM; 402 MB of q/k/v, larger than
+  the 126 MB L2, so no flush is needed between steps). FLOPs are counted as
+  4*D per visible (query, key) pair for the forward and 10*D for the
+  backward; masked pairs are not counted.
+* varlen forward: 65536 packed tokens, GQA 32/8, window (4096, 0), softcap 50.
+* paged decode: B=64, GQA 32/8, D=128, cache lengths 1024..32768, page 256,
+  num_splits 1, 4, 16; algorithmic bytes = every visible K and V row once.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
+torch.cuda.synchronize(), measured with CUDA events on the launching stream;
+with N > 1 ranks (torchrun) every rank runs its own replica and the maximum
+time over ranks is used. SM clocks and throttle reasons are sampled through
+NVML during the timed region.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import attn_workloads as W  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    out = dict(PEAKS_FALLBACK)
+    out["source"] = "fallback"
+    return out
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only: no data-path collective)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._stop.clear()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None):
+    """Run fn() warmup times, then time `steps` calls with CUDA events on the
+    current stream; returns max-over-ranks milliseconds per call."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if sampler is not None:
+        sampler.start()
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.stop()
+    dist.barrier()
+    ms = start.elapsed_time(end) / steps
+    return dist.max(ms)
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def prefill_inputs(dev):
+    c = W.CONFIGS[3]
+    inp = W.make_fwd_inputs(c.B, c.S, c.Hq, c.Hkv, c.D, c.dtype, seed=1000 + c.cid, with_do=True)
+    pairs = W.visible_pairs(c.S, c.S, c.causal, *c.window) * c.B
+    return c, inp, pairs
+
+
+def run_ours(args, dist: Dist):
+    import exact_attention_149_b200 as fa
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    res = {}
+    # -------------------- headline: causal prefill fwd + bwd --------------------
+    c, inp, pairs = prefill_inputs(dev)
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    fwd_flop = W.fwd_flops(pairs, c.D, c.Hq)
+    bwd_flop = W.bwd_flops(pairs, c.D, c.Hq)
+    have_bwd = True
+    out = torch.empty_like(q)
+    lse = torch.empty((c.B, c.Hq, c.S), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(c.B, c.Hq, c.S, c.D), dtype=torch.uint8, device=dev)
+
+    def step_fwd():
+        fa.fwd(q, k, v, scale=c.scale, causal=True, out=out, lse=lse)
+
+    def step_bwd():
+        fa.bwd(q, k, v, out, lse, do, scale=c.scale, causal=True, dq=dq, dk=dk, dv=dv,
+               workspace=ws)
+
+    step_fwd()
+    torch.cuda.synchronize()
+    try:
+        step_bwd()
+        torch.cuda.synchronize()
+    except fa.FaError:
+        have_bwd = False
+
+    def step():
+        step_fwd()
+        if have_bwd:
+            step_bwd()
+
+    sampler = ClockSampler(dev.index) if dist.rank == 0 else None
+    ms_step = timed(step, args.steps, args.warmup, dist, sampler)
+    ms_fwd = timed(step_fwd, args.steps, 1, dist)
+    ms_bwd = timed(step_bwd, args.steps, 1, dist) if have_bwd else None
+    flop_step = fwd_flop + (bwd_flop if have_bwd else 0)
+    value = dist.world * flop_step / (ms_step * 1e-3) / 1e12
+    res["fwd"] = {"ms": ms_fwd, "tflops": fwd_flop / (ms_fwd * 1e-3) / 1e12,
+                  "flop": fwd_flop}
+    res["fwd"]["frac_of_bf16_peak"] = res["fwd"]["tflops"] / peaks["bf16_tflops"]
+    if have_bwd:
+        res["bwd"] = {"ms": ms_bwd, "tflops": bwd_flop / (ms_bwd * 1e-3) / 1e12, "flop": bwd_flop}
+        res["bwd"]["frac_of_bf16_peak"] = res["bwd"]["tflops"] / peaks["bf16_tflops"]
+
+    # -------------------- end to end through the public API --------------------
+    hq_, hk_, hv_, hdo_ = (inp[n].pin_memory() for n in ("q", "k", "v", "do"))
+    h_out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    h_dq = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    h_dk = torch.empty(k.shape, dtype=k.dtype).pin_memory()
+    h_dv = torch.empty(v.shape, dtype=v.dtype).pin_memory()
+
+    def step_e2e():
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        do.copy_(hdo_, non_blocking=True)
+        step_fwd()
+        h_out.copy_(out, non_blocking=True)
+        if have_bwd:
+            step_bwd()
+            h_dq.copy_(dq, non_blocking=True)
+            h_dk.copy_(dk, non_blocking=True)
+            h_dv.copy_(dv, non_blocking=True)
+
+    ms_e2e = timed(step_e2e, max(2, args.steps // 2), 1, dist)
+    h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hdo_))
+    d2h = h_out.numel() * 2 + ((h_dq.numel() + h_dk.numel() + h_dv.numel()) * 2 if have_bwd else 0)
+    e2e = {"value": dist.world * flop_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del hq_, hk_, hv_, hdo_, h_out, h_dq, h_dk, h_dv
+
+    # -------------------- varlen forward (GQA, window, softcap) --------------------
+    cv = W.CONFIGS[4]
+    vin = W.make_varlen_inputs(None, cv.Hq, cv.Hkv, cv.D, cv.dtype, seed=1000 + cv.cid,
+                               total=cv.total, len_lo=cv.len_lo, len_hi=cv.len_hi)
+    vq, vk, vv = (vin[n].to(dev) for n in ("q", "k", "v"))
+    cu = vin["cu_seqlens"].to(dev)
+    vout = torch.empty_like(vq)
+    vlse = torch.empty((cv.Hq, cv.total), dtype=torch.float32, device=dev)
+    vpairs = W.varlen_visible_pairs(vin["lengths"], cv.causal, *cv.window)
+    vflop = W.fwd_flops(vpairs, cv.D, cv.Hq)
+
+    def step_varlen():
+        fa.fwd(vq, vk, vv, scale=cv.scale, causal=True, window=cv.window, softcap=cv.softcap,
+               cu_seqlens=cu, max_seqlen=max(vin["lengths"]), out=vout, lse=vlse)
+
+    ms_var = timed(step_varlen, args.steps, args.warmup, dist)
+    res["varlen_fwd"] = {"ms": ms_var, "tflops": vflop / (ms_var * 1e-3) / 1e12, "flop": vflop,
+                         "lengths": vin["lengths"]}
+    res["varlen_fwd"]["frac_of_bf16_peak"] = res["varlen_fwd"]["tflops"] / peaks["bf16_tflops"]
+    del vq, vk, vv, vout, vlse
+
+    # -------------------- paged split-KV decode --------------------
+    cd = W.CONFIGS[5]
+    st = W.make_decode_structure(cd.B, cd.Hq, cd.Hkv, cd.D, cd.len_lo, cd.len_hi, cd.page_size,
+                                 cd.dtype, seed=1000 + cd.cid)
+    shape = (st["num_pages"], st["page_size"], cd.Hkv, cd.D)
+    kc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    W.fill_paged_pool(st, kc, vc)
+    dq_ = st["q"].to(dev)
+    kn, vn = st["k_new"].to(dev), st["v_new"].to(dev)
+    cs, bt = st["cache_seqlens"].to(dev), st["block_table"].to(dev)
+    kv_bytes = W.decode_kv_bytes(st["cache_seqlens"], cd.Hkv, cd.D)
+    dec = {"kv_bytes": kv_bytes, "splits": {}}
+    dout = torch.empty_like(dq_)
+    dlse = torch.empty((cd.B, cd.Hq, 1), dtype=torch.float32, device=dev)
+    for splits in cd.splits:
+        wsd = fa.fa_kvcache_workspace_size(cd.B, cd.Hq, cd.D, splits)
+        wsb = torch.empty(max(wsd, 1), dtype=torch.uint8, device=dev)
+
+        def step_dec(splits=splits, wsb=wsb):
+            fa.fwd_kvcache(dq_, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale, causal=True,
+                           num_splits=splits, out=dout, lse=dlse, workspace=wsb)
+
+        ms_d = timed(step_dec, max(args.steps, 20), args.warmup, dist)
+        gbs = kv_bytes / (ms_d * 1e-3) / 1e9
+        dec["splits"][str(splits)] = {"ms": ms_d, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+    best = max(dec["splits"].values(), key=lambda d: d["gbs"])
+    dec["best_gbs"] = best["gbs"]
+    dec["best_frac_of_hbm"] = best["frac_of_hbm"]
+    res["decode"] = dec
+    del kc, vc
+    torch.cuda.empty_cache()
+
+    # -------------------- roofline of the dominant kernel --------------------
+    kern_times = {"fwd_kernel": ms_fwd}
+    if have_bwd:
+        kern_times["bwd (pre+main+post)"] = ms_bwd
+    dominant = max(kern_times, key=kern_times.get)
+    if dominant == "fwd_kernel":
+        achieved = fwd_flop / (ms_fwd * 1e-3) / 1e12
+    else:
+        achieved = bwd_flop / (ms_bwd * 1e-3) / 1e12
+    roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peaks["source"] + " burst bf16 (cuBLAS)"}
+
+    launches_per_step = 1 + (3 if have_bwd else 0)
+    line = {
+        "metric": "attention fwd+bwd TFLOP/s, causal B2 H32 S8192 D128 bf16 "
+                  "(decode KV GB/s and varlen fwd reported alongside)",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16, seeded (no dataset exists for this benchmark)",
+        "config": {"workload": "fwd+bwd causal B2 Hq32 Hkv32 S8192 D128 bf16" if have_bwd
+                   else "fwd causal B2 Hq32 Hkv32 S8192 D128 bf16",
+                   "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "S": c.S, "D": c.D, "causal": True,
+                   "l2": "inputs larger than L2 (q,k,v 402 MB), no flush",
+                   "parallelism": f"replicas x{dist.world}"},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "roofline": roofline,
+        "peaks": peaks,
+        "clocks": sampler.summary() if sampler is not None else None,
+        **res,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the headline workload
+# ---------------------------------------------------------------------------
+def _oracle_sample(c, inp, seconds_budget):
+    """Time the oracle's forward and backward on whole heads of the causal
+    S8192 workload until about `seconds_budget` seconds have passed."""
+    import numpy as np
+
+    from oracle import head_bwd, head_fwd
+
+    done_flop = 0
+    heads = 0
+    t0 = time.perf_counter()
+    pairs_head = W.visible_pairs(c.S, c.S, True)
+    for b in range(c.B):
+        for h in range(c.Hq):
+            qh = inp["q"][b, :, h]
+            kh = inp["k"][b, :, h]
+            vh = inp["v"][b, :, h]
+            doh = inp["do"][b, :, h]
+            head_fwd(qh, kh, vh, c.scale, True)
+            head_bwd(qh, kh, vh, doh, c.scale, True)
+            heads += 1
+            done_flop += W.fwd_flops(pairs_head, c.D, 1) + W.bwd_flops(pairs_head, c.D, 1)
+            if time.perf_counter() - t0 > seconds_budget:
+                break
+        else:
+            continue
+        break
+    dt = time.perf_counter() - t0
+    del np
+    return done_flop, dt, heads
+
+
+def cpu_baseline(seconds):
+    c = W.CONFIGS[3]
+    inp = W.make_fwd_inputs(c.B, c.S, c.Hq, c.Hkv, c.D, c.dtype, seed=1000 + c.cid, with_do=True)
+    flop, dt, heads = _oracle_sample(c, inp, seconds)
+    return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{heads} whole head(s) (b, h) of the causal B2 H32 S8192 D128 workload, "
+                      f"fwd + bwd in fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return None
+    c = W.CONFIGS[3]
+    inp = W.make_fwd_inputs(c.B, c.S, c.Hq, c.Hkv, c.D, c.dtype, seed=1000 + c.cid, with_do=True)
+    per_step = []
+    flop_total = 0
+    heads_total = 0
+    budget = max(2.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup and 1):
+        _oracle_sample(c, inp, 0.0)  # one head: warm BLAS
+    for _ in range(args.steps):
+        flop, dt, heads = _oracle_sample(c, inp, budget)
+        per_step.append(dt)
+        flop_total += flop
+        heads_total += heads
+    t = sum(per_step)
+    value = flop_total / t / 1e12
+    line = {
+        "impl": "reference",
+        "metric": "attention fwd+bwd TFLOP/s, causal B2 H32 S8192 D128 bf16 "
+                  "(decode KV GB/s and varlen fwd reported alongside)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic N(0,1) bf16 inputs, seeded; each step a bounded sample of whole heads",
+        "config": {"workload": "fwd+bwd causal B2 Hq32 Hkv32 S8192 D128 bf16", "B": c.B,
+                   "Hq": c.Hq, "Hkv": c.Hkv, "S": c.S, "D": c.D, "causal": True},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "kind": "oracle",
+                         "cores": len(os.sched_getaffinity(0)),
+                         "sample": f"{heads_total} head(s) over {args.steps} step(s), fp64 numpy"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, dist)
+        else:
+            line = run_ours(args, dist)
+        if dist.rank == 0 and line is not None:
+            print(json.dumps(line))
+            sys.stdout.flush()
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,3 +1,523 @@
-// Backward attention kernels (filled in below the forward path).
+// Backward attention kernels for sm_100a. The attention matrix is never
+// stored: P is recomputed from Q, K and the saved LSE ("FlashAttention 实战指南"
+// §长序列注意力为什么会爆内存: the backward pass recomputes the attention
+// matrix when it needs it instead of keeping it).
+//
+// With P the softmax probabilities of the forward pass,
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * O)),
+//   dQ = scale * dS K,  dK = scale * dS^T Q
+// (and dS picks up the factor 1 - tanh^2 under softcap).
+//
+//   bwd_pre_kernel   Drow = rowsum(dO * O) per (token, query head); zero the
+//                    float32 dQ accumulator.
+//   bwd_main_kernel  one CTA per (sequence, kv head, 128-key tile); K and V
+//                    stay resident while the CTA walks every query head of
+//                    the GQA group and every 128-row Q tile that can see the
+//                    keys, accumulating dK and dV in tensor memory; each
+//                    tile's dQ contribution is added to the accumulator with
+//                    float4 atomics.
+//   bwd_post_kernel  dQ accumulator -> 16-bit dq.
+//
+// bwd_main warp roles (320 threads):
+//   warp 0     TMA producer: K, V once; Q_i and dO_i into a 2-slot ring.
+//   warp 1     MMA issuer (one lane), TMEM owner.
+//   warps 2-5  "P/dS" group, one thread per key row: P^T = exp(S^T - LSE),
+//              dS^T = P^T * (dP^T - Drow); P^T -> TMEM (16-bit), dS^T -> smem.
+//   warps 6-9  "dQ" group, one thread per query row: dQ tile TMEM -> atomics;
+//              at the end both groups write dK and dV.
+// TMEM columns: A [0,128) S^T then P^T; B [128,256) dP^T then dQ;
+// dV [256, 256+D); dK [256+D, 256+2D).
 #pragma once
+
 #include "ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  int B, Hq, Hkv, S, total, group;
+  int n_ktiles;              // ceil(S / 128)
+  float scale;               // multiplies dS (so dQ, dK come out scaled)
+  float scale_log2;          // scale * log2(e)
+  float softcap, cap_in, cap_out_log2;
+  int wl, wr;                // window (causal folded into wr)
+  const void* o;
+  const void* dout;
+  const float* lse;
+  float* drow;               // LSE layout
+  float* dq_acc;             // (T, Hq, D) float32
+  void* dq;                  // (T, Hq, D) 16-bit
+  void* dk;                  // (T, Hkv, D)
+  void* dv;
+  const int* cu_seqlens;
+};
+
+// ---------------------------------------------------------------------------
+// pre: Drow and zeroed dQ accumulator. One warp per (token, head) row.
+// ---------------------------------------------------------------------------
+template <int kD, bool kBF16>
+__global__ void bwd_pre_kernel(const BwdParams p) {
+  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(p.total) * p.Hq;
+  if (gw >= rows) return;
+  const int tok = static_cast<int>(gw / p.Hq);
+  const int h = static_cast<int>(gw % p.Hq);
+  constexpr int kPer = kD / 32;  // elements per lane
+  const uint16_t* o = static_cast<const uint16_t*>(p.o) + gw * kD + lane * kPer;
+  const uint16_t* d = static_cast<const uint16_t*>(p.dout) + gw * kD + lane * kPer;
+  float acc = 0.f;
+  if constexpr (kPer == 4) {
+    const uint2 ov = *reinterpret_cast<const uint2*>(o);
+    const uint2 dv = *reinterpret_cast<const uint2*>(d);
+    const float2 o0 = unpack2<kBF16>(ov.x), o1 = unpack2<kBF16>(ov.y);
+    const float2 d0 = unpack2<kBF16>(dv.x), d1 = unpack2<kBF16>(dv.y);
+    acc = o0.x * d0.x + o0.y * d0.y + o1.x * d1.x + o1.y * d1.y;
+  } else {
+    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o);
+    const uint32_t dv = *reinterpret_cast<const uint32_t*>(d);
+    const float2 o0 = unpack2<kBF16>(ov), d0 = unpack2<kBF16>(dv);
+    acc = o0.x * d0.x + o0.y * d0.y;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  float4* z = reinterpret_cast<float4*>(p.dq_acc + gw * kD);
+  for (int i = lane; i < kD / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane == 0) {
+    size_t li;
+    if (p.cu_seqlens != nullptr) {
+      li = static_cast<size_t>(h) * p.total + tok;
+    } else {
+      const int b = tok / p.S, s = tok % p.S;
+      li = (static_cast<size_t>(b) * p.Hq + h) * p.S + s;
+    }
+    p.drow[li] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// post: dq = dq_acc (already scaled) -> 16-bit
+// ---------------------------------------------------------------------------
+template <bool kBF16>
+__global__ void bwd_post_kernel(const BwdParams p, long long n4) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = reinterpret_cast<const float4*>(p.dq_acc)[i];
+  uint2 w;
+  w.x = pack2<kBF16>(v.x, v.y);
+  w.y = pack2<kBF16>(v.z, v.w);
+  reinterpret_cast<uint2*>(p.dq)[i] = w;
+}
+
+// ---------------------------------------------------------------------------
+// main
+// ---------------------------------------------------------------------------
+template <int kD>
+struct BwdShape {
+  static constexpr int kChunks = kD / 64;
+  static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 B
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kDsBytes = 2 * kChunkBytes;     // 128 keys x 128 queries x 16 bit
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;         // + slot * 2 * kTileBytes (Q, dO)
+  static constexpr int kOffDs = 6 * kTileBytes;
+  static constexpr int kOffVec = kOffDs + kDsBytes;    // lse_log2[128], drow[128]
+  static constexpr int kOffBar = kOffVec + 1024;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr int kThreads = 320;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kColA = 0;
+  static constexpr int kColB = 128;
+  static constexpr int kColDV = 256;
+  static constexpr int kColDK = 256 + kD;
+};
+
+struct BwdBars {
+  uint64_t kv_full;
+  uint64_t qd_full[2];
+  uint64_t qd_empty[2];
+  uint64_t s_ready;
+  uint64_t pds_ready;
+  uint64_t dq_ready;
+  uint64_t dq_free;
+  uint64_t final_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        atomicExch(&g_device_status, kDevTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+template <int kD, bool kBF16>
+__global__ void __launch_bounds__(320, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using Sh = BwdShape<kD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + Sh::kOffBar);
+  float* vec_lse = reinterpret_cast<float*>(smem + Sh::kOffVec);
+  float* vec_drow = vec_lse + 128;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: key tiles with the most query tiles first ----------------
+  const int bk = p.B * p.Hkv;
+  const int kt = static_cast<int>(blockIdx.x) / bk;
+  const int rem = static_cast<int>(blockIdx.x) % bk;
+  const int kvh = rem % p.Hkv;
+  const int b = rem / p.Hkv;
+  int seq_start, seq_len;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    seq_len = p.cu_seqlens[b + 1] - seq_start;
+  } else {
+    seq_start = b * p.S;
+    seq_len = p.S;
+  }
+  const int k0 = kt * 128;
+  if (k0 >= seq_len) return;
+  // query rows that can see some key of [k0, k0 + 127]
+  int q_lo = 0;
+  if (p.wr >= 0) q_lo = max(0, k0 - p.wr);
+  int q_hi = seq_len - 1;
+  if (p.wl >= 0) q_hi = min(q_hi, k0 + 127 + p.wl);
+  const int i_begin = q_lo / 128;
+  const int i_cnt = q_hi >= q_lo ? q_hi / 128 + 1 - i_begin : 0;
+  const int n_items = i_cnt * p.group;  // (head, q tile) pairs
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->qd_full[s], 1);
+      mbar_init(&bars->qd_empty[s], 1);
+    }
+    mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->pds_ready, 4);
+    mbar_init(&bars->dq_ready, 1);
+    mbar_init(&bars->dq_free, 4);
+    mbar_init(&bars->final_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, Sh::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * Sh::kTileBytes);
+      for (int c = 0; c < Sh::kChunks; ++c) {
+        tma_load_3d(&tm_k, &bars->kv_full, smem + Sh::kOffK + c * Sh::kChunkBytes, c * 64, kvh,
+                    seq_start + k0);
+        tma_load_3d(&tm_v, &bars->kv_full, smem + Sh::kOffV + c * Sh::kChunkBytes, c * 64, kvh,
+                    seq_start + k0);
+      }
+      int it = 0;
+      for (; it < n_items && !*abort; ++it) {
+        const int slot = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+        if (!bwd_wait(&bars->qd_empty[slot], ph ^ 1u, abort)) break;
+        const int h = kvh * p.group + it / i_cnt;
+        const int tok = seq_start + (i_begin + it % i_cnt) * 128;
+        uint8_t* dst = smem + Sh::kOffQ + slot * 2 * Sh::kTileBytes;
+        mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kTileBytes);
+        for (int c = 0; c < Sh::kChunks; ++c) {
+          tma_load_3d(&tm_q, &bars->qd_full[slot], dst + c * Sh::kChunkBytes, c * 64, h, tok);
+          tma_load_3d(&tm_do, &bars->qd_full[slot], dst + Sh::kTileBytes + c * Sh::kChunkBytes,
+                      c * 64, h, tok);
+        }
+      }
+      for (int f = max(0, it - 2); f < it; ++f)
+        mbar_wait(&bars->qd_full[f & 1], static_cast<uint32_t>(f >> 1) & 1u);
+      mbar_wait(&bars->kv_full, 0);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (elect_one()) {
+      constexpr uint32_t id_s = idesc_f16(kBF16, 128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t id_dv = idesc_f16(kBF16, 128, kD, false, true);    // P^T (tmem) x dO
+      constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);    // dS^T x Q
+      constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, true, true);     // dS x K
+      const uint32_t sK = smem_u32(smem + Sh::kOffK);
+      const uint32_t sV = smem_u32(smem + Sh::kOffV);
+      const uint32_t sDs = smem_u32(smem + Sh::kOffDs);
+      bool ok = bwd_wait(&bars->kv_full, 0, abort);
+      tc_fence_after();
+      auto kmajor = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
+      };
+      auto mnmajor = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + kk * 2048, Sh::kChunkBytes, 1024);
+      };
+      auto issue_s = [&](uint32_t sQ) {
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColA, kmajor(sK, kk), kmajor(sQ, kk), id_s, kk > 0 ? 1u : 0u);
+      };
+      if (ok && n_items > 0) {
+        if ((ok = bwd_wait(&bars->qd_full[0], 0, abort))) {
+          tc_fence_after();
+          issue_s(smem_u32(smem + Sh::kOffQ));
+        }
+      }
+      for (int it = 0; it < n_items && ok; ++it) {
+        const int slot = it & 1;
+        const uint32_t sQ = smem_u32(smem + Sh::kOffQ + slot * 2 * Sh::kTileBytes);
+        const uint32_t sDO = sQ + Sh::kTileBytes;
+        // region B must be free: the dQ group has read the previous dQ
+        if (it > 0) {
+          if (!(ok = bwd_wait(&bars->dq_free, static_cast<uint32_t>(it - 1) & 1u, abort))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColB, kmajor(sV, kk), kmajor(sDO, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_ready);
+        if (!(ok = bwd_wait(&bars->pds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+        tc_fence_after();
+        const uint32_t acc_first = (it == 0) ? 0u : 1u;
+        // dV += P^T dO   (A = P^T from TMEM region A, 16 queries = 8 columns per step)
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + kk * 8, mnmajor(sDO, kk), id_dv,
+                  (kk == 0) ? acc_first : 1u);
+        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ss(tmem + Sh::kColDK, kmajor(sDs, kk), mnmajor(sQ, kk), id_dk,
+                  (kk == 0) ? acc_first : 1u);
+        // dQ = dS K  -> region B
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ss(tmem + Sh::kColB, mnmajor(sDs, kk), mnmajor(sK, kk), id_dq, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->dq_ready);
+        umma_commit(&bars->qd_empty[slot]);
+        // next S^T into region A (P^T of this item has been consumed in order)
+        if (it + 1 < n_items) {
+          const int ns = (it + 1) & 1;
+          if (!(ok = bwd_wait(&bars->qd_full[ns], static_cast<uint32_t>((it + 1) >> 1) & 1u, abort)))
+            break;
+          tc_fence_after();
+          issue_s(smem_u32(smem + Sh::kOffQ + ns * 2 * Sh::kTileBytes));
+        }
+      }
+      umma_commit(&bars->final_done);
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ======================= P / dS group =======================
+    const int lane_base = 32 * (warp & 3);
+    const int r = lane_base + lane;           // key row within the tile
+    const int key = k0 + r;                   // key position within the sequence
+    const uint32_t t_a = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColA;
+    const uint32_t t_b = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColB;
+    uint8_t* ds_row = smem + Sh::kOffDs;      // swizzled K-major tile, row r
+    const int tid = threadIdx.x - 64;         // 0..127
+    bool ok = true;
+    for (int it = 0; it < n_items; ++it) {
+      const int h = kvh * p.group + it / i_cnt;
+      const int i0 = (i_begin + it % i_cnt) * 128;
+      // query-row vectors of this item (LSE in the exp2 domain, Drow)
+      named_bar_sync(2, 128);  // previous item's readers are done
+      {
+        const int qi = i0 + tid;
+        float l2 = INFINITY, dr = 0.f;
+        if (qi < seq_len) {
+          size_t li = p.cu_seqlens != nullptr ? static_cast<size_t>(h) * p.total + seq_start + qi
+                                              : (static_cast<size_t>(b) * p.Hq + h) * p.S + qi;
+          const float l = p.lse[li];
+          l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+          dr = p.drow[li];
+        }
+        vec_lse[tid] = l2;
+        vec_drow[tid] = dr;
+      }
+      named_bar_sync(2, 128);
+      if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+      tc_fence_after();
+      // mask needed for this warp's 32 keys x 128 queries?
+      const int kw_lo = k0 + lane_base, kw_hi = kw_lo + 31;
+      bool need_mask = (kw_hi >= seq_len) || (i0 + 127 >= seq_len);
+      if (p.wr >= 0) need_mask |= (kw_hi > i0 + p.wr);
+      if (p.wl >= 0) need_mask |= (kw_lo < i0 + 127 - p.wl);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {  // 32 queries per chunk
+        uint32_t sr[32], dr[32];
+        tmem_ld32(t_a + c * 32, sr);
+        tmem_ld32(t_b + c * 32, dr);
+        tmem_ld_wait();
+        uint32_t pk[16];
+        uint32_t dk_[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = c * 32 + 2 * j2 + e;
+            const float s = __uint_as_float(sr[2 * j2 + e]);
+            float x, dfac = 1.f;
+            if (p.softcap > 0.f) {
+              const float t = tanhf(s * p.cap_in);
+              x = p.cap_out_log2 * t;
+              dfac = 1.f - t * t;
+            } else {
+              x = s * p.scale_log2;
+            }
+            bool vis = true;
+            if (need_mask) {
+              const int qi = i0 + j;
+              vis = key < seq_len && qi < seq_len;
+              if (p.wr >= 0) vis = vis && key <= qi + p.wr;
+              if (p.wl >= 0) vis = vis && key >= qi - p.wl;
+            }
+            const float pr = vis ? ex2_approx(x - vec_lse[j]) : 0.f;
+            pv[e] = pr;
+            dsv[e] = pr * (__uint_as_float(dr[2 * j2 + e]) - vec_drow[j]) * dfac * p.scale;
+          }
+          pk[j2] = pack2<kBF16>(pv[0], pv[1]);
+          dk_[j2] = pack2<kBF16>(dsv[0], dsv[1]);
+        }
+        // P^T chunk -> TMEM region A columns [16c, 16c+16) (S^T chunks < c
+        // have already been read)
+        tmem_st16(t_a + c * 16, pk);
+        // dS^T chunk -> shared memory row r, queries [32c, 32c+32): chunk
+        // (c >> 1) of 64 queries, 16-byte groups 4*(c&1) .. +3
+        uint8_t* rowp = ds_row + (c >> 1) * Sh::kChunkBytes + r * 128;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int gg = (c & 1) * 4 + g;
+          *reinterpret_cast<uint4*>(rowp + ((gg ^ (r & 7)) << 4)) =
+              make_uint4(dk_[4 * g], dk_[4 * g + 1], dk_[4 * g + 2], dk_[4 * g + 3]);
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->pds_ready);
+    }
+    // ---- epilogue: dV rows (keys) -> dv ----
+    if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
+    tc_fence_after();
+    uint8_t* dst = static_cast<uint8_t*>(p.dv) +
+                   (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
+    if (ok && n_items > 0) {
+      // every lane loads (the TMEM load is warp-collective); only rows of
+      // the sequence are stored
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColDV + c * 32, rr);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+        if (key < seq_len) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+    } else if (ok && key < seq_len) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+      for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else {
+    // ======================= dQ group =======================
+    const int lane_base = 32 * (warp & 3);
+    const int r = lane_base + lane;           // query row within the Q tile (dQ),
+                                              // key row for the final dK
+    const uint32_t t_b = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColB;
+    bool ok = true;
+    for (int it = 0; it < n_items; ++it) {
+      const int h = kvh * p.group + it / i_cnt;
+      const int qi = (i_begin + it % i_cnt) * 128 + r;
+      if (!(ok = bwd_wait(&bars->dq_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+      tc_fence_after();
+      float4* dst = reinterpret_cast<float4*>(p.dq_acc +
+                                              (static_cast<size_t>(seq_start + qi) * p.Hq + h) * kD);
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(t_b + c * 32, rr);
+        tmem_ld_wait();
+        if (qi < seq_len) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            atomicAdd(dst + c * 8 + i, make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
+                                                   __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_free);
+    }
+    // ---- epilogue: dK rows (keys) -> dk ----
+    if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
+    tc_fence_after();
+    const int key = k0 + r;
+    if (ok && n_items > 0) {
+      uint8_t* dst = static_cast<uint8_t*>(p.dk) +
+                     (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColDK + c * 32, rr);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+        if (key < seq_len) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+    } else if (ok && key < seq_len) {
+      uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dk) +
+                                           (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2);
+      for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Sh::kTmemCols);
+  }
+}
+
+}  // namespace fa
