@@ -184,6 +184,63 @@ def prefill_inputs(dev):
     return c, inp, pairs
 
 
+def run_only(args, dist: Dist):
+    """One kernel family on its headline workload, few launches: the command
+    the ncu captures in profiles/ run (`--only fwd|bwd|varlen|decode`)."""
+    import exact_attention_149_b200 as fa
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    out = {"impl": "ours", "only": args.only, "steps": args.steps, "warmup": args.warmup}
+    if args.only in ("fwd", "bwd"):
+        c, inp, pairs = prefill_inputs(dev)
+        q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+        o, lse = fa.fwd(q, k, v, scale=c.scale, causal=True)
+        if args.only == "fwd":
+            fn = lambda: fa.fwd(q, k, v, scale=c.scale, causal=True, out=o, lse=lse)  # noqa: E731
+            flop = W.fwd_flops(pairs, c.D, c.Hq)
+        else:
+            ws = torch.empty(fa.fa_bwd_workspace_size(c.B, c.Hq, c.S, c.D), dtype=torch.uint8,
+                             device=dev)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            fn = lambda: fa.bwd(q, k, v, o, lse, do, scale=c.scale, causal=True, dq=dq, dk=dk,  # noqa: E731
+                                dv=dv, workspace=ws)
+            flop = W.bwd_flops(pairs, c.D, c.Hq)
+        ms = timed(fn, args.steps, args.warmup, dist)
+        out.update(ms=ms, tflops=flop / (ms * 1e-3) / 1e12)
+        out["frac_of_bf16_peak"] = out["tflops"] / peaks["bf16_tflops"]
+    elif args.only == "varlen":
+        cv = W.CONFIGS[4]
+        vin = W.make_varlen_inputs(None, cv.Hq, cv.Hkv, cv.D, cv.dtype, seed=1000 + cv.cid,
+                                   total=cv.total, len_lo=cv.len_lo, len_hi=cv.len_hi)
+        vq, vk, vv = (vin[n].to(dev) for n in ("q", "k", "v"))
+        cu = vin["cu_seqlens"].to(dev)
+        flop = W.fwd_flops(W.varlen_visible_pairs(vin["lengths"], cv.causal, *cv.window), cv.D, cv.Hq)
+        fn = lambda: fa.fwd(vq, vk, vv, scale=cv.scale, causal=True, window=cv.window,  # noqa: E731
+                            softcap=cv.softcap, cu_seqlens=cu, max_seqlen=max(vin["lengths"]))
+        ms = timed(fn, args.steps, args.warmup, dist)
+        out.update(ms=ms, tflops=flop / (ms * 1e-3) / 1e12)
+    elif args.only == "decode":
+        cd = W.CONFIGS[5]
+        st = W.make_decode_structure(cd.B, cd.Hq, cd.Hkv, cd.D, cd.len_lo, cd.len_hi,
+                                     cd.page_size, cd.dtype, seed=1000 + cd.cid)
+        shape = (st["num_pages"], st["page_size"], cd.Hkv, cd.D)
+        kc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+        W.fill_paged_pool(st, kc, vc)
+        q = st["q"].to(dev)
+        kn, vn = st["k_new"].to(dev), st["v_new"].to(dev)
+        cs, bt = st["cache_seqlens"].to(dev), st["block_table"].to(dev)
+        kv_bytes = W.decode_kv_bytes(st["cache_seqlens"], cd.Hkv, cd.D)
+        fn = lambda: fa.fwd_kvcache(q, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale,  # noqa: E731
+                                    causal=True, num_splits=args.splits)
+        ms = timed(fn, args.steps, args.warmup, dist)
+        gbs = kv_bytes / (ms * 1e-3) / 1e9
+        out.update(ms=ms, gbs=gbs, frac_of_hbm=gbs / peaks["hbm_gbs"], splits=args.splits)
+    return out
+
+
 def run_ours(args, dist: Dist):
     import exact_attention_149_b200 as fa
 
@@ -451,13 +508,18 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None, choices=["fwd", "bwd", "varlen", "decode"],
+                    help="time one kernel family only (profiling runs)")
+    ap.add_argument("--splits", type=int, default=16, help="num_splits for --only decode")
     args = ap.parse_args()
-    if args.warmup < 3 and args.impl == "ours":
+    if args.warmup < 3 and args.impl == "ours" and args.only is None:
         args.warmup = 3
     dist = Dist()
     try:
         if args.impl == "reference":
             line = run_reference(args, dist)
+        elif args.only is not None:
+            line = run_only(args, dist)
         else:
             line = run_ours(args, dist)
         if dist.rank == 0 and line is not None:

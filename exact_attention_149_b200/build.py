@@ -1,6 +1,9 @@
 """Build libfa.so (the C-ABI attention library) in-tree for sm_100a.
 
-    python -m exact_attention_149_b200.build
+    python exact_attention_149_b200/build.py [--force] [-v]
+
+(run it as a script: importing the package would first bind the existing
+library, which may be stale).
 
 The library is one translation unit (csrc/fa_api.cu includes every kernel
 header), compiled with nvcc for sm_100a only and linked against the static

@@ -16,9 +16,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def fa():
-    from exact_attention_149_b200 import build
+    import importlib.util
 
-    build.build()
+    spec = importlib.util.spec_from_file_location(
+        "_fa_build", os.path.join(ROOT, "exact_attention_149_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
     import exact_attention_149_b200 as m
 
     return m
