@@ -21,7 +21,8 @@ import torch
 
 __all__ = [
     "LIB_PATH", "FaError", "lib",
-    "fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_bwd_workspace_size", "fa_kvcache_workspace_size",
+    "fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_fwd_kvcache_noalloc", "fa_bwd_workspace_size",
+    "fa_kvcache_workspace_size", "FA_NOALLOC_SCRATCH_BYTES",
     "fa_get_device_status", "fa_last_error", "fa_version",
     "fwd", "bwd", "fwd_kvcache",
 ]
@@ -42,7 +43,7 @@ class FaError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m exact_attention_149_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python exact_attention_149_b200/build.py` "
         "(nvcc, sm_100a). There is no CPU or library fallback.")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -60,6 +61,9 @@ lib.fa_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _
 lib.fa_fwd_kvcache.restype = _i
 lib.fa_fwd_kvcache.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
                                _i, _i, _i, _f, _i, _i, _p, _z, _p]
+lib.fa_fwd_kvcache_noalloc.restype = _i
+lib.fa_fwd_kvcache_noalloc.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                                       _i, _f, _i, _i, _i, _f, _i, _i, _p]
 lib.fa_bwd_workspace_size.restype = _z
 lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 lib.fa_kvcache_workspace_size.restype = _z
@@ -152,6 +156,24 @@ def fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens
                               Hkv, D, page_size, max_pages_per_seq, num_pages, scale, int(causal),
                               window_left, window_right, softcap, num_splits, dtype,
                               _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+# size of the library's static scratch array used by fa_fwd_kvcache_noalloc
+FA_NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
+
+
+def fa_fwd_kvcache_noalloc(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, out, lse,
+                           B, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
+                           window_left, window_right, softcap, num_splits, dtype, stream=None):
+    """fa_fwd_kvcache for callers that cannot allocate device memory: no
+    workspace argument; the split partials live in the library's own static
+    device array (see include/fa.h)."""
+    _check(lib.fa_fwd_kvcache_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                      _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens),
+                                      _ptr(out), _ptr(lse), B, Hq, Hkv, D, page_size,
+                                      max_pages_per_seq, num_pages, scale, int(causal),
+                                      window_left, window_right, softcap, num_splits, dtype,
+                                      _stream(stream)))
 
 
 def fa_get_device_status() -> int:

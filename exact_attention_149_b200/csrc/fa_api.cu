@@ -224,3 +224,4 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
 
 #include "bwd_api.inc"
 #include "decode_api.inc"
+#include "noalloc_api.inc"

@@ -144,6 +144,45 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_
                          fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_fwd_kvcache without a workspace argument, for callers that cannot
+ * allocate device memory on their decode path: a serving loop that has
+ * handed all free device memory to its KV-cache pool up front (so a late
+ * cudaMalloc would fail), code embedded in a host runtime that owns the
+ * allocator and passes in only input and output buffers, or a latency-bound
+ * loop that must not call cudaMalloc/cudaFree because those calls can
+ * synchronise the device. The source pages have no counterpart to this
+ * call; it exists only for such callers.
+ *
+ * Arguments, results and errors are those of fa_fwd_kvcache. The split
+ * partials that fa_fwd_kvcache keeps in the caller's workspace live instead
+ * in one statically sized device array inside this library,
+ * FA_NOALLOC_SCRATCH_BYTES (24 MiB) large, which every GPU that loads the
+ * library holds until the process exits. A call whose partials need more
+ * (fa_kvcache_workspace_size(B, Hq, D, num_splits) > FA_NOALLOC_SCRATCH_BYTES)
+ * is rejected with FA_ERR_INVALID_ARG before anything is launched. The call
+ * itself allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *
+ * - The first call on a device looks up the array's device address on that
+ *   device (cudaGetSymbolAddress, with that device current) and caches it;
+ *   make that first call outside any stream capture.
+ * - Every call on a device shares the one array and leaves its contents
+ *   behind. Nothing in it needs to start at zero: each call writes every
+ *   partial it later reads. Calls whose kernels overlap on the GPU (other
+ *   streams, other host threads) race on the array and must be serialised
+ *   by the caller, e.g. by issuing them on one stream.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
+FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const void* v_new,
+                                        void* k_cache, void* v_cache, const int32_t* block_table,
+                                        const int32_t* cache_seqlens, void* out, float* lse, int B,
+                                        int Hq, int Hkv, int D, int page_size,
+                                        int max_pages_per_seq, int num_pages, float scale,
+                                        int causal, int window_left, int window_right,
+                                        float softcap, int num_splits, fa_dtype dtype,
+                                        void* stream);
+
+/*
  * Reads and clears the library's device status word on the current device
  * (synchronous). *status_out = 0 if no kernel reported a problem since the
  * last call, FA_ERR_TIMEOUT if one gave up on a bounded wait, and
