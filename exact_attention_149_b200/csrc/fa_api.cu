@@ -135,11 +135,11 @@ fa_status set_smem(K kernel, int bytes) {
   return FA_OK;
 }
 
-template <int kD, bool kBF16>
+template <int kD, bool kBF16, bool kCap>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const fa::FwdParams& p, cudaStream_t st) {
   using Sh = fa::FwdShape<kD>;
-  auto kern = fa::fwd_kernel<kD, kBF16>;
+  auto kern = fa::fwd_kernel<kD, kBF16, kCap>;
   fa_status s = set_smem(kern, Sh::kSmemBytes);
   if (s != FA_OK) return s;
   const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
@@ -211,10 +211,17 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   p.lse = lse;
   p.cu_seqlens = cu_seqlens;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool cap = softcap > 0.f;
   if (D == 128) {
-    s = dtype == FA_BF16 ? launch_fwd<128, true>(tq, tk, tv, p, st) : launch_fwd<128, false>(tq, tk, tv, p, st);
+    if (dtype == FA_BF16)
+      s = cap ? launch_fwd<128, true, true>(tq, tk, tv, p, st) : launch_fwd<128, true, false>(tq, tk, tv, p, st);
+    else
+      s = cap ? launch_fwd<128, false, true>(tq, tk, tv, p, st) : launch_fwd<128, false, false>(tq, tk, tv, p, st);
   } else {
-    s = dtype == FA_BF16 ? launch_fwd<64, true>(tq, tk, tv, p, st) : launch_fwd<64, false>(tq, tk, tv, p, st);
+    if (dtype == FA_BF16)
+      s = cap ? launch_fwd<64, true, true>(tq, tk, tv, p, st) : launch_fwd<64, true, false>(tq, tk, tv, p, st);
+    else
+      s = cap ? launch_fwd<64, false, true>(tq, tk, tv, p, st) : launch_fwd<64, false, false>(tq, tk, tv, p, st);
   }
   if (s != FA_OK) return s;
   return ok();

@@ -6,13 +6,17 @@
 // V into on-chip memory, update the row max and row sum tile by tile, never
 // materialise the attention matrix).
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: Q tiles once, then K_j, V_j into a ring of
 //               shared-memory slots (128-byte swizzle).
 //   warp 1      MMA issuer (one lane): S_t = Q_t K_j^T into TMEM, then
 //               O_t += P_t V_j with P_t read from TMEM. Owns TMEM alloc.
-//   warps 2-5   softmax group 0 (Q tile 0), one thread per query row.
-//   warps 6-9   softmax group 1 (Q tile 1).
+//   warps 2-3   idle (they complete warpgroup 0, which gives its registers
+//               to the softmax groups: 88 per thread instead of 168)
+//   warps 4-7   softmax group 0 (Q tile 0), one thread per query row, 208
+//               registers per thread (the whole score row lives in registers).
+//   warps 8-11  softmax group 1 (Q tile 1).
+// Register pool: 384 x 168 at launch = 64512 = 128 x 88 + 256 x 208.
 // The two softmax groups alternate with the tensor core: while group 0
 // exponentiates S_0, the tensor core runs group 1's PV and QK, and so on.
 //
@@ -53,7 +57,9 @@ struct FwdShape {
   static constexpr int kStages = kD == 128 ? 4 : 8;  // K/V ring slots
   static constexpr int kBarOffset = (2 + kStages) * kTileBytes;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + align slack
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  static constexpr int kRegsLow = 88;   // warpgroup 0 after setmaxnreg.dec
+  static constexpr int kRegsHigh = 208; // softmax warpgroups after setmaxnreg.inc
   static constexpr int kTmemCols = 512;
   static constexpr int kColS = 0;      // + 128 * t
   static constexpr int kColP = 64;     // + 128 * t
@@ -89,14 +95,37 @@ __device__ __forceinline__ bool fwd_wait(uint64_t* bar, uint32_t parity, volatil
   }
 }
 
-// Logit transform in the exp2 domain: scale (and optional tanh softcap).
-__device__ __forceinline__ float fwd_logit(float s, const FwdParams& p) {
-  if (p.softcap > 0.f) return p.cap_out_log2 * tanhf(s * p.cap_in);
-  return s * p.scale_log2;
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
-template <int kD, bool kBF16>
-__global__ void __launch_bounds__(320, 1)
+// max (kMax) or min of 128 values, four independent chains
+template <bool kMax>
+__device__ __forceinline__ float reduce128(const float (&x)[128]) {
+  float a[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) a[c] = x[c];
+#pragma unroll
+  for (int i = 4; i + 8 <= 128; i += 8) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      a[c] = kMax ? max3(a[c], x[i + c], x[i + 4 + c]) : min3(a[c], x[i + c], x[i + 4 + c]);
+  }
+  // elements 124..127
+#pragma unroll
+  for (int c = 0; c < 4; ++c) a[c] = kMax ? fmaxf(a[c], x[124 + c]) : fminf(a[c], x[124 + c]);
+  return kMax ? max3(fmaxf(a[0], a[1]), a[2], a[3]) : min3(fminf(a[0], a[1]), a[2], a[3]);
+}
+
+template <int kD, bool kBF16, bool kCap>
+__global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Sh = FwdShape<kD>;
@@ -110,12 +139,12 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: heaviest query blocks first -------------------------------
-  const int bh = p.B * p.Hq;
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / bh;
-  const int rem = static_cast<int>(blockIdx.x) % bh;
-  const int h = rem % p.Hq;
-  const int b = rem / p.Hq;
+  // ---- work item: (sequence, head) major so the CTAs in flight share the
+  // K/V of a few heads in L2; heaviest query blocks first within a head
+  const int bh = static_cast<int>(blockIdx.x) / p.n_qblocks;
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) % p.n_qblocks;
+  const int h = bh % p.Hq;
+  const int b = bh / p.Hq;
   int seq_start, seq_len;
   if (p.cu_seqlens != nullptr) {
     seq_start = p.cu_seqlens[b];
@@ -162,7 +191,12 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-
+  static_assert(Sh::kThreads * 168 >= 128 * Sh::kRegsLow + 256 * Sh::kRegsHigh,
+                "register split exceeds the launch pool");
+  // register reallocation sits inside each role's branch so the compiler
+  // knows which limit every region runs under
+  if (warp < 4) {
+    regs_dec<Sh::kRegsLow>();
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (elect_one()) {
@@ -201,28 +235,32 @@ __global__ void __launch_bounds__(320, 1)
     if (elect_one()) {
       constexpr uint32_t id_qk = idesc_f16(kBF16, 128, 128, false, false);
       constexpr uint32_t id_pv = idesc_f16(kBF16, 128, kD, false, true);
-      const uint32_t sq_addr = smem_u32(sQ);
-      const uint32_t skv_addr = smem_u32(sKV);
+      // descriptors are built once; a tile or K-step offset is added to the
+      // start-address field (bits 0..13, in 16-byte units; every address
+      // stays below 256 KB, so the addition never carries out of the field)
+      const uint64_t dq_base = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk_base = sdesc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dv_base = sdesc_sw128(smem_u32(sKV), Sh::kChunkBytes, 1024);
       bool ok = fwd_wait(&bars->q_full, 0, abort);
       tc_fence_after();
       auto issue_qk = [&](int t, int slot) {
-        const uint32_t a0 = sq_addr + t * Sh::kTileBytes;
-        const uint32_t b0 = skv_addr + slot * Sh::kTileBytes;
+        const uint64_t a0 = dq_base + static_cast<uint64_t>((t * Sh::kTileBytes) >> 4);
+        const uint64_t b0 = dk_base + static_cast<uint64_t>((slot * Sh::kTileBytes) >> 4);
+        const uint32_t d = tmem + Sh::kColS + 128 * t;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32;
-          umma_ss(tmem + Sh::kColS + 128 * t, sdesc_sw128(a0 + off, 16, 1024),
-                  sdesc_sw128(b0 + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32) >> 4);
+          umma_ss(d, a0 + off, b0 + off, id_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int slot, bool first) {
-        const uint32_t b0 = skv_addr + slot * Sh::kTileBytes;
+        const uint64_t b0 = dv_base + static_cast<uint64_t>((slot * Sh::kTileBytes) >> 4);
+        const uint32_t d = tmem + Sh::kColO + kD * t;
+        const uint32_t a = tmem + Sh::kColS + 128 * t + Sh::kColP;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          umma_ts(tmem + Sh::kColO + kD * t, tmem + Sh::kColS + 128 * t + Sh::kColP + kk * 8,
-                  sdesc_sw128(b0 + kk * 2048, Sh::kChunkBytes, 1024), id_pv,
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), id_pv,
                   (first && kk == 0) ? 0u : 1u);
-        }
       };
       for (int it = 0; it < n_tiles && ok; ++it) {
         const int fk = 2 * it, fv = 2 * it + 1;
@@ -273,9 +311,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(&bars->drain, 0);
     }
     __syncwarp();
+  }
   } else {
+    regs_inc<Sh::kRegsHigh>();
     // ======================= softmax groups =======================
-    const int t = (warp - 2) >> 2;            // Q tile of this group
+    const int t = (warp - 4) >> 2;            // Q tile of this group
     const int lane_base = 32 * (warp & 3);    // TMEM lanes this warp may touch
     const int row = lane_base + lane;         // row within the Q tile
     const int qrow = q0 + t * 128 + row;      // row within the sequence
@@ -291,40 +331,44 @@ __global__ void __launch_bounds__(320, 1)
     for (int it = 0; it < n_tiles; ++it) {
       if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it) & 1u, abort))) break;
       tc_fence_after();
+      // ---- the row of S_t: 128 raw scores ----
       float x[128];
       {
-        uint32_t r[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(t_s + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
-        }
+        uint32_t* u = reinterpret_cast<uint32_t*>(x);
+        tmem_ld32(t_s + 0, reinterpret_cast<uint32_t(&)[32]>(u[0]));
+        tmem_ld32(t_s + 32, reinterpret_cast<uint32_t(&)[32]>(u[32]));
+        tmem_ld32(t_s + 64, reinterpret_cast<uint32_t(&)[32]>(u[64]));
+        tmem_ld32(t_s + 96, reinterpret_cast<uint32_t(&)[32]>(u[96]));
+        tmem_ld_wait();
       }
       const int k0 = (n_begin + it) * Sh::kBN;
       // does any (row, key) of this warp's 32 x 128 block need masking?
       bool need_mask = (k0 + 127 >= seq_len);
       if (p.wr >= 0) need_mask |= (k0 + 127 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
-      float mt = -INFINITY;
+      if constexpr (kCap) {
+        // logits in the exp2 domain: softcap * tanh(scale * s / softcap) * log2(e)
+#pragma unroll
+        for (int i = 0; i < 128; ++i) x[i] = p.cap_out_log2 * tanh_fast(x[i] * p.cap_in);
+      }
+      // masked entries become the value that the reduction ignores and whose
+      // exponential is 0 (-inf; +inf for raw scores under a negative scale)
+      const bool pos = kCap || p.scale_log2 >= 0.f;
       if (need_mask) {
-        int jmax = seq_len - 1;
-        if (p.wr >= 0) jmax = min(jmax, qrow + p.wr);
-        int jmin = p.wl >= 0 ? qrow - p.wl : INT32_MIN;
+        const float hide = pos ? -INFINITY : INFINITY;
+        int jmax = seq_len - 1 - k0;
+        if (p.wr >= 0) jmax = min(jmax, qrow + p.wr - k0);
+        const int jmin = p.wl >= 0 ? qrow - p.wl - k0 : INT32_MIN;
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const int j = k0 + i;
-          const float v = (j > jmax || j < jmin) ? -INFINITY : fwd_logit(x[i], p);
-          x[i] = v;
-          mt = fmaxf(mt, v);
-        }
+        for (int i = 0; i < 128; ++i) x[i] = (i > jmax || i < jmin) ? hide : x[i];
+      }
+      float mt;
+      if constexpr (kCap) {
+        mt = reduce128<true>(x);
       } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          x[i] = fwd_logit(x[i], p);
-          mt = fmaxf(mt, x[i]);
-        }
+        mt = pos ? reduce128<true>(x) : reduce128<false>(x);
+        mt *= p.scale_log2;  // +-inf stays -inf for a fully masked row
+        if (mt != mt) mt = -INFINITY;
       }
       const float m_new = fmaxf(m_run, mt);
       const bool grow = m_new > m_run + 8.0f;
@@ -336,30 +380,35 @@ __global__ void __launch_bounds__(320, 1)
           // O_t holds the previous PV results (complete: s_full commit
           // follows them); rescale it in place
 #pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(t_o + c * 32, r);
+          for (int c = 0; c < kD / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(t_o + c * 16, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(t_o + c * 32, r);
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st16(t_o + c * 16, r);
           }
         }
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      float lsum = 0.f;
+      // P = 2^(x - base): one packed FMA (or add) per pair, then MUFU ex2
+      const float2 nb2 = make_float2(-base, -base);
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float e0 = ex2_approx(x[c * 64 + 2 * i] - base);
-          const float e1 = ex2_approx(x[c * 64 + 2 * i + 1] - base);
-          lsum += e0 + e1;
-          r[i] = pack2<kBF16>(e0, e1);
+          const float2 xv = make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]);
+          const float2 d = kCap ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
+          const float2 e = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+          sum2 = __fadd2_rn(sum2, e);
+          r[i] = pack2<kBF16>(e.x, e.y);
         }
         tmem_st32(t_p + c * 32, r);
       }
+      const float lsum = sum2.x + sum2.y;
       l_run += lsum;
       tmem_st_wait();
       tc_fence_before();

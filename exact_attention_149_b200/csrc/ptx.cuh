@@ -119,6 +119,18 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Per-warpgroup register reallocation. All four warps of a warpgroup execute
+// it. The block's pool is fixed at launch (threads x registers at launch), so
+// the sum of the warpgroups' new limits must stay within it, or inc waits.
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // named barrier over a subset of warps (id 1..15; 0 is __syncthreads)
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -293,6 +305,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// tanh from the identity tanh(y) = sign(y) (1 - e) / (1 + e), e = exp(-2|y|),
+// with e taken as 2^(-2 |y| log2(e)). Absolute error ~2e-7 (the subtraction
+// 1 - e near y = 0 and the exp2/rcp approximations); with softcap c the
+// logit error is ~c * 2e-7.
+__device__ __forceinline__ float tanh_fast(float y) {
+  const float e = ex2_approx(fabsf(y) * -2.8853900817779268f);
+  return copysignf(__fdividef(1.f - e, 1.f + e), y);
 }
 
 template <bool kBF16>
