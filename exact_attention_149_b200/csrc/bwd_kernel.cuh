@@ -162,7 +162,7 @@ __device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatil
   }
 }
 
-template <int kD, bool kBF16>
+template <int kD, bool kBF16, bool kCap>
 __global__ void __launch_bounds__(320, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -178,12 +178,13 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: key tiles with the most query tiles first ----------------
-  const int bk = p.B * p.Hkv;
-  const int kt = static_cast<int>(blockIdx.x) / bk;
-  const int rem = static_cast<int>(blockIdx.x) % bk;
-  const int kvh = rem % p.Hkv;
-  const int b = rem / p.Hkv;
+  // ---- work item: (sequence, kv head) major, so the CTAs in flight add into
+  // the dQ rows of only a few heads (which then stay in L2); within a head,
+  // key tiles in increasing order, i.e. the ones with most query tiles first
+  const int bk = static_cast<int>(blockIdx.x) / p.n_ktiles;
+  const int kt = static_cast<int>(blockIdx.x) % p.n_ktiles;
+  const int kvh = bk % p.Hkv;
+  const int b = bk / p.Hkv;
   int seq_start, seq_len;
   if (p.cu_seqlens != nullptr) {
     seq_start = p.cu_seqlens[b];
@@ -346,26 +347,31 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t t_b = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColB;
     uint8_t* ds_row = smem + Sh::kOffDs;      // swizzled K-major tile, row r
     const int tid = threadIdx.x - 64;         // 0..127
+    // query-row vectors (LSE in the exp2 domain, Drow) of item `it`, loaded
+    // one item ahead so the global-load latency overlaps the previous item
+    auto load_vec = [&](int it, float& l2, float& dr) {
+      const int h = kvh * p.group + it / i_cnt;
+      const int qi = (i_begin + it % i_cnt) * 128 + tid;
+      l2 = INFINITY;
+      dr = 0.f;
+      if (it < n_items && qi < seq_len) {
+        const size_t li = p.cu_seqlens != nullptr ? static_cast<size_t>(h) * p.total + seq_start + qi
+                                                  : (static_cast<size_t>(b) * p.Hq + h) * p.S + qi;
+        const float l = p.lse[li];
+        l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+        dr = p.drow[li];
+      }
+    };
+    float nl2, ndr;
+    load_vec(0, nl2, ndr);
     bool ok = true;
     for (int it = 0; it < n_items; ++it) {
-      const int h = kvh * p.group + it / i_cnt;
       const int i0 = (i_begin + it % i_cnt) * 128;
-      // query-row vectors of this item (LSE in the exp2 domain, Drow)
       named_bar_sync(2, 128);  // previous item's readers are done
-      {
-        const int qi = i0 + tid;
-        float l2 = INFINITY, dr = 0.f;
-        if (qi < seq_len) {
-          size_t li = p.cu_seqlens != nullptr ? static_cast<size_t>(h) * p.total + seq_start + qi
-                                              : (static_cast<size_t>(b) * p.Hq + h) * p.S + qi;
-          const float l = p.lse[li];
-          l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-          dr = p.drow[li];
-        }
-        vec_lse[tid] = l2;
-        vec_drow[tid] = dr;
-      }
+      vec_lse[tid] = nl2;
+      vec_drow[tid] = ndr;
       named_bar_sync(2, 128);
+      load_vec(it + 1, nl2, ndr);
       if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
       tc_fence_after();
       // mask needed for this warp's 32 keys x 128 queries?
@@ -389,8 +395,8 @@ __global__ void __launch_bounds__(320, 1)
             const int j = c * 32 + 2 * j2 + e;
             const float s = __uint_as_float(sr[2 * j2 + e]);
             float x, dfac = 1.f;
-            if (p.softcap > 0.f) {
-              const float t = tanhf(s * p.cap_in);
+            if constexpr (kCap) {
+              const float t = tanh_fast(s * p.cap_in);
               x = p.cap_out_log2 * t;
               dfac = 1.f - t * t;
             } else {

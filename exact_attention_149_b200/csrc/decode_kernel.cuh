@@ -141,7 +141,7 @@ struct DecBars {
 };
 
 __device__ __forceinline__ float dec_logit(float s, const DecodeParams& p) {
-  if (p.softcap > 0.f) return p.cap_out_log2 * tanhf(s * p.cap_in);
+  if (p.softcap > 0.f) return p.cap_out_log2 * tanh_fast(s * p.cap_in);
   return s * p.scale_log2;
 }
 
