@@ -58,6 +58,28 @@ def load_peaks():
     return out
 
 
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the last ncu capture recorded in
+    profiles/kernel_traffic.json, or None when the kernel's source files have
+    changed since that capture (their SHA-256 no longer matches)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "kernel_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for rel in rec["source_files"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["source_sha256"]:
+        return None
+    return {"bytes_per_launch": rec["dram_bytes_per_launch"], "workload": rec["workload"]}
+
+
 # ---------------------------------------------------------------------------
 # distributed plumbing (replicas only: no data-path collective)
 # ---------------------------------------------------------------------------
@@ -149,9 +171,11 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
-def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None):
+def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None, fa_mod=None):
     """Run fn() warmup times, then time `steps` calls with CUDA events on the
-    current stream; returns max-over-ranks milliseconds per call."""
+    current stream; returns max-over-ranks milliseconds per call. With
+    `fa_mod`, the library's per-kernel event timing is switched on for the
+    timed calls only (reset first, so the records cover exactly those)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -160,6 +184,9 @@ def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None):
     stream = torch.cuda.current_stream()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    if fa_mod is not None:
+        fa_mod.fa_kernel_timing_reset()
+        fa_mod.fa_kernel_timing_enable(True)
     if sampler is not None:
         sampler.start()
     start.record(stream)
@@ -167,6 +194,8 @@ def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None):
         fn()
     end.record(stream)
     torch.cuda.synchronize()
+    if fa_mod is not None:
+        fa_mod.fa_kernel_timing_enable(False)
     if sampler is not None:
         sampler.stop()
     dist.barrier()
@@ -223,7 +252,8 @@ def run_only(args, dist: Dist):
         out.update(ms=ms, tflops=flop / (ms * 1e-3) / 1e12)
     elif args.only == "decode":
         cd = W.CONFIGS[5]
-        st = W.make_decode_structure(cd.B, cd.Hq, cd.Hkv, cd.D, cd.len_lo, cd.len_hi,
+        B = args.decode_batch or cd.B
+        st = W.make_decode_structure(B, cd.Hq, cd.Hkv, cd.D, cd.len_lo, cd.len_hi,
                                      cd.page_size, cd.dtype, seed=1000 + cd.cid)
         shape = (st["num_pages"], st["page_size"], cd.Hkv, cd.D)
         kc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
@@ -237,7 +267,7 @@ def run_only(args, dist: Dist):
                                     causal=True, num_splits=args.splits)
         ms = timed(fn, args.steps, args.warmup, dist)
         gbs = kv_bytes / (ms * 1e-3) / 1e9
-        out.update(ms=ms, gbs=gbs, frac_of_hbm=gbs / peaks["hbm_gbs"], splits=args.splits)
+        out.update(ms=ms, gbs=gbs, frac_of_hbm=gbs / peaks["hbm_gbs"], splits=args.splits, B=B)
     return out
 
 
@@ -280,7 +310,13 @@ def run_ours(args, dist: Dist):
             step_bwd()
 
     sampler = ClockSampler(dev.index) if dist.rank == 0 else None
-    ms_step = timed(step, args.steps, args.warmup, dist, sampler)
+    ms_step = timed(step, args.steps, args.warmup, dist, sampler, fa_mod=fa)
+    kern = {}
+    for name in ("fwd", "bwd_pre", "bwd_main", "bwd_post"):
+        tot, n = fa.fa_kernel_timing_read(name)
+        if n:
+            kern[name] = {"ms_avg": tot / n, "launches": n}
+    fa.fa_kernel_timing_reset()
     ms_fwd = timed(step_fwd, args.steps, 1, dist)
     ms_bwd = timed(step_bwd, args.steps, 1, dist) if have_bwd else None
     flop_step = fwd_flop + (bwd_flop if have_bwd else 0)
@@ -363,31 +399,52 @@ def run_ours(args, dist: Dist):
             fa.fwd_kvcache(dq_, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale, causal=True,
                            num_splits=splits, out=dout, lse=dlse, workspace=wsb)
 
-        ms_d = timed(step_dec, max(args.steps, 20), args.warmup, dist)
+        ms_d = timed(step_dec, max(args.steps, 20), args.warmup, dist, fa_mod=fa)
+        ksplit, nsplit = fa.fa_kernel_timing_read("decode_split")
+        fa.fa_kernel_timing_reset()
         gbs = kv_bytes / (ms_d * 1e-3) / 1e9
-        dec["splits"][str(splits)] = {"ms": ms_d, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+        entry = {"ms": ms_d, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+        if nsplit:
+            ks = ksplit / nsplit
+            entry["decode_split_kernel"] = {
+                "ms_avg": ks, "gbs": kv_bytes / (ks * 1e-3) / 1e9,
+                "frac_of_hbm": kv_bytes / (ks * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        dec["splits"][str(splits)] = entry
     best = max(dec["splits"].values(), key=lambda d: d["gbs"])
     dec["best_gbs"] = best["gbs"]
     dec["best_frac_of_hbm"] = best["frac_of_hbm"]
+    trd = kernel_traffic("decode_split")
+    dec["roofline"] = {"kernel": "decode_split", "bound": "hbm",
+                       "achieved": best.get("decode_split_kernel", best)["gbs"],
+                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": best.get("decode_split_kernel", best)["gbs"] / peaks["hbm_gbs"],
+                       "traffic": trd["bytes_per_launch"] if trd else None,
+                       "peak_source": peaks["source"] + " HBM copy"}
     res["decode"] = dec
     del kc, vc
     torch.cuda.empty_cache()
 
     # -------------------- roofline of the dominant kernel --------------------
-    kern_times = {"fwd_kernel": ms_fwd}
-    if have_bwd:
-        kern_times["bwd (pre+main+post)"] = ms_bwd
-    dominant = max(kern_times, key=kern_times.get)
-    if dominant == "fwd_kernel":
-        achieved = fwd_flop / (ms_fwd * 1e-3) / 1e12
+    # per-kernel averages come from CUDA events the library recorded around
+    # each launch on the launching stream during the headline loop
+    dominant = max(kern, key=lambda k: kern[k]["ms_avg"])
+    algo = {"fwd": fwd_flop, "bwd_main": bwd_flop}
+    if dominant in algo:
+        achieved = algo[dominant] / (kern[dominant]["ms_avg"] * 1e-3) / 1e12
+        roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"],
+                    "peak_source": peaks["source"] + " burst bf16 (cuBLAS)",
+                    "algorithmic": f"{algo[dominant]:.4e} FLOP per launch (4*D per visible pair "
+                                   f"per head fwd, 10*D bwd)"}
     else:
-        achieved = bwd_flop / (ms_bwd * 1e-3) / 1e12
-    roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                "peak_source": peaks["source"] + " burst bf16 (cuBLAS)"}
+        roofline = {"kernel": dominant, "bound": "hbm", "achieved": None, "peak": None}
+    tr = kernel_traffic(dominant)
+    roofline["traffic"] = tr["bytes_per_launch"] if tr else None
+    roofline["traffic_unit"] = "bytes per launch (dram read + write, ncu)"
+    res["kernels"] = kern
 
-    launches_per_step = 1 + (3 if have_bwd else 0)
+    launches_per_step = 1 + (3 if have_bwd else 0)  # fwd; bwd_pre, bwd_main, bwd_post
     line = {
         "metric": "attention fwd+bwd TFLOP/s, causal B2 H32 S8192 D128 bf16 "
                   "(decode KV GB/s and varlen fwd reported alongside)",
@@ -511,6 +568,8 @@ def main():
     ap.add_argument("--only", default=None, choices=["fwd", "bwd", "varlen", "decode"],
                     help="time one kernel family only (profiling runs)")
     ap.add_argument("--splits", type=int, default=16, help="num_splits for --only decode")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="batch for --only decode (default: the B64 workload); smaller for ncu")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and args.only is None:
         args.warmup = 3

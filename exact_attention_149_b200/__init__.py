@@ -24,6 +24,7 @@ __all__ = [
     "fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_fwd_kvcache_noalloc", "fa_bwd_workspace_size",
     "fa_kvcache_workspace_size", "FA_NOALLOC_SCRATCH_BYTES",
     "fa_get_device_status", "fa_last_error", "fa_version",
+    "fa_kernel_timing_enable", "fa_kernel_timing_read", "fa_kernel_timing_reset",
     "fwd", "bwd", "fwd_kvcache",
 ]
 
@@ -70,6 +71,12 @@ lib.fa_kvcache_workspace_size.restype = _z
 lib.fa_kvcache_workspace_size.argtypes = [_i, _i, _i, _i]
 lib.fa_get_device_status.restype = _i
 lib.fa_get_device_status.argtypes = [ctypes.POINTER(_i)]
+lib.fa_kernel_timing_enable.restype = _i
+lib.fa_kernel_timing_enable.argtypes = [_i]
+lib.fa_kernel_timing_read.restype = _i
+lib.fa_kernel_timing_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(_f), ctypes.POINTER(_i)]
+lib.fa_kernel_timing_reset.restype = _i
+lib.fa_kernel_timing_reset.argtypes = []
 lib.fa_last_error.restype = ctypes.c_char_p
 lib.fa_last_error.argtypes = []
 lib.fa_version.restype = ctypes.c_char_p
@@ -174,6 +181,23 @@ def fa_fwd_kvcache_noalloc(q, k_new, v_new, k_cache, v_cache, block_table, cache
                                       max_pages_per_seq, num_pages, scale, int(causal),
                                       window_left, window_right, softcap, num_splits, dtype,
                                       _stream(stream)))
+
+
+def fa_kernel_timing_enable(enable: bool = True):
+    _check(lib.fa_kernel_timing_enable(int(bool(enable))))
+
+
+def fa_kernel_timing_reset():
+    _check(lib.fa_kernel_timing_reset())
+
+
+def fa_kernel_timing_read(name: str):
+    """(total milliseconds, launches) of kernel `name` since the last reset,
+    from CUDA events the library recorded around each launch."""
+    ms = ctypes.c_float(0.0)
+    n = ctypes.c_int(0)
+    _check(lib.fa_kernel_timing_read(name.encode(), ctypes.byref(ms), ctypes.byref(n)))
+    return float(ms.value), int(n.value)
 
 
 def fa_get_device_status() -> int:

@@ -14,19 +14,22 @@
 //                    stay resident while the CTA walks every query head of
 //                    the GQA group and every 128-row Q tile that can see the
 //                    keys, accumulating dK and dV in tensor memory; each
-//                    tile's dQ contribution is added to the accumulator with
-//                    float4 atomics.
+//                    tile's dQ contribution is staged through shared memory
+//                    and added to the float32 accumulator with TMA bulk
+//                    reduce-add (atomic per element in L2).
 //   bwd_post_kernel  dQ accumulator -> 16-bit dq.
 //
 // bwd_main warp roles (320 threads):
 //   warp 0     TMA producer: K, V once; Q_i and dO_i into a 2-slot ring.
 //   warp 1     MMA issuer (one lane), TMEM owner.
-//   warps 2-5  "P/dS" group, one thread per key row: P^T = exp(S^T - LSE),
-//              dS^T = P^T * (dP^T - Drow); P^T -> TMEM (16-bit), dS^T -> smem.
-//   warps 6-9  "dQ" group, one thread per query row: dQ tile TMEM -> atomics;
-//              at the end both groups write dK and dV.
-// TMEM columns: A [0,128) S^T then P^T; B [128,256) dP^T then dQ;
-// dV [256, 256+D); dK [256+D, 256+2D).
+//   warps 2-9  two compute groups; group g owns query columns [64g, 64g+64):
+//              one thread per key row computes P^T = exp(S^T - LSE) and
+//              dS^T = P^T * (dP^T - Drow), P^T -> TMEM (16-bit), dS^T -> smem;
+//              then one thread per query row moves dQ columns [64g, 64g+64)
+//              from TMEM through smem to the reduce-add; at the end group 0
+//              writes dV, group 1 dK.
+// TMEM columns: A [0,128) S^T then P^T (queries [64g, 64g+64) packed into
+// [64g, 64g+32)); B [128,256) dP^T then dQ; dV [256, 256+D); dK [256+D, 256+2D).
 #pragma once
 
 #include "ptx.cuh"
@@ -166,7 +169,7 @@ template <int kD, bool kBF16, bool kCap>
 __global__ void __launch_bounds__(320, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Sh = BwdShape<kD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -211,9 +214,9 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->qd_empty[s], 1);
     }
     mbar_init(&bars->s_ready, 1);
-    mbar_init(&bars->pds_ready, 4);
+    mbar_init(&bars->pds_ready, 8);
     mbar_init(&bars->dq_ready, 1);
-    mbar_init(&bars->dq_free, 4);
+    mbar_init(&bars->dq_free, 2);
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -308,10 +311,11 @@ __global__ void __launch_bounds__(320, 1)
         if (!(ok = bwd_wait(&bars->pds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
         tc_fence_after();
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
-        // dV += P^T dO   (A = P^T from TMEM region A, 16 queries = 8 columns per step)
+        // dV += P^T dO (A = P^T from TMEM region A: queries [64g, 64g+64) are
+        // packed into columns [64g, 64g+32), 16 queries = 8 columns per step)
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + kk * 8, mnmajor(sDO, kk), id_dv,
+          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 2) * 64 + (kk & 3) * 8, mnmajor(sDO, kk), id_dv,
                   (kk == 0) ? acc_first : 1u);
         // dK += dS^T Q
 #pragma unroll
@@ -338,95 +342,119 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(&bars->drain, 0);
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ======================= P / dS group =======================
+  } else {
+    // ======================= compute groups =======================
+    // Group g (warps 2-5: g = 0; warps 6-9: g = 1) owns query columns
+    // [64g, 64g+64) of S^T and dP^T (one thread per key row), and columns
+    // [64g, 64g+64) of each dQ tile (one thread per query row).
+    const int g = (warp - 2) >> 2;
     const int lane_base = 32 * (warp & 3);
-    const int r = lane_base + lane;           // key row within the tile
-    const int key = k0 + r;                   // key position within the sequence
-    const uint32_t t_a = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColA;
-    const uint32_t t_b = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColB;
-    uint8_t* ds_row = smem + Sh::kOffDs;      // swizzled K-major tile, row r
-    const int tid = threadIdx.x - 64;         // 0..127
-    // query-row vectors (LSE in the exp2 domain, Drow) of item `it`, loaded
-    // one item ahead so the global-load latency overlaps the previous item
-    auto load_vec = [&](int it, float& l2, float& dr) {
-      const int h = kvh * p.group + it / i_cnt;
-      const int qi = (i_begin + it % i_cnt) * 128 + tid;
-      l2 = INFINITY;
-      dr = 0.f;
-      if (it < n_items && qi < seq_len) {
-        const size_t li = p.cu_seqlens != nullptr ? static_cast<size_t>(h) * p.total + seq_start + qi
-                                                  : (static_cast<size_t>(b) * p.Hq + h) * p.S + qi;
-        const float l = p.lse[li];
-        l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-        dr = p.drow[li];
+    const int r = lane_base + lane;
+    const int key = k0 + r;
+    const int gt = static_cast<int>(threadIdx.x) - 64 - 128 * g;  // 0..127 in the group
+    const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
+    const uint32_t t_a = tmem + lane_off + Sh::kColA;
+    const uint32_t t_b = tmem + lane_off + Sh::kColB;
+    float* glse = vec_lse + 64 * g;
+    float* gdrow = vec_drow + 64 * g;
+    const uint32_t bar_id = 2u + static_cast<uint32_t>(g);
+    // the group's query-row vectors of item `it` (threads 0..63: LSE in the
+    // exp2 domain; 64..127: Drow), loaded one item ahead
+    auto load_vec = [&](int it) -> float {
+      float v = gt < 64 ? INFINITY : 0.f;
+      if (it < n_items) {
+        const int h = kvh * p.group + it / i_cnt;
+        const int qi = (i_begin + it % i_cnt) * 128 + 64 * g + (gt & 63);
+        if (qi < seq_len) {
+          const size_t li = p.cu_seqlens != nullptr
+                                ? static_cast<size_t>(h) * p.total + seq_start + qi
+                                : (static_cast<size_t>(b) * p.Hq + h) * p.S + qi;
+          if (gt < 64) {
+            const float l = p.lse[li];
+            v = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+          } else {
+            v = p.drow[li];
+          }
+        }
       }
+      return v;
     };
-    float nl2, ndr;
-    load_vec(0, nl2, ndr);
+    float nv = load_vec(0);
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < n_items; ++it) {
+      const int h = kvh * p.group + it / i_cnt;
       const int i0 = (i_begin + it % i_cnt) * 128;
-      named_bar_sync(2, 128);  // previous item's readers are done
-      vec_lse[tid] = nl2;
-      vec_drow[tid] = ndr;
-      named_bar_sync(2, 128);
-      load_vec(it + 1, nl2, ndr);
+      named_bar_sync(bar_id, 128);  // the group is done with the previous vectors
+      if (gt < 64)
+        glse[gt] = nv;
+      else
+        gdrow[gt - 64] = nv;
+      named_bar_sync(bar_id, 128);
+      nv = load_vec(it + 1);
       if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
       tc_fence_after();
-      // mask needed for this warp's 32 keys x 128 queries?
+      // does any (key, query) of this warp's 32 keys x the group's 64 queries need masking?
       const int kw_lo = k0 + lane_base, kw_hi = kw_lo + 31;
-      bool need_mask = (kw_hi >= seq_len) || (i0 + 127 >= seq_len);
-      if (p.wr >= 0) need_mask |= (kw_hi > i0 + p.wr);
-      if (p.wl >= 0) need_mask |= (kw_lo < i0 + 127 - p.wl);
+      const int qg_lo = i0 + 64 * g, qg_hi = qg_lo + 63;
+      bool need_mask = (kw_hi >= seq_len) || (qg_hi >= seq_len);
+      if (p.wr >= 0) need_mask |= (kw_hi > qg_lo + p.wr);
+      if (p.wl >= 0) need_mask |= (kw_lo < qg_hi - p.wl);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {  // 32 queries per chunk
+      for (int cc = 0; cc < 2; ++cc) {  // 32 queries per chunk
+        const int c = 2 * g + cc;       // chunk index within the 128 queries
         uint32_t sr[32], dr[32];
         tmem_ld32(t_a + c * 32, sr);
         tmem_ld32(t_b + c * 32, dr);
         tmem_ld_wait();
-        uint32_t pk[16];
-        uint32_t dk_[16];
+        uint32_t pk[16], dsk[16];
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
-          float pv[2], dsv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = c * 32 + 2 * j2 + e;
-            const float s = __uint_as_float(sr[2 * j2 + e]);
-            float x, dfac = 1.f;
-            if constexpr (kCap) {
-              const float t = tanh_fast(s * p.cap_in);
-              x = p.cap_out_log2 * t;
-              dfac = 1.f - t * t;
-            } else {
-              x = s * p.scale_log2;
-            }
-            bool vis = true;
-            if (need_mask) {
-              const int qi = i0 + j;
-              vis = key < seq_len && qi < seq_len;
-              if (p.wr >= 0) vis = vis && key <= qi + p.wr;
-              if (p.wl >= 0) vis = vis && key >= qi - p.wl;
-            }
-            const float pr = vis ? ex2_approx(x - vec_lse[j]) : 0.f;
-            pv[e] = pr;
-            dsv[e] = pr * (__uint_as_float(dr[2 * j2 + e]) - vec_drow[j]) * dfac * p.scale;
+          const int jl = cc * 32 + 2 * j2;  // query within the group
+          const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
+          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
+          const float2 l2 = *reinterpret_cast<const float2*>(glse + jl);
+          const float2 d2 = *reinterpret_cast<const float2*>(gdrow + jl);
+          float2 arg, fac;
+          if constexpr (kCap) {
+            const float t0 = tanh_fast(s2.x * p.cap_in), t1 = tanh_fast(s2.y * p.cap_in);
+            arg = make_float2(p.cap_out_log2 * t0 - l2.x, p.cap_out_log2 * t1 - l2.y);
+            fac = make_float2((1.f - t0 * t0) * p.scale, (1.f - t1 * t1) * p.scale);
+          } else {
+            arg = __ffma2_rn(s2, sc2, make_float2(-l2.x, -l2.y));
+            fac = make_float2(p.scale, p.scale);
           }
-          pk[j2] = pack2<kBF16>(pv[0], pv[1]);
-          dk_[j2] = pack2<kBF16>(dsv[0], dsv[1]);
+          float2 pr = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+          if (need_mask) {
+            const int q0i = qg_lo + jl;
+            bool v0 = key < seq_len && q0i < seq_len;
+            bool v1 = key < seq_len && q0i + 1 < seq_len;
+            if (p.wr >= 0) {
+              v0 = v0 && key <= q0i + p.wr;
+              v1 = v1 && key <= q0i + 1 + p.wr;
+            }
+            if (p.wl >= 0) {
+              v0 = v0 && key >= q0i - p.wl;
+              v1 = v1 && key >= q0i + 1 - p.wl;
+            }
+            pr.x = v0 ? pr.x : 0.f;
+            pr.y = v1 ? pr.y : 0.f;
+          }
+          // dS = P (dP - Drow) scale [(1 - tanh^2)]
+          const float2 ds = __fmul2_rn(__fmul2_rn(__fadd2_rn(dp2, make_float2(-d2.x, -d2.y)), pr), fac);
+          pk[j2] = pack2<kBF16>(pr.x, pr.y);
+          dsk[j2] = pack2<kBF16>(ds.x, ds.y);
         }
-        // P^T chunk -> TMEM region A columns [16c, 16c+16) (S^T chunks < c
-        // have already been read)
-        tmem_st16(t_a + c * 16, pk);
-        // dS^T chunk -> shared memory row r, queries [32c, 32c+32): chunk
-        // (c >> 1) of 64 queries, 16-byte groups 4*(c&1) .. +3
-        uint8_t* rowp = ds_row + (c >> 1) * Sh::kChunkBytes + r * 128;
+        // P^T of queries [32c, 32c+32) -> TMEM region A columns [64g + 16cc, +16):
+        // only columns this group has already read are overwritten
+        tmem_st16(t_a + 64 * g + 16 * cc, pk);
+        // dS^T row r, queries [32c, 32c+32): 64-query chunk g, 16-byte groups 4cc..4cc+3
+        uint8_t* rowp = smem + Sh::kOffDs + g * Sh::kChunkBytes + r * 128;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int gg = (c & 1) * 4 + g;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int gg = cc * 4 + q4;
           *reinterpret_cast<uint4*>(rowp + ((gg ^ (r & 7)) << 4)) =
-              make_uint4(dk_[4 * g], dk_[4 * g + 1], dk_[4 * g + 2], dk_[4 * g + 3]);
+              make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
         }
       }
       tmem_st_wait();
@@ -434,19 +462,59 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pds_ready);
+
+      // ---- dQ tile: TMEM -> shared-memory staging -> TMA reduce-add ----
+      // The staging slot is this group's half of the dS^T buffer: dq_ready
+      // follows the dK and dQ MMAs that read dS^T, and the next dS^T is only
+      // written after dq_free (both groups) has let the next dP^T MMA run.
+      if (!(ok = bwd_wait(&bars->dq_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+      tc_fence_after();
+      uint8_t* stage = smem + Sh::kOffDs + g * Sh::kChunkBytes;
+      const bool valid = i0 + r < seq_len;
+#pragma unroll 1
+      for (int cc = 0; cc < kD / 64; ++cc) {
+        const int c = (kD / 64) * g + cc;  // 32-column dQ chunk
+        uint32_t rr[32];
+        tmem_ld32(t_b + c * 32, rr);
+        tmem_ld_wait();
+        if (cc > 0) {
+          if (gt == 0) bulk_wait_read<0>();  // previous chunk has left the slot
+          named_bar_sync(bar_id, 128);
+        }
+        uint8_t* rowp = stage + r * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = valid ? make_uint4(rr[4 * j], rr[4 * j + 1], rr[4 * j + 2], rr[4 * j + 3])
+                                : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(rowp + ((j ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(bar_id, 128);
+        if (gt == 0) {
+          tma_reduce_add_3d(&tm_dq, stage, c * 32, h, seq_start + i0);
+          bulk_commit();
+        }
+      }
+      if (gt == 0) bulk_wait_read<0>();
+      tc_fence_before();
+      named_bar_sync(bar_id, 128);
+      if (gt == 0) mbar_arrive(&bars->dq_free);
     }
-    // ---- epilogue: dV rows (keys) -> dv ----
+    if (gt == 0) bulk_wait<0>();  // every reduction has reached global memory
+
+    // ---- epilogue: group 0 writes the dV rows, group 1 the dK rows ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
-    uint8_t* dst = static_cast<uint8_t*>(p.dv) +
-                   (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
+    void* outp = g == 0 ? p.dv : p.dk;
+    const uint32_t col = g == 0 ? Sh::kColDV : Sh::kColDK;
+    uint8_t* dst = static_cast<uint8_t*>(outp) + (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
     if (ok && n_items > 0) {
       // every lane loads (the TMEM load is warp-collective); only rows of
       // the sequence are stored
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t rr[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColDV + c * 32, rr);
+        tmem_ld32(tmem + lane_off + col + c * 32, rr);
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
@@ -459,62 +527,6 @@ __global__ void __launch_bounds__(320, 1)
       }
     } else if (ok && key < seq_len) {
       uint4* d4 = reinterpret_cast<uint4*>(dst);
-      for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  } else {
-    // ======================= dQ group =======================
-    const int lane_base = 32 * (warp & 3);
-    const int r = lane_base + lane;           // query row within the Q tile (dQ),
-                                              // key row for the final dK
-    const uint32_t t_b = tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColB;
-    bool ok = true;
-    for (int it = 0; it < n_items; ++it) {
-      const int h = kvh * p.group + it / i_cnt;
-      const int qi = (i_begin + it % i_cnt) * 128 + r;
-      if (!(ok = bwd_wait(&bars->dq_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
-      tc_fence_after();
-      float4* dst = reinterpret_cast<float4*>(p.dq_acc +
-                                              (static_cast<size_t>(seq_start + qi) * p.Hq + h) * kD);
-#pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(t_b + c * 32, rr);
-        tmem_ld_wait();
-        if (qi < seq_len) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            atomicAdd(dst + c * 8 + i, make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
-                                                   __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->dq_free);
-    }
-    // ---- epilogue: dK rows (keys) -> dk ----
-    if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
-    tc_fence_after();
-    const int key = k0 + r;
-    if (ok && n_items > 0) {
-      uint8_t* dst = static_cast<uint8_t*>(p.dk) +
-                     (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
-#pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + Sh::kColDK + c * 32, rr);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
-        if (key < seq_len) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
-      }
-    } else if (ok && key < seq_len) {
-      uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.dk) +
-                                           (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2);
       for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/fa.h"
 #include "ptx.cuh"
@@ -105,6 +106,70 @@ fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, i
   return FA_OK;
 }
 
+// 3-D map over a (tokens, heads, D) row-major float32 tensor; box = 32
+// columns (128 B) x 1 head x `rows` tokens, 128-byte swizzle. Used for the
+// backward's bulk reduce-add of dQ tiles.
+fa_status make_map_thd_f32(CUtensorMap* map, const void* base, int D, int H, long long T, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H) * D * 4};
+  cuuint32_t box[3] = {32u, 1u, static_cast<cuuint32_t>(rows)};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (f32) failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// optional per-kernel timing (events around each launch on the caller's stream)
+// ---------------------------------------------------------------------------
+struct TimingRecord {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timing_mu;
+bool g_timing_on = false;
+std::vector<TimingRecord> g_timing_records;
+
+cudaEvent_t timing_event() {
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// RAII helper: records an event before the launch in its scope and one after.
+class KernelTimer {
+ public:
+  KernelTimer(const char* name, cudaStream_t st) : name_(name), st_(st) {
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    if (!g_timing_on) return;
+    start_ = timing_event();
+    if (start_ != nullptr) cudaEventRecord(start_, st_);
+  }
+  ~KernelTimer() {
+    if (start_ == nullptr) return;
+    cudaEvent_t stop = timing_event();
+    if (stop == nullptr) {
+      cudaEventDestroy(start_);
+      return;
+    }
+    cudaEventRecord(stop, st_);
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    g_timing_records.push_back({name_, start_, stop});
+  }
+  KernelTimer(const KernelTimer&) = delete;
+  KernelTimer& operator=(const KernelTimer&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t st_;
+  cudaEvent_t start_ = nullptr;
+};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // common option validation for fwd/bwd
@@ -144,7 +209,10 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   if (s != FA_OK) return s;
   const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
   if (grid > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "grid too large");
-  kern<<<static_cast<unsigned>(grid), Sh::kThreads, Sh::kSmemBytes, st>>>(tq, tk, tv, p);
+  {
+    KernelTimer timer("fwd", st);
+    kern<<<static_cast<unsigned>(grid), Sh::kThreads, Sh::kSmemBytes, st>>>(tq, tk, tv, p);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "fwd launch failed: %s", cudaGetErrorString(e));
   return FA_OK;
@@ -157,6 +225,42 @@ extern "C" {
 const char* fa_last_error(void) { return g_last_error.c_str(); }
 
 const char* fa_version(void) { return "exact-attention-b200 0.1.0 (sm_100a)"; }
+
+fa_status fa_kernel_timing_enable(int enable) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  g_timing_on = enable != 0;
+  return ok();
+}
+
+fa_status fa_kernel_timing_reset(void) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  for (auto& r : g_timing_records) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_timing_records.clear();
+  return ok();
+}
+
+fa_status fa_kernel_timing_read(const char* name, float* total_ms, int* launches) {
+  if (name == nullptr || total_ms == nullptr || launches == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "fa_kernel_timing_read: null argument");
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  float sum = 0.f;
+  int n = 0;
+  for (auto& r : g_timing_records) {
+    if (std::strcmp(r.name, name) != 0) continue;
+    cudaError_t e = cudaEventSynchronize(r.stop);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.start, r.stop);
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "timing event: %s", cudaGetErrorString(e));
+    sum += ms;
+    ++n;
+  }
+  *total_ms = sum;
+  *launches = n;
+  return ok();
+}
 
 fa_status fa_get_device_status(int* status_out) {
   if (status_out == nullptr) return fail(FA_ERR_INVALID_ARG, "status_out is NULL");

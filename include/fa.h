@@ -183,6 +183,24 @@ FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const 
                                         void* stream);
 
 /*
+ * Per-kernel timing, for profiling (off by default). While enabled, every
+ * call records a pair of CUDA events around each kernel it launches, on the
+ * caller's stream, so the durations are those of the kernels themselves as
+ * they ran in the caller's stream order.
+ *   fa_kernel_timing_enable(1/0) switches recording on or off (host-wide).
+ *   fa_kernel_timing_read(name, &total_ms, &launches) waits for the recorded
+ *     events and returns the summed duration and count of the launches of
+ *     the kernel `name` ("fwd", "bwd_pre", "bwd_main", "bwd_post",
+ *     "kv_append", "decode_split", "lse_combine") since the last reset.
+ *   fa_kernel_timing_reset() drops all records.
+ * Errors: FA_ERR_INVALID_ARG for null arguments, FA_ERR_CUDA if an event
+ * call fails.
+ */
+FA_API fa_status fa_kernel_timing_enable(int enable);
+FA_API fa_status fa_kernel_timing_read(const char* name, float* total_ms, int* launches);
+FA_API fa_status fa_kernel_timing_reset(void);
+
+/*
  * Reads and clears the library's device status word on the current device
  * (synchronous). *status_out = 0 if no kernel reported a problem since the
  * last call, FA_ERR_TIMEOUT if one gave up on a bounded wait, and
