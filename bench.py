@@ -84,18 +84,25 @@ def kernel_traffic(kernel: str):
 # distributed plumbing (replicas only: no data-path collective)
 # ---------------------------------------------------------------------------
 class Dist:
+    """One process per GPU (torchrun env vars). Every rank runs its own
+    replica of the workload; the process group is used only for barriers and
+    the max-over-ranks of the timings (NCCL on GPUs, gloo on CPU)."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.backend = None
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+            self.backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=300))
             self.pg = dist
 
     def barrier(self):
@@ -105,7 +112,8 @@ class Dist:
     def max(self, x: float) -> float:
         if self.pg is None:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
@@ -169,6 +177,12 @@ class ClockSampler:
         names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "reasons": names, "samples": len(self.samples)}
+
+
+def replica_throughput(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput of N independent replicas: all ranks' units over
+    the slowest rank's time (units per second)."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None, fa_mod=None):
@@ -320,7 +334,7 @@ def run_ours(args, dist: Dist):
     ms_fwd = timed(step_fwd, args.steps, 1, dist)
     ms_bwd = timed(step_bwd, args.steps, 1, dist) if have_bwd else None
     flop_step = fwd_flop + (bwd_flop if have_bwd else 0)
-    value = dist.world * flop_step / (ms_step * 1e-3) / 1e12
+    value = replica_throughput(flop_step, ms_step, dist.world) / 1e12
     res["fwd"] = {"ms": ms_fwd, "tflops": fwd_flop / (ms_fwd * 1e-3) / 1e12,
                   "flop": fwd_flop}
     res["fwd"]["frac_of_bf16_peak"] = res["fwd"]["tflops"] / peaks["bf16_tflops"]
