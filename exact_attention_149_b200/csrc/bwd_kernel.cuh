@@ -140,7 +140,8 @@ struct BwdBars {
   uint64_t qd_full[2];
   uint64_t qd_empty[2];
   uint64_t s_ready;
-  uint64_t pds_ready;
+  uint64_t p_ready;
+  uint64_t ds_ready;
   uint64_t dq_ready;
   uint64_t dq_free;
   uint64_t final_done;
@@ -214,7 +215,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->qd_empty[s], 1);
     }
     mbar_init(&bars->s_ready, 1);
-    mbar_init(&bars->pds_ready, 8);
+    mbar_init(&bars->p_ready, 8);
+    mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->dq_ready, 1);
     mbar_init(&bars->dq_free, 2);
     mbar_init(&bars->final_done, 1);
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < kD / 16; ++kk)
           umma_ss(tmem + Sh::kColB, kmajor(sV, kk), kmajor(sDO, kk), id_s, kk > 0 ? 1u : 0u);
         umma_commit(&bars->s_ready);
-        if (!(ok = bwd_wait(&bars->pds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+        if (!(ok = bwd_wait(&bars->p_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
         tc_fence_after();
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
         // dV += P^T dO (A = P^T from TMEM region A: queries [64g, 64g+64) are
@@ -317,7 +319,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < 128 / 16; ++kk)
           umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 2) * 64 + (kk & 3) * 8, mnmajor(sDO, kk), id_dv,
                   (kk == 0) ? acc_first : 1u);
-        // dK += dS^T Q
+        // dK += dS^T Q (after dS^T is in shared memory)
+        if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
           umma_ss(tmem + Sh::kColDK, kmajor(sDs, kk), mnmajor(sQ, kk), id_dk,
@@ -400,26 +404,38 @@ __global__ void __launch_bounds__(320, 1)
       bool need_mask = (kw_hi >= seq_len) || (qg_hi >= seq_len);
       if (p.wr >= 0) need_mask |= (kw_hi > qg_lo + p.wr);
       if (p.wl >= 0) need_mask |= (kw_lo < qg_hi - p.wl);
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {  // 32 queries per chunk
+      // pass 1: P^T from S^T (32 queries per chunk) -> TMEM; keep
+      // w = P * scale (* (1 - tanh^2) under softcap) for the dS pass
+      float w[64];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * g + cc;       // chunk index within the 128 queries
-        uint32_t sr[32], dr[32];
+        uint32_t sr[32];
         tmem_ld32(t_a + c * 32, sr);
-        tmem_ld32(t_b + c * 32, dr);
         tmem_ld_wait();
-        uint32_t pk[16], dsk[16];
+        bool poly = false;
+        if constexpr (kCap) {
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(sr[i])), fabsf(__uint_as_float(sr[i + 1]))));
+          poly = __all_sync(0xffffffffu, amax * fabsf(p.cap_in) <= kTanhPolyMax);
+        }
+        uint32_t pk[16];
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
           const int jl = cc * 32 + 2 * j2;  // query within the group
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
-          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
           const float2 l2 = *reinterpret_cast<const float2*>(glse + jl);
-          const float2 d2 = *reinterpret_cast<const float2*>(gdrow + jl);
           float2 arg, fac;
           if constexpr (kCap) {
-            const float t0 = tanh_fast(s2.x * p.cap_in), t1 = tanh_fast(s2.y * p.cap_in);
-            arg = make_float2(p.cap_out_log2 * t0 - l2.x, p.cap_out_log2 * t1 - l2.y);
-            fac = make_float2((1.f - t0 * t0) * p.scale, (1.f - t1 * t1) * p.scale);
+            float2 th;
+            if (poly)
+              th = tanh_poly2(__fmul2_rn(s2, make_float2(p.cap_in, p.cap_in)));
+            else
+              th = make_float2(tanh_fast(s2.x * p.cap_in), tanh_fast(s2.y * p.cap_in));
+            arg = make_float2(p.cap_out_log2 * th.x - l2.x, p.cap_out_log2 * th.y - l2.y);
+            fac = make_float2((1.f - th.x * th.x) * p.scale, (1.f - th.y * th.y) * p.scale);
           } else {
             arg = __ffma2_rn(s2, sc2, make_float2(-l2.x, -l2.y));
             fac = make_float2(p.scale, p.scale);
@@ -440,14 +456,35 @@ __global__ void __launch_bounds__(320, 1)
             pr.x = v0 ? pr.x : 0.f;
             pr.y = v1 ? pr.y : 0.f;
           }
-          // dS = P (dP - Drow) scale [(1 - tanh^2)]
-          const float2 ds = __fmul2_rn(__fmul2_rn(__fadd2_rn(dp2, make_float2(-d2.x, -d2.y)), pr), fac);
           pk[j2] = pack2<kBF16>(pr.x, pr.y);
-          dsk[j2] = pack2<kBF16>(ds.x, ds.y);
+          const float2 wv = __fmul2_rn(pr, fac);
+          w[jl] = wv.x;
+          w[jl + 1] = wv.y;
         }
         // P^T of queries [32c, 32c+32) -> TMEM region A columns [64g + 16cc, +16):
         // only columns this group has already read are overwritten
         tmem_st16(t_a + 64 * g + 16 * cc, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_ready);  // dV may start
+      // pass 2: dS^T = w * (dP^T - Drow) -> shared memory (the dK and dQ operand)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * g + cc;
+        uint32_t dr[32];
+        tmem_ld32(t_b + c * 32, dr);
+        tmem_ld_wait();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const int jl = cc * 32 + 2 * j2;
+          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
+          const float2 d2 = *reinterpret_cast<const float2*>(gdrow + jl);
+          const float2 ds = __fmul2_rn(__fadd2_rn(dp2, make_float2(-d2.x, -d2.y)), make_float2(w[jl], w[jl + 1]));
+          dsk[j2] = pack2<kBF16>(ds.x, ds.y);
+        }
         // dS^T row r, queries [32c, 32c+32): 64-query chunk g, 16-byte groups 4cc..4cc+3
         uint8_t* rowp = smem + Sh::kOffDs + g * Sh::kChunkBytes + r * 128;
 #pragma unroll
@@ -457,11 +494,10 @@ __global__ void __launch_bounds__(320, 1)
               make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
         }
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->pds_ready);
+      if (lane == 0) mbar_arrive(&bars->ds_ready);
 
       // ---- dQ tile: TMEM -> shared-memory staging -> TMA reduce-add ----
       // The staging slot is this group's half of the dS^T buffer: dq_ready

@@ -347,9 +347,27 @@ __global__ void __launch_bounds__(384, 1)
       if (p.wr >= 0) need_mask |= (k0 + 127 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
       if constexpr (kCap) {
-        // logits in the exp2 domain: softcap * tanh(scale * s / softcap) * log2(e)
+        // logits in the exp2 domain: softcap * tanh(scale * s / softcap) * log2(e).
+        // When every |scale * s / softcap| of the warp's rows is small, tanh
+        // is the FMA-pipe polynomial (two values per instruction); otherwise
+        // the exp-based identity.
+        float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < 128; ++i) x[i] = p.cap_out_log2 * tanh_fast(x[i] * p.cap_in);
+        for (int i = 0; i < 128; i += 2) amax = max3(amax, fabsf(x[i]), fabsf(x[i + 1]));
+        if (__all_sync(0xffffffffu, amax * fabsf(p.cap_in) <= kTanhPolyMax)) {
+          const float2 ci = make_float2(p.cap_in, p.cap_in);
+          const float2 co = make_float2(p.cap_out_log2, p.cap_out_log2);
+#pragma unroll
+          for (int i = 0; i < 128; i += 2) {
+            const float2 t = tanh_poly2(__fmul2_rn(make_float2(x[i], x[i + 1]), ci));
+            const float2 v = __fmul2_rn(t, co);
+            x[i] = v.x;
+            x[i + 1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) x[i] = p.cap_out_log2 * tanh_fast(x[i] * p.cap_in);
+        }
       }
       // masked entries become the value that the reduction ignores and whose
       // exponential is 0 (-inf; +inf for raw scores under a negative scale)
