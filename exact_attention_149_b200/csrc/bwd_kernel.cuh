@@ -8,28 +8,32 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q
 // (and dS picks up the factor 1 - tanh^2 under softcap).
 //
-//   bwd_pre_kernel   Drow = rowsum(dO * O) per (token, query head); zero the
-//                    float32 dQ accumulator.
-//   bwd_main_kernel  one CTA per (sequence, kv head, 128-key tile); K and V
-//                    stay resident while the CTA walks every query head of
-//                    the GQA group and every 128-row Q tile that can see the
-//                    keys, accumulating dK and dV in tensor memory; each
-//                    tile's dQ contribution is staged through shared memory
-//                    and added to the float32 accumulator with TMA bulk
-//                    reduce-add (atomic per element in L2).
-//   bwd_post_kernel  dQ accumulator -> 16-bit dq.
+//   bwd_pre_kernel   Drow = rowsum(dO * O) per (token, query head).
+//   bwd_dkdv_kernel  one CTA per (sequence, kv head, 128-key tile): K and V
+//                    stay resident while the CTA walks every query head of the
+//                    GQA group and every 128-row Q tile that can see the keys;
+//                    dK and dV accumulate in tensor memory (no atomics).
+//   bwd_dq_kernel    one CTA per (sequence, query head, 128-row Q tile): Q and
+//                    dO stay resident while the CTA walks the visible K/V
+//                    tiles; dQ accumulates in tensor memory and is written
+//                    once (no atomics, so the whole backward is deterministic).
+// dS is computed in both kernels (S and dP are recomputed twice): seven
+// 128x128xD products per (query tile, key tile) instead of five, in exchange
+// for no dQ reduction across CTAs and a pipeline with no write-back on the
+// critical path.
 //
-// bwd_main warp roles (320 threads):
+// bwd_dkdv warp roles (320 threads):
 //   warp 0     TMA producer: K, V once; Q_i and dO_i into a 2-slot ring.
 //   warp 1     MMA issuer (one lane), TMEM owner.
 //   warps 2-9  two compute groups; group g owns query columns [64g, 64g+64):
-//              one thread per key row computes P^T = exp(S^T - LSE) and
-//              dS^T = P^T * (dP^T - Drow), P^T -> TMEM (16-bit), dS^T -> smem;
-//              then one thread per query row moves dQ columns [64g, 64g+64)
-//              from TMEM through smem to the reduce-add; at the end group 0
-//              writes dV, group 1 dK.
+//              one thread per key row computes P^T = exp(S^T - LSE) (-> TMEM,
+//              16-bit, for the dV MMA) and then dS^T = P^T * (dP^T - Drow)
+//              (-> shared memory, for the dK MMA); at the end group 0 writes
+//              dV, group 1 dK.
 // TMEM columns: A [0,128) S^T then P^T (queries [64g, 64g+64) packed into
-// [64g, 64g+32)); B [128,256) dP^T then dQ; dV [256, 256+D); dK [256+D, 256+2D).
+// [64g, 64g+32)); B [128,256) dP^T; dV [256, 256+D); dK [256+D, 256+2D).
+// MMA order per item i: dV_i, S_{i+1}, dK_i, dP_{i+1}: the tensor core only
+// waits for the P pass of each item.
 #pragma once
 
 #include "ptx.cuh"
@@ -47,7 +51,6 @@ struct BwdParams {
   const void* dout;
   const float* lse;
   float* drow;               // LSE layout
-  float* dq_acc;             // (T, Hq, D) float32
   void* dq;                  // (T, Hq, D) 16-bit
   void* dk;                  // (T, Hkv, D)
   void* dv;
@@ -55,7 +58,7 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------------------
-// pre: Drow and zeroed dQ accumulator. One warp per (token, head) row.
+// pre: Drow = rowsum(dO * O). One warp per (token, head) row.
 // ---------------------------------------------------------------------------
 template <int kD, bool kBF16>
 __global__ void bwd_pre_kernel(const BwdParams p) {
@@ -83,8 +86,6 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  float4* z = reinterpret_cast<float4*>(p.dq_acc + gw * kD);
-  for (int i = lane; i < kD / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane == 0) {
     size_t li;
     if (p.cu_seqlens != nullptr) {
@@ -97,25 +98,56 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// post: dq = dq_acc (already scaled) -> 16-bit
-// ---------------------------------------------------------------------------
-template <bool kBF16>
-__global__ void bwd_post_kernel(const BwdParams p, long long n4) {
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n4) return;
-  const float4 v = reinterpret_cast<const float4*>(p.dq_acc)[i];
-  uint2 w;
-  w.x = pack2<kBF16>(v.x, v.y);
-  w.y = pack2<kBF16>(v.z, v.w);
-  reinterpret_cast<uint2*>(p.dq)[i] = w;
+__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        atomicExch(&g_device_status, kDevTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
 }
 
-// ---------------------------------------------------------------------------
-// main
-// ---------------------------------------------------------------------------
+// logit in the exp2 domain and the factor dS picks up (scale, and 1 - tanh^2
+// under softcap) for a pair of raw scores
+template <bool kCap>
+__device__ __forceinline__ void bwd_logit2(float2 s2, bool poly, const BwdParams& p, float2& x,
+                                           float2& fac) {
+  if constexpr (kCap) {
+    float2 th;
+    if (poly)
+      th = tanh_poly2(__fmul2_rn(s2, make_float2(p.cap_in, p.cap_in)));
+    else
+      th = make_float2(tanh_fast(s2.x * p.cap_in), tanh_fast(s2.y * p.cap_in));
+    x = make_float2(p.cap_out_log2 * th.x, p.cap_out_log2 * th.y);
+    fac = make_float2((1.f - th.x * th.x) * p.scale, (1.f - th.y * th.y) * p.scale);
+  } else {
+    x = __fmul2_rn(s2, make_float2(p.scale_log2, p.scale_log2));
+    fac = make_float2(p.scale, p.scale);
+  }
+}
+
+// is every |scale * s / softcap| of these 32 raw scores, in every lane of
+// the warp, small enough for the tanh polynomial?
+__device__ __forceinline__ bool poly_ok(const uint32_t (&sr)[32], float cap_in) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2)
+    amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(sr[i])), fabsf(__uint_as_float(sr[i + 1]))));
+  return __all_sync(0xffffffffu, amax * fabsf(cap_in) <= kTanhPolyMax);
+}
+
+// ===========================================================================
+// dK, dV
+// ===========================================================================
 template <int kD>
-struct BwdShape {
+struct DkdvShape {
   static constexpr int kChunks = kD / 64;
   static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
@@ -135,56 +167,37 @@ struct BwdShape {
   static constexpr int kColDK = 256 + kD;
 };
 
-struct BwdBars {
+struct DkdvBars {
   uint64_t kv_full;
   uint64_t qd_full[2];
   uint64_t qd_empty[2];
   uint64_t s_ready;
   uint64_t p_ready;
   uint64_t ds_ready;
-  uint64_t dq_ready;
-  uint64_t dq_free;
   uint64_t final_done;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 
-__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-        atomicExch(&g_device_status, kDevTimeout);
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-}
-
 template <int kD, bool kBF16, bool kCap>
 __global__ void __launch_bounds__(320, 1)
-    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using Sh = BwdShape<kD>;
+                    const BwdParams p) {
+  using Sh = DkdvShape<kD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + Sh::kOffBar);
+  DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem + Sh::kOffBar);
   float* vec_lse = reinterpret_cast<float*>(smem + Sh::kOffVec);
   float* vec_drow = vec_lse + 128;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (sequence, kv head) major, so the CTAs in flight add into
-  // the dQ rows of only a few heads (which then stay in L2); within a head,
-  // key tiles in increasing order, i.e. the ones with most query tiles first
+  // ---- work item: (sequence, kv head) major; within a head, key tiles in
+  // increasing order (under causal masking the first ones see the most rows)
   const int bk = static_cast<int>(blockIdx.x) / p.n_ktiles;
   const int kt = static_cast<int>(blockIdx.x) % p.n_ktiles;
   const int kvh = bk % p.Hkv;
@@ -217,8 +230,6 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&bars->s_ready, 1);
     mbar_init(&bars->p_ready, 8);
     mbar_init(&bars->ds_ready, 8);
-    mbar_init(&bars->dq_ready, 1);
-    mbar_init(&bars->dq_free, 2);
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -274,7 +285,6 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t id_s = idesc_f16(kBF16, 128, 128, false, false);   // S^T, dP^T
       constexpr uint32_t id_dv = idesc_f16(kBF16, 128, kD, false, true);    // P^T (tmem) x dO
       constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);    // dS^T x Q
-      constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, true, true);     // dS x K
       const uint32_t sK = smem_u32(smem + Sh::kOffK);
       const uint32_t sV = smem_u32(smem + Sh::kOffV);
       const uint32_t sDs = smem_u32(smem + Sh::kOffDs);
@@ -286,39 +296,49 @@ __global__ void __launch_bounds__(320, 1)
       auto mnmajor = [](uint32_t base, int kk) {
         return sdesc_sw128(base + kk * 2048, Sh::kChunkBytes, 1024);
       };
-      auto issue_s = [&](uint32_t sQ) {
+      auto q_addr = [&](int it) { return smem_u32(smem + Sh::kOffQ + (it & 1) * 2 * Sh::kTileBytes); };
+      auto issue_s = [&](int it) {  // S^T = K Q^T -> region A
+        const uint32_t sQ = q_addr(it);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           umma_ss(tmem + Sh::kColA, kmajor(sK, kk), kmajor(sQ, kk), id_s, kk > 0 ? 1u : 0u);
       };
+      auto issue_dp = [&](int it) {  // dP^T = V dO^T -> region B
+        const uint32_t sDO = q_addr(it) + Sh::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColB, kmajor(sV, kk), kmajor(sDO, kk), id_s, kk > 0 ? 1u : 0u);
+      };
       if (ok && n_items > 0) {
         if ((ok = bwd_wait(&bars->qd_full[0], 0, abort))) {
           tc_fence_after();
-          issue_s(smem_u32(smem + Sh::kOffQ));
+          issue_s(0);
+          issue_dp(0);
+          umma_commit(&bars->s_ready);
         }
       }
       for (int it = 0; it < n_items && ok; ++it) {
         const int slot = it & 1;
-        const uint32_t sQ = smem_u32(smem + Sh::kOffQ + slot * 2 * Sh::kTileBytes);
+        const uint32_t sQ = q_addr(it);
         const uint32_t sDO = sQ + Sh::kTileBytes;
-        // region B must be free: the dQ group has read the previous dQ
-        if (it > 0) {
-          if (!(ok = bwd_wait(&bars->dq_free, static_cast<uint32_t>(it - 1) & 1u, abort))) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ss(tmem + Sh::kColB, kmajor(sV, kk), kmajor(sDO, kk), id_s, kk > 0 ? 1u : 0u);
-        umma_commit(&bars->s_ready);
-        if (!(ok = bwd_wait(&bars->p_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
-        tc_fence_after();
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
         // dV += P^T dO (A = P^T from TMEM region A: queries [64g, 64g+64) are
         // packed into columns [64g, 64g+32), 16 queries = 8 columns per step)
+        if (!(ok = bwd_wait(&bars->p_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 2) * 64 + (kk & 3) * 8, mnmajor(sDO, kk), id_dv,
-                  (kk == 0) ? acc_first : 1u);
+          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 2) * 64 + (kk & 3) * 8,
+                  mnmajor(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
+        // next S^T into region A: P^T of this item has been consumed in order
+        const bool more = it + 1 < n_items;
+        if (more) {
+          if (!(ok = bwd_wait(&bars->qd_full[(it + 1) & 1], static_cast<uint32_t>((it + 1) >> 1) & 1u,
+                              abort)))
+            break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
         // dK += dS^T Q (after dS^T is in shared memory)
         if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
         tc_fence_after();
@@ -326,19 +346,12 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < 128 / 16; ++kk)
           umma_ss(tmem + Sh::kColDK, kmajor(sDs, kk), mnmajor(sQ, kk), id_dk,
                   (kk == 0) ? acc_first : 1u);
-        // dQ = dS K  -> region B
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ss(tmem + Sh::kColB, mnmajor(sDs, kk), mnmajor(sK, kk), id_dq, kk > 0 ? 1u : 0u);
-        umma_commit(&bars->dq_ready);
         umma_commit(&bars->qd_empty[slot]);
-        // next S^T into region A (P^T of this item has been consumed in order)
-        if (it + 1 < n_items) {
-          const int ns = (it + 1) & 1;
-          if (!(ok = bwd_wait(&bars->qd_full[ns], static_cast<uint32_t>((it + 1) >> 1) & 1u, abort)))
-            break;
-          tc_fence_after();
-          issue_s(smem_u32(smem + Sh::kOffQ + ns * 2 * Sh::kTileBytes));
+        // next dP^T into region B: the dS pass of this item has read dP^T.
+        // s_ready completes after dK, so the next dS^T write is safe too.
+        if (more) {
+          issue_dp(it + 1);
+          umma_commit(&bars->s_ready);
         }
       }
       umma_commit(&bars->final_done);
@@ -348,12 +361,9 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ======================= compute groups =======================
-    // Group g (warps 2-5: g = 0; warps 6-9: g = 1) owns query columns
-    // [64g, 64g+64) of S^T and dP^T (one thread per key row), and columns
-    // [64g, 64g+64) of each dQ tile (one thread per query row).
     const int g = (warp - 2) >> 2;
     const int lane_base = 32 * (warp & 3);
-    const int r = lane_base + lane;
+    const int r = lane_base + lane;             // key row within the tile
     const int key = k0 + r;
     const int gt = static_cast<int>(threadIdx.x) - 64 - 128 * g;  // 0..127 in the group
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
@@ -384,10 +394,8 @@ __global__ void __launch_bounds__(320, 1)
       return v;
     };
     float nv = load_vec(0);
-    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < n_items; ++it) {
-      const int h = kvh * p.group + it / i_cnt;
       const int i0 = (i_begin + it % i_cnt) * 128;
       named_bar_sync(bar_id, 128);  // the group is done with the previous vectors
       if (gt < 64)
@@ -413,34 +421,16 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t sr[32];
         tmem_ld32(t_a + c * 32, sr);
         tmem_ld_wait();
-        bool poly = false;
-        if constexpr (kCap) {
-          float amax = 0.f;
-#pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(sr[i])), fabsf(__uint_as_float(sr[i + 1]))));
-          poly = __all_sync(0xffffffffu, amax * fabsf(p.cap_in) <= kTanhPolyMax);
-        }
+        const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
         uint32_t pk[16];
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
           const int jl = cc * 32 + 2 * j2;  // query within the group
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
           const float2 l2 = *reinterpret_cast<const float2*>(glse + jl);
-          float2 arg, fac;
-          if constexpr (kCap) {
-            float2 th;
-            if (poly)
-              th = tanh_poly2(__fmul2_rn(s2, make_float2(p.cap_in, p.cap_in)));
-            else
-              th = make_float2(tanh_fast(s2.x * p.cap_in), tanh_fast(s2.y * p.cap_in));
-            arg = make_float2(p.cap_out_log2 * th.x - l2.x, p.cap_out_log2 * th.y - l2.y);
-            fac = make_float2((1.f - th.x * th.x) * p.scale, (1.f - th.y * th.y) * p.scale);
-          } else {
-            arg = __ffma2_rn(s2, sc2, make_float2(-l2.x, -l2.y));
-            fac = make_float2(p.scale, p.scale);
-          }
-          float2 pr = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+          float2 x, fac;
+          bwd_logit2<kCap>(s2, poly, p, x, fac);
+          float2 pr = make_float2(ex2_approx(x.x - l2.x), ex2_approx(x.y - l2.y));
           if (need_mask) {
             const int q0i = qg_lo + jl;
             bool v0 = key < seq_len && q0i < seq_len;
@@ -469,7 +459,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);  // dV may start
-      // pass 2: dS^T = w * (dP^T - Drow) -> shared memory (the dK and dQ operand)
+      // pass 2: dS^T = w * (dP^T - Drow) -> shared memory (the dK operand)
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * g + cc;
@@ -498,45 +488,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_ready);
-
-      // ---- dQ tile: TMEM -> shared-memory staging -> TMA reduce-add ----
-      // The staging slot is this group's half of the dS^T buffer: dq_ready
-      // follows the dK and dQ MMAs that read dS^T, and the next dS^T is only
-      // written after dq_free (both groups) has let the next dP^T MMA run.
-      if (!(ok = bwd_wait(&bars->dq_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
-      tc_fence_after();
-      uint8_t* stage = smem + Sh::kOffDs + g * Sh::kChunkBytes;
-      const bool valid = i0 + r < seq_len;
-#pragma unroll 1
-      for (int cc = 0; cc < kD / 64; ++cc) {
-        const int c = (kD / 64) * g + cc;  // 32-column dQ chunk
-        uint32_t rr[32];
-        tmem_ld32(t_b + c * 32, rr);
-        tmem_ld_wait();
-        if (cc > 0) {
-          if (gt == 0) bulk_wait_read<0>();  // previous chunk has left the slot
-          named_bar_sync(bar_id, 128);
-        }
-        uint8_t* rowp = stage + r * 128;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 v = valid ? make_uint4(rr[4 * j], rr[4 * j + 1], rr[4 * j + 2], rr[4 * j + 3])
-                                : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(rowp + ((j ^ (r & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(bar_id, 128);
-        if (gt == 0) {
-          tma_reduce_add_3d(&tm_dq, stage, c * 32, h, seq_start + i0);
-          bulk_commit();
-        }
-      }
-      if (gt == 0) bulk_wait_read<0>();
-      tc_fence_before();
-      named_bar_sync(bar_id, 128);
-      if (gt == 0) mbar_arrive(&bars->dq_free);
     }
-    if (gt == 0) bulk_wait<0>();  // every reduction has reached global memory
 
     // ---- epilogue: group 0 writes the dV rows, group 1 the dK rows ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
@@ -552,18 +504,341 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t rr[32];
         tmem_ld32(tmem + lane_off + col + c * 32, rr);
         tmem_ld_wait();
-        uint32_t w[16];
+        uint32_t wv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+        for (int i = 0; i < 16; ++i) wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
         if (key < seq_len) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
         }
       }
     } else if (ok && key < seq_len) {
       uint4* d4 = reinterpret_cast<uint4*>(dst);
       for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Sh::kTmemCols);
+  }
+}
+
+// ===========================================================================
+// dQ
+// ===========================================================================
+// One CTA per (sequence, query head, 128-row Q tile), structured like the
+// forward kernel:
+//   warp 0     TMA producer: Q, dO once; K_j, V_j into a ring of slots.
+//   warp 1     MMA issuer: S_j = Q K_j^T (two TMEM buffers, alternating),
+//              dP_j = dO V_j^T, then dQ += dS_j K_j with dS_j read from TMEM.
+//   warps 2-9  two compute groups, one thread per query row; group g owns key
+//              columns [64g, 64g+64) of S_j and dP_j and writes dS_j (16-bit)
+//              over the S columns it has read. LSE and Drow of the row live in
+//              registers.
+// TMEM columns: S buffers [0,128) and [128,256), dP [256,384), dQ [384, 384+D).
+// MMA order per tile j: S_{j+1}, dQ_j, dP_{j+1}: the tensor core computes the
+// next scores while the compute groups form dS_j.
+template <int kD>
+struct DqShape {
+  static constexpr int kChunks = kD / 64;
+  static constexpr int kChunkBytes = 128 * 128;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = kD == 128 ? 4 : 8;    // K/V ring slots
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kTileBytes;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr int kThreads = 320;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kColS = 0;      // + 128 * buffer
+  static constexpr int kColDP = 256;
+  static constexpr int kColDQ = 384;
+};
+
+struct DqBars {
+  uint64_t qd_full;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t s_ready;
+  uint64_t ds_ready;
+  uint64_t final_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int kD, bool kBF16, bool kCap>
+__global__ void __launch_bounds__(320, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+  using Sh = DqShape<kD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + Sh::kOffBar);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (sequence, head) major; Q tiles with most keys first
+  const int nq = p.n_ktiles;  // 128-row tiles per sequence
+  const int bh = static_cast<int>(blockIdx.x) / nq;
+  const int qt = nq - 1 - static_cast<int>(blockIdx.x) % nq;
+  const int h = bh % p.Hq;
+  const int b = bh / p.Hq;
+  int seq_start, seq_len;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    seq_len = p.cu_seqlens[b + 1] - seq_start;
+  } else {
+    seq_start = b * p.S;
+    seq_len = p.S;
+  }
+  const int q0 = qt * 128;
+  if (q0 >= seq_len) return;
+  const int kvh = h / p.group;
+  const int row_hi = min(q0 + 127, seq_len - 1);
+  int key_hi = seq_len - 1;
+  if (p.wr >= 0) key_hi = min(key_hi, row_hi + p.wr);
+  int key_lo = 0;
+  if (p.wl >= 0) key_lo = max(0, q0 - p.wl);
+  const int n_begin = key_lo / 128;
+  const int n_tiles = key_hi >= key_lo ? key_hi / 128 + 1 - n_begin : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->qd_full, 1);
+    for (int i = 0; i < Sh::kStages; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->ds_ready, 8);
+    mbar_init(&bars->final_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, Sh::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(&bars->qd_full, 2 * Sh::kTileBytes);
+      for (int c = 0; c < Sh::kChunks; ++c) {
+        tma_load_3d(&tm_q, &bars->qd_full, smem + Sh::kOffQ + c * Sh::kChunkBytes, c * 64, h,
+                    seq_start + q0);
+        tma_load_3d(&tm_do, &bars->qd_full, smem + Sh::kOffDO + c * Sh::kChunkBytes, c * 64, h,
+                    seq_start + q0);
+      }
+      int fill = 0;
+      for (int j = 0; j < n_tiles && !*abort; ++j) {
+        const int tok = seq_start + (n_begin + j) * 128;
+        for (int kv = 0; kv < 2; ++kv, ++fill) {
+          const int slot = fill % Sh::kStages;
+          const uint32_t ph = static_cast<uint32_t>(fill / Sh::kStages) & 1u;
+          if (!bwd_wait(&bars->kv_empty[slot], ph ^ 1u, abort)) break;
+          mbar_arrive_expect_tx(&bars->kv_full[slot], Sh::kTileBytes);
+          uint8_t* dst = smem + Sh::kOffKV + slot * Sh::kTileBytes;
+          const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+          for (int c = 0; c < Sh::kChunks; ++c)
+            tma_load_3d(tm, &bars->kv_full[slot], dst + c * Sh::kChunkBytes, c * 64, kvh, tok);
+        }
+      }
+      for (int f = max(0, fill - Sh::kStages); f < fill; ++f)
+        mbar_wait(&bars->kv_full[f % Sh::kStages], static_cast<uint32_t>(f / Sh::kStages) & 1u);
+      mbar_wait(&bars->qd_full, 0);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (elect_one()) {
+      constexpr uint32_t id_s = idesc_f16(kBF16, 128, 128, false, false);   // S, dP
+      constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, false, true);    // dS (tmem) x K
+      const uint32_t sQ = smem_u32(smem + Sh::kOffQ);
+      const uint32_t sDO = smem_u32(smem + Sh::kOffDO);
+      const uint32_t sKV = smem_u32(smem + Sh::kOffKV);
+      bool ok = bwd_wait(&bars->qd_full, 0, abort);
+      tc_fence_after();
+      auto kmajor = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
+      };
+      auto wait_slot = [&](int fill) {
+        return bwd_wait(&bars->kv_full[fill % Sh::kStages],
+                        static_cast<uint32_t>(fill / Sh::kStages) & 1u, abort);
+      };
+      auto slot_addr = [&](int fill) { return sKV + (fill % Sh::kStages) * Sh::kTileBytes; };
+      auto issue_s = [&](int j) {  // S_j = Q K_j^T -> buffer j & 1
+        const uint32_t sK = slot_addr(2 * j);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColS + 128 * (j & 1), kmajor(sQ, kk), kmajor(sK, kk), id_s,
+                  kk > 0 ? 1u : 0u);
+      };
+      auto issue_dp = [&](int j) {  // dP_j = dO V_j^T
+        const uint32_t sV = slot_addr(2 * j + 1);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColDP, kmajor(sDO, kk), kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+      };
+      if (ok && n_tiles > 0) {
+        if ((ok = wait_slot(0))) {
+          tc_fence_after();
+          issue_s(0);
+          if ((ok = wait_slot(1))) {
+            tc_fence_after();
+            issue_dp(0);
+            umma_commit(&bars->s_ready);
+          }
+        }
+      }
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const bool more = j + 1 < n_tiles;
+        // S_{j+1} into the other buffer (its previous dS was consumed by dQ_{j-1})
+        if (more) {
+          if (!(ok = wait_slot(2 * (j + 1)))) break;
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
+        tc_fence_after();
+        // dQ += dS_j K_j: A = dS_j from TMEM (keys [64g, 64g+64) packed into
+        // columns [64g, 64g+32) of buffer j & 1), B = K_j with N = D (MN-major)
+        {
+          const uint32_t sK = slot_addr(2 * j);
+          const uint32_t a = tmem + Sh::kColS + 128 * (j & 1);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            umma_ts(tmem + Sh::kColDQ, a + (kk >> 2) * 64 + (kk & 3) * 8,
+                    sdesc_sw128(sK + kk * 2048, Sh::kChunkBytes, 1024), id_dq,
+                    (j == 0 && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(&bars->kv_empty[(2 * j) % Sh::kStages]);      // K_j
+        umma_commit(&bars->kv_empty[(2 * j + 1) % Sh::kStages]);  // V_j
+        // dP_{j+1}: the compute groups have read dP_j before ds_ready
+        if (more) {
+          if (!(ok = wait_slot(2 * (j + 1) + 1))) break;
+          tc_fence_after();
+          issue_dp(j + 1);
+          umma_commit(&bars->s_ready);
+        }
+      }
+      umma_commit(&bars->final_done);
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ======================= compute groups =======================
+    const int g = (warp - 2) >> 2;
+    const int lane_base = 32 * (warp & 3);
+    const int r = lane_base + lane;          // query row within the tile
+    const int qrow = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
+    // the row's LSE (exp2 domain) and Drow
+    float lse2 = INFINITY, drow = 0.f;
+    if (qrow < seq_len) {
+      const size_t li = p.cu_seqlens != nullptr ? static_cast<size_t>(h) * p.total + seq_start + qrow
+                                                : (static_cast<size_t>(b) * p.Hq + h) * p.S + qrow;
+      const float l = p.lse[li];
+      lse2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+      drow = p.drow[li];
+    }
+    const float2 nl2 = make_float2(-lse2, -lse2);
+    const float2 nd2 = make_float2(-drow, -drow);
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
+      tc_fence_after();
+      const int k0 = (n_begin + j) * 128 + 64 * g;  // first key of this group's columns
+      const uint32_t t_s = tmem + lane_off + Sh::kColS + 128 * (j & 1) + 64 * g;
+      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 64 * g;
+      // mask needed for this warp's 32 rows x the group's 64 keys?
+      const int r_lo = q0 + lane_base, r_hi = r_lo + 31;
+      bool need_mask = (k0 + 63 >= seq_len) || (r_hi >= seq_len);
+      if (p.wr >= 0) need_mask |= (k0 + 63 > r_lo + p.wr);
+      if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {  // 32 keys per chunk
+        uint32_t sr[32], dr[32];
+        tmem_ld32(t_s + 32 * cc, sr);
+        tmem_ld32(t_dp + 32 * cc, dr);
+        tmem_ld_wait();
+        const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
+        uint32_t dsk[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
+          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
+          float2 x, fac;
+          bwd_logit2<kCap>(s2, poly, p, x, fac);
+          const float2 arg = __fadd2_rn(x, nl2);
+          float2 pr = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+          if (need_mask) {
+            const int kj = k0 + 32 * cc + 2 * j2;
+            bool v0 = qrow < seq_len && kj < seq_len;
+            bool v1 = qrow < seq_len && kj + 1 < seq_len;
+            if (p.wr >= 0) {
+              v0 = v0 && kj <= qrow + p.wr;
+              v1 = v1 && kj + 1 <= qrow + p.wr;
+            }
+            if (p.wl >= 0) {
+              v0 = v0 && kj >= qrow - p.wl;
+              v1 = v1 && kj + 1 >= qrow - p.wl;
+            }
+            pr.x = v0 ? pr.x : 0.f;
+            pr.y = v1 ? pr.y : 0.f;
+          }
+          const float2 ds = __fmul2_rn(__fmul2_rn(__fadd2_rn(dp2, nd2), pr), fac);
+          dsk[j2] = pack2<kBF16>(ds.x, ds.y);
+        }
+        // dS of keys [k0 + 32cc, +32) -> columns [64g + 16cc, +16) of the
+        // S buffer (columns this group has already read)
+        tmem_st16(t_s + 16 * cc, dsk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_ready);
+    }
+    // ---- epilogue: dQ row -> dq; group g writes columns [g D/2, (g+1) D/2) ----
+    if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
+    tc_fence_after();
+    uint8_t* dst = static_cast<uint8_t*>(p.dq) + (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD * 2;
+    if (ok && n_tiles > 0) {
+#pragma unroll 1
+      for (int c = g * (kD / 64); c < (g + 1) * (kD / 64); ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_off + Sh::kColDQ + c * 32, rr);
+        tmem_ld_wait();
+        uint32_t wv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+        if (qrow < seq_len) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+        }
+      }
+    } else if (ok && qrow < seq_len) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + g * kD);
+      for (int i = 0; i < kD / 16; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   tc_fence_before();

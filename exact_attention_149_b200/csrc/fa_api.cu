@@ -106,24 +106,6 @@ fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, i
   return FA_OK;
 }
 
-// 3-D map over a (tokens, heads, D) row-major float32 tensor; box = 32
-// columns (128 B) x 1 head x `rows` tokens, 128-byte swizzle. Used for the
-// backward's bulk reduce-add of dQ tiles.
-fa_status make_map_thd_f32(CUtensorMap* map, const void* base, int D, int H, long long T, int rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
-                        static_cast<cuuint64_t>(T)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H) * D * 4};
-  cuuint32_t box[3] = {32u, 1u, static_cast<cuuint32_t>(rows)};
-  cuuint32_t es[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
-                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (f32) failed (%d)", static_cast<int>(r));
-  return FA_OK;
-}
-
 // ---------------------------------------------------------------------------
 // optional per-kernel timing (events around each launch on the caller's stream)
 // ---------------------------------------------------------------------------

@@ -82,8 +82,9 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, 
                  fa_dtype dtype, void* stream);
 
 /*
- * Workspace bytes needed by fa_bwd for these sizes (float32 dQ accumulator
- * plus per-row dot(dO, O)); total_tokens as in fa_fwd (ignored if <= 0).
+ * Workspace bytes needed by fa_bwd for these sizes (the float32 per-row
+ * dot(dO, O), one per token and query head); total_tokens as in fa_fwd
+ * (ignored if <= 0).
  */
 FA_API size_t fa_bwd_workspace_size(int B, int Hq, int S, int D, int total_tokens);
 
@@ -97,6 +98,8 @@ FA_API size_t fa_bwd_workspace_size(int B, int Hq, int S, int D, int total_token
  *   head of a group are summed into the shared kv head).
  *   workspace: device memory of at least fa_bwd_workspace_size() bytes,
  *   256-byte aligned; its contents on entry do not matter.
+ *   The result is deterministic: no atomics; dK, dV come from one CTA per key
+ *   tile and dQ from one CTA per query tile.
  * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null dout/dq/dk/dv or a
  *   workspace that is null or too small.
  */
@@ -190,8 +193,8 @@ FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const 
  *   fa_kernel_timing_enable(1/0) switches recording on or off (host-wide).
  *   fa_kernel_timing_read(name, &total_ms, &launches) waits for the recorded
  *     events and returns the summed duration and count of the launches of
- *     the kernel `name` ("fwd", "bwd_pre", "bwd_main", "bwd_post",
- *     "kv_append", "decode_split", "lse_combine") since the last reset.
+ *     the kernel `name` ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq", "kv_append",
+ *     "decode_split", "lse_combine") since the last reset.
  *   fa_kernel_timing_reset() drops all records.
  * Errors: FA_ERR_INVALID_ARG for null arguments, FA_ERR_CUDA if an event
  * call fails.

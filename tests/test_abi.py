@@ -56,10 +56,10 @@ def test_version(fa):
 
 
 def test_workspace_sizes(fa):
-    # dQ accumulator (float32 T*Hq*D) + row dots (float32 T*Hq), each padded to 256 B
+    # row dots rowsum(dO * O): float32 per (token, query head), padded to 256 B
     n = fa.fa_bwd_workspace_size(2, 32, 8192, 128)
-    assert n == 2 * 8192 * 32 * 128 * 4 + 2 * 8192 * 32 * 4
-    assert fa.fa_bwd_workspace_size(3, 4, 0, 128, 1000) == 1000 * 4 * 128 * 4 + 16128 + 256 * 0
+    assert n == 2 * 8192 * 32 * 4
+    assert fa.fa_bwd_workspace_size(3, 4, 0, 128, 1000) == 16128
     assert fa.fa_kvcache_workspace_size(64, 32, 128, 1) == 0
     assert fa.fa_kvcache_workspace_size(64, 32, 128, 16) == 16 * 64 * 32 * 129 * 4
 

@@ -26,7 +26,7 @@ def test_timing_counts_each_launch(cuda_ok):
         fa.fa_kernel_timing_enable(False)
     ms, n = fa.fa_kernel_timing_read("fwd")
     assert n == 3 and ms > 0.0
-    for name in ("bwd_pre", "bwd_main", "bwd_post"):
+    for name in ("bwd_pre", "bwd_dkdv", "bwd_dq"):
         ms, n = fa.fa_kernel_timing_read(name)
         assert n == 1 and ms > 0.0, name
     assert fa.fa_kernel_timing_read("decode_split") == (0.0, 0)

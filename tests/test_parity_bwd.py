@@ -69,14 +69,15 @@ def test_bwd_varlen(cuda_ok, lengths, Hq, Hkv, D, causal, window, softcap):
     check_bwd(got, ref, f"varlen {lengths}")
 
 
-def test_bwd_is_stable_across_runs(cuda_ok):
-    """dK and dV come from one CTA each (no atomics): bitwise reproducible.
-    dQ uses float atomics, so it is only compared within tolerance."""
+def test_bwd_is_deterministic(cuda_ok):
+    """dK and dV come from one CTA per key tile and dQ from one CTA per query
+    tile, with no atomics: repeated runs are bitwise identical (a race would
+    show up here)."""
     inp = W.make_fwd_inputs(1, 600, 4, 2, 128, "bf16", seed=9, with_do=True)
     a = _gpu_fwd_bwd(inp, 0.088, True, (-1, -1), 0.0)
     b = _gpu_fwd_bwd(inp, 0.088, True, (-1, -1), 0.0)
-    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
-    assert rel_fro(to64(a[0]), to64(b[0])) < 1e-3
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
 
 
 @pytest.mark.slow
