@@ -32,8 +32,9 @@
 //              dV, group 1 dK.
 // TMEM columns: A [0,128) S^T then P^T (queries [64g, 64g+64) packed into
 // [64g, 64g+32)); B [128,256) dP^T; dV [256, 256+D); dK [256+D, 256+2D).
-// MMA order per item i: dV_i, S_{i+1}, dK_i, dP_{i+1}: the tensor core only
-// waits for the P pass of each item.
+// MMA order per item i: dV_i, S_{i+1}, dK_i, dP_{i+1}. S^T and dP^T signal
+// separately, so the P pass of item i+1 overlaps dK_i and dP_{i+1}, and the
+// dS pass of item i overlaps dV_i and S_{i+1}.
 #pragma once
 
 #include "ptx.cuh"
@@ -172,6 +173,7 @@ struct DkdvBars {
   uint64_t qd_full[2];
   uint64_t qd_empty[2];
   uint64_t s_ready;
+  uint64_t dp_ready;
   uint64_t p_ready;
   uint64_t ds_ready;
   uint64_t final_done;
@@ -228,6 +230,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->qd_empty[s], 1);
     }
     mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->dp_ready, 1);
     mbar_init(&bars->p_ready, 8);
     mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->final_done, 1);
@@ -313,8 +316,9 @@ __global__ void __launch_bounds__(320, 1)
         if ((ok = bwd_wait(&bars->qd_full[0], 0, abort))) {
           tc_fence_after();
           issue_s(0);
-          issue_dp(0);
           umma_commit(&bars->s_ready);
+          issue_dp(0);
+          umma_commit(&bars->dp_ready);
         }
       }
       for (int it = 0; it < n_items && ok; ++it) {
@@ -338,6 +342,7 @@ __global__ void __launch_bounds__(320, 1)
             break;
           tc_fence_after();
           issue_s(it + 1);
+          umma_commit(&bars->s_ready);  // the next P pass can start now
         }
         // dK += dS^T Q (after dS^T is in shared memory)
         if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
@@ -348,10 +353,10 @@ __global__ void __launch_bounds__(320, 1)
                   (kk == 0) ? acc_first : 1u);
         umma_commit(&bars->qd_empty[slot]);
         // next dP^T into region B: the dS pass of this item has read dP^T.
-        // s_ready completes after dK, so the next dS^T write is safe too.
+        // dp_ready completes after dK, so the next dS^T write is safe too.
         if (more) {
           issue_dp(it + 1);
-          umma_commit(&bars->s_ready);
+          umma_commit(&bars->dp_ready);
         }
       }
       umma_commit(&bars->final_done);
@@ -459,7 +464,11 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);  // dV may start
-      // pass 2: dS^T = w * (dP^T - Drow) -> shared memory (the dK operand)
+      // pass 2: dS^T = w * (dP^T - Drow) -> shared memory (the dK operand),
+      // once dP^T is in TMEM (which also means the previous dK has finished
+      // reading the dS^T buffer)
+      if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+      tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * g + cc;
@@ -539,8 +548,9 @@ __global__ void __launch_bounds__(320, 1)
 //              over the S columns it has read. LSE and Drow of the row live in
 //              registers.
 // TMEM columns: S buffers [0,128) and [128,256), dP [256,384), dQ [384, 384+D).
-// MMA order per tile j: S_{j+1}, dQ_j, dP_{j+1}: the tensor core computes the
-// next scores while the compute groups form dS_j.
+// MMA order per tile j: S_{j+1}, dQ_j, dP_{j+1}. S and dP signal separately:
+// the compute groups form P_{j+1} (needs S only) while the tensor core runs
+// dQ_j and dP_{j+1}, then dS_{j+1} once dP_{j+1} is there.
 template <int kD>
 struct DqShape {
   static constexpr int kChunks = kD / 64;
@@ -564,6 +574,7 @@ struct DqBars {
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint64_t s_ready;
+  uint64_t dp_ready;
   uint64_t ds_ready;
   uint64_t final_done;
   uint64_t drain;
@@ -617,6 +628,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->kv_empty[i], 1);
     }
     mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->dp_ready, 1);
     mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
@@ -701,10 +713,11 @@ __global__ void __launch_bounds__(320, 1)
         if ((ok = wait_slot(0))) {
           tc_fence_after();
           issue_s(0);
+          umma_commit(&bars->s_ready);
           if ((ok = wait_slot(1))) {
             tc_fence_after();
             issue_dp(0);
-            umma_commit(&bars->s_ready);
+            umma_commit(&bars->dp_ready);
           }
         }
       }
@@ -715,6 +728,7 @@ __global__ void __launch_bounds__(320, 1)
           if (!(ok = wait_slot(2 * (j + 1)))) break;
           tc_fence_after();
           issue_s(j + 1);
+          umma_commit(&bars->s_ready);
         }
         if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
         tc_fence_after();
@@ -736,7 +750,7 @@ __global__ void __launch_bounds__(320, 1)
           if (!(ok = wait_slot(2 * (j + 1) + 1))) break;
           tc_fence_after();
           issue_dp(j + 1);
-          umma_commit(&bars->s_ready);
+          umma_commit(&bars->dp_ready);
         }
       }
       umma_commit(&bars->final_done);
@@ -774,18 +788,18 @@ __global__ void __launch_bounds__(320, 1)
       bool need_mask = (k0 + 63 >= seq_len) || (r_hi >= seq_len);
       if (p.wr >= 0) need_mask |= (k0 + 63 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
-#pragma unroll 1
+      // pass 1 (needs S_j only): w = P * scale (* (1 - tanh^2)) for the
+      // group's 64 keys, kept in registers
+      float w[64];
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {  // 32 keys per chunk
-        uint32_t sr[32], dr[32];
+        uint32_t sr[32];
         tmem_ld32(t_s + 32 * cc, sr);
-        tmem_ld32(t_dp + 32 * cc, dr);
         tmem_ld_wait();
         const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
-        uint32_t dsk[16];
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
-          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
           float2 x, fac;
           bwd_logit2<kCap>(s2, poly, p, x, fac);
           const float2 arg = __fadd2_rn(x, nl2);
@@ -805,7 +819,25 @@ __global__ void __launch_bounds__(320, 1)
             pr.x = v0 ? pr.x : 0.f;
             pr.y = v1 ? pr.y : 0.f;
           }
-          const float2 ds = __fmul2_rn(__fmul2_rn(__fadd2_rn(dp2, nd2), pr), fac);
+          const float2 wv = __fmul2_rn(pr, fac);
+          w[32 * cc + 2 * j2] = wv.x;
+          w[32 * cc + 2 * j2 + 1] = wv.y;
+        }
+      }
+      // pass 2 (needs dP_j): dS = w * (dP - Drow) -> the S columns already read
+      if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t dr[32];
+        tmem_ld32(t_dp + 32 * cc, dr);
+        tmem_ld_wait();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
+          const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2),
+                                       make_float2(w[32 * cc + 2 * j2], w[32 * cc + 2 * j2 + 1]));
           dsk[j2] = pack2<kBF16>(ds.x, ds.y);
         }
         // dS of keys [k0 + 32cc, +32) -> columns [64g + 16cc, +16) of the

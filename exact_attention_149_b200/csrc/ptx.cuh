@@ -342,7 +342,7 @@ __device__ __forceinline__ float tanh_fast(float y) {
 }
 
 // tanh(y) = y * Q(y^2) for |y| <= kTanhPolyMax, Q of degree 4 fitted by the
-// Remez exchange algorithm for minimal relative error (fit_tanh_poly.py next
+// Remez exchange algorithm for minimal relative error (fit_polynomials.py next
 // to this file derives the coefficients; float64 relative error 1.3e-8,
 // float32 evaluation within 4e-8 absolute). Two values per call, on the FMA
 // pipe, instead of the two special-function operations of tanh_fast.
