@@ -26,12 +26,13 @@
 //   warp 0     TMA producer: K, V once; Q_i and dO_i into a 2-slot ring.
 //   warp 1     MMA issuer (one lane), TMEM owner.
 //   warps 2-9  two compute groups; group g owns query columns [64g, 64g+64):
-//              one thread per key row computes P^T = exp(S^T - LSE) (-> TMEM,
-//              16-bit, for the dV MMA) and then dS^T = P^T * (dP^T - Drow)
-//              (-> shared memory, for the dK MMA); at the end group 0 writes
-//              dV, group 1 dK.
-// TMEM columns: A [0,128) S^T then P^T (queries [64g, 64g+64) packed into
-// [64g, 64g+32)); B [128,256) dP^T; dV [256, 256+D); dK [256+D, 256+2D).
+//              one thread per key row computes P^T = exp(S^T - LSE) and then
+//              dS^T = P^T * (dP^T - Drow), each written back to TMEM as 16-bit
+//              over the columns it came from, where the dV and dK MMAs read
+//              their A operand; at the end group 0 writes dV, group 1 dK.
+// TMEM columns: A [0,128) S^T then P^T; B [128,256) dP^T then dS^T (queries
+// [64g, 64g+64) packed into [64g, 64g+32) of each); dV [256, 256+D);
+// dK [256+D, 256+2D).
 // MMA order per item i: dV_i, S_{i+1}, dK_i, dP_{i+1}. S^T and dP^T signal
 // separately, so the P pass of item i+1 overlaps dK_i and dP_{i+1}, and the
 // dS pass of item i overlaps dV_i and S_{i+1}.
@@ -152,12 +153,10 @@ struct DkdvShape {
   static constexpr int kChunks = kD / 64;
   static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kDsBytes = 2 * kChunkBytes;     // 128 keys x 128 queries x 16 bit
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;         // + slot * 2 * kTileBytes (Q, dO)
-  static constexpr int kOffDs = 6 * kTileBytes;
-  static constexpr int kOffVec = kOffDs + kDsBytes;    // lse_log2[128], drow[128]
+  static constexpr int kOffVec = 6 * kTileBytes;       // lse_log2[128], drow[128]
   static constexpr int kOffBar = kOffVec + 1024;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
   static constexpr int kThreads = 320;
@@ -287,10 +286,9 @@ __global__ void __launch_bounds__(320, 1)
     if (elect_one()) {
       constexpr uint32_t id_s = idesc_f16(kBF16, 128, 128, false, false);   // S^T, dP^T
       constexpr uint32_t id_dv = idesc_f16(kBF16, 128, kD, false, true);    // P^T (tmem) x dO
-      constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);    // dS^T x Q
+      constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);    // dS^T (tmem) x Q
       const uint32_t sK = smem_u32(smem + Sh::kOffK);
       const uint32_t sV = smem_u32(smem + Sh::kOffV);
-      const uint32_t sDs = smem_u32(smem + Sh::kOffDs);
       bool ok = bwd_wait(&bars->kv_full, 0, abort);
       tc_fence_after();
       auto kmajor = [](uint32_t base, int kk) {
@@ -344,16 +342,16 @@ __global__ void __launch_bounds__(320, 1)
           issue_s(it + 1);
           umma_commit(&bars->s_ready);  // the next P pass can start now
         }
-        // dK += dS^T Q (after dS^T is in shared memory)
+        // dK += dS^T Q (A = dS^T from TMEM region B, packed like P^T)
         if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ss(tmem + Sh::kColDK, kmajor(sDs, kk), mnmajor(sQ, kk), id_dk,
-                  (kk == 0) ? acc_first : 1u);
+          umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + (kk >> 2) * 64 + (kk & 3) * 8,
+                  mnmajor(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
         umma_commit(&bars->qd_empty[slot]);
-        // next dP^T into region B: the dS pass of this item has read dP^T.
-        // dp_ready completes after dK, so the next dS^T write is safe too.
+        // next dP^T into region B: dK (the reader of dS^T there) precedes it
+        // in issue order, and dp_ready completes after both.
         if (more) {
           issue_dp(it + 1);
           umma_commit(&bars->dp_ready);
@@ -428,11 +426,13 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait();
         const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
         uint32_t pk[16];
+        float4 l4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
           const int jl = cc * 32 + 2 * j2;  // query within the group
+          if ((j2 & 1) == 0) l4 = *reinterpret_cast<const float4*>(glse + jl);
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
-          const float2 l2 = *reinterpret_cast<const float2*>(glse + jl);
+          const float2 l2 = (j2 & 1) == 0 ? make_float2(l4.x, l4.y) : make_float2(l4.z, l4.w);
           float2 x, fac;
           bwd_logit2<kCap>(s2, poly, p, x, fac);
           float2 pr = make_float2(ex2_approx(x.x - l2.x), ex2_approx(x.y - l2.y));
@@ -464,9 +464,9 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);  // dV may start
-      // pass 2: dS^T = w * (dP^T - Drow) -> shared memory (the dK operand),
-      // once dP^T is in TMEM (which also means the previous dK has finished
-      // reading the dS^T buffer)
+      // pass 2: dS^T = w * (dP^T - Drow) -> TMEM region B (the dK operand),
+      // once dP^T is in TMEM (dK of the previous item, the last reader of the
+      // dS^T columns, precedes the dP^T MMA in issue order)
       if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
       tc_fence_after();
 #pragma unroll
@@ -477,23 +477,23 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait();
         uint32_t dsk[16];
 #pragma unroll
-        for (int j2 = 0; j2 < 16; ++j2) {
-          const int jl = cc * 32 + 2 * j2;
-          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
-          const float2 d2 = *reinterpret_cast<const float2*>(gdrow + jl);
-          const float2 ds = __fmul2_rn(__fadd2_rn(dp2, make_float2(-d2.x, -d2.y)), make_float2(w[jl], w[jl + 1]));
-          dsk[j2] = pack2<kBF16>(ds.x, ds.y);
-        }
-        // dS^T row r, queries [32c, 32c+32): 64-query chunk g, 16-byte groups 4cc..4cc+3
-        uint8_t* rowp = smem + Sh::kOffDs + g * Sh::kChunkBytes + r * 128;
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const int jl = cc * 32 + 4 * j4;
+          const float4 d4 = *reinterpret_cast<const float4*>(gdrow + jl);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int gg = cc * 4 + q4;
-          *reinterpret_cast<uint4*>(rowp + ((gg ^ (r & 7)) << 4)) =
-              make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int j2 = 2 * j4 + h2;
+            const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
+            const float2 d2 = h2 == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
+            const float2 ds = __fmul2_rn(__fadd2_rn(dp2, d2), make_float2(w[jl + 2 * h2], w[jl + 2 * h2 + 1]));
+            dsk[j2] = pack2<kBF16>(ds.x, ds.y);
+          }
         }
+        // dS^T of queries [32c, 32c+32) -> region B columns [64g + 16cc, +16)
+        // (dP^T columns this group has already read)
+        tmem_st16(t_b + 64 * g + 16 * cc, dsk);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_ready);
