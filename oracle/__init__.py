@@ -11,6 +11,8 @@ from .attention import (  # noqa: F401
     head_fwd,
     kvcache_decode,
     lse_combine,
+    rotary,
+    round_to,
     scores,
     visible_mask,
 )

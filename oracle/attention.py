@@ -61,6 +61,8 @@ __all__ = [
     "attention_bwd",
     "kvcache_decode",
     "lse_combine",
+    "rotary",
+    "round_to",
 ]
 
 
@@ -259,42 +261,104 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool = False, window=(-1, -
     return dq, dk, dv
 
 
+def round_to(x, dtype):
+    """Round float64 values to a 16-bit type (round to nearest even) and back.
+    "bf16": through float32 bits; "fp16": numpy float16; None: unchanged."""
+    x = np.asarray(x, dtype=np.float64)
+    if dtype is None:
+        return x
+    if dtype == "fp16":
+        return x.astype(np.float16).astype(np.float64)
+    if dtype == "bf16":
+        b = x.astype(np.float32).view(np.uint32).astype(np.uint64)
+        b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+        return b.astype(np.uint32).view(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def rotary(x, pos, cos, sin, interleaved=False):
+    """Rotary position embedding of the last dimension of x (..., T, H, D) at
+    integer positions pos (T,): with r = rotary dim (2 * cos.shape[1]) and
+    angle tables cos, sin of shape (positions, r/2), each pair (a, b) of the
+    first r dimensions becomes (a cos - b sin, a sin + b cos). Pairs are
+    (i, i + r/2) by default, (2i, 2i + 1) when interleaved; dimensions from r
+    on are unchanged. (Guide §增量解码场景: rotary_cos / rotary_sin apply the
+    rotary position encoding inside the call; the pairing is a reading.)"""
+    x = _f64(x).copy()
+    cos = _f64(cos)
+    sin = _f64(sin)
+    half = cos.shape[1]
+    c = cos[np.asarray(pos)][:, None, :]  # (T, 1, r/2)
+    sn = sin[np.asarray(pos)][:, None, :]
+    if interleaved:
+        a = x[..., 0:2 * half:2].copy()
+        b = x[..., 1:2 * half:2].copy()
+        x[..., 0:2 * half:2] = a * c - b * sn
+        x[..., 1:2 * half:2] = a * sn + b * c
+    else:
+        a = x[..., :half].copy()
+        b = x[..., half:2 * half].copy()
+        x[..., :half] = a * c - b * sn
+        x[..., half:2 * half] = a * sn + b * c
+    return x
+
+
 def kvcache_decode(q, k_new, v_new, k_cache_logical, v_cache_logical, cache_seqlens,
                    scale: float, causal: bool = True, window=(-1, -1), softcap: float = 0.0,
-                   heads=None):
-    """One decode step against a *logical, contiguous* per-sequence cache.
+                   heads=None, rotary_cos=None, rotary_sin=None, rotary_interleaved=False,
+                   rotated_dtype=None):
+    """One step against a *logical, contiguous* per-sequence cache.
 
-    q (B, 1, Hq, D); k_new, v_new (B, 1, Hkv, D); k/v_cache_logical: sequence
-    of B arrays, each holding at least cache_seqlens[b] rows of shape
-    (rows, Hkv, D). Following the notes' KVCache.update, the new k, v are
-    written at position L_b = cache_seqlens[b] and the prefix of length L_b+1
-    is returned; attention then runs for the single query at logical position
-    L_b over those L_b+1 keys (bottom-right alignment: causal lets it see all
-    of them). The paged layout and block_table are not used here at all.
+    q (B, Sq, Hq, D); k_new, v_new (B, Sq, Hkv, D) or None; k/v_cache_logical:
+    sequence of B arrays, each holding at least cache_seqlens[b] rows of shape
+    (rows, Hkv, D). Following the notes' KVCache.update, the Sq new keys and
+    values are written at positions L_b .. L_b + Sq - 1 (L_b =
+    cache_seqlens[b]) and the prefix of length Lk = L_b + Sq is used (without
+    an append, Lk = L_b). Query token t sits at position Lk - Sq + t and
+    attends over the Lk keys with bottom-right alignment (causal: keys up to
+    its own position). With rotary tables, q and the new keys are rotated at
+    those positions before the append (guide §增量解码场景); `rotated_dtype`
+    rounds the rotated values to the 16-bit type the cache and the matmul
+    operands hold. The paged layout and block_table are not used here.
 
     ``heads`` optionally restricts the query heads evaluated (others left 0).
-    Returns (O (B, 1, Hq, D), LSE (B, Hq, 1), appended_k list, appended_v list).
+    Returns (O (B, Sq, Hq, D), LSE (B, Hq, Sq), appended_k list, appended_v list).
     """
     q = _f64(q)
-    k_new = _f64(k_new)
-    v_new = _f64(v_new)
-    bsz, _, hq, d = q.shape
-    hkv = k_new.shape[2]
+    bsz, sq, hq, d = q.shape
+    append = k_new is not None
+    if append:
+        k_new = _f64(k_new)
+        v_new = _f64(v_new)
+        hkv = k_new.shape[2]
+    else:
+        hkv = _f64(k_cache_logical[0]).shape[1]
     g = hq // hkv
-    o = np.zeros((bsz, 1, hq, d))
-    lse = np.zeros((bsz, hq, 1))
+    o = np.zeros((bsz, sq, hq, d))
+    lse = np.zeros((bsz, hq, sq))
     ks, vs = [], []
     for b in range(bsz):
         n = int(cache_seqlens[b])
-        kb = np.concatenate([_f64(k_cache_logical[b])[:n], k_new[b]], axis=0)
-        vb = np.concatenate([_f64(v_cache_logical[b])[:n], v_new[b]], axis=0)
+        lk = n + (sq if append else 0)
+        pos = np.arange(lk - sq, lk)
+        qb = q[b]
+        kn = k_new[b] if append else None
+        if rotary_cos is not None:
+            qb = round_to(rotary(qb, pos, rotary_cos, rotary_sin, rotary_interleaved), rotated_dtype)
+            if append:
+                kn = round_to(rotary(kn, pos, rotary_cos, rotary_sin, rotary_interleaved),
+                              rotated_dtype)
+        kc = _f64(k_cache_logical[b])[:n]
+        vc = _f64(v_cache_logical[b])[:n]
+        kb = np.concatenate([kc, kn], axis=0) if append else kc
+        vb = np.concatenate([vc, v_new[b]], axis=0) if append else vc
         ks.append(kb)
         vs.append(vb)
         for h in (range(hq) if heads is None else heads):
-            ob, lb = head_fwd(q[b, :, h], kb[:, h // g], vb[:, h // g], scale, causal,
+            ob, lb = head_fwd(qb[:, h], kb[:, h // g], vb[:, h // g], scale, causal,
                               window[0], window[1], softcap)
-            o[b, 0, h] = ob[0]
-            lse[b, h, 0] = lb[0]
+            o[b, :, h] = ob
+            lse[b, h, :] = lb
     return o, lse, ks, vs
 
 

@@ -20,7 +20,7 @@ import torch
 
 import attn_workloads as W
 from oracle import (attention_bwd, attention_fwd, head_bwd, head_fwd, kvcache_decode,
-                    lse_combine, scores, visible_mask)
+                    lse_combine, rotary, round_to, scores, visible_mask)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
 
@@ -152,6 +152,10 @@ def test_golden_worked_examples(case):
         np.testing.assert_allclose(lse[0, :, 0], np.array(case["expect_lse_value"]), atol=1e-14)
         np.testing.assert_array_equal(ks[0], np.array(case["expect_k_after"]))
         np.testing.assert_array_equal(vs[0], np.array(case["expect_v_after"]))
+    elif kind == "rotary":
+        got = rotary(np.array(case["x"]), np.array(case["pos"]), np.array(case["cos"]),
+                     np.array(case["sin"]))
+        np.testing.assert_allclose(got, np.array(case["expect"]), atol=1e-15)
     elif kind == "combine":
         o, lse = lse_combine(np.array(case["o_parts"]), np.array(case["lse_parts"]))
         np.testing.assert_allclose(o, np.array(case["expect_o"]), atol=1e-14)
@@ -457,3 +461,100 @@ def test_oracle_is_independent_of_cuda_package():
             src = open(os.path.join(here, "oracle", fn), encoding="utf-8").read()
             assert "exact_attention_149_b200" not in src.replace(
                 "imports nothing from\nthe CUDA library", "")
+
+
+# ---------------------------------------------------------------------------
+# rotary embedding and multi-token decode
+# ---------------------------------------------------------------------------
+def rope_tables(positions, rdim, base=10000.0):
+    """Standard angle tables: theta(p, i) = p * base^(-2i / rdim)."""
+    inv = base ** (-np.arange(0, rdim, 2) / rdim)
+    ang = np.arange(positions)[:, None] * inv[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_rotary_preserves_pair_norms_and_tail(interleaved):
+    r = rng(97)
+    x = r.standard_normal((5, 3, 8))
+    cos, sin = rope_tables(40, 6)
+    pos = np.array([0, 3, 7, 20, 39])
+    y = rotary(x, pos, cos, sin, interleaved)
+    if interleaved:
+        px, py = (x[..., 0:6:2], x[..., 1:6:2]), (y[..., 0:6:2], y[..., 1:6:2])
+    else:
+        px, py = (x[..., :3], x[..., 3:6]), (y[..., :3], y[..., 3:6])
+    np.testing.assert_allclose(px[0] ** 2 + px[1] ** 2, py[0] ** 2 + py[1] ** 2, atol=1e-12)
+    np.testing.assert_array_equal(y[..., 6:], x[..., 6:])
+    np.testing.assert_array_equal(y[0], x[0])  # position 0: identity rotation
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_rotary_scores_depend_on_relative_position(interleaved):
+    """<R(m) q, R(n) k> depends on m - n only: the property that makes the
+    rotation a relative position encoding (fails for a sign or pairing slip
+    between the cos and sin terms)."""
+    r = rng(101)
+    q = r.standard_normal((1, 1, 16))
+    k = r.standard_normal((1, 1, 16))
+    cos, sin = rope_tables(100, 16)
+    s1 = np.sum(rotary(q, [10], cos, sin, interleaved) * rotary(k, [3], cos, sin, interleaved))
+    s2 = np.sum(rotary(q, [57], cos, sin, interleaved) * rotary(k, [50], cos, sin, interleaved))
+    s3 = np.sum(rotary(q, [10], cos, sin, interleaved) * rotary(k, [4], cos, sin, interleaved))
+    assert abs(s1 - s2) < 1e-10 and abs(s1 - s3) > 1e-3
+
+
+def test_rotary_interleaved_is_a_permutation_of_half_split():
+    r = rng(103)
+    x = r.standard_normal((4, 2, 8))
+    cos, sin = rope_tables(10, 8)
+    pos = np.array([1, 2, 5, 9])
+    perm = np.array([0, 2, 4, 6, 1, 3, 5, 7])  # interleaved slot -> half-split slot
+    half = rotary(x[..., perm], pos, cos, sin, interleaved=False)
+    inter = rotary(x, pos, cos, sin, interleaved=True)
+    np.testing.assert_allclose(half, inter[..., perm], atol=1e-14)
+
+
+def test_round_to_matches_torch_casts():
+    r = rng(107)
+    x = r.standard_normal(10000) * np.exp(r.uniform(-20, 20, 10000))
+    bf = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(round_to(x.astype(np.float32).astype(np.float64), "bf16"), bf)
+    hf = torch.tensor(x, dtype=torch.float32).to(torch.float16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(round_to(x.astype(np.float32).astype(np.float64), "fp16"), hf)
+
+
+@pytest.mark.parametrize("window,softcap,causal", [((-1, -1), 0.0, True), ((4, 0), 1.7, True),
+                                                   ((-1, -1), 0.0, False)])
+def test_multi_token_decode_equals_prefill_rows(window, softcap, causal):
+    """Sq new tokens appended after L cached ones: the outputs are the last Sq
+    rows of an ordinary (bottom-right aligned) attention over all L + Sq
+    tokens; with rotary, q and the new keys are rotated at their positions."""
+    r = rng(109)
+    B, Sq, hq, hkv, D = 2, 3, 4, 2, 8
+    lens = [5, 9]
+    kc = [r.standard_normal((n, hkv, D)) for n in lens]
+    vc = [r.standard_normal((n, hkv, D)) for n in lens]
+    q = r.standard_normal((B, Sq, hq, D))
+    kn = r.standard_normal((B, Sq, hkv, D))
+    vn = r.standard_normal((B, Sq, hkv, D))
+    cos, sin = rope_tables(32, 6)
+    for rot in (False, True):
+        kw = dict(rotary_cos=cos, rotary_sin=sin) if rot else {}
+        o, lse, ks, vs = kvcache_decode(q, kn, vn, kc, vc, lens, 0.37, causal, window, softcap, **kw)
+        for b in range(B):
+            n = lens[b] + Sq
+            pos = np.arange(lens[b], n)
+            kfull = np.concatenate([kc[b], rotary(kn[b], pos, cos, sin) if rot else kn[b]])
+            np.testing.assert_allclose(ks[b], kfull, atol=1e-14)
+            qb = rotary(q[b], pos, cos, sin) if rot else q[b]
+            for h in range(hq):
+                of, lf = head_fwd(qb[:, h], kfull[:, h // 2], vs[b][:, h // 2], 0.37, causal,
+                                  window[0], window[1], softcap)
+                # the same rows through a full-length prefill (bottom-right = top-left here)
+                qq = np.concatenate([r.standard_normal((lens[b], D)), qb[:, h]])
+                op, lp = head_fwd(qq, kfull[:, h // 2], vs[b][:, h // 2], 0.37, causal,
+                                  window[0], window[1], softcap)
+                np.testing.assert_allclose(o[b, :, h], of, atol=1e-13)
+                np.testing.assert_allclose(o[b, :, h], op[-Sq:], atol=1e-13)
+                np.testing.assert_allclose(lse[b, h], lp[-Sq:], atol=1e-13)
