@@ -23,6 +23,7 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass, field
 
+import numpy as np
 import torch
 
 __all__ = [
@@ -36,6 +37,7 @@ __all__ = [
     "make_decode_structure",
     "decode_sequence_cache",
     "fill_paged_pool",
+    "rotary_tables",
     "visible_pairs",
     "fwd_flops",
     "bwd_flops",
@@ -177,27 +179,27 @@ def make_varlen_inputs(lengths=None, Hq=32, Hkv=8, D=128, dtype="bf16", seed=0, 
 
 
 def make_decode_structure(B, Hq, Hkv, D, len_lo, len_hi, page_size, dtype="bf16", seed=0,
-                          cache_seqlens=None, pages_per_seq=None):
-    """Structure and per-step inputs of one decode step.
+                          cache_seqlens=None, pages_per_seq=None, sq=1):
+    """Structure and per-step inputs of one decode step with sq new tokens.
 
     Returns dict with cache_seqlens (int32, B), block_table (int32,
     B x pages_per_seq: a random permutation of all physical pages), q
-    (B,1,Hq,D), k_new, v_new (B,1,Hkv,D), num_pages, page_size, seed.
-    ``pages_per_seq`` defaults to ceil((len_hi + 1) / page_size) so the
-    appended token always has a page.
+    (B,sq,Hq,D), k_new, v_new (B,sq,Hkv,D), num_pages, page_size, seed.
+    ``pages_per_seq`` defaults to ceil((len_hi + sq) / page_size) so the
+    appended tokens always have a page.
     """
     g = _gen(seed)
     if cache_seqlens is None:
         cache_seqlens = torch.randint(len_lo, len_hi + 1, (B,), generator=g, dtype=torch.int64)
     cache_seqlens = torch.as_tensor(cache_seqlens, dtype=torch.int64)
     if pages_per_seq is None:
-        pages_per_seq = -(-(int(len_hi) + 1) // page_size)
+        pages_per_seq = -(-(int(len_hi) + sq) // page_size)
     num_pages = B * pages_per_seq
     perm = torch.randperm(num_pages, generator=g)
     block_table = perm.view(B, pages_per_seq).to(torch.int32)
-    q = _randn(g, (B, 1, Hq, D), dtype)
-    k_new = _randn(g, (B, 1, Hkv, D), dtype)
-    v_new = _randn(g, (B, 1, Hkv, D), dtype)
+    q = _randn(g, (B, sq, Hq, D), dtype)
+    k_new = _randn(g, (B, sq, Hkv, D), dtype)
+    v_new = _randn(g, (B, sq, Hkv, D), dtype)
     return {
         "cache_seqlens": cache_seqlens.to(torch.int32),
         "block_table": block_table,
@@ -242,6 +244,16 @@ def fill_paged_pool(st, k_pool, v_pool, batches=None):
             m = min(ps, n - p)
             k_pool[page, :m].copy_(kd[p:p + m])
             v_pool[page, :m].copy_(vd[p:p + m])
+
+
+def rotary_tables(rows, rotary_dim, base=10000.0):
+    """Angle tables a caller passes for the rotary encoding: float32 cos and
+    sin of shape (rows, rotary_dim / 2) with angle(p, i) = p * base^(-2i /
+    rotary_dim), the common frequency ladder (evaluated in float64)."""
+    inv = base ** (-np.arange(0, rotary_dim, 2, dtype=np.float64) / rotary_dim)
+    ang = np.arange(rows, dtype=np.float64)[:, None] * inv[None, :]
+    return (torch.from_numpy(np.cos(ang).astype(np.float32)),
+            torch.from_numpy(np.sin(ang).astype(np.float32)))
 
 
 # ---------------------------------------------------------------------------

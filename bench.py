@@ -417,7 +417,7 @@ def run_ours(args, dist: Dist):
     dout = torch.empty_like(dq_)
     dlse = torch.empty((cd.B, cd.Hq, 1), dtype=torch.float32, device=dev)
     for splits in cd.splits:
-        wsd = fa.fa_kvcache_workspace_size(cd.B, cd.Hq, cd.D, splits)
+        wsd = fa.fa_kvcache_workspace_size(cd.B, 1, cd.Hq, cd.D, splits)
         wsb = torch.empty(max(wsd, 1), dtype=torch.uint8, device=dev)
 
         def step_dec(splits=splits, wsb=wsb):

@@ -60,15 +60,18 @@ lib.fa_bwd.restype = _i
 lib.fa_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f,
                        _p, _i, _i, _p, _z, _p]
 lib.fa_fwd_kvcache.restype = _i
-lib.fa_fwd_kvcache.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f,
-                               _i, _i, _i, _f, _i, _i, _p, _z, _p]
+# q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos, rotary_sin, out, lse;
+# B, Sq, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+# rotary_interleaved; scale, causal, window_left, window_right, softcap, num_splits, dtype
+_KV_ARGS = [_p] * 11 + [_i] * 11 + [_f, _i, _i, _i, _f, _i, _i]
+lib.fa_fwd_kvcache.restype = _i
+lib.fa_fwd_kvcache.argtypes = _KV_ARGS + [_p, _z, _p]
 lib.fa_fwd_kvcache_noalloc.restype = _i
-lib.fa_fwd_kvcache_noalloc.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
-                                       _i, _f, _i, _i, _i, _f, _i, _i, _p]
+lib.fa_fwd_kvcache_noalloc.argtypes = _KV_ARGS + [_p]
 lib.fa_bwd_workspace_size.restype = _z
 lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 lib.fa_kvcache_workspace_size.restype = _z
-lib.fa_kvcache_workspace_size.argtypes = [_i, _i, _i, _i]
+lib.fa_kvcache_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.fa_get_device_status.restype = _i
 lib.fa_get_device_status.argtypes = [ctypes.POINTER(_i)]
 lib.fa_kernel_timing_enable.restype = _i
@@ -150,37 +153,43 @@ def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
                       _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
-def fa_kvcache_workspace_size(B, Hq, D, num_splits) -> int:
-    return int(lib.fa_kvcache_workspace_size(B, Hq, D, num_splits))
+def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rotary_dim=0) -> int:
+    return int(lib.fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rotary_dim))
 
 
-def fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, out, lse, B,
-                   Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
+def fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos,
+                   rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, max_pages_per_seq,
+                   num_pages, rotary_rows, rotary_dim, rotary_interleaved, scale, causal,
                    window_left, window_right, softcap, num_splits, dtype, workspace,
                    workspace_bytes, stream=None):
     _check(lib.fa_fwd_kvcache(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
-                              _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse), B, Hq,
-                              Hkv, D, page_size, max_pages_per_seq, num_pages, scale, int(causal),
-                              window_left, window_right, softcap, num_splits, dtype,
-                              _ptr(workspace), workspace_bytes, _stream(stream)))
+                              _ptr(block_table), _ptr(cache_seqlens), _ptr(rotary_cos),
+                              _ptr(rotary_sin), _ptr(out), _ptr(lse), B, Sq, Hq, Hkv, D, page_size,
+                              max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+                              int(rotary_interleaved), scale, int(causal), window_left,
+                              window_right, softcap, num_splits, dtype, _ptr(workspace),
+                              workspace_bytes, _stream(stream)))
 
 
 # size of the library's static scratch array used by fa_fwd_kvcache_noalloc
 FA_NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
 
 
-def fa_fwd_kvcache_noalloc(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, out, lse,
-                           B, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
-                           window_left, window_right, softcap, num_splits, dtype, stream=None):
+def fa_fwd_kvcache_noalloc(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens,
+                           rotary_cos, rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size,
+                           max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+                           rotary_interleaved, scale, causal, window_left, window_right, softcap,
+                           num_splits, dtype, stream=None):
     """fa_fwd_kvcache for callers that cannot allocate device memory: no
-    workspace argument; the split partials live in the library's own static
-    device array (see include/fa.h)."""
+    workspace argument; the split partials and rotated queries live in the
+    library's own static device array (see include/fa.h)."""
     _check(lib.fa_fwd_kvcache_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
                                       _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens),
-                                      _ptr(out), _ptr(lse), B, Hq, Hkv, D, page_size,
-                                      max_pages_per_seq, num_pages, scale, int(causal),
-                                      window_left, window_right, softcap, num_splits, dtype,
-                                      _stream(stream)))
+                                      _ptr(rotary_cos), _ptr(rotary_sin), _ptr(out), _ptr(lse), B,
+                                      Sq, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages,
+                                      rotary_rows, rotary_dim, int(rotary_interleaved), scale,
+                                      int(causal), window_left, window_right, softcap, num_splits,
+                                      dtype, _stream(stream)))
 
 
 def fa_kernel_timing_enable(enable: bool = True):
@@ -266,21 +275,32 @@ def bwd(q, k, v, out, lse, dout, scale=None, causal=False, window=(-1, -1), soft
 
 
 def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_new=None,
-                scale=None, causal=True, window=(-1, -1), softcap=0.0, num_splits=1, out=None,
-                lse=None, workspace=None, stream=None):
-    """One decode step: q (B,1,Hq,D); caches (num_pages, page_size, Hkv, D);
+                rotary_cos=None, rotary_sin=None, rotary_interleaved=False, scale=None,
+                causal=True, window=(-1, -1), softcap=0.0, num_splits=1, out=None, lse=None,
+                workspace=None, stream=None):
+    """One decode step: q (B,Sq,Hq,D); caches (num_pages, page_size, Hkv, D);
     block_table int32 (B, max_pages); cache_seqlens int32 (B). Appends
-    k_new/v_new (B,1,Hkv,D) in place, then attends. Returns (out, lse)."""
-    _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new)
-    B, _, Hq, D = q.shape
+    k_new/v_new (B,Sq,Hkv,D) in place, then attends. rotary_cos/rotary_sin:
+    float32 (rows, rotary_dim/2) tables that rotate q and k_new at their
+    positions. Returns (out (B,Sq,Hq,D), lse (B,Hq,Sq))."""
+    _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new, rotary_cos,
+               rotary_sin)
+    B, Sq, Hq, D = q.shape
     num_pages, page_size, Hkv, _ = k_cache.shape
+    if (rotary_cos is None) != (rotary_sin is None):
+        raise FaError(FA_ERR_INVALID_ARG, "rotary_cos and rotary_sin go together")
+    if rotary_cos is not None and (rotary_cos.dtype != torch.float32 or rotary_sin.dtype != torch.float32
+                                   or rotary_cos.shape != rotary_sin.shape or rotary_cos.dim() != 2):
+        raise FaError(FA_ERR_INVALID_ARG, "rotary tables must be float32 (rows, rotary_dim/2), same shape")
+    rot_rows, rot_dim = (0, 0) if rotary_cos is None else (rotary_cos.shape[0], 2 * rotary_cos.shape[1])
     out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device) if lse is None else lse
-    nbytes = fa_kvcache_workspace_size(B, Hq, D, num_splits)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    nbytes = fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rot_dim)
     if workspace is None and nbytes > 0:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, out, lse, B, Hq,
-                   Hkv, D, page_size, block_table.shape[1], num_pages, _scale(scale, D), causal,
+    fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos,
+                   rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, block_table.shape[1],
+                   num_pages, rot_rows, rot_dim, rotary_interleaved, _scale(scale, D), causal,
                    window[0], window[1], softcap, num_splits, _dt(q), workspace,
                    0 if workspace is None else workspace.numel(), stream)
     return out, lse

@@ -1,21 +1,27 @@
 // Paged split-KV decode for sm_100a ("FlashAttention 实战指南" §增量解码场景
 // flash_attn_with_kvcache: append the new K/V to the cache in place, attend
 // in place; cache_seqlens gives each sample's length, block_table pages the
-// cache, num_splits splits the KV range).
+// cache, num_splits splits the KV range; rotary_cos / rotary_sin rotate q and
+// the new keys inside the call).
 //
-//   kv_append_kernel     k_new/v_new -> their page slot (position cache_seqlens[b])
-//   decode_split_kernel  one CTA per (sequence, kv head, split): a TMA producer
-//                        warp streams 64-token K/V chunks of the split's range
-//                        through block_table into a shared-memory ring; four
-//                        consumer warps each own 16 tokens of a chunk and keep
-//                        an online softmax for all query heads of the GQA
-//                        group, so every K/V byte is read from HBM once.
+//   kv_append_kernel     the Sq new K/V rows -> their page slots (positions
+//                        cache_seqlens[b] ..), keys rotated when rotary tables
+//                        are given; with rotary, also the rotated queries into
+//                        the workspace
+//   decode_split_kernel  one CTA per (sequence, kv head, split, column block):
+//                        a TMA producer warp streams 64-token K/V chunks of
+//                        the split's range through block_table into a shared-
+//                        memory ring; four consumer warps each own 16 tokens of
+//                        a chunk and keep an online softmax for up to 32 query
+//                        columns, a column being one (new token, query head of
+//                        the GQA group) pair, so every K/V byte is read from
+//                        HBM once per column block.
 //   lse_combine_kernel   merges the splits' (O_s, LSE_s) partials.
 //
 // Decode is bound by HBM bandwidth (about 4 flops per K/V byte), so the dot
 // products run on mma.sync (m16n8k16) straight from the swizzled TMA tiles:
-//   S^T[16 tokens x 8 heads] = K[16 x 16 d] . Q^T[16 d x 8 heads]
-//   O^T[16 d x 8 heads]     += V^T[16 d x 16 tokens] . P^T[16 tokens x 8 heads]
+//   S^T[16 tokens x 8 columns] = K[16 x 16 d] . Q^T[16 d x 8 columns]
+//   O^T[16 d x 8 columns]     += V^T[16 d x 16 tokens] . P^T[16 tokens x 8 columns]
 // P^T's fragment is the transpose of S^T's accumulator fragment, done with
 // movmatrix.
 #pragma once
@@ -27,50 +33,142 @@ namespace fa {
 enum : int { kDevBadIndex = 2 };
 
 struct DecodeParams {
-  const void* q;          // (B, 1, Hq, D)
-  const void* k_new;      // (B, 1, Hkv, D) or null
+  const void* q;          // (B, Sq, Hq, D): the caller's q, or the rotated copy
+  const void* q_in;       // the caller's q (read by kv_append_kernel)
+  void* q_rot;            // (B, Sq, Hq, D) rotated queries (workspace), or null
+  const void* k_new;      // (B, Sq, Hkv, D) or null
   const void* v_new;
   void* k_cache;          // (num_pages, page_size, Hkv, D)
   void* v_cache;
   const int* block_table; // (B, max_pages)
   const int* cache_seqlens;
-  void* out;              // (B, 1, Hq, D)
-  float* lse;             // (B, Hq, 1)
-  float* part_o;          // (splits, B, Hq, D) fp32, used when splits > 1
-  float* part_lse;        // (splits, B, Hq)
-  int B, Hq, Hkv, D, group;
+  const float* rot_cos;   // (rot_rows, rot_dim / 2) fp32, or null
+  const float* rot_sin;
+  void* out;              // (B, Sq, Hq, D)
+  float* lse;             // (B, Hq, Sq)
+  float* part_o;          // (splits, B, Sq, Hq, D) fp32, used when splits > 1
+  float* part_lse;        // (splits, B, Sq, Hq)
+  int B, Sq, Hq, Hkv, D, group;
+  int n_cols;             // Sq * group query columns per (sequence, kv head)
+  int col_blocks;         // column blocks of 8 * kNT columns
   int page_size, max_pages, num_pages;
   int splits;
   int append;             // 1 when k_new/v_new are given
+  int rot_rows, rot_dim, rot_inter;
   float scale_log2, softcap, cap_in, cap_out_log2;
-  int wl;                 // window left (-1 = unbounded); the query is the last position
+  int wl;                 // window left (-1 = unbounded)
+  int right;              // visible keys end at position + right (-1 = unbounded; causal = 0)
 };
 
+// Keys visible to the query at position `qpos` of a sequence of Lk keys:
+// [key_lo, key_hi). Bottom-right alignment: the last query sits at Lk - 1.
+__device__ __forceinline__ int key_lo(const DecodeParams& p, int qpos) {
+  return p.wl >= 0 ? max(0, qpos - p.wl) : 0;
+}
+__device__ __forceinline__ int key_hi(const DecodeParams& p, int qpos, int Lk) {
+  return p.right >= 0 ? min(Lk, qpos + p.right + 1) : Lk;
+}
+
 // ---------------------------------------------------------------------------
-// append
+// append (+ rotary)
 // ---------------------------------------------------------------------------
-// grid B, block Hkv * D / 8 threads (16 bytes each, for both K and V)
+template <bool kBF16>
+__device__ __forceinline__ void unpack8(const uint4& r, float (&x)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = unpack2<kBF16>(w[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+template <bool kBF16>
+__device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
+  return make_uint4(pack2<kBF16>(x[0], x[1]), pack2<kBF16>(x[2], x[3]), pack2<kBF16>(x[4], x[5]),
+                    pack2<kBF16>(x[6], x[7]));
+}
+
+// Elements d0 .. d0+7 of one head row after the rotary rotation at the angle
+// row (cs, sn) (null: no rotation). A pair (a, b) becomes
+// (a cos - b sin, a sin + b cos); pairs are (i, i + rd/2), or (2i, 2i + 1)
+// when interleaved; dimensions from rd on pass through. rd is a multiple of
+// 16, so a group of 8 never straddles rd or rd/2.
+template <bool kBF16>
+__device__ __forceinline__ uint4 rotate8(const uint16_t* row, int d0, const float* cs,
+                                         const float* sn, const DecodeParams& p) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(row + d0);
+  if (cs == nullptr || d0 >= p.rot_dim) return raw;
+  float x[8], y[8];
+  unpack8<kBF16>(raw, x);
+  if (p.rot_inter) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float c = cs[(d0 >> 1) + j], s = sn[(d0 >> 1) + j];
+      y[2 * j] = x[2 * j] * c - x[2 * j + 1] * s;
+      y[2 * j + 1] = x[2 * j] * s + x[2 * j + 1] * c;
+    }
+  } else {
+    const int half = p.rot_dim >> 1;
+    const bool first = d0 < half;
+    const int i0 = first ? d0 : d0 - half;
+    float xp[8];
+    unpack8<kBF16>(*reinterpret_cast<const uint4*>(row + (first ? d0 + half : d0 - half)), xp);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float c = cs[i0 + j], s = sn[i0 + j];
+      y[j] = first ? x[j] * c - xp[j] * s : xp[j] * s + x[j] * c;
+    }
+  }
+  return pack8<kBF16>(y);
+}
+
+// grid B * Sq (one block per new token), block 128: 16 bytes per thread-step
+template <bool kBF16>
 __global__ void kv_append_kernel(const DecodeParams p) {
-  const int b = blockIdx.x;
+  const int b = blockIdx.x / p.Sq, t = blockIdx.x % p.Sq;
   const int L = p.cache_seqlens[b];
-  const int pi = L / p.page_size;
-  if (L < 0 || pi >= p.max_pages) {
+  const int Lk = L + (p.append ? p.Sq : 0);
+  const int pos = Lk - p.Sq + t;  // position of query t and of new key t
+  const float* cs = nullptr;
+  const float* sn = nullptr;
+  if (p.rot_dim > 0) {
+    if (L < 0 || pos < 0 || pos >= p.rot_rows) {
+      if (threadIdx.x == 0) atomicExch(&g_device_status, kDevBadIndex);
+    } else {
+      cs = p.rot_cos + static_cast<size_t>(pos) * (p.rot_dim >> 1);
+      sn = p.rot_sin + static_cast<size_t>(pos) * (p.rot_dim >> 1);
+    }
+    const int groups = p.D >> 3;
+    const size_t base = (static_cast<size_t>(b) * p.Sq + t) * p.Hq * p.D;
+    const uint16_t* src = static_cast<const uint16_t*>(p.q_in) + base;
+    uint16_t* dst = static_cast<uint16_t*>(p.q_rot) + base;
+    for (int i = threadIdx.x; i < p.Hq * groups; i += blockDim.x) {
+      const int h = i / groups, d0 = (i % groups) * 8;
+      *reinterpret_cast<uint4*>(dst + h * p.D + d0) = rotate8<kBF16>(src + h * p.D, d0, cs, sn, p);
+    }
+  }
+  if (!p.append) return;
+  if (L < 0 || Lk > p.max_pages * p.page_size) {
     if (threadIdx.x == 0) atomicExch(&g_device_status, kDevBadIndex);
     return;
   }
-  const int page = p.block_table[static_cast<size_t>(b) * p.max_pages + pi];
+  const int page = p.block_table[static_cast<size_t>(b) * p.max_pages + pos / p.page_size];
   if (page < 0 || page >= p.num_pages) {
     if (threadIdx.x == 0) atomicExch(&g_device_status, kDevBadIndex);
     return;
   }
-  const int row_elems = p.Hkv * p.D;
-  const size_t dst = (static_cast<size_t>(page) * p.page_size + (L % p.page_size)) * row_elems;
-  const size_t src = static_cast<size_t>(b) * row_elems;
-  for (int i = threadIdx.x * 8; i < row_elems; i += blockDim.x * 8) {
-    const uint4 kv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.k_new) + src + i);
-    const uint4 vv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.v_new) + src + i);
-    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.k_cache) + dst + i) = kv;
-    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.v_cache) + dst + i) = vv;
+  const int groups = p.D >> 3;
+  const size_t dst = (static_cast<size_t>(page) * p.page_size + (pos % p.page_size)) * p.Hkv * p.D;
+  const size_t src = (static_cast<size_t>(b) * p.Sq + t) * p.Hkv * p.D;
+  const uint16_t* kn = static_cast<const uint16_t*>(p.k_new) + src;
+  const uint16_t* vn = static_cast<const uint16_t*>(p.v_new) + src;
+  uint16_t* kc = static_cast<uint16_t*>(p.k_cache) + dst;
+  uint16_t* vc = static_cast<uint16_t*>(p.v_cache) + dst;
+  for (int i = threadIdx.x; i < p.Hkv * groups; i += blockDim.x) {
+    const int h = i / groups, d0 = (i % groups) * 8;
+    const int e = h * p.D + d0;
+    *reinterpret_cast<uint4*>(kc + e) = rotate8<kBF16>(kn + h * p.D, d0, cs, sn, p);
+    *reinterpret_cast<uint4*>(vc + e) = *reinterpret_cast<const uint4*>(vn + e);
   }
 }
 
@@ -145,7 +243,8 @@ __device__ __forceinline__ float dec_logit(float s, const DecodeParams& p) {
   return s * p.scale_log2;
 }
 
-// kNT: number of 8-wide head tiles (group size <= 8 * kNT)
+// kNT: number of 8-wide column tiles per CTA (a column block holds 8 * kNT
+// columns; column n is new token n / group, query head kvh * group + n % group)
 template <int kD, bool kBF16, int kNT>
 __global__ void __launch_bounds__(160)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -159,23 +258,34 @@ __global__ void __launch_bounds__(160)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // work item: split fastest, then kv head, then sequence
-  const int split = blockIdx.x % p.splits;
-  const int kvh = (blockIdx.x / p.splits) % p.Hkv;
-  const int b = blockIdx.x / (p.splits * p.Hkv);
+  constexpr int kH = 8 * kNT;
+  // work item: column block fastest (the blocks of one split read the same
+  // K/V, so they run together and share it through L2), then split, kv head,
+  // sequence
+  const int cb = blockIdx.x % p.col_blocks;
+  const int split = (blockIdx.x / p.col_blocks) % p.splits;
+  const int kvh = (blockIdx.x / (p.col_blocks * p.splits)) % p.Hkv;
+  const int b = blockIdx.x / (p.col_blocks * p.splits * p.Hkv);
+  const int n0 = cb * kH;                        // first column of the block
+  const int n_here = min(kH, p.n_cols - n0);     // real columns in the block
 
   const int L = p.cache_seqlens[b];
-  const int Lk = L + p.append;  // keys visible to the query (bottom-right causal)
-  int lo = 0;
-  if (p.wl >= 0) lo = max(0, Lk - 1 - p.wl);
-  const int hi = Lk;            // exclusive
+  const int Lk = L + (p.append ? p.Sq : 0);      // keys after the append
+  const int qbase = Lk - p.Sq;                   // position of new token 0
+  // union [lo, hi) and intersection [lo_in, hi_in) of the block's columns'
+  // key ranges: both bounds grow with the token index
+  const int t_first_col = n0 / p.group, t_last_col = (n0 + n_here - 1) / p.group;
+  const int lo = key_lo(p, qbase + t_first_col);
+  const int hi = key_hi(p, qbase + t_last_col, Lk);  // exclusive
+  const int lo_in = key_lo(p, qbase + t_last_col);
+  const int hi_in = key_hi(p, qbase + t_first_col, Lk);
   const int t_first = lo / Sh::kTok;
   const int t_all = hi > lo ? (hi - 1) / Sh::kTok + 1 - t_first : 0;
   const int per = (t_all + p.splits - 1) / p.splits;
   const int t_begin = t_first + split * per;
   const int t_end = min(t_first + t_all, t_begin + per);
   const int n_t = max(0, t_end - t_begin);
-  const bool bad_len = (L < 0) || (hi > p.max_pages * p.page_size);
+  const bool bad_len = (L < 0) || (Lk > p.max_pages * p.page_size);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < Sh::kStages; ++i) {
@@ -239,15 +349,16 @@ __global__ void __launch_bounds__(160)
   }
 
   // ======================= consumers (warps 0..3) =======================
-  // Q^T fragments: B[k = d][n = head], n = lane / 4 within each 8-head tile
+  // Q^T fragments: B[k = d][n = column], n = lane / 4 within each 8-column tile
   uint32_t qf[kNT][kD / 16][2];
   {
-    const uint16_t* qp = static_cast<const uint16_t*>(p.q) + (static_cast<size_t>(b) * p.Hq) * kD;
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
-      const int hl = nt * 8 + (lane >> 2);  // head within the group
-      const bool real = hl < p.group;
-      const uint16_t* row = qp + static_cast<size_t>(kvh * p.group + (real ? hl : 0)) * kD;
+      const int n = n0 + nt * 8 + (lane >> 2);
+      const bool real = n < p.n_cols;
+      const int t = real ? n / p.group : 0, hl = real ? n % p.group : 0;
+      const uint16_t* row = static_cast<const uint16_t*>(p.q) +
+                            ((static_cast<size_t>(b) * p.Sq + t) * p.Hq + kvh * p.group + hl) * kD;
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk) {
         const int d = kk * 16 + 2 * (lane & 3);
@@ -256,7 +367,7 @@ __global__ void __launch_bounds__(160)
       }
     }
   }
-  // running state per (head tile, column pair): heads nt*8 + 2*(lane&3) + {0,1}
+  // running state per (column tile, column pair): columns nt*8 + 2*(lane&3) + {0,1}
   float m_run[kNT][2], l_part[kNT][2];
   float acc[kNT][kD / 16][4];
 #pragma unroll
@@ -306,17 +417,29 @@ __global__ void __launch_bounds__(160)
       for (int nt = 0; nt < kNT; ++nt) mma16816<kBF16>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
     }
     // ---- logits, mask, online softmax ----
-    const int pos0 = (t_begin + i) * Sh::kTok + tok0 + (lane >> 2);  // token of s[.][0], s[.][1]
-    const bool v0 = pos0 >= lo && pos0 < hi;
-    const bool v1 = pos0 + 8 >= lo && pos0 + 8 < hi;
+    const int wtok = (t_begin + i) * Sh::kTok + tok0;  // first token of this warp's 16
+    const int pos0 = wtok + (lane >> 2);                // token of s[.][0], s[.][1]
+    // every column sees all 16 tokens: no mask (warp-uniform)
+    const bool all_visible = wtok >= lo_in && wtok + 16 <= hi_in;
     uint32_t pb[kNT][2];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
-      float x0 = v0 ? dec_logit(s[nt][0], p) : -INFINITY;
-      float x1 = v0 ? dec_logit(s[nt][1], p) : -INFINITY;
-      float x2 = v1 ? dec_logit(s[nt][2], p) : -INFINITY;
-      float x3 = v1 ? dec_logit(s[nt][3], p) : -INFINITY;
-      // column (head) maxima over the warp's 16 tokens: reduce over lane >> 2
+      float x0 = dec_logit(s[nt][0], p);
+      float x1 = dec_logit(s[nt][1], p);
+      float x2 = dec_logit(s[nt][2], p);
+      float x3 = dec_logit(s[nt][3], p);
+      if (!all_visible) {
+        // per-column key ranges (padding columns take the last real one's)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int n = min(n0 + nt * 8 + 2 * (lane & 3) + j, p.n_cols - 1);
+          const int qpos = qbase + n / p.group;
+          const int clo = key_lo(p, qpos), chi = key_hi(p, qpos, Lk);
+          if (pos0 < clo || pos0 >= chi) (j ? x1 : x0) = -INFINITY;
+          if (pos0 + 8 < clo || pos0 + 8 >= chi) (j ? x3 : x2) = -INFINITY;
+        }
+      }
+      // column maxima over the warp's 16 tokens: reduce over lane >> 2
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -360,8 +483,7 @@ __global__ void __launch_bounds__(160)
   }
 
   // ---- merge the four warps' states, then write the split's result ----
-  // per warp and head: m (log2 domain), l; per head and d: unnormalised O
-  constexpr int kH = 8 * kNT;
+  // per warp and column: m (log2 domain), l; per column and d: unnormalised O
   named_bar_sync(1, 128);  // every consumer is done reading the stage ring
   float* red_m = red;                        // [4][kH]
   float* red_l = red + 4 * kH;               // [4][kH]
@@ -391,33 +513,36 @@ __global__ void __launch_bounds__(160)
     }
   }
   named_bar_sync(1, 128);
-  // 128 threads: each (head, d-slice) combination
-  for (int idx = threadIdx.x; idx < p.group * kD; idx += 128) {
-    const int hl = idx / kD, d = idx % kD;
+  // 128 threads: each (column, d) combination
+  for (int idx = threadIdx.x; idx < n_here * kD; idx += 128) {
+    const int c = idx / kD, d = idx % kD;
     float m = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) m = fmaxf(m, red_m[w * kH + hl]);
+    for (int w = 0; w < 4; ++w) m = fmaxf(m, red_m[w * kH + c]);
     float l = 0.f, o = 0.f;
     if (m != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const float sc = ex2_approx(red_m[w * kH + hl] - m);
-        l += red_l[w * kH + hl] * sc;
-        o += red_o[(w * kH + hl) * kD + d] * sc;
+        const float sc = ex2_approx(red_m[w * kH + c] - m);
+        l += red_l[w * kH + c] * sc;
+        o += red_o[(w * kH + c) * kD + d] * sc;
       }
     }
     const float on = l > 0.f ? o / l : 0.f;
     const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-    const int hq = kvh * p.group + hl;
+    const int n = n0 + c;
+    const int t = n / p.group;
+    const int hq = kvh * p.group + n % p.group;
+    const size_t row = (static_cast<size_t>(b) * p.Sq + t) * p.Hq + hq;  // row of out
     if (p.splits == 1) {
-      const size_t oi = (static_cast<size_t>(b) * p.Hq + hq) * kD + d;
+      const size_t oi = row * kD + d;
       if constexpr (kBF16)
         static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(on);
       else
         static_cast<__half*>(p.out)[oi] = __float2half_rn(on);
-      if (d == 0) p.lse[static_cast<size_t>(b) * p.Hq + hq] = lse;
+      if (d == 0) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Sq + t] = lse;
     } else {
-      const size_t pi = (static_cast<size_t>(split) * p.B + b) * p.Hq + hq;
+      const size_t pi = static_cast<size_t>(split) * p.B * p.Sq * p.Hq + row;
       p.part_o[pi * kD + d] = on;
       if (d == 0) p.part_lse[pi] = lse;
     }
@@ -425,13 +550,13 @@ __global__ void __launch_bounds__(160)
   __syncthreads();
 }
 
-// one warp per (b, hq): merge the splits' partials
+// one warp per output row (b, t, hq): merge the splits' partials
 template <int kD, bool kBF16>
 __global__ void lse_combine_kernel(const DecodeParams p) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (gw >= p.B * p.Hq) return;
-  const size_t stride = static_cast<size_t>(p.B) * p.Hq;
+  const size_t stride = static_cast<size_t>(p.B) * p.Sq * p.Hq;
+  if (gw >= stride) return;
   float m = -INFINITY;
   for (int s = 0; s < p.splits; ++s) m = fmaxf(m, p.part_lse[s * stride + gw]);
   float wsum = 0.f;
@@ -457,7 +582,10 @@ __global__ void lse_combine_kernel(const DecodeParams p) {
     else
       static_cast<__half*>(p.out)[oi] = __float2half_rn(o[j] * inv);
   }
-  if (lane == 0) p.lse[gw] = wsum > 0.f ? m + __logf(wsum) : -INFINITY;
+  if (lane == 0) {
+    const int hq = gw % p.Hq, t = (gw / p.Hq) % p.Sq, b = gw / (p.Hq * p.Sq);
+    p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Sq + t] = wsum > 0.f ? m + __logf(wsum) : -INFINITY;
+  }
 }
 
 }  // namespace fa

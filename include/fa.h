@@ -109,18 +109,24 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype, void* workspace,
                  size_t workspace_bytes, void* stream);
 
-/* Workspace bytes needed by fa_fwd_kvcache (float32 per-split partial
- * outputs and log-sum-exps); 0 when num_splits == 1. */
-FA_API size_t fa_kvcache_workspace_size(int B, int Hq, int D, int num_splits);
+/* Workspace bytes needed by fa_fwd_kvcache: the float32 per-split partial
+ * results (num_splits > 1; 0 bytes for them otherwise) and, with rotary
+ * tables (rotary_dim > 0), the rotated queries in the input dtype. */
+FA_API size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits,
+                                        int rotary_dim);
 
 /*
  * One decode step against a paged KV cache (guide §增量解码场景
- * flash_attn_with_kvcache): the new key/value of each sequence is appended
- * IN PLACE at logical position cache_seqlens[b], then the single query
- * attends over the cache_seqlens[b] + 1 keys; the KV range is split into
- * num_splits parts whose partial results are merged by a log-sum-exp combine.
- *   q (B, 1, Hq, D); k_new, v_new (B, 1, Hkv, D), or both NULL for no append
- *     (the query then attends over cache_seqlens[b] keys).
+ * flash_attn_with_kvcache): the Sq new keys/values of each sequence are
+ * appended IN PLACE at logical positions L .. L + Sq - 1 (L =
+ * cache_seqlens[b]), then the Sq new queries attend over the Lk = L + Sq
+ * keys with bottom-right alignment: query t sits at position Lk - Sq + t and,
+ * when causal, sees the keys up to its own position; the window bounds are
+ * taken from that position (the convention of fa_fwd). The KV range is split
+ * into num_splits parts whose partial results are merged by a log-sum-exp
+ * combine.
+ *   q (B, Sq, Hq, D); k_new, v_new (B, Sq, Hkv, D), or both NULL for no append
+ *     (then Lk = L and the queries sit at L - Sq .. L - 1).
  *   k_cache, v_cache (num_pages, page_size, Hkv, D): the page pool; logical
  *     position p of sequence b lives in page block_table[b, p / page_size],
  *     slot p % page_size ("FlashAttention技术深度解析" §动态缓存架构: a page
@@ -129,22 +135,39 @@ FA_API size_t fa_kvcache_workspace_size(int B, int Hq, int D, int num_splits);
  *     in [0, num_pages).
  *   cache_seqlens: DEVICE int32 (B), valid length BEFORE the append; the
  *     library does not increment it (the caller advances its own position).
- *   out (B, 1, Hq, D); lse float32 (B, Hq, 1).
+ *   rotary_cos, rotary_sin: DEVICE float32 (rotary_rows, rotary_dim / 2)
+ *     angle tables, or NULL with rotary_dim = 0 for no rotary encoding (the
+ *     guide names rotary_cos / rotary_sin as the in-call rotary position
+ *     encoding). With them, q and the new keys of token t are rotated at
+ *     position Lk - Sq + t before the attention and the append: each pair
+ *     (a, b) of the first rotary_dim dimensions becomes
+ *     (a cos - b sin, a sin + b cos), pairs (i, i + rotary_dim/2), or
+ *     (2i, 2i + 1) when rotary_interleaved is nonzero; the rotated values are
+ *     rounded to the input dtype (the cache holds rotated keys). rotary_dim is
+ *     a multiple of 16 up to D; every rotated position must lie in
+ *     [0, rotary_rows).
+ *   out (B, Sq, Hq, D); lse float32 (B, Hq, Sq).
  *   page_size: a multiple of 64.
- *   workspace: at least fa_kvcache_workspace_size(B, Hq, D, num_splits)
- *     bytes of device memory (may be NULL when that is 0).
+ *   workspace: at least fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits,
+ *     rotary_dim) bytes of device memory (may be NULL when that is 0).
  * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null cache/table/lengths,
- *   num_splits < 1, page_size not a positive multiple of 64, or a workspace
- *   that is too small. Lengths and table entries live on the device and are
- *   not read by the host; cache_seqlens[b] (+1 with an append) must not
- *   exceed max_pages_per_seq * page_size.
+ *   Sq < 1, num_splits < 1, page_size not a positive multiple of 64, a bad
+ *   rotary_dim or missing tables, or a workspace that is too small. Lengths
+ *   and table entries live on the device and are not read by the host;
+ *   cache_seqlens[b] (+ Sq with an append) must not exceed
+ *   max_pages_per_seq * page_size. A device-side violation (length, page
+ *   index or rotary position out of range) is skipped and reported by
+ *   fa_get_device_status as FA_ERR_INVALID_ARG; the outputs are then invalid.
  */
 FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_new, void* k_cache,
-                         void* v_cache, const int32_t* block_table, const int32_t* cache_seqlens,
-                         void* out, float* lse, int B, int Hq, int Hkv, int D, int page_size,
-                         int max_pages_per_seq, int num_pages, float scale, int causal,
-                         int window_left, int window_right, float softcap, int num_splits,
-                         fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+                                void* v_cache, const int32_t* block_table,
+                                const int32_t* cache_seqlens, const float* rotary_cos,
+                                const float* rotary_sin, void* out, float* lse, int B, int Sq,
+                                int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                                int num_pages, int rotary_rows, int rotary_dim,
+                                int rotary_interleaved, float scale, int causal, int window_left,
+                                int window_right, float softcap, int num_splits, fa_dtype dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fa_fwd_kvcache without a workspace argument, for callers that cannot
@@ -157,11 +180,13 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_
  * call; it exists only for such callers.
  *
  * Arguments, results and errors are those of fa_fwd_kvcache. The split
- * partials that fa_fwd_kvcache keeps in the caller's workspace live instead
- * in one statically sized device array inside this library,
+ * partials and rotated queries that fa_fwd_kvcache keeps in the caller's
+ * workspace live instead in one statically sized device array inside this
+ * library,
  * FA_NOALLOC_SCRATCH_BYTES (24 MiB) large, which every GPU that loads the
  * library holds until the process exits. A call whose partials need more
- * (fa_kvcache_workspace_size(B, Hq, D, num_splits) > FA_NOALLOC_SCRATCH_BYTES)
+ * (fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rotary_dim) >
+ * FA_NOALLOC_SCRATCH_BYTES)
  * is rejected with FA_ERR_INVALID_ARG before anything is launched. The call
  * itself allocates nothing: no cudaMalloc, cudaFree or allocating library
  * routine.
@@ -178,9 +203,11 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_
 #define FA_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
 FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const void* v_new,
                                         void* k_cache, void* v_cache, const int32_t* block_table,
-                                        const int32_t* cache_seqlens, void* out, float* lse, int B,
-                                        int Hq, int Hkv, int D, int page_size,
-                                        int max_pages_per_seq, int num_pages, float scale,
+                                        const int32_t* cache_seqlens, const float* rotary_cos,
+                                        const float* rotary_sin, void* out, float* lse, int B,
+                                        int Sq, int Hq, int Hkv, int D, int page_size,
+                                        int max_pages_per_seq, int num_pages, int rotary_rows,
+                                        int rotary_dim, int rotary_interleaved, float scale,
                                         int causal, int window_left, int window_right,
                                         float softcap, int num_splits, fa_dtype dtype,
                                         void* stream);

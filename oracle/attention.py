@@ -288,6 +288,9 @@ def rotary(x, pos, cos, sin, interleaved=False):
     cos = _f64(cos)
     sin = _f64(sin)
     half = cos.shape[1]
+    pos = np.asarray(pos)
+    if pos.size and (pos.min() < 0 or pos.max() >= cos.shape[0]):
+        raise ValueError("rotary position outside the angle table")
     c = cos[np.asarray(pos)][:, None, :]  # (T, 1, r/2)
     sn = sin[np.asarray(pos)][:, None, :]
     if interleaved:

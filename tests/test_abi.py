@@ -60,8 +60,13 @@ def test_workspace_sizes(fa):
     n = fa.fa_bwd_workspace_size(2, 32, 8192, 128)
     assert n == 2 * 8192 * 32 * 4
     assert fa.fa_bwd_workspace_size(3, 4, 0, 128, 1000) == 16128
-    assert fa.fa_kvcache_workspace_size(64, 32, 128, 1) == 0
-    assert fa.fa_kvcache_workspace_size(64, 32, 128, 16) == 16 * 64 * 32 * 129 * 4
+    # kv-cache: float32 split partials (O and LSE per split and output row),
+    # padded to 256 B, then the rotated queries in the 16-bit input type
+    assert fa.fa_kvcache_workspace_size(64, 1, 32, 128, 1) == 0
+    assert fa.fa_kvcache_workspace_size(64, 1, 32, 128, 16) == 16 * 64 * 32 * 129 * 4
+    assert fa.fa_kvcache_workspace_size(3, 5, 7, 64, 2) == (2 * 105 * 65 * 4 + 255) // 256 * 256
+    assert fa.fa_kvcache_workspace_size(3, 5, 7, 64, 1, 64) == 105 * 64 * 2
+    assert fa.fa_kvcache_workspace_size(3, 5, 7, 64, 2, 32) == 54784 + 105 * 64 * 2
 
 
 def _fwd_status(fa, **kw):
@@ -112,13 +117,15 @@ def test_kvcache_rejects_bad_arguments(fa):
     lib = fa.lib
 
     def call(**kw):
-        a = dict(q=16, kn=16, vn=16, kc=16, vc=16, bt=16, cs=16, out=16, lse=16, B=2, Hq=4,
-                 Hkv=2, D=128, ps=256, mp=4, npg=8, scale=0.1, causal=1, wl=-1, wr=-1,
-                 softcap=0.0, splits=1, dtype=0, ws=None, wsb=0)
+        a = dict(q=16, kn=16, vn=16, kc=16, vc=16, bt=16, cs=16, cos=None, sin=None, out=16,
+                 lse=16, B=2, Sq=1, Hq=4, Hkv=2, D=128, ps=256, mp=4, npg=8, rrows=0, rd=0,
+                 rint=0, scale=0.1, causal=1, wl=-1, wr=-1, softcap=0.0, splits=1, dtype=0,
+                 ws=None, wsb=0)
         a.update(kw)
         return lib.fa_fwd_kvcache(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["bt"], a["cs"],
-                                  a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["D"], a["ps"],
-                                  a["mp"], a["npg"], a["scale"], a["causal"], a["wl"], a["wr"],
+                                  a["cos"], a["sin"], a["out"], a["lse"], a["B"], a["Sq"], a["Hq"],
+                                  a["Hkv"], a["D"], a["ps"], a["mp"], a["npg"], a["rrows"], a["rd"],
+                                  a["rint"], a["scale"], a["causal"], a["wl"], a["wr"],
                                   a["softcap"], a["splits"], a["dtype"], a["ws"], a["wsb"], None)
 
     assert call(kc=None) == 1
@@ -130,6 +137,14 @@ def test_kvcache_rejects_bad_arguments(fa):
     assert call(kn=None) == 1 or call(kn=None) == 3  # k_new without v_new is invalid
     assert call(splits=4, ws=None, wsb=0) == 1        # workspace required
     assert call(D=80) == 2
+    assert call(Sq=0) == 1
+    rot = dict(cos=16, sin=16, rrows=100, ws=256, wsb=1 << 20)
+    assert call(rd=24, **rot) == 1                    # not a multiple of 16
+    assert call(rd=256, **rot) == 1                   # wider than D
+    assert call(rd=64, **dict(rot, cos=None)) == 1    # table missing
+    assert call(rd=64, **dict(rot, rrows=0)) == 1     # empty table
+    assert call(rd=64, **dict(rot, sin=18)) == 1      # misaligned table
+    assert call(rd=64, **dict(rot, ws=None, wsb=0)) == 1  # rotated queries need a workspace
 
 
 def test_valid_call_without_gpu_reports_cuda_error(fa):

@@ -1,7 +1,11 @@
-"""GPU decode parity: fa_fwd_kvcache (paged, split-KV, in-place append) vs the
-oracle, which attends over a logical contiguous cache and never reads the
-page table. The page pool after the call must equal the pool before it with
-exactly the appended slots changed (bitwise)."""
+"""GPU decode parity: fa_fwd_kvcache (paged, split-KV, in-place append, Sq
+new tokens, rotary) vs the oracle, which attends over a logical contiguous
+cache and never reads the page table. The page pool after the call must equal
+the pool before it with exactly the appended slots changed: bitwise for plain
+appends; with rotary, rotated keys within one 16-bit rounding step of the
+oracle's (the GPU rotates in float32, the oracle in float64, and both round
+the result to the storage type, so a value lying within float32 error of a
+rounding boundary may round the other way)."""
 
 import math
 
@@ -10,21 +14,27 @@ import pytest
 import torch
 
 import attn_workloads as W
-from oracle import head_fwd, kvcache_decode
+from oracle import kvcache_decode
 from parity_utils import check_fwd, to64
 
 pytestmark = pytest.mark.gpu
 
 fa = pytest.importorskip("exact_attention_149_b200")
 
+# one rounding step of the storage type, relative, plus the float32 error of
+# a rotation of O(1) values (a cos - b sin can cancel)
+ROT_RTOL = {"bf16": 2.0 ** -7, "fp16": 2.0 ** -10}
+ROT_ATOL = 1e-5
+
 
 def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True, scale=None,
-              heads=None, check_pool=True):
+              heads=None, check_pool=True, rotary_dim=0, interleaved=False):
     dev = torch.device("cuda")
     D = st["D"]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     Hkv = st["Hkv"]
     dt = W.DTYPES[st["dtype"]]
+    B, Sq, Hq, _ = st["q"].shape
     shape = (st["num_pages"], st["page_size"], Hkv, D)
     # unused slots hold a recognisable non-zero pattern so stray reads show up
     kc = torch.full(shape, 3.0, dtype=dt, device=dev)
@@ -35,32 +45,31 @@ def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True
     q = st["q"].to(dev)
     kn = st["k_new"].to(dev) if append else None
     vn = st["v_new"].to(dev) if append else None
+    cos = sin = None
+    if rotary_dim:
+        cos, sin = W.rotary_tables(st["pages_per_seq"] * st["page_size"], rotary_dim)
     out, lse = fa.fwd_kvcache(q, kc, vc, st["cache_seqlens"].to(dev), st["block_table"].to(dev),
-                              k_new=kn, v_new=vn, scale=scale, causal=causal, window=window,
-                              softcap=softcap, num_splits=splits)
+                              k_new=kn, v_new=vn,
+                              rotary_cos=None if cos is None else cos.to(dev),
+                              rotary_sin=None if sin is None else sin.to(dev),
+                              rotary_interleaved=interleaved, scale=scale, causal=causal,
+                              window=window, softcap=softcap, num_splits=splits)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
-    B = st["q"].shape[0]
-    Hq = st["q"].shape[2]
-    g = Hq // Hkv
+    assert out.shape == (B, Sq, Hq, D) and lse.shape == (B, Hq, Sq)
     logical = [W.decode_sequence_cache(st, b) for b in range(B)]
-    if append:
-        o_ref, l_ref, ks, vs = kvcache_decode(st["q"], st["k_new"], st["v_new"],
-                                              [c[0] for c in logical], [c[1] for c in logical],
-                                              st["cache_seqlens"].tolist(), scale, causal, window,
-                                              softcap, heads=heads)
-    else:
-        o_ref = np.zeros((B, 1, Hq, D))
-        l_ref = np.zeros((B, Hq, 1))
-        for b in range(B):
-            for h in (range(Hq) if heads is None else heads):
-                o1, l1 = head_fwd(st["q"][b, :, h], logical[b][0][:, h // g], logical[b][1][:, h // g],
-                                  scale, causal, window[0], window[1], softcap)
-                o_ref[b, 0, h] = o1[0]
-                l_ref[b, h, 0] = l1[0]
+    rot = {}
+    if rotary_dim:
+        rot = dict(rotary_cos=cos.double().numpy(), rotary_sin=sin.double().numpy(),
+                   rotary_interleaved=interleaved, rotated_dtype=st["dtype"])
+    o_ref, l_ref, ks, vs = kvcache_decode(st["q"], st["k_new"] if append else None,
+                                          st["v_new"] if append else None,
+                                          [c[0] for c in logical], [c[1] for c in logical],
+                                          st["cache_seqlens"].tolist(), scale, causal, window,
+                                          softcap, heads=heads, **rot)
     hs = list(range(Hq)) if heads is None else list(heads)
     check_fwd(out[:, :, hs], lse[:, hs], o_ref[:, :, hs], l_ref[:, hs],
-              f"decode splits={splits}")
+              f"decode Sq={Sq} splits={splits} rot={rotary_dim}")
     if check_pool:
         ps = st["page_size"]
         changed_k = (kc != k_before).any(dim=(2, 3))
@@ -69,10 +78,19 @@ def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True
         if append:
             for b in range(B):
                 L = int(st["cache_seqlens"][b])
-                page = int(st["block_table"][b, L // ps])
-                expect[page, L % ps] = True
-                assert torch.equal(kc[page, L % ps].cpu(), st["k_new"][b, 0])
-                assert torch.equal(vc[page, L % ps].cpu(), st["v_new"][b, 0])
+                for t in range(Sq):
+                    pos = L + t
+                    page = int(st["block_table"][b, pos // ps])
+                    expect[page, pos % ps] = True
+                    assert torch.equal(vc[page, pos % ps].cpu(), st["v_new"][b, t])
+                    got_k = kc[page, pos % ps].cpu()
+                    if rotary_dim:
+                        ref_k = ks[b][pos]
+                        err = np.abs(to64(got_k) - ref_k)
+                        assert np.all(err <= ROT_RTOL[st["dtype"]] * np.abs(ref_k) + ROT_ATOL), \
+                            f"rotated key b{b} t{t}: max err {err.max():.3e}"
+                    else:
+                        assert torch.equal(got_k, st["k_new"][b, t])
         # a slot may also legitimately keep its value if k_new equals the old one
         assert not (changed_k & ~expect).any() and not (changed_v & ~expect).any()
     return out, lse
@@ -111,6 +129,64 @@ def test_decode_without_append(cuda_ok):
                                  cache_seqlens=[1, 129, 500])
     _run_case(st, 1, append=False)
     _run_case(st, 5, append=False)
+
+
+@pytest.mark.parametrize("Sq,Hq,Hkv,D,dtype,lengths,ps", [
+    (2, 8, 2, 128, "bf16", [5, 64, 200], 64),        # 8 columns: one tile
+    (4, 8, 2, 128, "bf16", [0, 61, 1000], 64),       # 16 columns
+    (5, 16, 4, 64, "fp16", [3, 300], 128),           # 20 columns, ragged tiles
+    (9, 8, 1, 128, "bf16", [700, 31], 64),           # 72 columns: three column blocks
+    (3, 32, 1, 128, "bf16", [129, 2000], 256),       # group 32 x 3 tokens
+])
+@pytest.mark.parametrize("splits", [1, 3])
+def test_decode_multi_token(cuda_ok, Sq, Hq, Hkv, D, dtype, lengths, ps, splits):
+    """Sq new tokens per sequence: bottom-right causal over the L + Sq keys."""
+    st = W.make_decode_structure(len(lengths), Hq, Hkv, D, 0, max(lengths), ps, dtype,
+                                 seed=Sq * 100 + sum(lengths), cache_seqlens=lengths, sq=Sq)
+    _run_case(st, splits)
+
+
+@pytest.mark.parametrize("window,softcap,causal", [((7, 0), 0.0, True), ((-1, -1), 5.0, True),
+                                                   ((-1, -1), 0.0, False), ((20, 2), 0.0, False),
+                                                   ((0, 0), 0.0, True)])
+def test_decode_multi_token_options(cuda_ok, window, softcap, causal):
+    st = W.make_decode_structure(3, 8, 2, 128, 0, 300, 64, "bf16", seed=41,
+                                 cache_seqlens=[300, 3, 128], sq=6)
+    for splits in (1, 4):
+        _run_case(st, splits, causal=causal, window=window, softcap=softcap)
+
+
+def test_decode_multi_token_without_append(cuda_ok):
+    """No append: the Sq queries sit at L - Sq .. L - 1; with L < Sq the first
+    queries precede every key and (causal) see none: O = 0, LSE = -inf."""
+    st = W.make_decode_structure(3, 8, 2, 64, 1, 400, 64, "bf16", seed=43,
+                                 cache_seqlens=[2, 65, 400], sq=4)
+    _run_case(st, 1, append=False)
+    _run_case(st, 3, append=False)
+    _run_case(st, 2, append=False, causal=False)
+
+
+@pytest.mark.parametrize("Sq,D,rd,interleaved,dtype", [
+    (1, 128, 128, False, "bf16"),
+    (1, 128, 128, True, "bf16"),
+    (3, 128, 64, False, "bf16"),   # rotary on the first half of the dims only
+    (2, 64, 32, True, "fp16"),
+    (4, 64, 64, False, "fp16"),
+])
+@pytest.mark.parametrize("splits", [1, 4])
+def test_decode_rotary(cuda_ok, Sq, D, rd, interleaved, dtype, splits):
+    """q and the new keys rotated at their positions; the cache keeps the
+    rotated keys."""
+    st = W.make_decode_structure(3, 8, 2, D, 0, 500, 64, dtype, seed=rd + Sq + splits,
+                                 cache_seqlens=[0, 77, 500], sq=Sq)
+    _run_case(st, splits, rotary_dim=rd, interleaved=interleaved)
+
+
+def test_decode_rotary_without_append(cuda_ok):
+    """Rotary without k_new: only q is rotated (at L - Sq + t)."""
+    st = W.make_decode_structure(2, 8, 2, 128, 4, 300, 64, "bf16", seed=47,
+                                 cache_seqlens=[4, 300], sq=3)
+    _run_case(st, 2, append=False, rotary_dim=128)
 
 
 def test_decode_split_counts_agree(cuda_ok):

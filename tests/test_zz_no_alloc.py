@@ -27,10 +27,10 @@ pytestmark = pytest.mark.gpu
 fa = pytest.importorskip("exact_attention_149_b200")
 
 
-def _decode_both_ways(B, Hq, Hkv, D, lengths, page_size, splits, seed):
+def _decode_both_ways(B, Hq, Hkv, D, lengths, page_size, splits, seed, sq=1, rotary_dim=0):
     dev = torch.device("cuda")
     st = W.make_decode_structure(B, Hq, Hkv, D, 0, max(lengths), page_size, "bf16", seed=seed,
-                                 cache_seqlens=lengths)
+                                 cache_seqlens=lengths, sq=sq)
     shape = (st["num_pages"], page_size, Hkv, D)
     kc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
     vc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
@@ -39,23 +39,29 @@ def _decode_both_ways(B, Hq, Hkv, D, lengths, page_size, splits, seed):
     q = st["q"].to(dev)
     kn, vn = st["k_new"].to(dev), st["v_new"].to(dev)
     cs, bt = st["cache_seqlens"].to(dev), st["block_table"].to(dev)
+    rows = st["pages_per_seq"] * page_size
+    cos = sin = None
+    if rotary_dim:
+        cos, sin = (t.to(dev) for t in W.rotary_tables(rows, rotary_dim))
     scale = 1.0 / math.sqrt(D)
     # reference: the workspace entry point
-    ws = torch.empty(fa.fa_kvcache_workspace_size(B, Hq, D, splits), dtype=torch.uint8, device=dev)
+    ws = torch.empty(fa.fa_kvcache_workspace_size(B, sq, Hq, D, splits, rotary_dim),
+                     dtype=torch.uint8, device=dev)
     out_ref = torch.empty_like(q)
-    lse_ref = torch.empty((B, Hq, 1), dtype=torch.float32, device=dev)
-    fa.fa_fwd_kvcache(q, kn, vn, kc, vc, bt, cs, out_ref, lse_ref, B, Hq, Hkv, D, page_size,
-                      bt.shape[1], st["num_pages"], scale, True, -1, -1, 0.0, splits, 0, ws,
-                      ws.numel())
+    lse_ref = torch.empty((B, Hq, sq), dtype=torch.float32, device=dev)
+    fa.fa_fwd_kvcache(q, kn, vn, kc, vc, bt, cs, cos, sin, out_ref, lse_ref, B, sq, Hq, Hkv, D,
+                      page_size, bt.shape[1], st["num_pages"], rows, rotary_dim, False, scale,
+                      True, -1, -1, 0.0, splits, 0, ws, ws.numel())
     # the allocation-free entry point, called straight through the C ABI
     out = torch.full_like(q, float("nan"))
-    lse = torch.full((B, Hq, 1), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((B, Hq, sq), float("nan"), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream().cuda_stream
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
     status = fa.lib.fa_fwd_kvcache_noalloc(
         q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc2.data_ptr(), vc2.data_ptr(), bt.data_ptr(),
-        cs.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, D, page_size, bt.shape[1],
-        st["num_pages"], ctypes.c_float(scale), 1, -1, -1, ctypes.c_float(0.0), splits, 0,
-        ctypes.c_void_p(stream))
+        cs.data_ptr(), ptr(cos), ptr(sin), out.data_ptr(), lse.data_ptr(), B, sq, Hq, Hkv, D,
+        page_size, bt.shape[1], st["num_pages"], rows if rotary_dim else 0, rotary_dim, 0,
+        ctypes.c_float(scale), 1, -1, -1, ctypes.c_float(0.0), splits, 0, ctypes.c_void_p(stream))
     assert status == 0, fa.fa_last_error()
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
@@ -66,14 +72,15 @@ def _decode_both_ways(B, Hq, Hkv, D, lengths, page_size, splits, seed):
 
 def test_noalloc_matches_workspace_entry_point_twice(cuda_ok):
     _decode_both_ways(4, 32, 8, 128, [1500, 64, 777, 3000], 256, 4, seed=101)
-    _decode_both_ways(3, 8, 2, 128, [200, 1000, 5], 64, 7, seed=202)
+    # the second call also keeps rotated queries of 3 new tokens in the scratch
+    _decode_both_ways(3, 8, 2, 128, [200, 1000, 5], 64, 7, seed=202, sq=3, rotary_dim=128)
 
 
 def test_noalloc_rejects_oversized_partials(cuda_ok):
     # B=64, Hq=64, D=128, 32 splits need 64*64*129*4*32 bytes > 24 MiB
-    need = fa.fa_kvcache_workspace_size(64, 64, 128, 32)
+    need = fa.fa_kvcache_workspace_size(64, 1, 64, 128, 32)
     assert need > fa.FA_NOALLOC_SCRATCH_BYTES
-    status = fa.lib.fa_fwd_kvcache_noalloc(16, 16, 16, 16, 16, 16, 16, 16, 16, 64, 64, 8, 128,
-                                           256, 4, 8, ctypes.c_float(0.1), 1, -1, -1,
-                                           ctypes.c_float(0.0), 32, 0, None)
+    status = fa.lib.fa_fwd_kvcache_noalloc(16, 16, 16, 16, 16, 16, 16, None, None, 16, 16, 64, 1,
+                                           64, 8, 128, 256, 4, 8, 0, 0, 0, ctypes.c_float(0.1), 1,
+                                           -1, -1, ctypes.c_float(0.0), 32, 0, None)
     assert status == 1 and "scratch" in fa.fa_last_error()
