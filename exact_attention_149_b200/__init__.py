@@ -278,8 +278,9 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
                 rotary_cos=None, rotary_sin=None, rotary_interleaved=False, scale=None,
                 causal=True, window=(-1, -1), softcap=0.0, num_splits=1, out=None, lse=None,
                 workspace=None, stream=None):
-    """One decode step: q (B,Sq,Hq,D); caches (num_pages, page_size, Hkv, D);
-    block_table int32 (B, max_pages); cache_seqlens int32 (B). Appends
+    """One decode step: q (B,Sq,Hq,D); caches (num_pages, page_size, Hkv, D)
+    with block_table int32 (B, max_pages), or block_table None and contiguous
+    caches (B, capacity, Hkv, D); cache_seqlens int32 (B). Appends
     k_new/v_new (B,Sq,Hkv,D) in place, then attends. rotary_cos/rotary_sin:
     float32 (rows, rotary_dim/2) tables that rotate q and k_new at their
     positions. Returns (out (B,Sq,Hq,D), lse (B,Hq,Sq))."""
@@ -287,6 +288,7 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
                rotary_sin)
     B, Sq, Hq, D = q.shape
     num_pages, page_size, Hkv, _ = k_cache.shape
+    max_pages = 1 if block_table is None else block_table.shape[1]
     if (rotary_cos is None) != (rotary_sin is None):
         raise FaError(FA_ERR_INVALID_ARG, "rotary_cos and rotary_sin go together")
     if rotary_cos is not None and (rotary_cos.dtype != torch.float32 or rotary_sin.dtype != torch.float32
@@ -299,8 +301,8 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
     if workspace is None and nbytes > 0:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos,
-                   rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, block_table.shape[1],
-                   num_pages, rot_rows, rot_dim, rotary_interleaved, _scale(scale, D), causal,
-                   window[0], window[1], softcap, num_splits, _dt(q), workspace,
+                   rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, max_pages, num_pages,
+                   rot_rows, rot_dim, rotary_interleaved, _scale(scale, D), causal, window[0],
+                   window[1], softcap, num_splits, _dt(q), workspace,
                    0 if workspace is None else workspace.numel(), stream)
     return out, lse

@@ -40,7 +40,7 @@ struct DecodeParams {
   const void* v_new;
   void* k_cache;          // (num_pages, page_size, Hkv, D)
   void* v_cache;
-  const int* block_table; // (B, max_pages)
+  const int* block_table; // (B, max_pages); null: contiguous cache, page b = sequence b
   const int* cache_seqlens;
   const float* rot_cos;   // (rot_rows, rot_dim / 2) fp32, or null
   const float* rot_sin;
@@ -152,7 +152,8 @@ __global__ void kv_append_kernel(const DecodeParams p) {
     if (threadIdx.x == 0) atomicExch(&g_device_status, kDevBadIndex);
     return;
   }
-  const int page = p.block_table[static_cast<size_t>(b) * p.max_pages + pos / p.page_size];
+  const int page =
+      p.block_table ? p.block_table[static_cast<size_t>(b) * p.max_pages + pos / p.page_size] : b;
   if (page < 0 || page >= p.num_pages) {
     if (threadIdx.x == 0) atomicExch(&g_device_status, kDevBadIndex);
     return;
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(160)
     if (elect_one()) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
+      const int* bt = p.block_table ? p.block_table + static_cast<size_t>(b) * p.max_pages : nullptr;
       int i = 0;
       for (; i < n_iter; ++i) {
         const int slot = i % Sh::kStages;
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(160)
         }
         if (!ok) break;
         const int pos = (t_begin + i) * Sh::kTok;
-        int page = bt[pos / p.page_size];
+        int page = bt ? bt[pos / p.page_size] : b;
         if (page < 0 || page >= p.num_pages) {
           atomicExch(&g_device_status, kDevBadIndex);
           page = 0;  // stay in bounds; the result is flagged as invalid
@@ -468,6 +469,18 @@ __global__ void __launch_bounds__(160)
       pb[nt][1] = movmatrix_t(pack2<kBF16>(e2, e3));
     }
     // ---- O^T += V^T P^T ----
+    // Slots at positions >= Lk (the rest of the last page, or the next
+    // sequence of a contiguous cache) may hold anything, NaN included; P is 0
+    // there but 0 * NaN is not, so those V elements are zeroed. Fragment
+    // registers a0, a1 hold tokens wtok + 2*(lane&3) + {0, 1} (low, high
+    // half), a2, a3 the same tokens + 8.
+    const bool tail = wtok + 16 > Lk;  // warp-uniform
+    uint32_t vm01 = 0xffffffffu, vm23 = 0xffffffffu;
+    if (tail) {
+      const int k0 = wtok + 2 * (lane & 3);
+      vm01 = (k0 < Lk ? 0x0000ffffu : 0u) | (k0 + 1 < Lk ? 0xffff0000u : 0u);
+      vm23 = (k0 + 8 < Lk ? 0x0000ffffu : 0u) | (k0 + 9 < Lk ? 0xffff0000u : 0u);
+    }
 #pragma unroll
     for (int mt = 0; mt < kD / 16; ++mt) {
       const int mi = lane >> 3, r = lane & 7;
@@ -475,6 +488,12 @@ __global__ void __launch_bounds__(160)
       const int dcol = mt * 16 + (mi & 1) * 8;
       uint32_t a0, a1, a2, a3;
       ldsm_x4_t(sw128(vbase + (dcol >> 6) * Sh::kBoxBytes, tok, (dcol & 63) >> 3), a0, a1, a2, a3);
+      if (tail) {
+        a0 &= vm01;
+        a1 &= vm01;
+        a2 &= vm23;
+        a3 &= vm23;
+      }
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) mma16816<kBF16>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
     }

@@ -116,7 +116,7 @@ FA_API size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_sp
                                         int rotary_dim);
 
 /*
- * One decode step against a paged KV cache (guide §增量解码场景
+ * One decode step against a paged (or contiguous) KV cache (guide §增量解码场景
  * flash_attn_with_kvcache): the Sq new keys/values of each sequence are
  * appended IN PLACE at logical positions L .. L + Sq - 1 (L =
  * cache_seqlens[b]), then the Sq new queries attend over the Lk = L + Sq
@@ -132,7 +132,10 @@ FA_API size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_sp
  *     slot p % page_size ("FlashAttention技术深度解析" §动态缓存架构: a page
  *     table maps logical blocks to physical ones).
  *   block_table: DEVICE int32 (B, max_pages_per_seq), every referenced entry
- *     in [0, num_pages).
+ *     in [0, num_pages). NULL selects a contiguous (non-paged) cache:
+ *     k_cache, v_cache (B, capacity, Hkv, D) with page_size = capacity (any
+ *     value >= 1), max_pages_per_seq = 1 and num_pages = B, so that sequence
+ *     b is page b.
  *   cache_seqlens: DEVICE int32 (B), valid length BEFORE the append; the
  *     library does not increment it (the caller advances its own position).
  *   rotary_cos, rotary_sin: DEVICE float32 (rotary_rows, rotary_dim / 2)
@@ -147,11 +150,13 @@ FA_API size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_sp
  *     a multiple of 16 up to D; every rotated position must lie in
  *     [0, rotary_rows).
  *   out (B, Sq, Hq, D); lse float32 (B, Hq, Sq).
- *   page_size: a multiple of 64.
+ *   page_size: a multiple of 64 (paged cache). Cache slots at positions
+ *     >= Lk are never read into a result, whatever they hold (NaN included).
  *   workspace: at least fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits,
  *     rotary_dim) bytes of device memory (may be NULL when that is 0).
- * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null cache/table/lengths,
- *   Sq < 1, num_splits < 1, page_size not a positive multiple of 64, a bad
+ * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null cache/lengths, Sq < 1,
+ *   num_splits < 1, page_size not a positive multiple of 64 (or a
+ *   contiguous cache described otherwise than above), a bad
  *   rotary_dim or missing tables, or a workspace that is too small. Lengths
  *   and table entries live on the device and are not read by the host;
  *   cache_seqlens[b] (+ Sq with an append) must not exceed

@@ -27,19 +27,40 @@ ROT_RTOL = {"bf16": 2.0 ** -7, "fp16": 2.0 ** -10}
 ROT_ATOL = 1e-5
 
 
+def _slot(st, b, pos, contiguous):
+    """(page, slot) of logical position pos of sequence b."""
+    if contiguous:
+        return b, pos
+    ps = st["page_size"]
+    return int(st["block_table"][b, pos // ps]), pos % ps
+
+
 def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True, scale=None,
-              heads=None, check_pool=True, rotary_dim=0, interleaved=False):
+              heads=None, check_pool=True, rotary_dim=0, interleaved=False, fill=(3.0, -5.0),
+              contiguous_capacity=0):
+    """contiguous_capacity > 0: a contiguous (B, capacity, Hkv, D) cache and no
+    block table instead of the paged pool."""
     dev = torch.device("cuda")
     D = st["D"]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     Hkv = st["Hkv"]
     dt = W.DTYPES[st["dtype"]]
     B, Sq, Hq, _ = st["q"].shape
-    shape = (st["num_pages"], st["page_size"], Hkv, D)
-    # unused slots hold a recognisable non-zero pattern so stray reads show up
-    kc = torch.full(shape, 3.0, dtype=dt, device=dev)
-    vc = torch.full(shape, -5.0, dtype=dt, device=dev)
-    W.fill_paged_pool(st, kc, vc)
+    contiguous = contiguous_capacity > 0
+    if contiguous:
+        shape = (B, contiguous_capacity, Hkv, D)
+    else:
+        shape = (st["num_pages"], st["page_size"], Hkv, D)
+    # unused slots hold a recognisable pattern (or NaN) so stray reads show up
+    kc = torch.full(shape, fill[0], dtype=dt, device=dev)
+    vc = torch.full(shape, fill[1], dtype=dt, device=dev)
+    if contiguous:
+        for b in range(B):
+            k, v = W.decode_sequence_cache(st, b)
+            kc[b, :k.shape[0]].copy_(k.to(dev))
+            vc[b, :v.shape[0]].copy_(v.to(dev))
+    else:
+        W.fill_paged_pool(st, kc, vc)
     k_before = kc.clone() if check_pool else None
     v_before = vc.clone() if check_pool else None
     q = st["q"].to(dev)
@@ -48,7 +69,8 @@ def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True
     cos = sin = None
     if rotary_dim:
         cos, sin = W.rotary_tables(st["pages_per_seq"] * st["page_size"], rotary_dim)
-    out, lse = fa.fwd_kvcache(q, kc, vc, st["cache_seqlens"].to(dev), st["block_table"].to(dev),
+    bt = None if contiguous else st["block_table"].to(dev)
+    out, lse = fa.fwd_kvcache(q, kc, vc, st["cache_seqlens"].to(dev), bt,
                               k_new=kn, v_new=vn,
                               rotary_cos=None if cos is None else cos.to(dev),
                               rotary_sin=None if sin is None else sin.to(dev),
@@ -71,19 +93,22 @@ def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True
     check_fwd(out[:, :, hs], lse[:, hs], o_ref[:, :, hs], l_ref[:, hs],
               f"decode Sq={Sq} splits={splits} rot={rotary_dim}")
     if check_pool:
-        ps = st["page_size"]
-        changed_k = (kc != k_before).any(dim=(2, 3))
-        changed_v = (vc != v_before).any(dim=(2, 3))
+        def changed(a, b):
+            same = (a == b) | (torch.isnan(a) & torch.isnan(b))
+            return (~same).any(dim=(2, 3))
+
+        changed_k = changed(kc, k_before)
+        changed_v = changed(vc, v_before)
         expect = torch.zeros_like(changed_k)
         if append:
             for b in range(B):
                 L = int(st["cache_seqlens"][b])
                 for t in range(Sq):
+                    page, slot = _slot(st, b, L + t, contiguous)
                     pos = L + t
-                    page = int(st["block_table"][b, pos // ps])
-                    expect[page, pos % ps] = True
-                    assert torch.equal(vc[page, pos % ps].cpu(), st["v_new"][b, t])
-                    got_k = kc[page, pos % ps].cpu()
+                    expect[page, slot] = True
+                    assert torch.equal(vc[page, slot].cpu(), st["v_new"][b, t])
+                    got_k = kc[page, slot].cpu()
                     if rotary_dim:
                         ref_k = ks[b][pos]
                         err = np.abs(to64(got_k) - ref_k)
@@ -187,6 +212,31 @@ def test_decode_rotary_without_append(cuda_ok):
     st = W.make_decode_structure(2, 8, 2, 128, 4, 300, 64, "bf16", seed=47,
                                  cache_seqlens=[4, 300], sq=3)
     _run_case(st, 2, append=False, rotary_dim=128)
+
+
+@pytest.mark.parametrize("Sq,splits", [(1, 1), (1, 4), (3, 2)])
+def test_decode_ignores_nan_in_unused_slots(cuda_ok, Sq, splits):
+    """A pool straight from an uninitialised allocation may hold NaN bit
+    patterns past each sequence's end; they must not reach the result (the
+    kernel reads whole 64-token chunks of the last page)."""
+    st = W.make_decode_structure(3, 8, 2, 128, 0, 300, 64, "bf16", seed=53,
+                                 cache_seqlens=[5, 64, 299], sq=Sq)
+    nan = float("nan")
+    _run_case(st, splits, fill=(nan, nan))
+    _run_case(st, splits, fill=(nan, nan), append=False)
+
+
+@pytest.mark.parametrize("Sq,splits,capacity,rd", [(1, 1, 301, 0), (1, 4, 1000, 0), (4, 3, 310, 64),
+                                                    (2, 1, 64, 0)])
+def test_decode_contiguous_cache(cuda_ok, Sq, splits, capacity, rd):
+    """block_table NULL: a contiguous (B, capacity, Hkv, D) cache, capacity not
+    a multiple of the 64-token chunk; the slots past each sequence (and the
+    next sequence's rows that a chunk straddles) hold NaN."""
+    lens = [0, 57, capacity - Sq]
+    st = W.make_decode_structure(3, 8, 2, 128, 0, max(lens), 64, "bf16", seed=59 + capacity,
+                                 cache_seqlens=lens, sq=Sq)
+    nan = float("nan")
+    _run_case(st, splits, fill=(nan, nan), contiguous_capacity=capacity, rotary_dim=rd)
 
 
 def test_decode_split_counts_agree(cuda_ok):
