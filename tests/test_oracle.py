@@ -558,3 +558,12 @@ def test_multi_token_decode_equals_prefill_rows(window, softcap, causal):
                 np.testing.assert_allclose(o[b, :, h], of, atol=1e-13)
                 np.testing.assert_allclose(o[b, :, h], op[-Sq:], atol=1e-13)
                 np.testing.assert_allclose(lse[b, h], lp[-Sq:], atol=1e-13)
+
+
+def test_rotary_rejects_positions_outside_the_table():
+    cos, sin = rope_tables(8, 4)
+    x = np.ones((1, 1, 4))
+    with pytest.raises(ValueError):
+        rotary(x, [-1], cos, sin)  # numpy would silently wrap to the last row
+    with pytest.raises(ValueError):
+        rotary(x, [8], cos, sin)
