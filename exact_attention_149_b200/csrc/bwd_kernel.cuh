@@ -8,7 +8,8 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q
 // (and dS picks up the factor 1 - tanh^2 under softcap).
 //
-//   bwd_pre_kernel   Drow = rowsum(dO * O) per (token, query head).
+//   bwd_pre_kernel   Drow = rowsum(dO * O) and -LSE (exp2 domain) per
+//                    (token, query head), into a padded per-row layout.
 //   bwd_dkdv_kernel  one CTA per (sequence, kv head, 128-key tile): K and V
 //                    stay resident while the CTA walks every query head of the
 //                    GQA group and every 128-row Q tile that can see the keys;
@@ -22,16 +23,19 @@
 // for no dQ reduction across CTAs and a pipeline with no write-back on the
 // critical path.
 //
-// bwd_dkdv warp roles (320 threads):
-//   warp 0     TMA producer: K, V once; Q_i and dO_i into a 2-slot ring.
-//   warp 1     MMA issuer (one lane), TMEM owner.
-//   warps 2-9  two compute groups; group g owns query columns [64g, 64g+64):
-//              one thread per key row computes P^T = exp(S^T - LSE) and then
-//              dS^T = P^T * (dP^T - Drow), each written back to TMEM as 16-bit
-//              over the columns it came from, where the dV and dK MMAs read
-//              their A operand; at the end group 0 writes dV, group 1 dK.
+// bwd_dkdv warp roles (576 threads):
+//   warp 0      TMA producer: K, V once; Q_i, dO_i and the rows' -LSE and Drow
+//               into a 2-slot ring.
+//   warp 1      MMA issuer (one lane), TMEM owner.
+//   warps 2-17  four compute groups; group g owns query columns [32g, 32g+32):
+//               one thread per key row computes P^T = exp(S^T - LSE) and then
+//               dS^T = P^T * (dP^T - Drow), each written back to TMEM as 16-bit
+//               pairs over the first half of the columns it came from, where
+//               the dV and dK MMAs read their A operand. Four warps per SM
+//               sub-partition hide the latency of the exponentials and of the
+//               TMEM round trips. At the end groups 0-1 write dV, 2-3 dK.
 // TMEM columns: A [0,128) S^T then P^T; B [128,256) dP^T then dS^T (queries
-// [64g, 64g+64) packed into [64g, 64g+32) of each); dV [256, 256+D);
+// [32g, 32g+32) packed into [32g, 32g+16) of each); dV [256, 256+D);
 // dK [256+D, 256+2D).
 // MMA order per item i: dV_i, S_{i+1}, dK_i, dP_{i+1}. S^T and dP^T signal
 // separately, so the P pass of item i+1 overlaps dK_i and dP_{i+1}, and the
@@ -45,22 +49,35 @@ namespace fa {
 struct BwdParams {
   int B, Hq, Hkv, S, total, group;
   int n_ktiles;              // ceil(S / 128)
-  float scale;               // multiplies dS (so dQ, dK come out scaled)
+  float scale;               // multiplies dK and dQ in the epilogues
   float scale_log2;          // scale * log2(e)
   float softcap, cap_in, cap_out_log2;
   int wl, wr;                // window (causal folded into wr)
   const void* o;
   const void* dout;
-  const float* lse;
-  float* drow;               // LSE layout
+  const float* lse;          // forward LSE, (B, Hq, S) or (Hq, total)
+  float* vec_nlse;           // -LSE * log2(e) (-inf for an empty row), padded layout
+  float* vec_drow;           // rowsum(dO * O), padded layout
+  int tpad;                  // per-head stride of the padded layout
   void* dq;                  // (T, Hq, D) 16-bit
   void* dk;                  // (T, Hkv, D)
   void* dv;
   const int* cu_seqlens;
 };
 
+// Padded layout of the per-row vectors: query row q of sequence b (first
+// token seq_start) and query head h sits at
+//   h * tpad + 128 * (seq_start / 128 + b) + q,  tpad = 128 * (T / 128 + B + 1).
+// Each 128-row tile of a sequence is then contiguous and 512-byte aligned (one
+// bulk copy), and the tiles of different sequences never overlap:
+// seq_start / 128 + ceil(len / 128) <= (seq_start + len) / 128 + 1.
+__device__ __forceinline__ size_t vec_index(const BwdParams& p, int h, int b, int seq_start, int q) {
+  return static_cast<size_t>(h) * p.tpad + 128 * static_cast<size_t>(seq_start / 128 + b) + q;
+}
+
 // ---------------------------------------------------------------------------
-// pre: Drow = rowsum(dO * O). One warp per (token, head) row.
+// pre: Drow = rowsum(dO * O) and -LSE in the exp2 domain, both into the padded
+// layout. One warp per (token, head) row.
 // ---------------------------------------------------------------------------
 template <int kD, bool kBF16>
 __global__ void bwd_pre_kernel(const BwdParams p) {
@@ -90,13 +107,29 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
     size_t li;
+    int b, seq_start;
     if (p.cu_seqlens != nullptr) {
+      // the sequence holding tok: the largest b with cu_seqlens[b] <= tok
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cu_seqlens[mid] <= tok)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      b = lo;
+      seq_start = p.cu_seqlens[b];
       li = static_cast<size_t>(h) * p.total + tok;
     } else {
-      const int b = tok / p.S, s = tok % p.S;
-      li = (static_cast<size_t>(b) * p.Hq + h) * p.S + s;
+      b = tok / p.S;
+      seq_start = b * p.S;
+      li = (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
     }
-    p.drow[li] = acc;
+    const float l = p.lse[li];
+    const size_t vi = vec_index(p, h, b, seq_start, tok - seq_start);
+    p.vec_nlse[vi] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+    p.vec_drow[vi] = acc;
   }
 }
 
@@ -116,22 +149,24 @@ __device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatil
   }
 }
 
-// logit in the exp2 domain and the factor dS picks up (scale, and 1 - tanh^2
-// under softcap) for a pair of raw scores
+// For a pair of raw scores s = q.k: the exponent of P in the exp2 domain,
+// x = logit * log2(e) - LSE * log2(e) (nl2 holds the second term), and the
+// factor dS picks up from the softcap, 1 - tanh^2 (1 without softcap). The
+// common factor `scale` of dS is applied to dK and dQ in the epilogues.
 template <bool kCap>
-__device__ __forceinline__ void bwd_logit2(float2 s2, bool poly, const BwdParams& p, float2& x,
-                                           float2& fac) {
+__device__ __forceinline__ void bwd_logit2(float2 s2, bool poly, const BwdParams& p, float2 nl2,
+                                           float2& x, float2& fac) {
   if constexpr (kCap) {
     float2 th;
     if (poly)
       th = tanh_poly2(__fmul2_rn(s2, make_float2(p.cap_in, p.cap_in)));
     else
       th = make_float2(tanh_fast(s2.x * p.cap_in), tanh_fast(s2.y * p.cap_in));
-    x = make_float2(p.cap_out_log2 * th.x, p.cap_out_log2 * th.y);
-    fac = make_float2((1.f - th.x * th.x) * p.scale, (1.f - th.y * th.y) * p.scale);
+    x = __ffma2_rn(th, make_float2(p.cap_out_log2, p.cap_out_log2), nl2);
+    fac = __ffma2_rn(make_float2(-th.x, -th.y), th, make_float2(1.f, 1.f));
   } else {
-    x = __fmul2_rn(s2, make_float2(p.scale_log2, p.scale_log2));
-    fac = make_float2(p.scale, p.scale);
+    x = __ffma2_rn(s2, make_float2(p.scale_log2, p.scale_log2), nl2);
+    fac = make_float2(1.f, 1.f);
   }
 }
 
@@ -156,10 +191,15 @@ struct DkdvShape {
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;         // + slot * 2 * kTileBytes (Q, dO)
-  static constexpr int kOffVec = 6 * kTileBytes;       // lse_log2[128], drow[128]
-  static constexpr int kOffBar = kOffVec + 1024;
+  // per Q/dO slot: -LSE (exp2 domain)[128], Drow[128] of the slot's query rows
+  static constexpr int kOffVec = 6 * kTileBytes;
+  static constexpr int kVecBytes = 1024;
+  static constexpr int kOffBar = kOffVec + 2 * kVecBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  static constexpr int kThreads = 320;
+  // warp 0 TMA, warp 1 MMA, then kGroups compute groups of 4 warps; group g
+  // owns the 32 query columns [32g, 32g + 32) of every item
+  static constexpr int kGroups = 4;
+  static constexpr int kThreads = 64 + 128 * kGroups;
   static constexpr int kTmemCols = 512;
   static constexpr int kColA = 0;
   static constexpr int kColB = 128;
@@ -182,7 +222,7 @@ struct DkdvBars {
 };
 
 template <int kD, bool kBF16, bool kCap>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
@@ -191,8 +231,6 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem + Sh::kOffBar);
-  float* vec_lse = reinterpret_cast<float*>(smem + Sh::kOffVec);
-  float* vec_drow = vec_lse + 128;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -230,8 +268,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(&bars->s_ready, 1);
     mbar_init(&bars->dp_ready, 1);
-    mbar_init(&bars->p_ready, 8);
-    mbar_init(&bars->ds_ready, 8);
+    mbar_init(&bars->p_ready, 4 * Sh::kGroups);
+    mbar_init(&bars->ds_ready, 4 * Sh::kGroups);
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -267,14 +305,21 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
         if (!bwd_wait(&bars->qd_empty[slot], ph ^ 1u, abort)) break;
         const int h = kvh * p.group + it / i_cnt;
-        const int tok = seq_start + (i_begin + it % i_cnt) * 128;
+        const int q0 = (i_begin + it % i_cnt) * 128;
+        const int tok = seq_start + q0;
         uint8_t* dst = smem + Sh::kOffQ + slot * 2 * Sh::kTileBytes;
-        mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kTileBytes);
+        uint8_t* vdst = smem + Sh::kOffVec + slot * Sh::kVecBytes;
+        const size_t vi = vec_index(p, h, b, seq_start, q0);
+        mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kTileBytes + Sh::kVecBytes);
         for (int c = 0; c < Sh::kChunks; ++c) {
           tma_load_3d(&tm_q, &bars->qd_full[slot], dst + c * Sh::kChunkBytes, c * 64, h, tok);
           tma_load_3d(&tm_do, &bars->qd_full[slot], dst + Sh::kTileBytes + c * Sh::kChunkBytes,
                       c * 64, h, tok);
         }
+        // the rows' vectors (rows past the sequence end hold stale values;
+        // the compute groups mask those columns)
+        bulk_load(vdst, p.vec_nlse + vi, 512, &bars->qd_full[slot]);
+        bulk_load(vdst + 512, p.vec_drow + vi, 512, &bars->qd_full[slot]);
       }
       for (int f = max(0, it - 2); f < it; ++f)
         mbar_wait(&bars->qd_full[f & 1], static_cast<uint32_t>(f >> 1) & 1u);
@@ -324,13 +369,13 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t sQ = q_addr(it);
         const uint32_t sDO = sQ + Sh::kTileBytes;
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
-        // dV += P^T dO (A = P^T from TMEM region A: queries [64g, 64g+64) are
-        // packed into columns [64g, 64g+32), 16 queries = 8 columns per step)
+        // dV += P^T dO (A = P^T from TMEM region A: queries [32c, 32c+32) are
+        // packed into columns [32c, 32c+16), 16 queries = 8 columns per step)
         if (!(ok = bwd_wait(&bars->p_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 2) * 64 + (kk & 3) * 8,
+          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 1) * 32 + (kk & 1) * 8,
                   mnmajor(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
         // next S^T into region A: P^T of this item has been consumed in order
         const bool more = it + 1 < n_items;
@@ -347,7 +392,7 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + (kk >> 2) * 64 + (kk & 3) * 8,
+          umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + (kk >> 1) * 32 + (kk & 1) * 8,
                   mnmajor(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
         umma_commit(&bars->qd_empty[slot]);
         // next dP^T into region B: dK (the reader of dS^T there) precedes it
@@ -368,74 +413,57 @@ __global__ void __launch_bounds__(320, 1)
     const int lane_base = 32 * (warp & 3);
     const int r = lane_base + lane;             // key row within the tile
     const int key = k0 + r;
-    const int gt = static_cast<int>(threadIdx.x) - 64 - 128 * g;  // 0..127 in the group
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
-    const uint32_t t_a = tmem + lane_off + Sh::kColA;
-    const uint32_t t_b = tmem + lane_off + Sh::kColB;
-    float* glse = vec_lse + 64 * g;
-    float* gdrow = vec_drow + 64 * g;
-    const uint32_t bar_id = 2u + static_cast<uint32_t>(g);
-    // the group's query-row vectors of item `it` (threads 0..63: LSE in the
-    // exp2 domain; 64..127: Drow), loaded one item ahead
-    auto load_vec = [&](int it) -> float {
-      float v = gt < 64 ? INFINITY : 0.f;
-      if (it < n_items) {
-        const int h = kvh * p.group + it / i_cnt;
-        const int qi = (i_begin + it % i_cnt) * 128 + 64 * g + (gt & 63);
-        if (qi < seq_len) {
-          const size_t li = p.cu_seqlens != nullptr
-                                ? static_cast<size_t>(h) * p.total + seq_start + qi
-                                : (static_cast<size_t>(b) * p.Hq + h) * p.S + qi;
-          if (gt < 64) {
-            const float l = p.lse[li];
-            v = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-          } else {
-            v = p.drow[li];
-          }
-        }
-      }
-      return v;
-    };
-    float nv = load_vec(0);
+    // this group's 32 query columns of S^T / dP^T, and the 16 columns its
+    // P^T / dS^T (16-bit pairs) overwrite: only columns it has read itself
+    const uint32_t t_a = tmem + lane_off + Sh::kColA + 32 * g;
+    const uint32_t t_b = tmem + lane_off + Sh::kColB + 32 * g;
     bool ok = true;
     for (int it = 0; it < n_items; ++it) {
       const int i0 = (i_begin + it % i_cnt) * 128;
-      named_bar_sync(bar_id, 128);  // the group is done with the previous vectors
-      if (gt < 64)
-        glse[gt] = nv;
-      else
-        gdrow[gt - 64] = nv;
-      named_bar_sync(bar_id, 128);
-      nv = load_vec(it + 1);
+      // the group's 32 query columns of -LSE and Drow, bulk-loaded with the
+      // item's Q/dO into its slot (the slot is refilled only after dK of this
+      // item, which waits for this group's dS pass)
+      const int slot = it & 1;
+      const float* glse = reinterpret_cast<const float*>(smem + Sh::kOffVec + slot * Sh::kVecBytes) + 32 * g;
+      const float* gdrow = glse + 128;
+      // w first holds the 32 columns' -LSE, loaded while S^T is computed
+      // (shared-memory loads are slow while the tensor core reads its
+      // operands), then P (* (1 - tanh^2)) for the dS pass
+      float w[32];
+      if (!(ok = bwd_wait(&bars->qd_full[slot], static_cast<uint32_t>(it >> 1) & 1u, abort))) break;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(glse + 4 * j4);
+        w[4 * j4] = l4.x;
+        w[4 * j4 + 1] = l4.y;
+        w[4 * j4 + 2] = l4.z;
+        w[4 * j4 + 3] = l4.w;
+      }
       if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
       tc_fence_after();
-      // does any (key, query) of this warp's 32 keys x the group's 64 queries need masking?
+      // does any (key, query) of this warp's 32 keys x the group's 32 queries need masking?
       const int kw_lo = k0 + lane_base, kw_hi = kw_lo + 31;
-      const int qg_lo = i0 + 64 * g, qg_hi = qg_lo + 63;
+      const int qg_lo = i0 + 32 * g, qg_hi = qg_lo + 31;
       bool need_mask = (kw_hi >= seq_len) || (qg_hi >= seq_len);
       if (p.wr >= 0) need_mask |= (kw_hi > qg_lo + p.wr);
       if (p.wl >= 0) need_mask |= (kw_lo < qg_hi - p.wl);
-      // pass 1: P^T from S^T (32 queries per chunk) -> TMEM; keep
-      // w = P * scale (* (1 - tanh^2) under softcap) for the dS pass
-      float w[64];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * g + cc;       // chunk index within the 128 queries
+      // pass 1: P^T from S^T -> TMEM; keep w = P (* (1 - tanh^2) under
+      // softcap) for the dS pass
+      {
         uint32_t sr[32];
-        tmem_ld32(t_a + c * 32, sr);
+        tmem_ld32(t_a, sr);
         tmem_ld_wait();
         const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
         uint32_t pk[16];
-        float4 l4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
-          const int jl = cc * 32 + 2 * j2;  // query within the group
-          if ((j2 & 1) == 0) l4 = *reinterpret_cast<const float4*>(glse + jl);
+          const int jl = 2 * j2;  // query within the group
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
-          const float2 l2 = (j2 & 1) == 0 ? make_float2(l4.x, l4.y) : make_float2(l4.z, l4.w);
+          const float2 nl2 = make_float2(w[jl], w[jl + 1]);
           float2 x, fac;
-          bwd_logit2<kCap>(s2, poly, p, x, fac);
-          float2 pr = make_float2(ex2_approx(x.x - l2.x), ex2_approx(x.y - l2.y));
+          bwd_logit2<kCap>(s2, poly, p, nl2, x, fac);
+          float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           if (need_mask) {
             const int q0i = qg_lo + jl;
             bool v0 = key < seq_len && q0i < seq_len;
@@ -451,14 +479,12 @@ __global__ void __launch_bounds__(320, 1)
             pr.x = v0 ? pr.x : 0.f;
             pr.y = v1 ? pr.y : 0.f;
           }
-          pk[j2] = pack2<kBF16>(pr.x, pr.y);
-          const float2 wv = __fmul2_rn(pr, fac);
+          pk[j2] = pack2_alu<kBF16>(pr.x, pr.y);
+          const float2 wv = kCap ? __fmul2_rn(pr, fac) : pr;
           w[jl] = wv.x;
           w[jl + 1] = wv.y;
         }
-        // P^T of queries [32c, 32c+32) -> TMEM region A columns [64g + 16cc, +16):
-        // only columns this group has already read are overwritten
-        tmem_st16(t_a + 64 * g + 16 * cc, pk);
+        tmem_st16(t_a, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -469,29 +495,33 @@ __global__ void __launch_bounds__(320, 1)
       // dS^T columns, precedes the dP^T MMA in issue order)
       if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
       tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * g + cc;
+      {
         uint32_t dr[32];
-        tmem_ld32(t_b + c * 32, dr);
+        tmem_ld32(t_b, dr);
         tmem_ld_wait();
         uint32_t dsk[16];
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
-          const int jl = cc * 32 + 4 * j4;
-          const float4 d4 = *reinterpret_cast<const float4*>(gdrow + jl);
+          const int jl = 4 * j4;
+          float4 d4 = *reinterpret_cast<const float4*>(gdrow + jl);
+          if (need_mask) {
+            // rows past the sequence end: the slot holds stale values (w = 0)
+            const int q4 = qg_lo + jl;
+            d4.x = q4 < seq_len ? d4.x : 0.f;
+            d4.y = q4 + 1 < seq_len ? d4.y : 0.f;
+            d4.z = q4 + 2 < seq_len ? d4.z : 0.f;
+            d4.w = q4 + 3 < seq_len ? d4.w : 0.f;
+          }
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int j2 = 2 * j4 + h2;
             const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
             const float2 d2 = h2 == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
             const float2 ds = __fmul2_rn(__fadd2_rn(dp2, d2), make_float2(w[jl + 2 * h2], w[jl + 2 * h2 + 1]));
-            dsk[j2] = pack2<kBF16>(ds.x, ds.y);
+            dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
           }
         }
-        // dS^T of queries [32c, 32c+32) -> region B columns [64g + 16cc, +16)
-        // (dP^T columns this group has already read)
-        tmem_st16(t_b + 64 * g + 16 * cc, dsk);
+        tmem_st16(t_b, dsk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -499,23 +529,29 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive(&bars->ds_ready);
     }
 
-    // ---- epilogue: group 0 writes the dV rows, group 1 the dK rows ----
+    // ---- epilogue: groups 0, 1 write the two column halves of the dV rows,
+    // groups 2, 3 those of the dK rows ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
-    void* outp = g == 0 ? p.dv : p.dk;
-    const uint32_t col = g == 0 ? Sh::kColDV : Sh::kColDK;
+    const bool is_dk = g >= Sh::kGroups / 2;
+    void* outp = is_dk ? p.dk : p.dv;
+    const uint32_t col = is_dk ? Sh::kColDK : Sh::kColDV;
+    const float osc = is_dk ? p.scale : 1.f;  // dK = scale * dS^T Q
+    constexpr int kHalfChunks = kD / 64;      // 32-column chunks per half row
+    const int c_begin = (g & 1) * kHalfChunks;
     uint8_t* dst = static_cast<uint8_t*>(outp) + (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
     if (ok && n_items > 0) {
       // every lane loads (the TMEM load is warp-collective); only rows of
       // the sequence are stored
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = c_begin; c < c_begin + kHalfChunks; ++c) {
         uint32_t rr[32];
         tmem_ld32(tmem + lane_off + col + c * 32, rr);
         tmem_ld_wait();
         uint32_t wv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+        for (int i = 0; i < 16; ++i)
+          wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]) * osc, __uint_as_float(rr[2 * i + 1]) * osc);
         if (key < seq_len) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
 #pragma unroll
@@ -523,8 +559,8 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     } else if (ok && key < seq_len) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst);
-      for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c_begin * 64);
+      for (int i = 0; i < kHalfChunks * 4; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   tc_fence_before();
@@ -765,16 +801,14 @@ __global__ void __launch_bounds__(320, 1)
     const int r = lane_base + lane;          // query row within the tile
     const int qrow = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
-    // the row's LSE (exp2 domain) and Drow
-    float lse2 = INFINITY, drow = 0.f;
+    // the row's -LSE (exp2 domain) and Drow
+    float nlse = -INFINITY, drow = 0.f;
     if (qrow < seq_len) {
-      const size_t li = p.cu_seqlens != nullptr ? static_cast<size_t>(h) * p.total + seq_start + qrow
-                                                : (static_cast<size_t>(b) * p.Hq + h) * p.S + qrow;
-      const float l = p.lse[li];
-      lse2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-      drow = p.drow[li];
+      const size_t vi = vec_index(p, h, b, seq_start, qrow);
+      nlse = p.vec_nlse[vi];
+      drow = p.vec_drow[vi];
     }
-    const float2 nl2 = make_float2(-lse2, -lse2);
+    const float2 nl2 = make_float2(nlse, nlse);
     const float2 nd2 = make_float2(-drow, -drow);
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -788,8 +822,8 @@ __global__ void __launch_bounds__(320, 1)
       bool need_mask = (k0 + 63 >= seq_len) || (r_hi >= seq_len);
       if (p.wr >= 0) need_mask |= (k0 + 63 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
-      // pass 1 (needs S_j only): w = P * scale (* (1 - tanh^2)) for the
-      // group's 64 keys, kept in registers
+      // pass 1 (needs S_j only): w = P (* (1 - tanh^2)) for the group's 64
+      // keys, kept in registers
       float w[64];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {  // 32 keys per chunk
@@ -801,9 +835,8 @@ __global__ void __launch_bounds__(320, 1)
         for (int j2 = 0; j2 < 16; ++j2) {
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
           float2 x, fac;
-          bwd_logit2<kCap>(s2, poly, p, x, fac);
-          const float2 arg = __fadd2_rn(x, nl2);
-          float2 pr = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+          bwd_logit2<kCap>(s2, poly, p, nl2, x, fac);
+          float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           if (need_mask) {
             const int kj = k0 + 32 * cc + 2 * j2;
             bool v0 = qrow < seq_len && kj < seq_len;
@@ -819,7 +852,7 @@ __global__ void __launch_bounds__(320, 1)
             pr.x = v0 ? pr.x : 0.f;
             pr.y = v1 ? pr.y : 0.f;
           }
-          const float2 wv = __fmul2_rn(pr, fac);
+          const float2 wv = kCap ? __fmul2_rn(pr, fac) : pr;
           w[32 * cc + 2 * j2] = wv.x;
           w[32 * cc + 2 * j2 + 1] = wv.y;
         }
@@ -838,7 +871,7 @@ __global__ void __launch_bounds__(320, 1)
           const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
           const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2),
                                        make_float2(w[32 * cc + 2 * j2], w[32 * cc + 2 * j2 + 1]));
-          dsk[j2] = pack2<kBF16>(ds.x, ds.y);
+          dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
         }
         // dS of keys [k0 + 32cc, +32) -> columns [64g + 16cc, +16) of the
         // S buffer (columns this group has already read)
@@ -861,7 +894,8 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait();
         uint32_t wv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+        for (int i = 0; i < 16; ++i)
+          wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]) * p.scale, __uint_as_float(rr[2 * i + 1]) * p.scale);
         if (qrow < seq_len) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
 #pragma unroll

@@ -161,29 +161,15 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
-// Element-wise add of a shared-memory tile into global memory through a
-// tensor map (the add is atomic per element at L2). Commit and wait are per
-// issuing thread.
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int c0,
-                                                  int c1, int c2) {
+// Untiled bulk copy of `bytes` from global to this CTA's shared memory,
+// completing on `bar` (no multicast). Both addresses 16-byte aligned, bytes
+// a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
-      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// wait until at most N committed bulk groups still read shared memory
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-// wait until at most N committed bulk groups are incomplete
-template <int N>
-__device__ __forceinline__ void bulk_wait() {
-  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -365,6 +351,25 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   } else {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+// Two finite floats -> packed 16-bit pair like pack2, but for bf16 on the
+// integer pipe: add half a bf16 ulp (0x8000) to each bit pattern and keep the
+// high halves (one prmt). That rounds half away from zero instead of to even:
+// the same half-ulp error bound, different only on exact ties. The
+// conversion instruction shares its unit with ex2, which the softmax keeps
+// busy; fp16 keeps the conversion.
+template <bool kBF16>
+__device__ __forceinline__ uint32_t pack2_alu(float lo, float hi) {
+  if constexpr (kBF16) {
+    const uint32_t a = __float_as_uint(lo) + 0x8000u;
+    const uint32_t b = __float_as_uint(hi) + 0x8000u;
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  } else {
+    return pack2<false>(lo, hi);
   }
 }
 

@@ -82,9 +82,11 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, 
                  fa_dtype dtype, void* stream);
 
 /*
- * Workspace bytes needed by fa_bwd for these sizes (the float32 per-row
- * dot(dO, O), one per token and query head); total_tokens as in fa_fwd
- * (ignored if <= 0).
+ * Workspace bytes needed by fa_bwd for these sizes: two float32 values per
+ * token and query head (the row's dot(dO, O) and its LSE in the exp2
+ * domain), each sequence's rows padded to a multiple of 128, i.e.
+ * 2 * Hq * 128 * (T / 128 + B + 1) * 4 bytes with T = B * S or total_tokens;
+ * total_tokens as in fa_fwd (ignored if <= 0).
  */
 FA_API size_t fa_bwd_workspace_size(int B, int Hq, int S, int D, int total_tokens);
 

@@ -56,10 +56,11 @@ def test_version(fa):
 
 
 def test_workspace_sizes(fa):
-    # row dots rowsum(dO * O): float32 per (token, query head), padded to 256 B
+    # -LSE and rowsum(dO * O): two float32 vectors per query head, each row
+    # of a sequence in a padded layout of 128 * (T / 128 + B + 1) rows per head
     n = fa.fa_bwd_workspace_size(2, 32, 8192, 128)
-    assert n == 2 * 8192 * 32 * 4
-    assert fa.fa_bwd_workspace_size(3, 4, 0, 128, 1000) == 16128
+    assert n == 2 * 32 * 128 * (16384 // 128 + 2 + 1) * 4
+    assert fa.fa_bwd_workspace_size(3, 4, 0, 128, 1000) == 2 * 4 * 128 * (1000 // 128 + 3 + 1) * 4
     # kv-cache: float32 split partials (O and LSE per split and output row),
     # padded to 256 B, then the rotated queries in the 16-bit input type
     assert fa.fa_kvcache_workspace_size(64, 1, 32, 128, 1) == 0
