@@ -23,23 +23,24 @@
 // for no dQ reduction across CTAs and a pipeline with no write-back on the
 // critical path.
 //
-// bwd_dkdv warp roles (576 threads):
+// bwd_dkdv warp roles (576 threads); an item is one (query head, 64-row
+// query block) against the CTA's 128 keys:
 //   warp 0      TMA producer: K, V once; Q_i, dO_i and the rows' -LSE and Drow
-//               into a 2-slot ring.
+//               into a 4-slot ring.
 //   warp 1      MMA issuer (one lane), TMEM owner.
-//   warps 2-17  four compute groups; group g owns query columns [32g, 32g+32):
-//               one thread per key row computes P^T = exp(S^T - LSE) and then
-//               dS^T = P^T * (dP^T - Drow), each written back to TMEM as 16-bit
-//               pairs over the first half of the columns it came from, where
-//               the dV and dK MMAs read their A operand. Four warps per SM
-//               sub-partition hide the latency of the exponentials and of the
-//               TMEM round trips. At the end groups 0-1 write dV, 2-3 dK.
-// TMEM columns: A [0,128) S^T then P^T; B [128,256) dP^T then dS^T (queries
-// [32g, 32g+32) packed into [32g, 32g+16) of each); dV [256, 256+D);
-// dK [256+D, 256+2D).
-// MMA order per item i: dV_i, S_{i+1}, dK_i, dP_{i+1}. S^T and dP^T signal
-// separately, so the P pass of item i+1 overlaps dK_i and dP_{i+1}, and the
-// dS pass of item i overlaps dV_i and S_{i+1}.
+//   warps 2-17  two teams of two compute groups; team t takes the items with
+//               i % 2 == t, group g of a team the item's query columns
+//               [32g, 32g+32): one thread per key row computes
+//               P^T = exp(S^T - LSE) and then dS^T = P^T * (dP^T - Drow), each
+//               written back to TMEM as 16-bit pairs over the first half of
+//               the columns it came from, where the dV and dK MMAs read their
+//               A operand. While one team computes, the tensor core runs the
+//               other team's MMAs. At the end warps 2-9 write dV, 10-17 dK.
+// TMEM columns: A_t [64t, 64t+64) S^T then P^T; B_t [128+64t, +64) dP^T then
+// dS^T (queries [32g, 32g+32) packed into [32g, 32g+16) of each);
+// dV [256, 256+D); dK [256+D, 256+2D).
+// MMA order per item i (team t = i % 2): dV_i, S_{i+2} -> A_t, dK_i,
+// dP_{i+2} -> B_t.
 #pragma once
 
 #include "ptx.cuh"
@@ -186,35 +187,39 @@ __device__ __forceinline__ bool poly_ok(const uint32_t (&sr)[32], float cap_in) 
 template <int kD>
 struct DkdvShape {
   static constexpr int kChunks = kD / 64;
-  static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 B
+  static constexpr int kChunkBytes = 128 * 128;        // K/V: 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kQRows = 64;                    // query rows per item
+  static constexpr int kQChunkBytes = kQRows * 128;
+  static constexpr int kQTileBytes = kChunks * kQChunkBytes;
+  static constexpr int kSlots = 4;                     // Q/dO ring
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;         // + slot * 2 * kTileBytes (Q, dO)
-  // per Q/dO slot: -LSE (exp2 domain)[128], Drow[128] of the slot's query rows
-  static constexpr int kOffVec = 6 * kTileBytes;
-  static constexpr int kVecBytes = 1024;
-  static constexpr int kOffBar = kOffVec + 2 * kVecBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;         // + slot * 2 * kQTileBytes (Q, dO)
+  // per slot: -LSE (exp2 domain)[64], Drow[64] of the slot's query rows
+  static constexpr int kOffVec = kOffQ + kSlots * 2 * kQTileBytes;
+  static constexpr int kVecBytes = 512;
+  static constexpr int kOffBar = kOffVec + kSlots * kVecBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  // warp 0 TMA, warp 1 MMA, then kGroups compute groups of 4 warps; group g
-  // owns the 32 query columns [32g, 32g + 32) of every item
-  static constexpr int kGroups = 4;
-  static constexpr int kThreads = 64 + 128 * kGroups;
+  // warp 0 TMA, warp 1 MMA, then two teams of two compute groups (4 warps
+  // each); team t takes the items it with it % 2 == t, group g of a team the
+  // 32 query columns [32g, 32g + 32) of the item
+  static constexpr int kThreads = 64 + 4 * 128;
   static constexpr int kTmemCols = 512;
-  static constexpr int kColA = 0;
-  static constexpr int kColB = 128;
+  static constexpr int kColA = 0;    // + 64 t: team t's S^T, then P^T
+  static constexpr int kColB = 128;  // + 64 t: team t's dP^T, then dS^T
   static constexpr int kColDV = 256;
   static constexpr int kColDK = 256 + kD;
 };
 
 struct DkdvBars {
   uint64_t kv_full;
-  uint64_t qd_full[2];
-  uint64_t qd_empty[2];
-  uint64_t s_ready;
-  uint64_t dp_ready;
-  uint64_t p_ready;
-  uint64_t ds_ready;
+  uint64_t qd_full[4];
+  uint64_t qd_empty[4];
+  uint64_t s_ready[2];   // per team
+  uint64_t dp_ready[2];
+  uint64_t p_ready[2];
+  uint64_t ds_ready[2];
   uint64_t final_done;
   uint64_t drain;
   uint32_t tmem_base;
@@ -251,25 +256,27 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
   }
   const int k0 = kt * 128;
   if (k0 >= seq_len) return;
-  // query rows that can see some key of [k0, k0 + 127]
+  // query rows that can see some key of [k0, k0 + 127], in 64-row blocks
   int q_lo = 0;
   if (p.wr >= 0) q_lo = max(0, k0 - p.wr);
   int q_hi = seq_len - 1;
   if (p.wl >= 0) q_hi = min(q_hi, k0 + 127 + p.wl);
-  const int i_begin = q_lo / 128;
-  const int i_cnt = q_hi >= q_lo ? q_hi / 128 + 1 - i_begin : 0;
-  const int n_items = i_cnt * p.group;  // (head, q tile) pairs
+  const int i_begin = q_lo / Sh::kQRows;
+  const int i_cnt = q_hi >= q_lo ? q_hi / Sh::kQRows + 1 - i_begin : 0;
+  const int n_items = i_cnt * p.group;  // (head, 64-row query block) pairs
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Sh::kSlots; ++s) {
       mbar_init(&bars->qd_full[s], 1);
       mbar_init(&bars->qd_empty[s], 1);
     }
-    mbar_init(&bars->s_ready, 1);
-    mbar_init(&bars->dp_ready, 1);
-    mbar_init(&bars->p_ready, 4 * Sh::kGroups);
-    mbar_init(&bars->ds_ready, 4 * Sh::kGroups);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_ready[t], 1);
+      mbar_init(&bars->dp_ready[t], 1);
+      mbar_init(&bars->p_ready[t], 8);
+      mbar_init(&bars->ds_ready[t], 8);
+    }
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -301,106 +308,116 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       }
       int it = 0;
       for (; it < n_items && !*abort; ++it) {
-        const int slot = it & 1;
-        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+        const int slot = it % Sh::kSlots;
+        const uint32_t ph = static_cast<uint32_t>(it / Sh::kSlots) & 1u;
         if (!bwd_wait(&bars->qd_empty[slot], ph ^ 1u, abort)) break;
         const int h = kvh * p.group + it / i_cnt;
-        const int q0 = (i_begin + it % i_cnt) * 128;
+        const int q0 = (i_begin + it % i_cnt) * Sh::kQRows;
         const int tok = seq_start + q0;
-        uint8_t* dst = smem + Sh::kOffQ + slot * 2 * Sh::kTileBytes;
+        uint8_t* dst = smem + Sh::kOffQ + slot * 2 * Sh::kQTileBytes;
         uint8_t* vdst = smem + Sh::kOffVec + slot * Sh::kVecBytes;
         const size_t vi = vec_index(p, h, b, seq_start, q0);
-        mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kTileBytes + Sh::kVecBytes);
+        mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kQTileBytes + Sh::kVecBytes);
         for (int c = 0; c < Sh::kChunks; ++c) {
-          tma_load_3d(&tm_q, &bars->qd_full[slot], dst + c * Sh::kChunkBytes, c * 64, h, tok);
-          tma_load_3d(&tm_do, &bars->qd_full[slot], dst + Sh::kTileBytes + c * Sh::kChunkBytes,
+          tma_load_3d(&tm_q, &bars->qd_full[slot], dst + c * Sh::kQChunkBytes, c * 64, h, tok);
+          tma_load_3d(&tm_do, &bars->qd_full[slot], dst + Sh::kQTileBytes + c * Sh::kQChunkBytes,
                       c * 64, h, tok);
         }
         // the rows' vectors (rows past the sequence end hold stale values;
         // the compute groups mask those columns)
-        bulk_load(vdst, p.vec_nlse + vi, 512, &bars->qd_full[slot]);
-        bulk_load(vdst + 512, p.vec_drow + vi, 512, &bars->qd_full[slot]);
+        bulk_load(vdst, p.vec_nlse + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
+        bulk_load(vdst + Sh::kVecBytes / 2, p.vec_drow + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
       }
-      for (int f = max(0, it - 2); f < it; ++f)
-        mbar_wait(&bars->qd_full[f & 1], static_cast<uint32_t>(f >> 1) & 1u);
+      for (int f = max(0, it - Sh::kSlots); f < it; ++f)
+        mbar_wait(&bars->qd_full[f % Sh::kSlots], static_cast<uint32_t>(f / Sh::kSlots) & 1u);
       mbar_wait(&bars->kv_full, 0);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
+    // Issue order per item i (team t = i % 2, regions A_t, B_t):
+    //   dV_i (after the P pass of i), S_{i+2} -> A_t, dK_i (after the dS pass
+    //   of i), dP_{i+2} -> B_t.
+    // S_{i+2} overwrites A_t only after dV_i, its last reader, in issue
+    // order; dP_{i+2} overwrites B_t after dK_i. The other team's item i+1
+    // is in its P or dS pass meanwhile, so the tensor core has work while
+    // each team computes. The order is fixed, so the sums are deterministic.
     if (elect_one()) {
-      constexpr uint32_t id_s = idesc_f16(kBF16, 128, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t id_dv = idesc_f16(kBF16, 128, kD, false, true);    // P^T (tmem) x dO
-      constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);    // dS^T (tmem) x Q
+      constexpr uint32_t id_s = idesc_f16(kBF16, 128, Sh::kQRows, false, false);  // S^T, dP^T
+      constexpr uint32_t id_dv = idesc_f16(kBF16, 128, kD, false, true);          // P^T (tmem) x dO
+      constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);          // dS^T (tmem) x Q
       const uint32_t sK = smem_u32(smem + Sh::kOffK);
       const uint32_t sV = smem_u32(smem + Sh::kOffV);
       bool ok = bwd_wait(&bars->kv_full, 0, abort);
       tc_fence_after();
-      auto kmajor = [](uint32_t base, int kk) {
+      auto kmajor_kv = [](uint32_t base, int kk) {
         return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
       };
-      auto mnmajor = [](uint32_t base, int kk) {
-        return sdesc_sw128(base + kk * 2048, Sh::kChunkBytes, 1024);
+      auto kmajor_q = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + (kk >> 2) * Sh::kQChunkBytes + (kk & 3) * 32, 16, 1024);
       };
-      auto q_addr = [&](int it) { return smem_u32(smem + Sh::kOffQ + (it & 1) * 2 * Sh::kTileBytes); };
-      auto issue_s = [&](int it) {  // S^T = K Q^T -> region A
+      auto mnmajor_q = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + kk * 2048, Sh::kQChunkBytes, 1024);
+      };
+      auto q_addr = [&](int it) {
+        return smem_u32(smem + Sh::kOffQ + (it % Sh::kSlots) * 2 * Sh::kQTileBytes);
+      };
+      auto wait_q = [&](int it) {
+        const bool r = bwd_wait(&bars->qd_full[it % Sh::kSlots],
+                                static_cast<uint32_t>(it / Sh::kSlots) & 1u, abort);
+        tc_fence_after();
+        return r;
+      };
+      auto issue_s = [&](int it) {  // S^T = K Q^T -> region A of the item's team
         const uint32_t sQ = q_addr(it);
+        const uint32_t d = tmem + Sh::kColA + 64 * (it & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ss(tmem + Sh::kColA, kmajor(sK, kk), kmajor(sQ, kk), id_s, kk > 0 ? 1u : 0u);
+          umma_ss(d, kmajor_kv(sK, kk), kmajor_q(sQ, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_ready[it & 1]);
       };
-      auto issue_dp = [&](int it) {  // dP^T = V dO^T -> region B
-        const uint32_t sDO = q_addr(it) + Sh::kTileBytes;
+      auto issue_dp = [&](int it) {  // dP^T = V dO^T -> region B of the item's team
+        const uint32_t sDO = q_addr(it) + Sh::kQTileBytes;
+        const uint32_t d = tmem + Sh::kColB + 64 * (it & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ss(tmem + Sh::kColB, kmajor(sV, kk), kmajor(sDO, kk), id_s, kk > 0 ? 1u : 0u);
+          umma_ss(d, kmajor_kv(sV, kk), kmajor_q(sDO, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->dp_ready[it & 1]);
       };
-      if (ok && n_items > 0) {
-        if ((ok = bwd_wait(&bars->qd_full[0], 0, abort))) {
-          tc_fence_after();
-          issue_s(0);
-          umma_commit(&bars->s_ready);
-          issue_dp(0);
-          umma_commit(&bars->dp_ready);
+      for (int it = 0; it < 2 && it < n_items && ok; ++it) {
+        if ((ok = wait_q(it))) {
+          issue_s(it);
+          issue_dp(it);
         }
       }
       for (int it = 0; it < n_items && ok; ++it) {
-        const int slot = it & 1;
+        const int t = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
         const uint32_t sQ = q_addr(it);
-        const uint32_t sDO = sQ + Sh::kTileBytes;
+        const uint32_t sDO = sQ + Sh::kQTileBytes;
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
-        // dV += P^T dO (A = P^T from TMEM region A: queries [32c, 32c+32) are
+        // dV += P^T dO: A = P^T of the team's region (queries [32c, 32c+32)
         // packed into columns [32c, 32c+16), 16 queries = 8 columns per step)
-        if (!(ok = bwd_wait(&bars->p_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+        if (!(ok = bwd_wait(&bars->p_ready[t], ph, abort))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + (kk >> 1) * 32 + (kk & 1) * 8,
-                  mnmajor(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
-        // next S^T into region A: P^T of this item has been consumed in order
-        const bool more = it + 1 < n_items;
+        for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
+          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + 64 * t + (kk >> 1) * 32 + (kk & 1) * 8,
+                  mnmajor_q(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
+        const bool more = it + 2 < n_items;
         if (more) {
-          if (!(ok = bwd_wait(&bars->qd_full[(it + 1) & 1], static_cast<uint32_t>((it + 1) >> 1) & 1u,
-                              abort)))
-            break;
-          tc_fence_after();
-          issue_s(it + 1);
-          umma_commit(&bars->s_ready);  // the next P pass can start now
+          if (!(ok = wait_q(it + 2))) break;
+          issue_s(it + 2);
         }
-        // dK += dS^T Q (A = dS^T from TMEM region B, packed like P^T)
-        if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+        // dK += dS^T Q: A = dS^T of the team's region B, packed like P^T
+        if (!(ok = bwd_wait(&bars->ds_ready[t], ph, abort))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + (kk >> 1) * 32 + (kk & 1) * 8,
-                  mnmajor(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
-        umma_commit(&bars->qd_empty[slot]);
-        // next dP^T into region B: dK (the reader of dS^T there) precedes it
-        // in issue order, and dp_ready completes after both.
-        if (more) {
-          issue_dp(it + 1);
-          umma_commit(&bars->dp_ready);
-        }
+        for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
+          umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + 64 * t + (kk >> 1) * 32 + (kk & 1) * 8,
+                  mnmajor_q(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
+        umma_commit(&bars->qd_empty[it % Sh::kSlots]);
+        if (more) issue_dp(it + 2);
       }
       umma_commit(&bars->final_done);
       umma_commit(&bars->drain);
@@ -408,30 +425,33 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ======================= compute groups =======================
-    const int g = (warp - 2) >> 2;
+    // ======================= compute teams =======================
+    const int team = (warp - 2) >> 3;
+    const int g = ((warp - 2) >> 2) & 1;       // group within the team
     const int lane_base = 32 * (warp & 3);
     const int r = lane_base + lane;             // key row within the tile
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
-    // this group's 32 query columns of S^T / dP^T, and the 16 columns its
-    // P^T / dS^T (16-bit pairs) overwrite: only columns it has read itself
-    const uint32_t t_a = tmem + lane_off + Sh::kColA + 32 * g;
-    const uint32_t t_b = tmem + lane_off + Sh::kColB + 32 * g;
+    // this group's 32 query columns of the team's S^T / dP^T, and the 16
+    // columns its P^T / dS^T (16-bit pairs) overwrite: only columns it has
+    // read itself
+    const uint32_t t_a = tmem + lane_off + Sh::kColA + 64 * team + 32 * g;
+    const uint32_t t_b = tmem + lane_off + Sh::kColB + 64 * team + 32 * g;
     bool ok = true;
-    for (int it = 0; it < n_items; ++it) {
-      const int i0 = (i_begin + it % i_cnt) * 128;
+    for (int it = team; it < n_items; it += 2) {
+      const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
+      const int q0 = (i_begin + it % i_cnt) * Sh::kQRows;
       // the group's 32 query columns of -LSE and Drow, bulk-loaded with the
       // item's Q/dO into its slot (the slot is refilled only after dK of this
-      // item, which waits for this group's dS pass)
-      const int slot = it & 1;
+      // item, which waits for this team's dS pass)
+      const int slot = it % Sh::kSlots;
       const float* glse = reinterpret_cast<const float*>(smem + Sh::kOffVec + slot * Sh::kVecBytes) + 32 * g;
-      const float* gdrow = glse + 128;
-      // w first holds the 32 columns' -LSE, loaded while S^T is computed
+      const float* gdrow = glse + Sh::kQRows;
+      // w first holds the 32 columns' -LSE, loaded before S^T is ready
       // (shared-memory loads are slow while the tensor core reads its
       // operands), then P (* (1 - tanh^2)) for the dS pass
       float w[32];
-      if (!(ok = bwd_wait(&bars->qd_full[slot], static_cast<uint32_t>(it >> 1) & 1u, abort))) break;
+      if (!(ok = bwd_wait(&bars->qd_full[slot], static_cast<uint32_t>(it / Sh::kSlots) & 1u, abort))) break;
 #pragma unroll
       for (int j4 = 0; j4 < 8; ++j4) {
         const float4 l4 = *reinterpret_cast<const float4*>(glse + 4 * j4);
@@ -440,11 +460,11 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
         w[4 * j4 + 2] = l4.z;
         w[4 * j4 + 3] = l4.w;
       }
-      if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+      if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort))) break;
       tc_fence_after();
       // does any (key, query) of this warp's 32 keys x the group's 32 queries need masking?
       const int kw_lo = k0 + lane_base, kw_hi = kw_lo + 31;
-      const int qg_lo = i0 + 32 * g, qg_hi = qg_lo + 31;
+      const int qg_lo = q0 + 32 * g, qg_hi = qg_lo + 31;
       bool need_mask = (kw_hi >= seq_len) || (qg_hi >= seq_len);
       if (p.wr >= 0) need_mask |= (kw_hi > qg_lo + p.wr);
       if (p.wl >= 0) need_mask |= (kw_lo < qg_hi - p.wl);
@@ -489,11 +509,11 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_ready);  // dV may start
+      if (lane == 0) mbar_arrive(&bars->p_ready[team]);  // dV may start
       // pass 2: dS^T = w * (dP^T - Drow) -> TMEM region B (the dK operand),
-      // once dP^T is in TMEM (dK of the previous item, the last reader of the
-      // dS^T columns, precedes the dP^T MMA in issue order)
-      if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(it) & 1u, abort))) break;
+      // once dP^T is in TMEM (dK two items back, the last reader of these
+      // columns, precedes the dP^T MMA in issue order)
+      if (!(ok = bwd_wait(&bars->dp_ready[team], ph, abort))) break;
       tc_fence_after();
       {
         uint32_t dr[32];
@@ -526,19 +546,20 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ds_ready);
+      if (lane == 0) mbar_arrive(&bars->ds_ready[team]);
     }
 
-    // ---- epilogue: groups 0, 1 write the two column halves of the dV rows,
-    // groups 2, 3 those of the dK rows ----
+    // ---- epilogue: the four groups write the two column halves of the dV
+    // rows (warps 2-9) and of the dK rows (warps 10-17) ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
-    const bool is_dk = g >= Sh::kGroups / 2;
+    const int e = (warp - 2) >> 2;
+    const bool is_dk = e >= 2;
     void* outp = is_dk ? p.dk : p.dv;
     const uint32_t col = is_dk ? Sh::kColDK : Sh::kColDV;
     const float osc = is_dk ? p.scale : 1.f;  // dK = scale * dS^T Q
     constexpr int kHalfChunks = kD / 64;      // 32-column chunks per half row
-    const int c_begin = (g & 1) * kHalfChunks;
+    const int c_begin = (e & 1) * kHalfChunks;
     uint8_t* dst = static_cast<uint8_t*>(outp) + (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
     if (ok && n_items > 0) {
       // every lane loads (the TMEM load is warp-collective); only rows of
