@@ -600,10 +600,11 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
 //   warp 0     TMA producer: Q, dO once; K_j, V_j into a ring of slots.
 //   warp 1     MMA issuer: S_j = Q K_j^T (two TMEM buffers, alternating),
 //              dP_j = dO V_j^T, then dQ += dS_j K_j with dS_j read from TMEM.
-//   warps 2-9  two compute groups, one thread per query row; group g owns key
-//              columns [64g, 64g+64) of S_j and dP_j and writes dS_j (16-bit)
-//              over the S columns it has read. LSE and Drow of the row live in
-//              registers.
+//   warps 2-17 four compute groups, one thread per query row; group g owns
+//              key columns [32g, 32g+32) of S_j and dP_j and writes dS_j
+//              (16-bit pairs) over the first half of the S columns it has
+//              read. LSE and Drow of the row live in registers. Four warps
+//              per SM sub-partition hide the latency of the exponentials.
 // TMEM columns: S buffers [0,128) and [128,256), dP [256,384), dQ [384, 384+D).
 // MMA order per tile j: S_{j+1}, dQ_j, dP_{j+1}. S and dP signal separately:
 // the compute groups form P_{j+1} (needs S only) while the tensor core runs
@@ -619,7 +620,8 @@ struct DqShape {
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  static constexpr int kThreads = 320;
+  static constexpr int kGroups = 4;
+  static constexpr int kThreads = 64 + 128 * kGroups;
   static constexpr int kTmemCols = 512;
   static constexpr int kColS = 0;      // + 128 * buffer
   static constexpr int kColDP = 256;
@@ -640,7 +642,7 @@ struct DqBars {
 };
 
 template <int kD, bool kBF16, bool kCap>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p) {
@@ -686,7 +688,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(&bars->s_ready, 1);
     mbar_init(&bars->dp_ready, 1);
-    mbar_init(&bars->ds_ready, 8);
+    mbar_init(&bars->ds_ready, 4 * Sh::kGroups);
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -789,14 +791,14 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
         tc_fence_after();
-        // dQ += dS_j K_j: A = dS_j from TMEM (keys [64g, 64g+64) packed into
-        // columns [64g, 64g+32) of buffer j & 1), B = K_j with N = D (MN-major)
+        // dQ += dS_j K_j: A = dS_j from TMEM (keys [32c, 32c+32) packed into
+        // columns [32c, 32c+16) of buffer j & 1), B = K_j with N = D (MN-major)
         {
           const uint32_t sK = slot_addr(2 * j);
           const uint32_t a = tmem + Sh::kColS + 128 * (j & 1);
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
-            umma_ts(tmem + Sh::kColDQ, a + (kk >> 2) * 64 + (kk & 3) * 8,
+            umma_ts(tmem + Sh::kColDQ, a + (kk >> 1) * 32 + (kk & 1) * 8,
                     sdesc_sw128(sK + kk * 2048, Sh::kChunkBytes, 1024), id_dq,
                     (j == 0 && kk == 0) ? 0u : 1u);
         }
@@ -835,21 +837,20 @@ __global__ void __launch_bounds__(320, 1)
     for (int j = 0; j < n_tiles; ++j) {
       if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
       tc_fence_after();
-      const int k0 = (n_begin + j) * 128 + 64 * g;  // first key of this group's columns
-      const uint32_t t_s = tmem + lane_off + Sh::kColS + 128 * (j & 1) + 64 * g;
-      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 64 * g;
-      // mask needed for this warp's 32 rows x the group's 64 keys?
+      const int k0 = (n_begin + j) * 128 + 32 * g;  // first key of this group's columns
+      const uint32_t t_s = tmem + lane_off + Sh::kColS + 128 * (j & 1) + 32 * g;
+      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 32 * g;
+      // mask needed for this warp's 32 rows x the group's 32 keys?
       const int r_lo = q0 + lane_base, r_hi = r_lo + 31;
-      bool need_mask = (k0 + 63 >= seq_len) || (r_hi >= seq_len);
-      if (p.wr >= 0) need_mask |= (k0 + 63 > r_lo + p.wr);
+      bool need_mask = (k0 + 31 >= seq_len) || (r_hi >= seq_len);
+      if (p.wr >= 0) need_mask |= (k0 + 31 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
-      // pass 1 (needs S_j only): w = P (* (1 - tanh^2)) for the group's 64
+      // pass 1 (needs S_j only): w = P (* (1 - tanh^2)) for the group's 32
       // keys, kept in registers
-      float w[64];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {  // 32 keys per chunk
+      float w[32];
+      {
         uint32_t sr[32];
-        tmem_ld32(t_s + 32 * cc, sr);
+        tmem_ld32(t_s, sr);
         tmem_ld_wait();
         const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
 #pragma unroll
@@ -859,7 +860,7 @@ __global__ void __launch_bounds__(320, 1)
           bwd_logit2<kCap>(s2, poly, p, nl2, x, fac);
           float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           if (need_mask) {
-            const int kj = k0 + 32 * cc + 2 * j2;
+            const int kj = k0 + 2 * j2;
             bool v0 = qrow < seq_len && kj < seq_len;
             bool v1 = qrow < seq_len && kj + 1 < seq_len;
             if (p.wr >= 0) {
@@ -874,58 +875,56 @@ __global__ void __launch_bounds__(320, 1)
             pr.y = v1 ? pr.y : 0.f;
           }
           const float2 wv = kCap ? __fmul2_rn(pr, fac) : pr;
-          w[32 * cc + 2 * j2] = wv.x;
-          w[32 * cc + 2 * j2 + 1] = wv.y;
+          w[2 * j2] = wv.x;
+          w[2 * j2 + 1] = wv.y;
         }
       }
       // pass 2 (needs dP_j): dS = w * (dP - Drow) -> the S columns already read
       if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
       tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      {
         uint32_t dr[32];
-        tmem_ld32(t_dp + 32 * cc, dr);
+        tmem_ld32(t_dp, dr);
         tmem_ld_wait();
         uint32_t dsk[16];
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
           const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
-          const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2),
-                                       make_float2(w[32 * cc + 2 * j2], w[32 * cc + 2 * j2 + 1]));
+          const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2), make_float2(w[2 * j2], w[2 * j2 + 1]));
           dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
         }
-        // dS of keys [k0 + 32cc, +32) -> columns [64g + 16cc, +16) of the
-        // S buffer (columns this group has already read)
-        tmem_st16(t_s + 16 * cc, dsk);
+        // dS of keys [k0, k0 + 32) -> columns [32g, 32g + 16) of the S buffer
+        // (columns this group has already read)
+        tmem_st16(t_s, dsk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_ready);
     }
-    // ---- epilogue: dQ row -> dq; group g writes columns [g D/2, (g+1) D/2) ----
+    // ---- epilogue: dQ row -> dq; group g writes the 32 columns [32g, 32g+32)
+    // (D = 64: groups 0 and 1) ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
     uint8_t* dst = static_cast<uint8_t*>(p.dq) + (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD * 2;
-    if (ok && n_tiles > 0) {
-#pragma unroll 1
-      for (int c = g * (kD / 64); c < (g + 1) * (kD / 64); ++c) {
+    if (g < kD / 32) {
+      if (ok && n_tiles > 0) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_off + Sh::kColDQ + c * 32, rr);
+        tmem_ld32(tmem + lane_off + Sh::kColDQ + g * 32, rr);
         tmem_ld_wait();
         uint32_t wv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]) * p.scale, __uint_as_float(rr[2 * i + 1]) * p.scale);
         if (qrow < seq_len) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + g * 64);
 #pragma unroll
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
         }
+      } else if (ok && qrow < seq_len) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + g * 64);
+        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
       }
-    } else if (ok && qrow < seq_len) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst + g * kD);
-      for (int i = 0; i < kD / 16; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   tc_fence_before();

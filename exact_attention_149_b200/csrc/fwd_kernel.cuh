@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(384, 1)
           const float2 d = kCap ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
           const float2 e = make_float2(ex2_approx(d.x), ex2_approx(d.y));
           sum2 = __fadd2_rn(sum2, e);
-          r[i] = pack2<kBF16>(e.x, e.y);
+          r[i] = pack2_alu<kBF16>(e.x, e.y);
         }
         tmem_st32(t_p + c * 32, r);
       }
