@@ -54,6 +54,7 @@ struct BwdParams {
   float scale_log2;          // scale * log2(e)
   float softcap, cap_in, cap_out_log2;
   int wl, wr;                // window (causal folded into wr)
+  const void* q;
   const void* o;
   const void* dout;
   const float* lse;          // forward LSE, (B, Hq, S) or (Hq, total)
@@ -179,6 +180,33 @@ __device__ __forceinline__ bool poly_ok(const uint32_t (&sr)[32], float cap_in) 
   for (int i = 0; i < 32; i += 2)
     amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(sr[i])), fabsf(__uint_as_float(sr[i + 1]))));
   return __all_sync(0xffffffffu, amax * fabsf(cap_in) <= kTanhPolyMax);
+}
+
+// P (or P * (1 - tanh^2) under softcap) of 32 raw scores sharing one -LSE
+// (nl2, in the exp2 domain): all exponentials are issued before any result
+// is consumed, so they pipeline through the special-function unit.
+template <bool kCap>
+__device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, const BwdParams& p,
+                                            float (&w)[32]) {
+  const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
+#pragma unroll
+  for (int j2 = 0; j2 < 16; ++j2) {
+    const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
+    float2 x, fac;
+    bwd_logit2<kCap>(s2, poly, p, nl2, x, fac);
+    w[2 * j2] = x.x;
+    w[2 * j2 + 1] = x.y;
+    if constexpr (kCap) {  // the raw scores are no longer needed
+      sr[2 * j2] = __float_as_uint(fac.x);
+      sr[2 * j2 + 1] = __float_as_uint(fac.y);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
+  if constexpr (kCap) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] *= __uint_as_float(sr[i]);
+  }
 }
 
 // ===========================================================================
@@ -475,36 +503,40 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
         tmem_ld32(t_a, sr);
         tmem_ld_wait();
         const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
-        uint32_t pk[16];
+        // exponents first (w holds -LSE per column), then every exponential
+        // before any result is consumed, so they pipeline
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
-          const int jl = 2 * j2;  // query within the group
           const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
-          const float2 nl2 = make_float2(w[jl], w[jl + 1]);
           float2 x, fac;
-          bwd_logit2<kCap>(s2, poly, p, nl2, x, fac);
-          float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (need_mask) {
-            const int q0i = qg_lo + jl;
-            bool v0 = key < seq_len && q0i < seq_len;
-            bool v1 = key < seq_len && q0i + 1 < seq_len;
-            if (p.wr >= 0) {
-              v0 = v0 && key <= q0i + p.wr;
-              v1 = v1 && key <= q0i + 1 + p.wr;
-            }
-            if (p.wl >= 0) {
-              v0 = v0 && key >= q0i - p.wl;
-              v1 = v1 && key >= q0i + 1 - p.wl;
-            }
-            pr.x = v0 ? pr.x : 0.f;
-            pr.y = v1 ? pr.y : 0.f;
+          bwd_logit2<kCap>(s2, poly, p, make_float2(w[2 * j2], w[2 * j2 + 1]), x, fac);
+          w[2 * j2] = x.x;
+          w[2 * j2 + 1] = x.y;
+          if constexpr (kCap) {  // the raw scores are no longer needed
+            sr[2 * j2] = __float_as_uint(fac.x);
+            sr[2 * j2 + 1] = __float_as_uint(fac.y);
           }
-          pk[j2] = pack2_alu<kBF16>(pr.x, pr.y);
-          const float2 wv = kCap ? __fmul2_rn(pr, fac) : pr;
-          w[jl] = wv.x;
-          w[jl + 1] = wv.y;
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int qi = qg_lo + i;
+            bool v = key < seq_len && qi < seq_len;
+            if (p.wr >= 0) v = v && key <= qi + p.wr;
+            if (p.wl >= 0) v = v && key >= qi - p.wl;
+            w[i] = v ? w[i] : 0.f;
+          }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) pk[j2] = pack2_alu<kBF16>(w[2 * j2], w[2 * j2 + 1]);
         tmem_st16(t_a, pk);
+        if constexpr (kCap) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] *= __uint_as_float(sr[i]);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
@@ -595,46 +627,49 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
 // ===========================================================================
 // dQ
 // ===========================================================================
-// One CTA per (sequence, query head, 128-row Q tile), structured like the
-// forward kernel:
-//   warp 0     TMA producer: Q, dO once; K_j, V_j into a ring of slots.
-//   warp 1     MMA issuer: S_j = Q K_j^T (two TMEM buffers, alternating),
-//              dP_j = dO V_j^T, then dQ += dS_j K_j with dS_j read from TMEM.
-//   warps 2-17 four compute groups, one thread per query row; group g owns
-//              key columns [32g, 32g+32) of S_j and dP_j and writes dS_j
-//              (16-bit pairs) over the first half of the S columns it has
-//              read. LSE and Drow of the row live in registers. Four warps
-//              per SM sub-partition hide the latency of the exponentials.
-// TMEM columns: S buffers [0,128) and [128,256), dP [256,384), dQ [384, 384+D).
-// MMA order per tile j: S_{j+1}, dQ_j, dP_{j+1}. S and dP signal separately:
-// the compute groups form P_{j+1} (needs S only) while the tensor core runs
-// dQ_j and dP_{j+1}, then dS_{j+1} once dP_{j+1} is there.
+// One CTA per (sequence, query head, 128-row Q tile). Q and dO stay in tensor
+// memory as the A operands of S = Q K^T and dP = dO V^T, so shared memory
+// carries only the streamed K/V blocks; an item is one 64-key block:
+//   warp 0      TMA producer: K_j, V_j (64 rows each) into a ring of slots.
+//   warp 1      MMA issuer: S_j -> S_t, dP_j -> dP_t (t = j % 2), then
+//               dQ += dS_j K_j with dS_j read from S_t.
+//   warps 2-17  two teams of two compute groups, one thread per query row;
+//               team t takes the items with j % 2 == t, group g of a team the
+//               item's key columns [32g, 32g+32): P = exp(S - LSE), then
+//               dS = P * (dP - Drow) (16-bit pairs) over the first half of the
+//               S columns it has read. LSE and Drow of the row live in
+//               registers. At the start warps 2-9 write Q and dO into TMEM.
+// TMEM columns: Q [0, D/2), dO [D/2, D), S_t [128+64t, +64), dP_t
+// [256+64t, +64), dQ [384, 384+D).
+// MMA order per item j (team t): dQ_j (after the dS pass of j), S_{j+2} -> S_t,
+// dP_{j+2} -> dP_t. While one team computes, the tensor core runs the other
+// team's products; the order is fixed, so dQ is deterministic.
 template <int kD>
 struct DqShape {
   static constexpr int kChunks = kD / 64;
-  static constexpr int kChunkBytes = 128 * 128;
+  static constexpr int kKRows = 64;                    // keys per item
+  static constexpr int kChunkBytes = kKRows * 128;     // 64 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = kD == 128 ? 4 : 8;    // K/V ring slots
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffDO = kTileBytes;
-  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kStages = kD == 128 ? 6 : 12;   // K/V ring slots (one tile each)
+  static constexpr int kOffKV = 0;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-  static constexpr int kGroups = 4;
-  static constexpr int kThreads = 64 + 128 * kGroups;
+  static constexpr int kThreads = 64 + 4 * 128;
   static constexpr int kTmemCols = 512;
-  static constexpr int kColS = 0;      // + 128 * buffer
-  static constexpr int kColDP = 256;
+  static constexpr int kColQ = 0;
+  static constexpr int kColDO = kD / 2;
+  static constexpr int kColS = 128;    // + 64 t
+  static constexpr int kColDP = 256;   // + 64 t
   static constexpr int kColDQ = 384;
 };
 
 struct DqBars {
-  uint64_t qd_full;
-  uint64_t kv_full[8];
-  uint64_t kv_empty[8];
-  uint64_t s_ready;
-  uint64_t dp_ready;
-  uint64_t ds_ready;
+  uint64_t qd_tmem;      // Q and dO written to TMEM (8 warps)
+  uint64_t kv_full[12];
+  uint64_t kv_empty[12];
+  uint64_t s_ready[2];
+  uint64_t dp_ready[2];
+  uint64_t ds_ready[2];
   uint64_t final_done;
   uint64_t drain;
   uint32_t tmem_base;
@@ -643,8 +678,7 @@ struct DqBars {
 
 template <int kD, bool kBF16, bool kCap>
 __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p) {
   using Sh = DqShape<kD>;
   extern __shared__ uint8_t smem_raw[];
@@ -677,18 +711,20 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
   if (p.wr >= 0) key_hi = min(key_hi, row_hi + p.wr);
   int key_lo = 0;
   if (p.wl >= 0) key_lo = max(0, q0 - p.wl);
-  const int n_begin = key_lo / 128;
-  const int n_tiles = key_hi >= key_lo ? key_hi / 128 + 1 - n_begin : 0;
+  const int n_begin = key_lo / Sh::kKRows;
+  const int n_tiles = key_hi >= key_lo ? key_hi / Sh::kKRows + 1 - n_begin : 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->qd_full, 1);
+    mbar_init(&bars->qd_tmem, 8);
     for (int i = 0; i < Sh::kStages; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
-    mbar_init(&bars->s_ready, 1);
-    mbar_init(&bars->dp_ready, 1);
-    mbar_init(&bars->ds_ready, 4 * Sh::kGroups);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_ready[t], 1);
+      mbar_init(&bars->dp_ready[t], 1);
+      mbar_init(&bars->ds_ready[t], 8);
+    }
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -707,20 +743,11 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (elect_one()) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&bars->qd_full, 2 * Sh::kTileBytes);
-      for (int c = 0; c < Sh::kChunks; ++c) {
-        tma_load_3d(&tm_q, &bars->qd_full, smem + Sh::kOffQ + c * Sh::kChunkBytes, c * 64, h,
-                    seq_start + q0);
-        tma_load_3d(&tm_do, &bars->qd_full, smem + Sh::kOffDO + c * Sh::kChunkBytes, c * 64, h,
-                    seq_start + q0);
-      }
       int fill = 0;
       for (int j = 0; j < n_tiles && !*abort; ++j) {
-        const int tok = seq_start + (n_begin + j) * 128;
+        const int tok = seq_start + (n_begin + j) * Sh::kKRows;
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % Sh::kStages;
           const uint32_t ph = static_cast<uint32_t>(fill / Sh::kStages) & 1u;
@@ -734,82 +761,72 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       }
       for (int f = max(0, fill - Sh::kStages); f < fill; ++f)
         mbar_wait(&bars->kv_full[f % Sh::kStages], static_cast<uint32_t>(f / Sh::kStages) & 1u);
-      mbar_wait(&bars->qd_full, 0);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (elect_one()) {
-      constexpr uint32_t id_s = idesc_f16(kBF16, 128, 128, false, false);   // S, dP
-      constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, false, true);    // dS (tmem) x K
-      const uint32_t sQ = smem_u32(smem + Sh::kOffQ);
-      const uint32_t sDO = smem_u32(smem + Sh::kOffDO);
+      constexpr uint32_t id_s = idesc_f16(kBF16, 128, Sh::kKRows, false, false);  // S, dP
+      constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, false, true);          // dS (tmem) x K
       const uint32_t sKV = smem_u32(smem + Sh::kOffKV);
-      bool ok = bwd_wait(&bars->qd_full, 0, abort);
+      bool ok = bwd_wait(&bars->qd_tmem, 0, abort);
       tc_fence_after();
       auto kmajor = [](uint32_t base, int kk) {
         return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
       };
       auto wait_slot = [&](int fill) {
-        return bwd_wait(&bars->kv_full[fill % Sh::kStages],
-                        static_cast<uint32_t>(fill / Sh::kStages) & 1u, abort);
+        const bool r = bwd_wait(&bars->kv_full[fill % Sh::kStages],
+                                static_cast<uint32_t>(fill / Sh::kStages) & 1u, abort);
+        tc_fence_after();
+        return r;
       };
       auto slot_addr = [&](int fill) { return sKV + (fill % Sh::kStages) * Sh::kTileBytes; };
-      auto issue_s = [&](int j) {  // S_j = Q K_j^T -> buffer j & 1
+      auto issue_s = [&](int j) {  // S_j = Q K_j^T -> S_{j%2}
         const uint32_t sK = slot_addr(2 * j);
+        const uint32_t d = tmem + Sh::kColS + 64 * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ss(tmem + Sh::kColS + 128 * (j & 1), kmajor(sQ, kk), kmajor(sK, kk), id_s,
-                  kk > 0 ? 1u : 0u);
+          umma_ts(d, tmem + Sh::kColQ + 8 * kk, kmajor(sK, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_ready[j & 1]);
       };
-      auto issue_dp = [&](int j) {  // dP_j = dO V_j^T
+      auto issue_dp = [&](int j) {  // dP_j = dO V_j^T -> dP_{j%2}
         const uint32_t sV = slot_addr(2 * j + 1);
+        const uint32_t d = tmem + Sh::kColDP + 64 * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ss(tmem + Sh::kColDP, kmajor(sDO, kk), kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+          umma_ts(d, tmem + Sh::kColDO + 8 * kk, kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->dp_ready[j & 1]);
       };
-      if (ok && n_tiles > 0) {
-        if ((ok = wait_slot(0))) {
-          tc_fence_after();
-          issue_s(0);
-          umma_commit(&bars->s_ready);
-          if ((ok = wait_slot(1))) {
-            tc_fence_after();
-            issue_dp(0);
-            umma_commit(&bars->dp_ready);
-          }
-        }
+      for (int j = 0; j < 2 && j < n_tiles && ok; ++j) {
+        if (!(ok = wait_slot(2 * j))) break;
+        issue_s(j);
+        if (!(ok = wait_slot(2 * j + 1))) break;
+        issue_dp(j);
       }
       for (int j = 0; j < n_tiles && ok; ++j) {
-        const bool more = j + 1 < n_tiles;
-        // S_{j+1} into the other buffer (its previous dS was consumed by dQ_{j-1})
-        if (more) {
-          if (!(ok = wait_slot(2 * (j + 1)))) break;
-          tc_fence_after();
-          issue_s(j + 1);
-          umma_commit(&bars->s_ready);
-        }
-        if (!(ok = bwd_wait(&bars->ds_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
+        const int t = j & 1;
+        if (!(ok = bwd_wait(&bars->ds_ready[t], static_cast<uint32_t>(j >> 1) & 1u, abort))) break;
         tc_fence_after();
-        // dQ += dS_j K_j: A = dS_j from TMEM (keys [32c, 32c+32) packed into
-        // columns [32c, 32c+16) of buffer j & 1), B = K_j with N = D (MN-major)
+        // dQ += dS_j K_j: A = dS_j from S_t (keys [32c, 32c+32) packed into
+        // columns [32c, 32c+16)), B = K_j with N = D (MN-major)
         {
           const uint32_t sK = slot_addr(2 * j);
-          const uint32_t a = tmem + Sh::kColS + 128 * (j & 1);
+          const uint32_t a = tmem + Sh::kColS + 64 * t;
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
+          for (int kk = 0; kk < Sh::kKRows / 16; ++kk)
             umma_ts(tmem + Sh::kColDQ, a + (kk >> 1) * 32 + (kk & 1) * 8,
                     sdesc_sw128(sK + kk * 2048, Sh::kChunkBytes, 1024), id_dq,
                     (j == 0 && kk == 0) ? 0u : 1u);
         }
         umma_commit(&bars->kv_empty[(2 * j) % Sh::kStages]);      // K_j
         umma_commit(&bars->kv_empty[(2 * j + 1) % Sh::kStages]);  // V_j
-        // dP_{j+1}: the compute groups have read dP_j before ds_ready
-        if (more) {
-          if (!(ok = wait_slot(2 * (j + 1) + 1))) break;
-          tc_fence_after();
-          issue_dp(j + 1);
-          umma_commit(&bars->dp_ready);
+        // S_{j+2} and dP_{j+2}: dQ_j, the last reader of S_t, precedes them;
+        // the team read dP_t before signalling ds_ready
+        if (j + 2 < n_tiles) {
+          if (!(ok = wait_slot(2 * (j + 2)))) break;
+          issue_s(j + 2);
+          if (!(ok = wait_slot(2 * (j + 2) + 1))) break;
+          issue_dp(j + 2);
         }
       }
       umma_commit(&bars->final_done);
@@ -818,12 +835,39 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ======================= compute groups =======================
-    const int g = (warp - 2) >> 2;
+    // ======================= compute teams =======================
+    const int team = (warp - 2) >> 3;
+    const int g = ((warp - 2) >> 2) & 1;     // group within the team
     const int lane_base = 32 * (warp & 3);
     const int r = lane_base + lane;          // query row within the tile
     const int qrow = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
+    if (team == 0) {
+      // Q (group 0) or dO (group 1) row -> TMEM, two 16-bit values per column
+      // (the A-operand layout: K-step kk of 16 values at columns 8kk..8kk+7);
+      // rows past the sequence end are zero
+      const uint16_t* src = static_cast<const uint16_t*>(g == 0 ? p.q : p.dout) +
+                            (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD;
+      const uint32_t col = g == 0 ? Sh::kColQ : Sh::kColDO;
+#pragma unroll
+      for (int c = 0; c < kD / 64; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint4 u = make_uint4(0u, 0u, 0u, 0u);
+          if (qrow < seq_len) u = reinterpret_cast<const uint4*>(src + c * 64)[i];
+          v[4 * i] = u.x;
+          v[4 * i + 1] = u.y;
+          v[4 * i + 2] = u.z;
+          v[4 * i + 3] = u.w;
+        }
+        tmem_st32(tmem + lane_off + col + 32 * c, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qd_tmem);
+    }
     // the row's -LSE (exp2 domain) and Drow
     float nlse = -INFINITY, drow = 0.f;
     if (qrow < seq_len) {
@@ -834,12 +878,13 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     const float2 nl2 = make_float2(nlse, nlse);
     const float2 nd2 = make_float2(-drow, -drow);
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
+    for (int j = team; j < n_tiles; j += 2) {
+      const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
+      if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort))) break;
       tc_fence_after();
-      const int k0 = (n_begin + j) * 128 + 32 * g;  // first key of this group's columns
-      const uint32_t t_s = tmem + lane_off + Sh::kColS + 128 * (j & 1) + 32 * g;
-      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 32 * g;
+      const int k0 = (n_begin + j) * Sh::kKRows + 32 * g;  // first key of this group's columns
+      const uint32_t t_s = tmem + lane_off + Sh::kColS + 64 * team + 32 * g;
+      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 64 * team + 32 * g;
       // mask needed for this warp's 32 rows x the group's 32 keys?
       const int r_lo = q0 + lane_base, r_hi = r_lo + 31;
       bool need_mask = (k0 + 31 >= seq_len) || (r_hi >= seq_len);
@@ -852,35 +897,20 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         uint32_t sr[32];
         tmem_ld32(t_s, sr);
         tmem_ld_wait();
-        const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
+        bwd_probs32<kCap>(sr, nl2, p, w);
+        if (need_mask) {
 #pragma unroll
-        for (int j2 = 0; j2 < 16; ++j2) {
-          const float2 s2 = make_float2(__uint_as_float(sr[2 * j2]), __uint_as_float(sr[2 * j2 + 1]));
-          float2 x, fac;
-          bwd_logit2<kCap>(s2, poly, p, nl2, x, fac);
-          float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (need_mask) {
-            const int kj = k0 + 2 * j2;
-            bool v0 = qrow < seq_len && kj < seq_len;
-            bool v1 = qrow < seq_len && kj + 1 < seq_len;
-            if (p.wr >= 0) {
-              v0 = v0 && kj <= qrow + p.wr;
-              v1 = v1 && kj + 1 <= qrow + p.wr;
-            }
-            if (p.wl >= 0) {
-              v0 = v0 && kj >= qrow - p.wl;
-              v1 = v1 && kj + 1 >= qrow - p.wl;
-            }
-            pr.x = v0 ? pr.x : 0.f;
-            pr.y = v1 ? pr.y : 0.f;
+          for (int i = 0; i < 32; ++i) {
+            const int kj = k0 + i;
+            bool v = qrow < seq_len && kj < seq_len;
+            if (p.wr >= 0) v = v && kj <= qrow + p.wr;
+            if (p.wl >= 0) v = v && kj >= qrow - p.wl;
+            w[i] = v ? w[i] : 0.f;
           }
-          const float2 wv = kCap ? __fmul2_rn(pr, fac) : pr;
-          w[2 * j2] = wv.x;
-          w[2 * j2 + 1] = wv.y;
         }
       }
       // pass 2 (needs dP_j): dS = w * (dP - Drow) -> the S columns already read
-      if (!(ok = bwd_wait(&bars->dp_ready, static_cast<uint32_t>(j) & 1u, abort))) break;
+      if (!(ok = bwd_wait(&bars->dp_ready[team], ph, abort))) break;
       tc_fence_after();
       {
         uint32_t dr[32];
@@ -893,36 +923,37 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
           const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2), make_float2(w[2 * j2], w[2 * j2 + 1]));
           dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
         }
-        // dS of keys [k0, k0 + 32) -> columns [32g, 32g + 16) of the S buffer
+        // dS of keys [k0, k0 + 32) -> columns [32g, 32g + 16) of S_t
         // (columns this group has already read)
         tmem_st16(t_s, dsk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ds_ready);
+      if (lane == 0) mbar_arrive(&bars->ds_ready[team]);
     }
-    // ---- epilogue: dQ row -> dq; group g writes the 32 columns [32g, 32g+32)
-    // (D = 64: groups 0 and 1) ----
+    // ---- epilogue: dQ row -> dq; warps 2-5, 6-9, 10-13, 14-17 write the
+    // 32-column chunks 0..3 (D = 64: the first two) ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
+    const int e = (warp - 2) >> 2;
     uint8_t* dst = static_cast<uint8_t*>(p.dq) + (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD * 2;
-    if (g < kD / 32) {
+    if (e < kD / 32) {
       if (ok && n_tiles > 0) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_off + Sh::kColDQ + g * 32, rr);
+        tmem_ld32(tmem + lane_off + Sh::kColDQ + e * 32, rr);
         tmem_ld_wait();
         uint32_t wv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]) * p.scale, __uint_as_float(rr[2 * i + 1]) * p.scale);
         if (qrow < seq_len) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + g * 64);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + e * 64);
 #pragma unroll
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
         }
       } else if (ok && qrow < seq_len) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + g * 64);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + e * 64);
         for (int i = 0; i < 4; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
