@@ -409,24 +409,35 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(x - base): one packed FMA (or add) per pair, then MUFU ex2
+      // P = 2^(x - base): one packed FMA (or add) per pair, then the 128
+      // exponentials, all issued before any result is used so that they
+      // pipeline through the special-function unit; then the row sum and
+      // the 16-bit P tile
       const float2 nb2 = make_float2(-base, -base);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-      float2 sum2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float2 xv = make_float2(x[i], x[i + 1]);
+        const float2 d = kCap ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
+        x[i] = d.x;
+        x[i + 1] = d.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 128; ++i) x[i] = ex2_approx(x[i]);
+      float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) sum2[(i >> 1) & 3] = __fadd2_rn(sum2[(i >> 1) & 3], make_float2(x[i], x[i + 1]));
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 xv = make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]);
-          const float2 d = kCap ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
-          const float2 e = make_float2(ex2_approx(d.x), ex2_approx(d.y));
-          sum2 = __fadd2_rn(sum2, e);
-          r[i] = pack2_alu<kBF16>(e.x, e.y);
-        }
+        for (int i = 0; i < 32; ++i) r[i] = pack2_alu<kBF16>(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]);
         tmem_st32(t_p + c * 32, r);
       }
-      const float lsum = sum2.x + sum2.y;
+      const float2 s01 = __fadd2_rn(sum2[0], sum2[1]), s23 = __fadd2_rn(sum2[2], sum2[3]);
+      const float2 s4 = __fadd2_rn(s01, s23);
+      const float lsum = s4.x + s4.y;
       l_run += lsum;
       tmem_st_wait();
       tc_fence_before();
