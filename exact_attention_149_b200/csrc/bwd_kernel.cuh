@@ -228,7 +228,8 @@ struct DkdvShape {
   static constexpr int kOffVec = kOffQ + kSlots * 2 * kQTileBytes;
   static constexpr int kVecBytes = 512;
   static constexpr int kOffBar = kOffVec + kSlots * kVecBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
   // warp 0 TMA, warp 1 MMA, then two teams of two compute groups (4 warps
   // each); team t takes the items it with it % 2 == t, group g of a team the
   // 32 query columns [32g, 32g + 32) of the item
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using Sh = DkdvShape<kD>;
+  static_assert(sizeof(DkdvBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -650,10 +652,13 @@ struct DqShape {
   static constexpr int kKRows = 64;                    // keys per item
   static constexpr int kChunkBytes = kKRows * 128;     // 64 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = kD == 128 ? 6 : 12;   // K/V ring slots (one tile each)
+  // K/V ring slots (one tile each): six items in flight hide the L2 -> shared
+  // latency of the next blocks behind about 1.3k cycles per item
+  static constexpr int kStages = kD == 128 ? 12 : 24;
   static constexpr int kOffKV = 0;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
   static constexpr int kThreads = 64 + 4 * 128;
   static constexpr int kTmemCols = 512;
   static constexpr int kColQ = 0;
@@ -665,8 +670,8 @@ struct DqShape {
 
 struct DqBars {
   uint64_t qd_tmem;      // Q and dO written to TMEM (8 warps)
-  uint64_t kv_full[12];
-  uint64_t kv_empty[12];
+  uint64_t kv_full[24];
+  uint64_t kv_empty[24];
   uint64_t s_ready[2];
   uint64_t dp_ready[2];
   uint64_t ds_ready[2];
@@ -681,6 +686,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p) {
   using Sh = DqShape<kD>;
+  static_assert(sizeof(DqBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

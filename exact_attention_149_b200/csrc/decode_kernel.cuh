@@ -251,6 +251,7 @@ __global__ void __launch_bounds__(160)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using Sh = DecShape<kD>;
+  static_assert(sizeof(DecBars) <= 256, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
