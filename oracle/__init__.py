@@ -5,6 +5,7 @@ Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
 """
 
 from .attention import (  # noqa: F401
+    alibi_bias,
     attention_bwd,
     attention_fwd,
     head_bwd,

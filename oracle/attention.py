@@ -110,8 +110,30 @@ def scores(q_h: np.ndarray, k_h: np.ndarray, scale: float, softcap: float):
     return x, y
 
 
+def alibi_bias(sq: int, sk: int, slope: float, rows=None) -> np.ndarray:
+    """ALiBi bias of one head, [len(rows), sk]: -slope * |i + (sk - sq) - j|,
+    the distance between query i and key j under the bottom-right alignment
+    of visible_mask. Guide §进阶参数: alibi_slopes is a position bias that
+    makes attention to distant keys decay, with no explicit position
+    encoding; the linear-in-distance form is the reading."""
+    if rows is None:
+        rows = np.arange(sq)
+    i = np.asarray(rows, dtype=np.int64)[:, None]
+    j = np.arange(sk, dtype=np.int64)[None, :]
+    return -float(slope) * np.abs(i + (sk - sq) - j).astype(np.float64)
+
+
+def _slope(alibi_slopes, b: int, h: int) -> float:
+    """Slope of (batch b, head h) from a (Hq,) or (B, Hq) array, 0 if None."""
+    if alibi_slopes is None:
+        return 0.0
+    a = np.asarray(alibi_slopes, dtype=np.float64)
+    return float(a[h] if a.ndim == 1 else a[b, h])
+
+
 def head_fwd(q_h, k_h, v_h, scale: float, causal: bool = False, window_left: int = -1,
-             window_right: int = -1, softcap: float = 0.0, rows=None, _score_hook=None):
+             window_right: int = -1, softcap: float = 0.0, rows=None, _score_hook=None,
+             alibi_slope: float = 0.0):
     """One head of the forward pass.
 
     q_h: [Sq, D]; k_h, v_h: [Sk, D]. ``rows`` optionally selects query rows
@@ -130,6 +152,8 @@ def head_fwd(q_h, k_h, v_h, scale: float, causal: bool = False, window_left: int
         rows = np.arange(sq)
     rows = np.asarray(rows, dtype=np.int64)
     x, _ = scores(q_h[rows], k_h, scale, softcap)
+    if alibi_slope != 0.0:
+        x = x + alibi_bias(sq, sk, alibi_slope, rows)
     if _score_hook is not None:
         x = _score_hook(x)
     vis = visible_mask(sq, sk, causal, window_left, window_right, rows)
@@ -147,7 +171,7 @@ def head_fwd(q_h, k_h, v_h, scale: float, causal: bool = False, window_left: int
 
 
 def head_bwd(q_h, k_h, v_h, do_h, scale: float, causal: bool = False, window_left: int = -1,
-             window_right: int = -1, softcap: float = 0.0):
+             window_right: int = -1, softcap: float = 0.0, alibi_slope: float = 0.0):
     """One head of the backward pass of ``head_fwd`` (all rows).
 
     With P the row-normalised softmax probabilities (zero where masked):
@@ -155,7 +179,8 @@ def head_bwd(q_h, k_h, v_h, do_h, scale: float, causal: bool = False, window_lef
     and through softcap X = c tanh(Y / c): dY = dX * (1 - tanh(Y / c)^2),
       dQ = scale * dY K,  dK = scale * dY^T Q.
     This is the chain rule of the definition; the guide (§长序列…) says the
-    tiled backward recomputes these quantities rather than storing P.
+    tiled backward recomputes these quantities rather than storing P. The
+    ALiBi bias is a constant added to X, so it changes P and nothing else.
     """
     q_h = _f64(q_h)
     k_h = _f64(k_h)
@@ -163,6 +188,8 @@ def head_bwd(q_h, k_h, v_h, do_h, scale: float, causal: bool = False, window_lef
     do_h = _f64(do_h)
     sq, sk = q_h.shape[0], k_h.shape[0]
     x, y = scores(q_h, k_h, scale, softcap)
+    if alibi_slope != 0.0:
+        x = x + alibi_bias(sq, sk, alibi_slope)
     vis = visible_mask(sq, sk, causal, window_left, window_right)
     x = np.where(vis, x, -np.inf)
     m = np.max(x, axis=1, initial=-np.inf)
@@ -198,14 +225,14 @@ def _segments(q, cu_seqlens):
 
 
 def attention_fwd(q, k, v, scale: float, causal: bool = False, window=(-1, -1),
-                  softcap: float = 0.0, cu_seqlens=None):
+                  softcap: float = 0.0, cu_seqlens=None, alibi_slopes=None):
     """Full forward over all batches and heads.
 
     Fixed length: q (B, S, Hq, D), k/v (B, S, Hkv, D) -> O (B, S, Hq, D),
     LSE (B, Hq, S). Varlen (cu_seqlens given, int prefix sums of length B+1):
     q (total, Hq, D), k/v (total, Hkv, D) -> O (total, Hq, D), LSE (Hq, total);
     each segment is an independent sequence with Sq = Sk = its length (guide
-    §上手…三步走, varlen family).
+    §上手…三步走, varlen family). alibi_slopes: None, (Hq,) or (B, Hq).
     """
     q = _f64(q)
     k = _f64(k)
@@ -222,7 +249,8 @@ def attention_fwd(q, k, v, scale: float, causal: bool = False, window=(-1, -1),
         qb, kb, vb = q[sl], k[sl], v[sl]
         for h in range(hq):
             ob, lb = head_fwd(qb[:, h], kb[:, h // g], vb[:, h // g], scale, causal,
-                              window[0], window[1], softcap)
+                              window[0], window[1], softcap,
+                              alibi_slope=_slope(alibi_slopes, b, h))
             if cu_seqlens is None:
                 o[b, :, h] = ob
                 lse[b, h] = lb
@@ -233,7 +261,7 @@ def attention_fwd(q, k, v, scale: float, causal: bool = False, window=(-1, -1),
 
 
 def attention_bwd(q, k, v, do, scale: float, causal: bool = False, window=(-1, -1),
-                  softcap: float = 0.0, cu_seqlens=None):
+                  softcap: float = 0.0, cu_seqlens=None, alibi_slopes=None):
     """Gradients (dQ, dK, dV) of sum(O * dO); same layouts as attention_fwd.
     For GQA the per-query-head dK/dV contributions of a group are summed into
     their shared kv head."""
@@ -249,7 +277,8 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool = False, window=(-1, -
     for b, sl in _segments(q, cu_seqlens):
         for h in range(hq):
             a, bb, c = head_bwd(q[sl][:, h], k[sl][:, h // g], v[sl][:, h // g], do[sl][:, h],
-                                scale, causal, window[0], window[1], softcap)
+                                scale, causal, window[0], window[1], softcap,
+                                alibi_slope=_slope(alibi_slopes, b, h))
             if cu_seqlens is None:
                 dq[b, :, h] = a
                 dk[b, :, h // g] += bb
@@ -309,7 +338,7 @@ def rotary(x, pos, cos, sin, interleaved=False):
 def kvcache_decode(q, k_new, v_new, k_cache_logical, v_cache_logical, cache_seqlens,
                    scale: float, causal: bool = True, window=(-1, -1), softcap: float = 0.0,
                    heads=None, rotary_cos=None, rotary_sin=None, rotary_interleaved=False,
-                   rotated_dtype=None):
+                   rotated_dtype=None, alibi_slopes=None):
     """One step against a *logical, contiguous* per-sequence cache.
 
     q (B, Sq, Hq, D); k_new, v_new (B, Sq, Hkv, D) or None; k/v_cache_logical:
@@ -359,7 +388,8 @@ def kvcache_decode(q, k_new, v_new, k_cache_logical, v_cache_logical, cache_seql
         vs.append(vb)
         for h in (range(hq) if heads is None else heads):
             ob, lb = head_fwd(qb[:, h], kb[:, h // g], vb[:, h // g], scale, causal,
-                              window[0], window[1], softcap)
+                              window[0], window[1], softcap,
+                              alibi_slope=_slope(alibi_slopes, b, h))
             o[b, :, h] = ob
             lse[b, h, :] = lb
     return o, lse, ks, vs

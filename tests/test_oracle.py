@@ -19,8 +19,8 @@ import pytest
 import torch
 
 import attn_workloads as W
-from oracle import (attention_bwd, attention_fwd, head_bwd, head_fwd, kvcache_decode,
-                    lse_combine, rotary, round_to, scores, visible_mask)
+from oracle import (alibi_bias, attention_bwd, attention_fwd, head_bwd, head_fwd,
+                    kvcache_decode, lse_combine, rotary, round_to, scores, visible_mask)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
 
@@ -32,7 +32,7 @@ def rng(seed):
 # ---------------------------------------------------------------------------
 # independent brute force: pure Python loops, math.fsum, no numpy in the math
 # ---------------------------------------------------------------------------
-def brute_head(q, k, v, scale, causal, wl, wr, softcap):
+def brute_head(q, k, v, scale, causal, wl, wr, softcap, slope=0.0):
     sq, sk, d = len(q), len(k), len(q[0])
     outs, lses = [], []
     for i in range(sq):
@@ -47,6 +47,7 @@ def brute_head(q, k, v, scale, causal, wl, wr, softcap):
             s = scale * math.fsum(q[i][t] * k[j][t] for t in range(d))
             if softcap > 0:
                 s = softcap * math.tanh(s / softcap)
+            s -= slope * abs(i + delta - j)
             logits.append((j, s))
         if not logits:
             outs.append([0.0] * d)
@@ -152,6 +153,11 @@ def test_golden_worked_examples(case):
         np.testing.assert_allclose(lse[0, :, 0], np.array(case["expect_lse_value"]), atol=1e-14)
         np.testing.assert_array_equal(ks[0], np.array(case["expect_k_after"]))
         np.testing.assert_array_equal(vs[0], np.array(case["expect_v_after"]))
+    elif kind == "alibi":
+        o, lse = head_fwd(np.array(case["q"]), np.array(case["k"]), np.array(case["v"]),
+                          case["scale"], True, alibi_slope=case["slope"])
+        np.testing.assert_allclose(o, np.array(case["expect_o"]), atol=1e-12)
+        np.testing.assert_allclose(lse, np.array(case["expect_lse"]), atol=1e-12)
     elif kind == "rotary":
         got = rotary(np.array(case["x"]), np.array(case["pos"]), np.array(case["cos"]),
                      np.array(case["sin"]))
@@ -567,3 +573,122 @@ def test_rotary_rejects_positions_outside_the_table():
         rotary(x, [-1], cos, sin)  # numpy would silently wrap to the last row
     with pytest.raises(ValueError):
         rotary(x, [8], cos, sin)
+
+
+# ---------------------------------------------------------------------------
+# ALiBi (guide §进阶参数 alibi_slopes; the linear-distance form is a reading)
+# ---------------------------------------------------------------------------
+ALIBI_CASES = [
+    # sq, sk, causal, wl, wr, softcap, slope
+    (6, 6, True, -1, -1, 0.0, 0.5),
+    (5, 5, False, -1, -1, 0.0, 0.25),
+    (7, 7, True, 2, 0, 1.2, 0.7),
+    (3, 8, True, -1, -1, 0.0, 1.5),   # Sq < Sk: distances from the bottom-right diagonal
+    (6, 6, False, 1, 2, 0.0, 0.3),
+]
+
+
+@pytest.mark.parametrize("sq,sk,causal,wl,wr,softcap,slope", ALIBI_CASES)
+def test_alibi_brute_force(sq, sk, causal, wl, wr, softcap, slope):
+    r = rng(sq * 7 + sk)
+    q, k, v = r.standard_normal((sq, 4)), r.standard_normal((sk, 4)), r.standard_normal((sk, 4))
+    o, lse = head_fwd(q, k, v, 0.6, causal, wl, wr, softcap, alibi_slope=slope)
+    bo, bl = brute_head(q.tolist(), k.tolist(), v.tolist(), 0.6, causal, wl, wr, softcap, slope)
+    np.testing.assert_allclose(o, np.array(bo), atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(bl), atol=1e-12)
+
+
+def _alibi_mask(sq, sk, slopes, causal):
+    """(H, sq, sk) additive float mask for SDPA: the bias, -inf where hidden."""
+    m = np.stack([alibi_bias(sq, sk, sl) for sl in slopes])
+    if causal:
+        vis = visible_mask(sq, sk, True, -1, -1)
+        m = np.where(vis[None], m, -np.inf)
+    return torch.tensor(m)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_alibi_sdpa_pin(causal):
+    """SDPA with the bias as an additive float mask (a library routine that
+    knows nothing of ALiBi), per-head slopes and GQA."""
+    r = rng(71 + causal)
+    B, S, hq, hkv, D = 2, 19, 4, 2, 8
+    q = r.standard_normal((B, S, hq, D))
+    k = r.standard_normal((B, S, hkv, D))
+    v = r.standard_normal((B, S, hkv, D))
+    slopes = np.array([0.5, 0.25, 0.125, 0.0625])
+    o, _ = attention_fwd(q, k, v, 0.35, causal=causal, alibi_slopes=slopes)
+    g = hq // hkv
+    qt = torch.tensor(q).permute(0, 2, 1, 3)
+    kt = torch.tensor(np.repeat(k, g, axis=2)).permute(0, 2, 1, 3)
+    vt = torch.tensor(np.repeat(v, g, axis=2)).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt, vt, attn_mask=_alibi_mask(S, S, slopes, causal), scale=0.35)
+    np.testing.assert_allclose(o, ref.permute(0, 2, 1, 3).numpy(), atol=1e-10)
+
+
+def test_alibi_autograd_pin_backward():
+    r = rng(73)
+    B, S, hq, hkv, D = 1, 13, 4, 2, 8
+    q = r.standard_normal((B, S, hq, D))
+    k = r.standard_normal((B, S, hkv, D))
+    v = r.standard_normal((B, S, hkv, D))
+    do = r.standard_normal((B, S, hq, D))
+    slopes = np.array([0.9, 0.3, 0.1, 0.05])
+    dq, dk, dv = attention_bwd(q, k, v, do, 0.45, causal=True, alibi_slopes=slopes)
+    qt = torch.tensor(q, requires_grad=True)
+    kt = torch.tensor(k, requires_grad=True)
+    vt = torch.tensor(v, requires_grad=True)
+    g = hq // hkv
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt.permute(0, 2, 1, 3), kt.repeat_interleave(g, dim=2).permute(0, 2, 1, 3),
+        vt.repeat_interleave(g, dim=2).permute(0, 2, 1, 3), attn_mask=_alibi_mask(S, S, slopes, True),
+        scale=0.45)
+    (o.permute(0, 2, 1, 3) * torch.tensor(do)).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-10)
+
+
+def test_alibi_finite_difference_with_softcap_and_window():
+    r = rng(79)
+    B, S, hq, hkv, D = 1, 6, 2, 1, 3
+    q = r.standard_normal((B, S, hq, D))
+    k = r.standard_normal((B, S, hkv, D))
+    v = r.standard_normal((B, S, hkv, D))
+    do = r.standard_normal((B, S, hq, D))
+    slopes = np.array([[0.8, 0.2]])  # (B, Hq) layout
+    args = (0.7, True, (3, 0), 1.1)
+    dq, dk, dv = attention_bwd(q, k, v, do, *args, alibi_slopes=slopes)
+
+    def f(q_, k_, v_):
+        return float(np.sum(attention_fwd(q_, k_, v_, *args, alibi_slopes=slopes)[0] * do))
+
+    h = 1e-6
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        x = {"q": q, "k": k, "v": v}[name]
+        num = np.zeros_like(x)
+        for idx in itertools.product(*map(range, x.shape)):
+            pl = {"q": q, "k": k, "v": v}
+            mi = {"q": q, "k": k, "v": v}
+            pl[name] = x.copy()
+            mi[name] = x.copy()
+            pl[name][idx] += h
+            mi[name][idx] -= h
+            num[idx] = (f(pl["q"], pl["k"], pl["v"]) - f(mi["q"], mi["k"], mi["v"])) / (2 * h)
+        assert np.linalg.norm(num - grad) / np.linalg.norm(num) < 1e-6, name
+
+
+def test_alibi_per_batch_slopes_and_zero_slope():
+    r = rng(83)
+    B, S, H, D = 2, 9, 2, 4
+    q, k, v = (r.standard_normal((B, S, H, D)) for _ in range(3))
+    o2, l2 = attention_fwd(q, k, v, 0.5, True, alibi_slopes=np.array([[0.3, 0.6], [1.2, 0.1]]))
+    for b, sl in ((0, [0.3, 0.6]), (1, [1.2, 0.1])):
+        o1, l1 = attention_fwd(q[b:b + 1], k[b:b + 1], v[b:b + 1], 0.5, True, alibi_slopes=np.array(sl))
+        np.testing.assert_allclose(o2[b:b + 1], o1, atol=1e-14)
+        np.testing.assert_allclose(l2[b:b + 1], l1, atol=1e-14)
+    o0, l0 = attention_fwd(q, k, v, 0.5, True, alibi_slopes=np.zeros(H))
+    on, ln = attention_fwd(q, k, v, 0.5, True)
+    np.testing.assert_array_equal(o0, on)
+    np.testing.assert_array_equal(l0, ln)
