@@ -38,6 +38,7 @@ __all__ = [
     "decode_sequence_cache",
     "fill_paged_pool",
     "rotary_tables",
+    "alibi_slopes",
     "visible_pairs",
     "fwd_flops",
     "bwd_flops",
@@ -254,6 +255,17 @@ def rotary_tables(rows, rotary_dim, base=10000.0):
     ang = np.arange(rows, dtype=np.float64)[:, None] * inv[None, :]
     return (torch.from_numpy(np.cos(ang).astype(np.float32)),
             torch.from_numpy(np.sin(ang).astype(np.float32)))
+
+
+def alibi_slopes(H, B=None, scale=1.0):
+    """ALiBi slopes a caller passes: the geometric sequence 2^(-8 (h+1) / H)
+    for H heads (times `scale`), float32 (H,); with B, a (B, H) array whose
+    row b is scaled by (b + 1), so that every sequence has its own slopes."""
+    base = scale * 2.0 ** (-8.0 * (np.arange(H, dtype=np.float64) + 1.0) / H)
+    if B is None:
+        return torch.from_numpy(base.astype(np.float32))
+    rows = np.stack([base * (b + 1) for b in range(B)])
+    return torch.from_numpy(rows.astype(np.float32))
 
 
 # ---------------------------------------------------------------------------

@@ -55,15 +55,17 @@ _f = ctypes.c_float
 _z = ctypes.c_size_t
 
 lib.fa_fwd.restype = _i
-lib.fa_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _p, _i, _i, _p]
+lib.fa_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _p, _i, _p, _i,
+                       _i, _p]
 lib.fa_bwd.restype = _i
 lib.fa_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f,
-                       _p, _i, _i, _p, _z, _p]
+                       _p, _i, _p, _i, _i, _p, _z, _p]
 lib.fa_fwd_kvcache.restype = _i
 # q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos, rotary_sin, out, lse;
 # B, Sq, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
-# rotary_interleaved; scale, causal, window_left, window_right, softcap, num_splits, dtype
-_KV_ARGS = [_p] * 11 + [_i] * 11 + [_f, _i, _i, _i, _f, _i, _i]
+# rotary_interleaved; scale, causal, window_left, window_right, softcap, alibi_slopes,
+# alibi_batch_stride, num_splits, dtype
+_KV_ARGS = [_p] * 11 + [_i] * 11 + [_f, _i, _i, _i, _f, _p, _i, _i, _i]
 lib.fa_fwd_kvcache.restype = _i
 lib.fa_fwd_kvcache.argtypes = _KV_ARGS + [_p, _z, _p]
 lib.fa_fwd_kvcache_noalloc.restype = _i
@@ -134,10 +136,10 @@ def _need_cuda(*ts):
 # C-ABI mirrors
 # ---------------------------------------------------------------------------
 def fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, scale, causal, window_left, window_right,
-           softcap, cu_seqlens, total_tokens, dtype, stream=None):
+           softcap, alibi_slopes, alibi_batch_stride, cu_seqlens, total_tokens, dtype, stream=None):
     _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, scale,
-                      int(causal), window_left, window_right, softcap, _ptr(cu_seqlens),
-                      total_tokens, dtype, _stream(stream)))
+                      int(causal), window_left, window_right, softcap, _ptr(alibi_slopes),
+                      alibi_batch_stride, _ptr(cu_seqlens), total_tokens, dtype, _stream(stream)))
 
 
 def fa_bwd_workspace_size(B, Hq, S, D, total_tokens=0) -> int:
@@ -145,12 +147,13 @@ def fa_bwd_workspace_size(B, Hq, S, D, total_tokens=0) -> int:
 
 
 def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, window_left,
-           window_right, softcap, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes,
-           stream=None):
+           window_right, softcap, alibi_slopes, alibi_batch_stride, cu_seqlens, total_tokens, dtype,
+           workspace, workspace_bytes, stream=None):
     _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
                       _ptr(dk), _ptr(dv), B, Hq, Hkv, S, D, scale, int(causal), window_left,
-                      window_right, softcap, _ptr(cu_seqlens), total_tokens, dtype,
-                      _ptr(workspace), workspace_bytes, _stream(stream)))
+                      window_right, softcap, _ptr(alibi_slopes), alibi_batch_stride,
+                      _ptr(cu_seqlens), total_tokens, dtype, _ptr(workspace), workspace_bytes,
+                      _stream(stream)))
 
 
 def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rotary_dim=0) -> int:
@@ -160,15 +163,16 @@ def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rotary_dim=0) -> int:
 def fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos,
                    rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, max_pages_per_seq,
                    num_pages, rotary_rows, rotary_dim, rotary_interleaved, scale, causal,
-                   window_left, window_right, softcap, num_splits, dtype, workspace,
-                   workspace_bytes, stream=None):
+                   window_left, window_right, softcap, alibi_slopes, alibi_batch_stride,
+                   num_splits, dtype, workspace, workspace_bytes, stream=None):
     _check(lib.fa_fwd_kvcache(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
                               _ptr(block_table), _ptr(cache_seqlens), _ptr(rotary_cos),
                               _ptr(rotary_sin), _ptr(out), _ptr(lse), B, Sq, Hq, Hkv, D, page_size,
                               max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
                               int(rotary_interleaved), scale, int(causal), window_left,
-                              window_right, softcap, num_splits, dtype, _ptr(workspace),
-                              workspace_bytes, _stream(stream)))
+                              window_right, softcap, _ptr(alibi_slopes), alibi_batch_stride,
+                              num_splits, dtype, _ptr(workspace), workspace_bytes,
+                              _stream(stream)))
 
 
 # size of the library's static scratch array used by fa_fwd_kvcache_noalloc
@@ -179,7 +183,7 @@ def fa_fwd_kvcache_noalloc(q, k_new, v_new, k_cache, v_cache, block_table, cache
                            rotary_cos, rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size,
                            max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
                            rotary_interleaved, scale, causal, window_left, window_right, softcap,
-                           num_splits, dtype, stream=None):
+                           alibi_slopes, alibi_batch_stride, num_splits, dtype, stream=None):
     """fa_fwd_kvcache for callers that cannot allocate device memory: no
     workspace argument; the split partials and rotated queries live in the
     library's own static device array (see include/fa.h)."""
@@ -188,8 +192,9 @@ def fa_fwd_kvcache_noalloc(q, k_new, v_new, k_cache, v_cache, block_table, cache
                                       _ptr(rotary_cos), _ptr(rotary_sin), _ptr(out), _ptr(lse), B,
                                       Sq, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages,
                                       rotary_rows, rotary_dim, int(rotary_interleaved), scale,
-                                      int(causal), window_left, window_right, softcap, num_splits,
-                                      dtype, _stream(stream)))
+                                      int(causal), window_left, window_right, softcap,
+                                      _ptr(alibi_slopes), alibi_batch_stride, num_splits, dtype,
+                                      _stream(stream)))
 
 
 def fa_kernel_timing_enable(enable: bool = True):
@@ -222,10 +227,22 @@ def _scale(scale, D):
     return float(D) ** -0.5 if scale is None else float(scale)
 
 
+def _alibi(alibi_slopes, Hq):
+    """(tensor, batch stride) for the C ABI: None, a float32 (Hq,) vector
+    (stride 0) or a float32 (B, Hq) array with contiguous rows."""
+    if alibi_slopes is None:
+        return None, 0
+    _need_cuda(alibi_slopes)
+    if alibi_slopes.dtype != torch.float32 or alibi_slopes.shape[-1] != Hq or alibi_slopes.dim() > 2:
+        raise FaError(FA_ERR_INVALID_ARG, "alibi_slopes must be float32 (Hq,) or (B, Hq)")
+    return alibi_slopes, (0 if alibi_slopes.dim() == 1 else alibi_slopes.stride(0))
+
+
 def fwd(q, k, v, scale=None, causal=False, window=(-1, -1), softcap=0.0, cu_seqlens=None,
-        max_seqlen=None, out=None, lse=None, stream=None):
+        max_seqlen=None, out=None, lse=None, alibi_slopes=None, stream=None):
     """q (B,S,Hq,D), k/v (B,S,Hkv,D) -> (out, lse (B,Hq,S)); varlen: q (T,Hq,D),
-    cu_seqlens int32 (B+1) on the device, lse (Hq,T)."""
+    cu_seqlens int32 (B+1) on the device, lse (Hq,T). alibi_slopes: float32
+    (Hq,) or (B, Hq) on the device."""
     _need_cuda(q, k, v, cu_seqlens)
     if cu_seqlens is None:
         B, S, Hq, D = q.shape
@@ -244,13 +261,15 @@ def fwd(q, k, v, scale=None, causal=False, window=(-1, -1), softcap=0.0, cu_seql
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    al, als = _alibi(alibi_slopes, Hq)
     fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, _scale(scale, D), causal, window[0], window[1],
-           softcap, cu_seqlens, T, _dt(q), stream)
+           softcap, al, als, cu_seqlens, T, _dt(q), stream)
     return out, lse
 
 
 def bwd(q, k, v, out, lse, dout, scale=None, causal=False, window=(-1, -1), softcap=0.0,
-        cu_seqlens=None, max_seqlen=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+        cu_seqlens=None, max_seqlen=None, dq=None, dk=None, dv=None, workspace=None,
+        alibi_slopes=None, stream=None):
     """Gradients (dq, dk, dv) of sum(out * dout); layouts as in fwd."""
     _need_cuda(q, k, v, out, lse, dout, cu_seqlens)
     if cu_seqlens is None:
@@ -268,16 +287,17 @@ def bwd(q, k, v, out, lse, dout, scale=None, causal=False, window=(-1, -1), soft
     nbytes = fa_bwd_workspace_size(B, Hq, S, D, T)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    al, als = _alibi(alibi_slopes, Hq)
     fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, _scale(scale, D), causal,
-           window[0], window[1], softcap, cu_seqlens, T, _dt(q), workspace, workspace.numel(),
-           stream)
+           window[0], window[1], softcap, al, als, cu_seqlens, T, _dt(q), workspace,
+           workspace.numel(), stream)
     return dq, dk, dv
 
 
 def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_new=None,
                 rotary_cos=None, rotary_sin=None, rotary_interleaved=False, scale=None,
                 causal=True, window=(-1, -1), softcap=0.0, num_splits=1, out=None, lse=None,
-                workspace=None, stream=None):
+                workspace=None, alibi_slopes=None, stream=None):
     """One decode step: q (B,Sq,Hq,D); caches (num_pages, page_size, Hkv, D)
     with block_table int32 (B, max_pages), or block_table None and contiguous
     caches (B, capacity, Hkv, D); cache_seqlens int32 (B). Appends
@@ -303,6 +323,6 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
     fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos,
                    rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, max_pages, num_pages,
                    rot_rows, rot_dim, rotary_interleaved, _scale(scale, D), causal, window[0],
-                   window[1], softcap, num_splits, _dt(q), workspace,
+                   window[1], softcap, *_alibi(alibi_slopes, Hq), num_splits, _dt(q), workspace,
                    0 if workspace is None else workspace.numel(), stream)
     return out, lse

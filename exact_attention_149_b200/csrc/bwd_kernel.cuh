@@ -65,7 +65,14 @@ struct BwdParams {
   void* dk;                  // (T, Hkv, D)
   void* dv;
   const int* cu_seqlens;
+  const float* alibi;        // ALiBi slopes, nullable: slope of (b, h) = alibi[b * alibi_bstride + h]
+  int alibi_bstride;
 };
+
+// ALiBi slope of (sequence b, query head h) in the exp2 domain, 0 without ALiBi
+__device__ __forceinline__ float alibi_slope2(const BwdParams& p, int b, int h) {
+  return p.alibi ? p.alibi[static_cast<size_t>(b) * p.alibi_bstride + h] * 1.4426950408889634f : 0.f;
+}
 
 // Padded layout of the per-row vectors: query row q of sequence b (first
 // token seq_start) and query head h sits at
@@ -184,10 +191,12 @@ __device__ __forceinline__ bool poly_ok(const uint32_t (&sr)[32], float cap_in) 
 
 // P (or P * (1 - tanh^2) under softcap) of 32 raw scores sharing one -LSE
 // (nl2, in the exp2 domain): all exponentials are issued before any result
-// is consumed, so they pipeline through the special-function unit.
+// is consumed, so they pipeline through the special-function unit. With
+// ALiBi, entry i gets -sl2 * |d0 - i| added to its exponent (sl2: slope in
+// the exp2 domain, d0: query position minus the first key's).
 template <bool kCap>
 __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, const BwdParams& p,
-                                            float (&w)[32]) {
+                                            bool alibi, float sl2, float d0, float (&w)[32]) {
   const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
 #pragma unroll
   for (int j2 = 0; j2 < 16; ++j2) {
@@ -200,6 +209,10 @@ __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, cons
       sr[2 * j2] = __float_as_uint(fac.x);
       sr[2 * j2 + 1] = __float_as_uint(fac.y);
     }
+  }
+  if (alibi) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = fmaf(-sl2, fabsf(d0 - static_cast<float>(i)), w[i]);
   }
 #pragma unroll
   for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
@@ -255,7 +268,7 @@ struct DkdvBars {
   int abort;
 };
 
-template <int kD, bool kBF16, bool kCap>
+template <int kD, bool kBF16, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -467,10 +480,12 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     // read itself
     const uint32_t t_a = tmem + lane_off + Sh::kColA + 64 * team + 32 * g;
     const uint32_t t_b = tmem + lane_off + Sh::kColB + 64 * team + 32 * g;
+    constexpr bool alibi = kAlibi;  // compiled in only where used
     bool ok = true;
     for (int it = team; it < n_items; it += 2) {
       const uint32_t ph = static_cast<uint32_t>(it >> 1) & 1u;
       const int q0 = (i_begin + it % i_cnt) * Sh::kQRows;
+      const float sl2 = alibi_slope2(p, b, kvh * p.group + it / i_cnt);
       // the group's 32 query columns of -LSE and Drow, bulk-loaded with the
       // item's Q/dO into its slot (the slot is refilled only after dK of this
       // item, which waits for this team's dS pass)
@@ -518,6 +533,11 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
             sr[2 * j2] = __float_as_uint(fac.x);
             sr[2 * j2 + 1] = __float_as_uint(fac.y);
           }
+        }
+        if constexpr (alibi) {  // -slope * |query - key| in the exp2 domain
+          const float d0 = static_cast<float>(qg_lo - key);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = fmaf(-sl2, fabsf(d0 + static_cast<float>(i)), w[i]);
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
@@ -681,7 +701,7 @@ struct DqBars {
   int abort;
 };
 
-template <int kD, bool kBF16, bool kCap>
+template <int kD, bool kBF16, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p) {
@@ -883,6 +903,8 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     }
     const float2 nl2 = make_float2(nlse, nlse);
     const float2 nd2 = make_float2(-drow, -drow);
+    constexpr bool alibi = kAlibi;  // compiled in only where used
+    const float sl2 = alibi_slope2(p, b, h);
     bool ok = true;
     for (int j = team; j < n_tiles; j += 2) {
       const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
@@ -903,7 +925,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         uint32_t sr[32];
         tmem_ld32(t_s, sr);
         tmem_ld_wait();
-        bwd_probs32<kCap>(sr, nl2, p, w);
+        bwd_probs32<kCap>(sr, nl2, p, alibi, sl2, static_cast<float>(qrow - k0), w);
         if (need_mask) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {

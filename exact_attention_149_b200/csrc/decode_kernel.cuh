@@ -58,6 +58,8 @@ struct DecodeParams {
   float scale_log2, softcap, cap_in, cap_out_log2;
   int wl;                 // window left (-1 = unbounded)
   int right;              // visible keys end at position + right (-1 = unbounded; causal = 0)
+  const float* alibi;     // ALiBi slopes, nullable: slope of (b, hq) = alibi[b * alibi_bstride + hq]
+  int alibi_bstride;
 };
 
 // Keys visible to the query at position `qpos` of a sequence of Lk keys:
@@ -369,6 +371,19 @@ __global__ void __launch_bounds__(160)
       }
     }
   }
+  // ALiBi: slope (exp2 domain) and query position of this lane's columns
+  const bool alibi = p.alibi != nullptr;
+  float asl[kNT][2], aqp[kNT][2];
+#pragma unroll
+  for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int n = min(n0 + nt * 8 + 2 * (lane & 3) + j, p.n_cols - 1);
+      const int hq = kvh * p.group + n % p.group;
+      asl[nt][j] = alibi ? p.alibi[static_cast<size_t>(b) * p.alibi_bstride + hq] * 1.4426950408889634f : 0.f;
+      aqp[nt][j] = static_cast<float>(qbase + n / p.group);
+    }
+  }
   // running state per (column tile, column pair): columns nt*8 + 2*(lane&3) + {0,1}
   float m_run[kNT][2], l_part[kNT][2];
   float acc[kNT][kD / 16][4];
@@ -430,6 +445,13 @@ __global__ void __launch_bounds__(160)
       float x1 = dec_logit(s[nt][1], p);
       float x2 = dec_logit(s[nt][2], p);
       float x3 = dec_logit(s[nt][3], p);
+      if (alibi) {  // -slope * |query - key|, after softcap
+        const float pf = static_cast<float>(pos0);
+        x0 = fmaf(-asl[nt][0], fabsf(aqp[nt][0] - pf), x0);
+        x1 = fmaf(-asl[nt][1], fabsf(aqp[nt][1] - pf), x1);
+        x2 = fmaf(-asl[nt][0], fabsf(aqp[nt][0] - pf - 8.f), x2);
+        x3 = fmaf(-asl[nt][1], fabsf(aqp[nt][1] - pf - 8.f), x3);
+      }
       if (!all_visible) {
         // per-column key ranges (padding columns take the last real one's)
 #pragma unroll

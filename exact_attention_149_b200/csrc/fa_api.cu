@@ -155,6 +155,17 @@ class KernelTimer {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // common option validation for fwd/bwd
+// ALiBi slopes: NULL, or a 4-byte aligned device float array read at
+// b * batch_stride + h (batch_stride 0: one (Hq) vector for every sequence).
+fa_status check_alibi(const float* slopes, int batch_stride, int Hq) {
+  if (slopes == nullptr) return FA_OK;
+  if (reinterpret_cast<uintptr_t>(slopes) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "alibi_slopes must be 4-byte aligned");
+  if (batch_stride != 0 && batch_stride < Hq)
+    return fail(FA_ERR_INVALID_ARG, "alibi_batch_stride must be 0 or >= Hq (got %d)", batch_stride);
+  return FA_OK;
+}
+
 fa_status check_common(int B, int Hq, int Hkv, int S, int D, float scale, int wl, int wr,
                        float softcap, fa_dtype dt, const int32_t* cu, int total) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1)
@@ -186,7 +197,7 @@ template <int kD, bool kBF16, bool kCap>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const fa::FwdParams& p, cudaStream_t st) {
   using Sh = fa::FwdShape<kD>;
-  auto kern = fa::fwd_kernel<kD, kBF16, kCap>;
+  auto kern = p.alibi ? fa::fwd_kernel<kD, kBF16, kCap, true> : fa::fwd_kernel<kD, kBF16, kCap, false>;
   fa_status s = set_smem(kern, Sh::kSmemBytes);
   if (s != FA_OK) return s;
   const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
@@ -261,14 +272,15 @@ fa_status fa_get_device_status(int* status_out) {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
                  int Hkv, int S, int D, float scale, int causal, int window_left, int window_right,
-                 float softcap, const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype,
-                 void* stream) {
+                 float softcap, const float* alibi_slopes, int alibi_batch_stride,
+                 const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype, void* stream) {
   if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd: null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be 16-byte aligned");
   fa_status s = check_common(B, Hq, Hkv, S, D, scale, window_left, window_right, softcap, dtype,
                              cu_seqlens, total_tokens);
   if (s != FA_OK) return s;
+  if ((s = check_alibi(alibi_slopes, alibi_batch_stride, Hq)) != FA_OK) return s;
   if ((s = check_device()) != FA_OK) return s;
 
   const long long T = cu_seqlens ? total_tokens : static_cast<long long>(B) * S;
@@ -296,6 +308,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   p.o = out;
   p.lse = lse;
   p.cu_seqlens = cu_seqlens;
+  p.alibi = alibi_slopes;
+  p.alibi_bstride = alibi_batch_stride;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool cap = softcap > 0.f;
   if (D == 128) {

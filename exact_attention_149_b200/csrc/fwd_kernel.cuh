@@ -45,6 +45,8 @@ struct FwdParams {
   void* o;
   float* lse;
   const int* cu_seqlens;     // nullable
+  const float* alibi;        // ALiBi slopes, nullable: slope of (b, h) = alibi[b * alibi_bstride + h]
+  int alibi_bstride;
 };
 
 template <int kD>
@@ -124,7 +126,9 @@ __device__ __forceinline__ float reduce128(const float (&x)[128]) {
   return kMax ? max3(fmaxf(a[0], a[1]), a[2], a[3]) : min3(fminf(a[0], a[1]), a[2], a[3]);
 }
 
-template <int kD, bool kBF16, bool kCap>
+// kAlibi: the ALiBi bias is compiled in only where it is used, so the
+// common instantiations keep their register allocation
+template <int kD, bool kBF16, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -328,6 +332,9 @@ __global__ void __launch_bounds__(384, 1)
     const int r_hi = r_lo + 31;
     float m_run = -INFINITY;
     float l_run = 0.f;
+    // ALiBi slope of this head in the exp2 domain (uniform across the CTA)
+    constexpr bool alibi = kAlibi;
+    const float sl2 = alibi ? p.alibi[static_cast<size_t>(b) * p.alibi_bstride + h] * 1.4426950408889634f : 0.f;
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
       if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it) & 1u, abort))) break;
@@ -370,9 +377,23 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 128; ++i) x[i] = p.cap_out_log2 * tanh_fast(x[i] * p.cap_in);
         }
       }
+      if constexpr (alibi) {
+        // ALiBi: -slope * |query - key| added to the logit, in the exp2
+        // domain (after softcap); x then holds exp2-domain logits
+        const float dq = static_cast<float>(qrow - k0);
+        if constexpr (kCap) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) x[i] = fmaf(-sl2, fabsf(dq - static_cast<float>(i)), x[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            x[i] = fmaf(x[i], p.scale_log2, -sl2 * fabsf(dq - static_cast<float>(i)));
+        }
+      }
+      constexpr bool lg = kCap || alibi;  // x holds exp2-domain logits
       // masked entries become the value that the reduction ignores and whose
       // exponential is 0 (-inf; +inf for raw scores under a negative scale)
-      const bool pos = kCap || p.scale_log2 >= 0.f;
+      const bool pos = lg || p.scale_log2 >= 0.f;
       if (need_mask) {
         const float hide = pos ? -INFINITY : INFINITY;
         int jmax = seq_len - 1 - k0;
@@ -382,7 +403,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 128; ++i) x[i] = (i > jmax || i < jmin) ? hide : x[i];
       }
       float mt;
-      if constexpr (kCap) {
+      if constexpr (lg) {
         mt = reduce128<true>(x);
       } else {
         mt = pos ? reduce128<true>(x) : reduce128<false>(x);
@@ -419,7 +440,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
         const float2 xv = make_float2(x[i], x[i + 1]);
-        const float2 d = kCap ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
+        const float2 d = lg ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
         x[i] = d.x;
         x[i + 1] = d.y;
       }

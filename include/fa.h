@@ -31,8 +31,14 @@
  *   an integer multiple of Hkv and query head h reads kv head h / (Hq / Hkv).
  *   When the query and key lengths differ (decode) the causal diagonal is
  *   aligned to the bottom-right corner.
- * - LSE is the natural-log log-sum-exp of each row's scaled (and softcapped)
- *   logits; a row with no visible key gets O = 0 and LSE = -inf.
+ * - ALiBi (guide §进阶参数 alibi_slopes: a position bias that decays the
+ *   scores of distant keys): alibi_slopes is NULL or a DEVICE float32 array;
+ *   query head h of sequence b uses slope s = alibi_slopes[b *
+ *   alibi_batch_stride + h] (batch stride 0: one (Hq) vector for every
+ *   sequence; Hq: a (B, Hq) array), and every logit of query i and key j gets
+ *   -s * |i + Sk - Sq - j| added after scaling and softcap, before masking.
+ * - LSE is the natural-log log-sum-exp of each row's scaled (and softcapped,
+ *   biased) logits; a row with no visible key gets O = 0 and LSE = -inf.
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *   default stream) and returns after the launch. Errors never abort: the
  *   call returns a status and fa_last_error() describes it. Invalid
@@ -73,12 +79,14 @@ typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
  *   total_tokens: number of packed tokens when cu_seqlens != NULL, else ignored.
  * Errors: FA_ERR_INVALID_ARG for null q/k/v/out/lse, B/Hq/Hkv/S < 1,
  *   Hq % Hkv != 0, window < -1, softcap < 0 or not finite, scale not finite,
- *   misaligned pointers; FA_ERR_UNSUPPORTED for D not in {64, 128} or a
+ *   misaligned pointers, alibi_batch_stride neither 0 nor >= Hq;
+ *   FA_ERR_UNSUPPORTED for D not in {64, 128} or a
  *   device other than compute capability 10.0; FA_ERR_CUDA on launch failure.
  */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                  int Hq, int Hkv, int S, int D, float scale, int causal, int window_left,
-                 int window_right, float softcap, const int32_t* cu_seqlens, int total_tokens,
+                 int window_right, float softcap, const float* alibi_slopes,
+                 int alibi_batch_stride, const int32_t* cu_seqlens, int total_tokens,
                  fa_dtype dtype, void* stream);
 
 /*
@@ -108,8 +116,9 @@ FA_API size_t fa_bwd_workspace_size(int B, int Hq, int S, int D, int total_token
 FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                  const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S,
                  int D, float scale, int causal, int window_left, int window_right, float softcap,
-                 const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype, void* workspace,
-                 size_t workspace_bytes, void* stream);
+                 const float* alibi_slopes, int alibi_batch_stride, const int32_t* cu_seqlens,
+                 int total_tokens, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                 void* stream);
 
 /* Workspace bytes needed by fa_fwd_kvcache: the float32 per-split partial
  * results (num_splits > 1; 0 bytes for them otherwise) and, with rotary
@@ -173,7 +182,8 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_
                                 int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
                                 int num_pages, int rotary_rows, int rotary_dim,
                                 int rotary_interleaved, float scale, int causal, int window_left,
-                                int window_right, float softcap, int num_splits, fa_dtype dtype,
+                                int window_right, float softcap, const float* alibi_slopes,
+                                int alibi_batch_stride, int num_splits, fa_dtype dtype,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
@@ -216,7 +226,8 @@ FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const 
                                         int max_pages_per_seq, int num_pages, int rotary_rows,
                                         int rotary_dim, int rotary_interleaved, float scale,
                                         int causal, int window_left, int window_right,
-                                        float softcap, int num_splits, fa_dtype dtype,
+                                        float softcap, const float* alibi_slopes,
+                                        int alibi_batch_stride, int num_splits, fa_dtype dtype,
                                         void* stream);
 
 /*

@@ -72,12 +72,12 @@ def test_workspace_sizes(fa):
 
 def _fwd_status(fa, **kw):
     args = dict(q=16, k=16, v=16, out=16, lse=16, B=1, Hq=2, Hkv=2, S=128, D=64, scale=0.125,
-                causal=0, wl=-1, wr=-1, softcap=0.0, cu=None, total=0, dtype=0)
+                causal=0, wl=-1, wr=-1, softcap=0.0, al=None, als=0, cu=None, total=0, dtype=0)
     args.update(kw)
     return fa.lib.fa_fwd(args["q"], args["k"], args["v"], args["out"], args["lse"], args["B"],
                          args["Hq"], args["Hkv"], args["S"], args["D"], args["scale"],
-                         args["causal"], args["wl"], args["wr"], args["softcap"], args["cu"],
-                         args["total"], args["dtype"], None)
+                         args["causal"], args["wl"], args["wr"], args["softcap"], args["al"],
+                         args["als"], args["cu"], args["total"], args["dtype"], None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -95,6 +95,8 @@ def _fwd_status(fa, **kw):
     (dict(D=96), 2),                # unsupported head dim
     (dict(D=256), 2),
     (dict(cu=16, total=0), 1),
+    (dict(al=18), 1),               # misaligned slopes
+    (dict(al=16, als=1), 1),        # batch stride neither 0 nor >= Hq
 ])
 def test_fwd_rejects_bad_arguments(fa, kw, status):
     assert _fwd_status(fa, **kw) == status
@@ -103,7 +105,7 @@ def test_fwd_rejects_bad_arguments(fa, kw, status):
 
 def test_bwd_rejects_bad_arguments(fa):
     lib = fa.lib
-    base = [16] * 9 + [1, 2, 2, 128, 64, 0.125, 0, -1, -1, 0.0, None, 0, 0]
+    base = [16] * 9 + [1, 2, 2, 128, 64, 0.125, 0, -1, -1, 0.0, None, 0, None, 0, 0]
     # null dout
     a = list(base)
     a[5] = None
@@ -112,6 +114,10 @@ def test_bwd_rejects_bad_arguments(fa):
     assert lib.fa_bwd(*base, 16, 8, None) in (1, 2)
     # workspace missing
     assert lib.fa_bwd(*base, None, 1 << 20, None) in (1, 2)
+    # misaligned ALiBi slopes
+    a = list(base)
+    a[19] = 18
+    assert lib.fa_bwd(*a, 16, 1 << 20, None) == 1
 
 
 def test_kvcache_rejects_bad_arguments(fa):
@@ -120,16 +126,18 @@ def test_kvcache_rejects_bad_arguments(fa):
     def call(**kw):
         a = dict(q=16, kn=16, vn=16, kc=16, vc=16, bt=16, cs=16, cos=None, sin=None, out=16,
                  lse=16, B=2, Sq=1, Hq=4, Hkv=2, D=128, ps=256, mp=4, npg=8, rrows=0, rd=0,
-                 rint=0, scale=0.1, causal=1, wl=-1, wr=-1, softcap=0.0, splits=1, dtype=0,
-                 ws=None, wsb=0)
+                 rint=0, scale=0.1, causal=1, wl=-1, wr=-1, softcap=0.0, al=None, als=0, splits=1,
+                 dtype=0, ws=None, wsb=0)
         a.update(kw)
         return lib.fa_fwd_kvcache(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["bt"], a["cs"],
                                   a["cos"], a["sin"], a["out"], a["lse"], a["B"], a["Sq"], a["Hq"],
                                   a["Hkv"], a["D"], a["ps"], a["mp"], a["npg"], a["rrows"], a["rd"],
                                   a["rint"], a["scale"], a["causal"], a["wl"], a["wr"],
-                                  a["softcap"], a["splits"], a["dtype"], a["ws"], a["wsb"], None)
+                                  a["softcap"], a["al"], a["als"], a["splits"], a["dtype"], a["ws"],
+                                  a["wsb"], None)
 
     assert call(kc=None) == 1
+    assert call(al=18) == 1                           # misaligned ALiBi slopes
     assert call(bt=None) == 1
     assert call(cs=None) == 1
     assert call(splits=0) == 1

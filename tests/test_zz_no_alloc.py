@@ -51,7 +51,7 @@ def _decode_both_ways(B, Hq, Hkv, D, lengths, page_size, splits, seed, sq=1, rot
     lse_ref = torch.empty((B, Hq, sq), dtype=torch.float32, device=dev)
     fa.fa_fwd_kvcache(q, kn, vn, kc, vc, bt, cs, cos, sin, out_ref, lse_ref, B, sq, Hq, Hkv, D,
                       page_size, bt.shape[1], st["num_pages"], rows, rotary_dim, False, scale,
-                      True, -1, -1, 0.0, splits, 0, ws, ws.numel())
+                      True, -1, -1, 0.0, None, 0, splits, 0, ws, ws.numel())
     # the allocation-free entry point, called straight through the C ABI
     out = torch.full_like(q, float("nan"))
     lse = torch.full((B, Hq, sq), float("nan"), dtype=torch.float32, device=dev)
@@ -61,7 +61,8 @@ def _decode_both_ways(B, Hq, Hkv, D, lengths, page_size, splits, seed, sq=1, rot
         q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc2.data_ptr(), vc2.data_ptr(), bt.data_ptr(),
         cs.data_ptr(), ptr(cos), ptr(sin), out.data_ptr(), lse.data_ptr(), B, sq, Hq, Hkv, D,
         page_size, bt.shape[1], st["num_pages"], rows if rotary_dim else 0, rotary_dim, 0,
-        ctypes.c_float(scale), 1, -1, -1, ctypes.c_float(0.0), splits, 0, ctypes.c_void_p(stream))
+        ctypes.c_float(scale), 1, -1, -1, ctypes.c_float(0.0), None, 0, splits, 0,
+        ctypes.c_void_p(stream))
     assert status == 0, fa.fa_last_error()
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
@@ -82,5 +83,5 @@ def test_noalloc_rejects_oversized_partials(cuda_ok):
     assert need > fa.FA_NOALLOC_SCRATCH_BYTES
     status = fa.lib.fa_fwd_kvcache_noalloc(16, 16, 16, 16, 16, 16, 16, None, None, 16, 16, 64, 1,
                                            64, 8, 128, 256, 4, 8, 0, 0, 0, ctypes.c_float(0.1), 1,
-                                           -1, -1, ctypes.c_float(0.0), 32, 0, None)
+                                           -1, -1, ctypes.c_float(0.0), None, 0, 32, 0, None)
     assert status == 1 and "scratch" in fa.fa_last_error()
