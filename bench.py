@@ -353,6 +353,20 @@ def run_ours(args, dist: Dist):
         res["bwd"] = {"ms": ms_bwd, "tflops": bwd_flop / (ms_bwd * 1e-3) / 1e12, "flop": bwd_flop}
         res["bwd"]["frac_of_bf16_peak"] = res["bwd"]["tflops"] / peaks["bf16_tflops"]
 
+    # -------------------- the same step with ALiBi slopes --------------------
+    if have_bwd:
+        slopes = W.alibi_slopes(c.Hq).to(dev)
+
+        def step_alibi():
+            fa.fwd(q, k, v, scale=c.scale, causal=True, out=out, lse=lse, alibi_slopes=slopes)
+            fa.bwd(q, k, v, out, lse, do, scale=c.scale, causal=True, dq=dq, dk=dk, dv=dv,
+                   workspace=ws, alibi_slopes=slopes)
+
+        ms_al = timed(step_alibi, args.steps, args.warmup, dist)
+        res["alibi_fwd_bwd"] = {"ms": ms_al, "tflops": flop_step / (ms_al * 1e-3) / 1e12,
+                                "slopes": "2^(-8(h+1)/Hq)"}
+        res["alibi_fwd_bwd"]["frac_of_bf16_peak"] = res["alibi_fwd_bwd"]["tflops"] / peaks["bf16_tflops"]
+
     # -------------------- end to end through the public API --------------------
     hq_, hk_, hv_, hdo_ = (inp[n].pin_memory() for n in ("q", "k", "v", "do"))
     h_out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
