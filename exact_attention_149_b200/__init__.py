@@ -25,7 +25,8 @@ __all__ = [
     "fa_kvcache_workspace_size", "FA_NOALLOC_SCRATCH_BYTES",
     "fa_get_device_status", "fa_last_error", "fa_version",
     "fa_kernel_timing_enable", "fa_kernel_timing_read", "fa_kernel_timing_reset",
-    "fwd", "bwd", "fwd_kvcache",
+    "fwd", "bwd", "fwd_kvcache", "fwd_qkvpacked", "bwd_qkvpacked", "fa_fwd_qkvpacked",
+    "fa_bwd_qkvpacked",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -60,6 +61,12 @@ lib.fa_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _
 lib.fa_bwd.restype = _i
 lib.fa_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f,
                        _p, _i, _p, _i, _i, _p, _z, _p]
+lib.fa_fwd_qkvpacked.restype = _i
+lib.fa_fwd_qkvpacked.argtypes = [_p, _p, _p, _i, _i, _i, _i, _f, _i, _i, _i, _f, _p, _i, _p, _i, _i,
+                                 _p]
+lib.fa_bwd_qkvpacked.restype = _i
+lib.fa_bwd_qkvpacked.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _f, _i, _i, _i, _f, _p, _i, _p,
+                                 _i, _i, _p, _z, _p]
 lib.fa_fwd_kvcache.restype = _i
 # q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos, rotary_sin, out, lse;
 # B, Sq, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
@@ -140,6 +147,24 @@ def fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, scale, causal, window_left, wind
     _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, scale,
                       int(causal), window_left, window_right, softcap, _ptr(alibi_slopes),
                       alibi_batch_stride, _ptr(cu_seqlens), total_tokens, dtype, _stream(stream)))
+
+
+def fa_fwd_qkvpacked(qkv, out, lse, B, H, S, D, scale, causal, window_left, window_right, softcap,
+                     alibi_slopes, alibi_batch_stride, cu_seqlens, total_tokens, dtype, stream=None):
+    _check(lib.fa_fwd_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), B, H, S, D, scale, int(causal),
+                                window_left, window_right, softcap, _ptr(alibi_slopes),
+                                alibi_batch_stride, _ptr(cu_seqlens), total_tokens, dtype,
+                                _stream(stream)))
+
+
+def fa_bwd_qkvpacked(qkv, out, lse, dout, dqkv, B, H, S, D, scale, causal, window_left,
+                     window_right, softcap, alibi_slopes, alibi_batch_stride, cu_seqlens,
+                     total_tokens, dtype, workspace, workspace_bytes, stream=None):
+    _check(lib.fa_bwd_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dqkv), B, H, S, D,
+                                scale, int(causal), window_left, window_right, softcap,
+                                _ptr(alibi_slopes), alibi_batch_stride, _ptr(cu_seqlens),
+                                total_tokens, dtype, _ptr(workspace), workspace_bytes,
+                                _stream(stream)))
 
 
 def fa_bwd_workspace_size(B, Hq, S, D, total_tokens=0) -> int:
@@ -292,6 +317,50 @@ def bwd(q, k, v, out, lse, dout, scale=None, causal=False, window=(-1, -1), soft
            window[0], window[1], softcap, al, als, cu_seqlens, T, _dt(q), workspace,
            workspace.numel(), stream)
     return dq, dk, dv
+
+
+def _packed_dims(qkv, cu_seqlens, max_seqlen):
+    if cu_seqlens is None:
+        B, S, three, H, D = qkv.shape
+        return B, S, H, D, 0
+    T, three, H, D = qkv.shape
+    if max_seqlen is None:
+        raise FaError(FA_ERR_INVALID_ARG, "max_seqlen is required with cu_seqlens")
+    return cu_seqlens.numel() - 1, int(max_seqlen), H, D, T
+
+
+def fwd_qkvpacked(qkv, scale=None, causal=False, window=(-1, -1), softcap=0.0, cu_seqlens=None,
+                  max_seqlen=None, out=None, lse=None, alibi_slopes=None, stream=None):
+    """qkv (B,S,3,H,D) (varlen: (T,3,H,D)) -> (out (B,S,H,D), lse (B,H,S));
+    the three tensors are read in place."""
+    _need_cuda(qkv, cu_seqlens)
+    B, S, H, D, T = _packed_dims(qkv, cu_seqlens, max_seqlen)
+    if out is None:
+        out = torch.empty(qkv.shape[:-3] + (H, D), dtype=qkv.dtype, device=qkv.device)
+    if lse is None:
+        shape = (B, H, S) if cu_seqlens is None else (H, T)
+        lse = torch.empty(shape, dtype=torch.float32, device=qkv.device)
+    al, als = _alibi(alibi_slopes, H)
+    fa_fwd_qkvpacked(qkv, out, lse, B, H, S, D, _scale(scale, D), causal, window[0], window[1],
+                     softcap, al, als, cu_seqlens, T, _dt(qkv), stream)
+    return out, lse
+
+
+def bwd_qkvpacked(qkv, out, lse, dout, scale=None, causal=False, window=(-1, -1), softcap=0.0,
+                  cu_seqlens=None, max_seqlen=None, dqkv=None, workspace=None, alibi_slopes=None,
+                  stream=None):
+    """Gradient dqkv, packed like qkv, of sum(out * dout)."""
+    _need_cuda(qkv, out, lse, dout, cu_seqlens)
+    B, S, H, D, T = _packed_dims(qkv, cu_seqlens, max_seqlen)
+    dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
+    nbytes = fa_bwd_workspace_size(B, H, S, D, T)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=qkv.device)
+    al, als = _alibi(alibi_slopes, H)
+    fa_bwd_qkvpacked(qkv, out, lse, dout, dqkv, B, H, S, D, _scale(scale, D), causal, window[0],
+                     window[1], softcap, al, als, cu_seqlens, T, _dt(qkv), workspace,
+                     workspace.numel(), stream)
+    return dqkv
 
 
 def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_new=None,

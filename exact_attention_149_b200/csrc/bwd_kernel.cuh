@@ -67,6 +67,9 @@ struct BwdParams {
   const int* cu_seqlens;
   const float* alibi;        // ALiBi slopes, nullable: slope of (b, h) = alibi[b * alibi_bstride + h]
   int alibi_bstride;
+  // elements from one token's row to the next: q and dq (Hq * D unpacked),
+  // dk and dv (Hkv * D unpacked); the qkv-packed layout uses 3 * H * D
+  long long q_tok, dq_tok, dkv_tok;
 };
 
 // ALiBi slope of (sequence b, query head h) in the exp2 domain, 0 without ALiBi
@@ -614,7 +617,8 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     const float osc = is_dk ? p.scale : 1.f;  // dK = scale * dS^T Q
     constexpr int kHalfChunks = kD / 64;      // 32-column chunks per half row
     const int c_begin = (e & 1) * kHalfChunks;
-    uint8_t* dst = static_cast<uint8_t*>(outp) + (static_cast<size_t>(seq_start + key) * p.Hkv + kvh) * kD * 2;
+    uint8_t* dst = static_cast<uint8_t*>(outp) +
+                   (static_cast<size_t>(seq_start + key) * p.dkv_tok + static_cast<size_t>(kvh) * kD) * 2;
     if (ok && n_items > 0) {
       // every lane loads (the TMEM load is warp-collective); only rows of
       // the sequence are stored
@@ -872,8 +876,10 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       // Q (group 0) or dO (group 1) row -> TMEM, two 16-bit values per column
       // (the A-operand layout: K-step kk of 16 values at columns 8kk..8kk+7);
       // rows past the sequence end are zero
-      const uint16_t* src = static_cast<const uint16_t*>(g == 0 ? p.q : p.dout) +
-                            (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD;
+      const uint16_t* src = g == 0 ? static_cast<const uint16_t*>(p.q) +
+                                         static_cast<size_t>(seq_start + qrow) * p.q_tok + static_cast<size_t>(h) * kD
+                                   : static_cast<const uint16_t*>(p.dout) +
+                                         (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD;
       const uint32_t col = g == 0 ? Sh::kColQ : Sh::kColDO;
 #pragma unroll
       for (int c = 0; c < kD / 64; ++c) {
@@ -965,7 +971,8 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
     const int e = (warp - 2) >> 2;
-    uint8_t* dst = static_cast<uint8_t*>(p.dq) + (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD * 2;
+    uint8_t* dst = static_cast<uint8_t*>(p.dq) +
+                   (static_cast<size_t>(seq_start + qrow) * p.dq_tok + static_cast<size_t>(h) * kD) * 2;
     if (e < kD / 32) {
       if (ok && n_tiles > 0) {
         uint32_t rr[32];

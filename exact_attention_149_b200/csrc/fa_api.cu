@@ -89,13 +89,16 @@ EncodeTiledFn encode_fn() {
 
 // 3-D map over a (tokens, heads, D) row-major 16-bit tensor; box = 64 columns
 // (128 B, one swizzle row) x 1 head x `rows` tokens, 128-byte swizzle.
+// tok_stride: elements from one token's row to the next (default H * D; the
+// qkv-packed layout interleaves three tensors per token)
 fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, int H, long long T,
-                       int rows) {
+                       int rows, long long tok_stride = -1) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(T)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  const long long ts = tok_stride >= 0 ? tok_stride : static_cast<long long>(H) * D;
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(ts) * 2};
   cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(rows)};
   cuuint32_t es[3] = {1u, 1u, 1u};
   CUresult r = enc(map, dt == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
@@ -213,6 +216,69 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 
 }  // namespace
 
+namespace {
+
+// q, k, v rows of token t start at t * q_tok (t * kv_tok) elements
+fa_status fwd_impl(const void* q, const void* k, const void* v, long long q_tok, long long kv_tok,
+                   void* out, float* lse, int B, int Hq, int Hkv, int S, int D, float scale,
+                   int causal, int window_left, int window_right, float softcap,
+                   const float* alibi_slopes, int alibi_batch_stride, const int32_t* cu_seqlens,
+                   int total_tokens, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd: null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be 16-byte aligned");
+  fa_status s = check_common(B, Hq, Hkv, S, D, scale, window_left, window_right, softcap, dtype,
+                             cu_seqlens, total_tokens);
+  if (s != FA_OK) return s;
+  if ((s = check_alibi(alibi_slopes, alibi_batch_stride, Hq)) != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+
+  const long long T = cu_seqlens ? total_tokens : static_cast<long long>(B) * S;
+  CUtensorMap tq, tk, tv;
+  if ((s = make_map_thd(&tq, q, dtype, D, Hq, T, 128, q_tok)) != FA_OK) return s;
+  if ((s = make_map_thd(&tk, k, dtype, D, Hkv, T, 128, kv_tok)) != FA_OK) return s;
+  if ((s = make_map_thd(&tv, v, dtype, D, Hkv, T, 128, kv_tok)) != FA_OK) return s;
+
+  fa::FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.total = static_cast<int>(T);
+  p.group = Hq / Hkv;
+  p.n_qblocks = (S + 255) / 256;
+  const float log2e = 1.4426950408889634f;
+  p.scale_log2 = scale * log2e;
+  p.softcap = softcap;
+  p.cap_in = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_out_log2 = softcap * log2e;
+  p.wl = window_left;
+  p.wr = causal ? 0 : window_right;
+  p.o = out;
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.alibi = alibi_slopes;
+  p.alibi_bstride = alibi_batch_stride;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool cap = softcap > 0.f;
+  if (D == 128) {
+    if (dtype == FA_BF16)
+      s = cap ? launch_fwd<128, true, true>(tq, tk, tv, p, st) : launch_fwd<128, true, false>(tq, tk, tv, p, st);
+    else
+      s = cap ? launch_fwd<128, false, true>(tq, tk, tv, p, st) : launch_fwd<128, false, false>(tq, tk, tv, p, st);
+  } else {
+    if (dtype == FA_BF16)
+      s = cap ? launch_fwd<64, true, true>(tq, tk, tv, p, st) : launch_fwd<64, true, false>(tq, tk, tv, p, st);
+    else
+      s = cap ? launch_fwd<64, false, true>(tq, tk, tv, p, st) : launch_fwd<64, false, false>(tq, tk, tv, p, st);
+  }
+  if (s != FA_OK) return s;
+  return ok();
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* fa_last_error(void) { return g_last_error.c_str(); }
@@ -274,57 +340,25 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
                  int Hkv, int S, int D, float scale, int causal, int window_left, int window_right,
                  float softcap, const float* alibi_slopes, int alibi_batch_stride,
                  const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype, void* stream) {
-  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd: null tensor pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
-    return fail(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be 16-byte aligned");
-  fa_status s = check_common(B, Hq, Hkv, S, D, scale, window_left, window_right, softcap, dtype,
-                             cu_seqlens, total_tokens);
-  if (s != FA_OK) return s;
-  if ((s = check_alibi(alibi_slopes, alibi_batch_stride, Hq)) != FA_OK) return s;
-  if ((s = check_device()) != FA_OK) return s;
+  return fwd_impl(q, k, v, -1, -1, out, lse, B, Hq, Hkv, S, D, scale, causal, window_left,
+                  window_right, softcap, alibi_slopes, alibi_batch_stride, cu_seqlens, total_tokens,
+                  dtype, stream);
+}
 
-  const long long T = cu_seqlens ? total_tokens : static_cast<long long>(B) * S;
-  CUtensorMap tq, tk, tv;
-  if ((s = make_map_thd(&tq, q, dtype, D, Hq, T, 128)) != FA_OK) return s;
-  if ((s = make_map_thd(&tk, k, dtype, D, Hkv, T, 128)) != FA_OK) return s;
-  if ((s = make_map_thd(&tv, v, dtype, D, Hkv, T, 128)) != FA_OK) return s;
-
-  fa::FwdParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.S = S;
-  p.total = static_cast<int>(T);
-  p.group = Hq / Hkv;
-  p.n_qblocks = (S + 255) / 256;
-  const float log2e = 1.4426950408889634f;
-  p.scale_log2 = scale * log2e;
-  p.softcap = softcap;
-  p.cap_in = softcap > 0.f ? scale / softcap : 0.f;
-  p.cap_out_log2 = softcap * log2e;
-  p.wl = window_left;
-  p.wr = causal ? 0 : window_right;
-  p.o = out;
-  p.lse = lse;
-  p.cu_seqlens = cu_seqlens;
-  p.alibi = alibi_slopes;
-  p.alibi_bstride = alibi_batch_stride;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool cap = softcap > 0.f;
-  if (D == 128) {
-    if (dtype == FA_BF16)
-      s = cap ? launch_fwd<128, true, true>(tq, tk, tv, p, st) : launch_fwd<128, true, false>(tq, tk, tv, p, st);
-    else
-      s = cap ? launch_fwd<128, false, true>(tq, tk, tv, p, st) : launch_fwd<128, false, false>(tq, tk, tv, p, st);
-  } else {
-    if (dtype == FA_BF16)
-      s = cap ? launch_fwd<64, true, true>(tq, tk, tv, p, st) : launch_fwd<64, true, false>(tq, tk, tv, p, st);
-    else
-      s = cap ? launch_fwd<64, false, true>(tq, tk, tv, p, st) : launch_fwd<64, false, false>(tq, tk, tv, p, st);
-  }
-  if (s != FA_OK) return s;
-  return ok();
+fa_status fa_fwd_qkvpacked(const void* qkv, void* out, float* lse, int B, int H, int S, int D,
+                           float scale, int causal, int window_left, int window_right,
+                           float softcap, const float* alibi_slopes, int alibi_batch_stride,
+                           const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype,
+                           void* stream) {
+  if (!qkv) return fail(FA_ERR_INVALID_ARG, "fa_fwd_qkvpacked: null qkv");
+  if (H < 1 || (D != 64 && D != 128))
+    return fail(D != 64 && D != 128 ? FA_ERR_UNSUPPORTED : FA_ERR_INVALID_ARG,
+                "fa_fwd_qkvpacked: H must be >= 1 and D 64 or 128");
+  const long long hd = static_cast<long long>(H) * D;
+  const uint16_t* base = static_cast<const uint16_t*>(qkv);
+  return fwd_impl(base, base + hd, base + 2 * hd, 3 * hd, 3 * hd, out, lse, B, H, H, S, D, scale,
+                  causal, window_left, window_right, softcap, alibi_slopes, alibi_batch_stride,
+                  cu_seqlens, total_tokens, dtype, stream);
 }
 
 }  // extern "C"

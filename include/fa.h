@@ -90,6 +90,20 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, 
                  fa_dtype dtype, void* stream);
 
 /*
+ * fa_fwd on a qkv-packed input (guide §上手…三步走: when Q, K and V are
+ * already one tensor, the packed entry avoids splitting it): qkv is
+ * (B, S, 3, H, D) (varlen: (total, 3, H, D)), i.e. token t holds its q heads,
+ * then its k heads, then its v heads; Hq = Hkv = H. out (B, S, H, D) and lse
+ * as in fa_fwd. The kernels read the three tensors in place through strided
+ * tensor maps: no copy. Arguments and errors otherwise as fa_fwd.
+ */
+FA_API fa_status fa_fwd_qkvpacked(const void* qkv, void* out, float* lse, int B, int H, int S,
+                                  int D, float scale, int causal, int window_left,
+                                  int window_right, float softcap, const float* alibi_slopes,
+                                  int alibi_batch_stride, const int32_t* cu_seqlens,
+                                  int total_tokens, fa_dtype dtype, void* stream);
+
+/*
  * Workspace bytes needed by fa_bwd for these sizes: two float32 values per
  * token and query head (the row's dot(dO, O) and its LSE in the exp2
  * domain), each sequence's rows padded to a multiple of 128, i.e.
@@ -119,6 +133,19 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  const float* alibi_slopes, int alibi_batch_stride, const int32_t* cu_seqlens,
                  int total_tokens, fa_dtype dtype, void* workspace, size_t workspace_bytes,
                  void* stream);
+
+/*
+ * fa_bwd for fa_fwd_qkvpacked: qkv (B, S, 3, H, D) as in the forward, out,
+ * lse, dout unpacked; the gradients are written packed into dqkv, the same
+ * layout as qkv. Workspace as fa_bwd_workspace_size(B, H, S, D, ...).
+ * Arguments and errors otherwise as fa_bwd.
+ */
+FA_API fa_status fa_bwd_qkvpacked(const void* qkv, const void* out, const float* lse,
+                                  const void* dout, void* dqkv, int B, int H, int S, int D,
+                                  float scale, int causal, int window_left, int window_right,
+                                  float softcap, const float* alibi_slopes, int alibi_batch_stride,
+                                  const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype,
+                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes needed by fa_fwd_kvcache: the float32 per-split partial
  * results (num_splits > 1; 0 bytes for them otherwise) and, with rotary
