@@ -3,9 +3,10 @@
 A minimax fit (Remez exchange algorithm, minimal maximum *relative* error)
 written for this library: tanh(y) = y * Q(y^2) for |y| <= 0.5, Q of degree 4
 on t = y^2 in [0, 0.25], used for softcap when every |y| of a warp's rows is
-small. The same routine also reports a degree-3 fit of 2^f on [-0.5, 0.5]
-(relative error 7.5e-5); replacing a quarter of the forward's special-function
-exponentials with it was measured and did not pay off, so no kernel uses it.
+small. The same routine also gives the degree-3 fit of 2^f on [-0.5, 0.5]
+(relative error 7.5e-5) that the forward kernel evaluates for a quarter of
+its exponentials (ex2_poly2), moving that share of the work from the
+special-function unit, which bounds the softmax, to the FMA pipe.
 
     python exact_attention_149_b200/csrc/fit_polynomials.py
 

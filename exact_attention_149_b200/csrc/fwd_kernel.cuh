@@ -63,6 +63,9 @@ struct FwdShape {
   static constexpr int kRegsLow = 88;   // warpgroup 0 after setmaxnreg.dec
   static constexpr int kRegsHigh = 208; // softmax warpgroups after setmaxnreg.inc
   static constexpr int kTmemCols = 512;
+  // of every 8 pairs of exponentials, this many run as a cubic on the FMA
+  // pipe instead of the special-function unit (which bounds the softmax)
+  static constexpr int kPolyOf8 = 2;
   static constexpr int kColS = 0;      // + 128 * t
   static constexpr int kColP = 64;     // + 128 * t
   static constexpr int kColO = 256;    // + kD * t
@@ -74,12 +77,24 @@ struct FwdBars {
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint64_t s_full[2];
-  uint64_t p_ready[2];
+  uint64_t p_ready[2][2];  // [Q tile][key half]: P of keys [64h, 64h+64) in TMEM
   uint64_t o_final[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  // the CTA's work item, written by thread 0 during setup and read back by
+  // every role after its register reallocation (so that no value crosses it)
+  int item[8];
 };
+
+struct FwdItem {
+  int seq_start, seq_len, q0, h, b, kvh, n_begin, n_tiles;
+};
+
+__device__ __forceinline__ FwdItem load_item(const FwdBars* bars) {
+  const volatile int* v = bars->item;
+  return FwdItem{v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]};
+}
 
 __device__ __forceinline__ bool fwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -144,6 +159,7 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  {
   // ---- work item: (sequence, head) major so the CTAs in flight share the
   // K/V of a few heads in L2; heaviest query blocks first within a head
   const int bh = static_cast<int>(blockIdx.x) / p.n_qblocks;
@@ -180,12 +196,16 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_ready[t], 4);
+      mbar_init(&bars->p_ready[t][0], 4);
+      mbar_init(&bars->p_ready[t][1], 4);
       mbar_init(&bars->o_final[t], 1);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
+    const int item[8] = {seq_start, seq_len, q0, h, b, kvh, n_begin, n_tiles};
+    for (int i = 0; i < 8; ++i) bars->item[i] = item[i];
     fence_mbar_init();
+  }
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, Sh::kTmemCols);
@@ -194,7 +214,6 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
   static_assert(Sh::kThreads * 168 >= 128 * Sh::kRegsLow + 256 * Sh::kRegsHigh,
                 "register split exceeds the launch pool");
@@ -205,6 +224,9 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (elect_one()) {
+      const FwdItem w = load_item(bars);
+      const int seq_start = w.seq_start, q0 = w.q0, h = w.h, kvh = w.kvh;
+      const int n_begin = w.n_begin, n_tiles = w.n_tiles;
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -238,6 +260,8 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (elect_one()) {
+      const int n_tiles = load_item(bars).n_tiles;
+      const uint32_t tmem = *static_cast<volatile uint32_t*>(&bars->tmem_base);
       constexpr uint32_t id_qk = idesc_f16(kBF16, 128, 128, false, false);
       constexpr uint32_t id_pv = idesc_f16(kBF16, 128, kD, false, true);
       // descriptors are built once; a tile or K-step offset is added to the
@@ -258,14 +282,24 @@ __global__ void __launch_bounds__(384, 1)
           umma_ss(d, a0 + off, b0 + off, id_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool first) {
+      // O_t += P_t V over keys [64 hf, 64 hf + 64) (K-steps 4 hf .. 4 hf + 3)
+      auto issue_pv = [&](int t, int slot, int hf, bool first) {
         const uint64_t b0 = dv_base + static_cast<uint64_t>((slot * Sh::kTileBytes) >> 4);
         const uint32_t d = tmem + Sh::kColO + kD * t;
         const uint32_t a = tmem + Sh::kColS + 128 * t + Sh::kColP;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
+        for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
           umma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), id_pv,
                   (first && kk == 0) ? 0u : 1u);
+      };
+      // both halves of PV_t, each as soon as its half of P is in TMEM
+      auto wait_issue_pv = [&](int t, int slot, uint32_t ph, bool first) {
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!fwd_wait(&bars->p_ready[t][hf], ph, abort)) return false;
+          tc_fence_after();
+          issue_pv(t, slot, hf, first);
+        }
+        return true;
       };
       for (int it = 0; it < n_tiles && ok; ++it) {
         const int fk = 2 * it, fv = 2 * it + 1;
@@ -276,14 +310,11 @@ __global__ void __launch_bounds__(384, 1)
         if (it > 0) {
           const int fvp = fv - 2, svp = fvp % Sh::kStages;
           // PV_0 of the previous tile, then QK_0 of this tile
-          if (!(ok = fwd_wait(&bars->p_ready[0], static_cast<uint32_t>(it - 1) & 1u, abort))) break;
-          tc_fence_after();
-          issue_pv(0, svp, it == 1);
+          const uint32_t ph = static_cast<uint32_t>(it - 1) & 1u;
+          if (!(ok = wait_issue_pv(0, svp, ph, it == 1))) break;
           issue_qk(0, sk);
           umma_commit(&bars->s_full[0]);
-          if (!(ok = fwd_wait(&bars->p_ready[1], static_cast<uint32_t>(it - 1) & 1u, abort))) break;
-          tc_fence_after();
-          issue_pv(1, svp, it == 1);
+          if (!(ok = wait_issue_pv(1, svp, ph, it == 1))) break;
           umma_commit(&bars->kv_empty[svp]);
           issue_qk(1, sk);
           umma_commit(&bars->s_full[1]);
@@ -303,10 +334,8 @@ __global__ void __launch_bounds__(384, 1)
       if (ok && n_tiles > 0) {
         const int fvl = 2 * (n_tiles - 1) + 1, svl = fvl % Sh::kStages;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = fwd_wait(&bars->p_ready[t], static_cast<uint32_t>(n_tiles - 1) & 1u, abort)))
+          if (!(ok = wait_issue_pv(t, svl, static_cast<uint32_t>(n_tiles - 1) & 1u, n_tiles == 1)))
             break;
-          tc_fence_after();
-          issue_pv(t, svl, n_tiles == 1);
           umma_commit(&bars->o_final[t]);
         }
         umma_commit(&bars->kv_empty[svl]);
@@ -319,6 +348,10 @@ __global__ void __launch_bounds__(384, 1)
   }
   } else {
     regs_inc<Sh::kRegsHigh>();
+    const FwdItem w = load_item(bars);
+    const uint32_t tmem = *static_cast<volatile uint32_t*>(&bars->tmem_base);
+    const int seq_start = w.seq_start, seq_len = w.seq_len, q0 = w.q0, h = w.h, b = w.b;
+    const int n_begin = w.n_begin, n_tiles = w.n_tiles;
     // ======================= softmax groups =======================
     const int t = (warp - 4) >> 2;            // Q tile of this group
     const int lane_base = 32 * (warp & 3);    // TMEM lanes this warp may touch
@@ -431,10 +464,9 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(x - base): one packed FMA (or add) per pair, then the 128
-      // exponentials, all issued before any result is used so that they
-      // pipeline through the special-function unit; then the row sum and
-      // the 16-bit P tile
+      // P = 2^(x - base): one packed FMA (or add) per pair, then the
+      // exponentials, 64 at a time, all issued before any of their results is
+      // used so that they pipeline through the special-function unit
       const float2 nb2 = make_float2(-base, -base);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
@@ -444,27 +476,40 @@ __global__ void __launch_bounds__(384, 1)
         x[i] = d.x;
         x[i + 1] = d.y;
       }
-#pragma unroll
-      for (int i = 0; i < 128; ++i) x[i] = ex2_approx(x[i]);
+      // the two halves of the row in turn: 64 exponentials, then their 16-bit
+      // P into TMEM and a signal, so that the tensor core starts on the first
+      // half of PV while the second half is exponentiated
       float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) sum2[(i >> 1) & 3] = __fadd2_rn(sum2[(i >> 1) & 3], make_float2(x[i], x[i + 1]));
+      for (int hf = 0; hf < 2; ++hf) {
+        float* xh = x + 64 * hf;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+        for (int i = 0; i < 64; i += 2) {
+          if (((i >> 1) & 7) < Sh::kPolyOf8) {
+            const float2 e = ex2_poly2(make_float2(xh[i], xh[i + 1]));
+            xh[i] = e.x;
+            xh[i + 1] = e.y;
+          } else {
+            xh[i] = ex2_approx(xh[i]);
+            xh[i + 1] = ex2_approx(xh[i + 1]);
+          }
+        }
         uint32_t r[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = pack2_alu<kBF16>(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]);
-        tmem_st32(t_p + c * 32, r);
+        for (int i = 0; i < 32; ++i) {
+          r[i] = pack2_alu<kBF16>(xh[2 * i], xh[2 * i + 1]);
+          sum2[i & 3] = __fadd2_rn(sum2[i & 3], make_float2(xh[2 * i], xh[2 * i + 1]));
+        }
+        tmem_st32(t_p + hf * 32, r);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_ready[t][hf]);
       }
       const float2 s01 = __fadd2_rn(sum2[0], sum2[1]), s23 = __fadd2_rn(sum2[2], sum2[3]);
       const float2 s4 = __fadd2_rn(s01, s23);
-      const float lsum = s4.x + s4.y;
-      l_run += lsum;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_ready[t]);
+      l_run += s4.x + s4.y;
     }
     // ---- epilogue: O / l and LSE ----
     if (ok && n_tiles > 0) ok = fwd_wait(&bars->o_final[t], 0, abort);
@@ -506,7 +551,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, Sh::kTmemCols);
+    tmem_dealloc(*static_cast<volatile uint32_t*>(&bars->tmem_base), Sh::kTmemCols);
   }
 }
 

@@ -318,6 +318,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for a pair of values on the FMA and integer pipes instead of the
+// special-function unit. x = n + f with n = round(x) (adding 1.5 * 2^23
+// rounds to an integer held in the low mantissa bits) and f in [-1/2, 1/2];
+// 2^f is a cubic fitted for minimal relative error by the Remez exchange
+// algorithm (fit_polynomials.py next to this file; float32 relative error
+// 7.5e-5), and n is added into the exponent field: the low 9 bits of the
+// rounded value's bit pattern, shifted by 23, are n << 23 modulo 2^32.
+// x is clamped at -126 so that the exponent cannot underflow: smaller inputs
+// (masked logits, -inf) give a value below 2^-125 rather than 0.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 j = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(j, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(f, make_float2(5.517166906e-02f, 5.517166906e-02f),
+                        make_float2(2.426111222e-01f, 2.426111222e-01f));
+  q = __ffma2_rn(q, f, make_float2(6.932609855e-01f, 6.932609855e-01f));
+  q = __ffma2_rn(q, f, make_float2(9.999280735e-01f, 9.999280735e-01f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(j.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(j.y) << 23)));
+}
+
 // tanh from the identity tanh(y) = sign(y) (1 - e) / (1 + e), e = exp(-2|y|),
 // with e taken as 2^(-2 |y| log2(e)). Absolute error ~2e-7 (the subtraction
 // 1 - e near y = 0 and the exp2/rcp approximations); with softcap c the
