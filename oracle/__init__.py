@@ -10,8 +10,11 @@ from .attention import (  # noqa: F401
     attention_fwd,
     head_bwd,
     head_fwd,
+    dequantize_int8,
     kvcache_decode,
+    kvcache_decode_int8,
     lse_combine,
+    quantize_int8,
     rotary,
     round_to,
     scores,

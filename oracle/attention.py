@@ -42,6 +42,14 @@ notes of the repository):
 * ``cache_seqlens[b]`` is the length *before* the append; the new token lands
   at position ``cache_seqlens[b]`` and attention covers ``cache_seqlens[b]+1``
   keys.
+* "FlashAttention技术深度解析：重塑LLM推理性能的新范式" §发展趋势 /
+  量化技术融合 mentions an INT8/INT4 quantised KV cache but gives no format; the int8 cache here is symmetric with one
+  float32 scale per (token, kv head) row: ``scale = max|x| / 127`` and
+  ``code = round-half-even(x / scale)``, both in float32 (the precision the
+  kernel takes the integer decision in), an all-zero row having scale 0 and
+  codes 0. A cached row stands for ``code * scale``; a new key is rotated (with
+  rotary) and rounded to the 16-bit input type first, as the 16-bit cache
+  stores it, then quantised.
 
 Every array is float64. 16-bit inputs are converted exactly (every bf16 and
 fp16 value is representable in float64), so the oracle sees the same values
@@ -60,6 +68,9 @@ __all__ = [
     "attention_fwd",
     "attention_bwd",
     "kvcache_decode",
+    "kvcache_decode_int8",
+    "quantize_int8",
+    "dequantize_int8",
     "lse_combine",
     "rotary",
     "round_to",
@@ -393,6 +404,76 @@ def kvcache_decode(q, k_new, v_new, k_cache_logical, v_cache_logical, cache_seql
             o[b, :, h] = ob
             lse[b, h, :] = lb
     return o, lse, ks, vs
+
+
+def quantize_int8(x):
+    """Symmetric int8 quantisation of each row (the last axis) of ``x``.
+
+    In float32, as the reading in the module header states: ``scale = max|x| /
+    127`` and ``code = round-half-even(x / scale)`` (IEEE division, numpy's
+    ``rint``); a row of zeros gets scale 0 and codes 0. Returns (codes int8 of
+    x's shape, scales float32 of x's shape without the last axis).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    div = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    codes = np.rint((x32 / div[..., None]).astype(np.float32))
+    codes = np.where(scale[..., None] > 0, codes, np.float32(0.0))
+    return np.clip(codes, -127, 127).astype(np.int8), scale
+
+
+def dequantize_int8(codes, scales):
+    """The values an int8 cache stands for: ``code * scale`` per row (float64)."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def kvcache_decode_int8(q, k_new, v_new, k_codes_logical, k_scales_logical, v_codes_logical,
+                        v_scales_logical, cache_seqlens, scale: float, causal: bool = True,
+                        window=(-1, -1), softcap: float = 0.0, heads=None, rotary_cos=None,
+                        rotary_sin=None, rotary_interleaved=False, rotated_dtype=None,
+                        alibi_slopes=None):
+    """kvcache_decode against an int8 cache (the quantised-cache reading above).
+
+    k/v_codes_logical: B arrays of at least cache_seqlens[b] rows (rows, Hkv, D)
+    of int8 codes; k/v_scales_logical: B arrays (rows, Hkv) of float32 scales.
+    The Sq new rows are quantised (keys after rotation and rounding to
+    ``rotated_dtype``) and appended; then every cached row is replaced by the
+    value it stands for and the step is kvcache_decode's, with the appended
+    rows already in the cache. Returns (O, LSE, appended k codes, k scales,
+    v codes, v scales), the last four as lists of the B sequences' new rows.
+    """
+    bsz, sq = np.asarray(q).shape[:2]
+    append = k_new is not None
+    kd, vd, kc_new, ks_new, vc_new, vs_new = [], [], [], [], [], []
+    lengths = []
+    for b in range(bsz):
+        n = int(cache_seqlens[b])
+        kc = np.asarray(k_codes_logical[b])[:n]
+        ksc = np.asarray(k_scales_logical[b])[:n]
+        vc = np.asarray(v_codes_logical[b])[:n]
+        vsc = np.asarray(v_scales_logical[b])[:n]
+        if append:
+            kn = _f64(k_new[b])
+            if rotary_cos is not None:
+                pos = np.arange(n, n + sq)
+                kn = round_to(rotary(kn, pos, rotary_cos, rotary_sin, rotary_interleaved),
+                              rotated_dtype)
+            a_kc, a_ks = quantize_int8(kn)
+            a_vc, a_vs = quantize_int8(_f64(v_new[b]))
+            kc_new.append(a_kc)
+            ks_new.append(a_ks)
+            vc_new.append(a_vc)
+            vs_new.append(a_vs)
+            kc, ksc = np.concatenate([kc, a_kc]), np.concatenate([ksc, a_ks])
+            vc, vsc = np.concatenate([vc, a_vc]), np.concatenate([vsc, a_vs])
+        kd.append(dequantize_int8(kc, ksc))
+        vd.append(dequantize_int8(vc, vsc))
+        lengths.append(kc.shape[0])
+    o, lse, _, _ = kvcache_decode(q, None, None, kd, vd, np.asarray(lengths), scale, causal,
+                                  window, softcap, heads, rotary_cos, rotary_sin,
+                                  rotary_interleaved, rotated_dtype, alibi_slopes)
+    return o, lse, kc_new, ks_new, vc_new, vs_new
 
 
 def lse_combine(o_parts, lse_parts):
