@@ -311,3 +311,10 @@ def decode_kv_bytes(cache_seqlens, Hkv, D, elem_bytes=2):
     value row of every kv head, once (L_b + 1 keys per sequence)."""
     n = int(torch.as_tensor(cache_seqlens, dtype=torch.int64).sum().item()) + len(cache_seqlens)
     return 2 * n * Hkv * D * elem_bytes
+
+
+def decode_kv_bytes_int8(cache_seqlens, Hkv, D):
+    """The same for an int8 cache: per row D one-byte codes and a 4-byte
+    float32 scale."""
+    n = int(torch.as_tensor(cache_seqlens, dtype=torch.int64).sum().item()) + len(cache_seqlens)
+    return 2 * n * Hkv * (D + 4)

@@ -277,11 +277,20 @@ def run_only(args, dist: Dist):
         kn, vn = st["k_new"].to(dev), st["v_new"].to(dev)
         cs, bt = st["cache_seqlens"].to(dev), st["block_table"].to(dev)
         kv_bytes = W.decode_kv_bytes(st["cache_seqlens"], cd.Hkv, cd.D)
-        fn = lambda: fa.fwd_kvcache(q, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale,  # noqa: E731
-                                    causal=True, num_splits=args.splits)
+        if args.int8:
+            kc, ksc = fa.kv_quantize_int8(kc)
+            vc, vsc = fa.kv_quantize_int8(vc)
+            kv_bytes = W.decode_kv_bytes_int8(st["cache_seqlens"], cd.Hkv, cd.D)
+            fn = lambda: fa.fwd_kvcache(q, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale,  # noqa: E731
+                                        causal=True, num_splits=args.splits, k_scale=ksc,
+                                        v_scale=vsc)
+        else:
+            fn = lambda: fa.fwd_kvcache(q, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale,  # noqa: E731
+                                        causal=True, num_splits=args.splits)
         ms = timed(fn, args.steps, args.warmup, dist)
         gbs = kv_bytes / (ms * 1e-3) / 1e9
-        out.update(ms=ms, gbs=gbs, frac_of_hbm=gbs / peaks["hbm_gbs"], splits=args.splits, B=B)
+        out.update(ms=ms, gbs=gbs, frac_of_hbm=gbs / peaks["hbm_gbs"], splits=args.splits, B=B,
+                   int8=bool(args.int8))
     return out
 
 
@@ -460,7 +469,43 @@ def run_ours(args, dist: Dist):
                        "traffic": trd["bytes_per_launch"] if trd else None,
                        "peak_source": peaks["source"] + " HBM copy"}
     res["decode"] = dec
+
+    # -------------------- the same decode step on an int8 cache --------------------
+    # the 16-bit pool quantised on the device (fa_kv_quantize_int8); the step
+    # then reads D + 4 bytes per cached row instead of 2 D
+    kq, ksq = fa.kv_quantize_int8(kc)
+    vq, vsq = fa.kv_quantize_int8(vc)
     del kc, vc
+    torch.cuda.empty_cache()
+    kv8 = W.decode_kv_bytes_int8(st["cache_seqlens"], cd.Hkv, cd.D)
+    dec8 = {"kv_bytes": kv8, "format": "int8 codes + one float32 scale per (token, kv head) row",
+            "splits": {}}
+    for splits in cd.splits:
+        wsd = fa.fa_kvcache_workspace_size(cd.B, 1, cd.Hq, cd.D, splits)
+        wsb = torch.empty(max(wsd, 1), dtype=torch.uint8, device=dev)
+
+        def step_dec8(splits=splits, wsb=wsb):
+            fa.fwd_kvcache(dq_, kq, vq, cs, bt, k_new=kn, v_new=vn, scale=cd.scale, causal=True,
+                           num_splits=splits, out=dout, lse=dlse, workspace=wsb, k_scale=ksq,
+                           v_scale=vsq)
+
+        ms_d = timed(step_dec8, max(args.steps, 20), args.warmup, dist, fa_mod=fa)
+        ksplit, nsplit = fa.fa_kernel_timing_read("decode_split")
+        fa.fa_kernel_timing_reset()
+        gbs = kv8 / (ms_d * 1e-3) / 1e9
+        entry = {"ms": ms_d, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                 "speedup_vs_16bit": dec["splits"][str(splits)]["ms"] / ms_d}
+        if nsplit:
+            ks = ksplit / nsplit
+            entry["decode_split_kernel"] = {
+                "ms_avg": ks, "gbs": kv8 / (ks * 1e-3) / 1e9,
+                "frac_of_hbm": kv8 / (ks * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        dec8["splits"][str(splits)] = entry
+    best8 = max(dec8["splits"].values(), key=lambda d: d["gbs"])
+    dec8["best_gbs"] = best8["gbs"]
+    dec8["best_frac_of_hbm"] = best8["frac_of_hbm"]
+    res["decode_int8"] = dec8
+    del kq, vq, ksq, vsq
     torch.cuda.empty_cache()
 
     # -------------------- roofline of the dominant kernel --------------------
@@ -607,6 +652,7 @@ def main():
     ap.add_argument("--only", default=None, choices=["fwd", "bwd", "varlen", "decode"],
                     help="time one kernel family only (profiling runs)")
     ap.add_argument("--splits", type=int, default=16, help="num_splits for --only decode")
+    ap.add_argument("--int8", action="store_true", help="--only decode on an int8 cache")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="batch for --only decode (default: the B64 workload); smaller for ncu")
     args = ap.parse_args()

@@ -26,7 +26,7 @@ __all__ = [
     "fa_get_device_status", "fa_last_error", "fa_version",
     "fa_kernel_timing_enable", "fa_kernel_timing_read", "fa_kernel_timing_reset",
     "fwd", "bwd", "fwd_kvcache", "fwd_qkvpacked", "bwd_qkvpacked", "fa_fwd_qkvpacked",
-    "fa_bwd_qkvpacked",
+    "fa_bwd_qkvpacked", "fa_fwd_kvcache_int8", "fa_kv_quantize_int8", "kv_quantize_int8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -77,6 +77,11 @@ lib.fa_fwd_kvcache.restype = _i
 lib.fa_fwd_kvcache.argtypes = _KV_ARGS + [_p, _z, _p]
 lib.fa_fwd_kvcache_noalloc.restype = _i
 lib.fa_fwd_kvcache_noalloc.argtypes = _KV_ARGS + [_p]
+# as _KV_ARGS with k_scale, v_scale after v_cache
+lib.fa_fwd_kvcache_int8.restype = _i
+lib.fa_fwd_kvcache_int8.argtypes = [_p] * 13 + _KV_ARGS[11:] + [_p, _z, _p]
+lib.fa_kv_quantize_int8.restype = _i
+lib.fa_kv_quantize_int8.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.fa_bwd_workspace_size.restype = _z
 lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 lib.fa_kvcache_workspace_size.restype = _z
@@ -198,6 +203,28 @@ def fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens
                               window_right, softcap, _ptr(alibi_slopes), alibi_batch_stride,
                               num_splits, dtype, _ptr(workspace), workspace_bytes,
                               _stream(stream)))
+
+
+def fa_fwd_kvcache_int8(q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_table,
+                        cache_seqlens, rotary_cos, rotary_sin, out, lse, B, Sq, Hq, Hkv, D,
+                        page_size, max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+                        rotary_interleaved, scale, causal, window_left, window_right, softcap,
+                        alibi_slopes, alibi_batch_stride, num_splits, dtype, workspace,
+                        workspace_bytes, stream=None):
+    _check(lib.fa_fwd_kvcache_int8(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+                                   _ptr(cache_seqlens), _ptr(rotary_cos), _ptr(rotary_sin),
+                                   _ptr(out), _ptr(lse), B, Sq, Hq, Hkv, D, page_size,
+                                   max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+                                   int(rotary_interleaved), scale, int(causal), window_left,
+                                   window_right, softcap, _ptr(alibi_slopes), alibi_batch_stride,
+                                   num_splits, dtype, _ptr(workspace), workspace_bytes,
+                                   _stream(stream)))
+
+
+def fa_kv_quantize_int8(src, codes, scales, num_pages, page_size, Hkv, D, dtype, stream=None):
+    _check(lib.fa_kv_quantize_int8(_ptr(src), _ptr(codes), _ptr(scales), num_pages, page_size,
+                                   Hkv, D, dtype, _stream(stream)))
 
 
 # size of the library's static scratch array used by fa_fwd_kvcache_noalloc
@@ -366,15 +393,20 @@ def bwd_qkvpacked(qkv, out, lse, dout, scale=None, causal=False, window=(-1, -1)
 def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_new=None,
                 rotary_cos=None, rotary_sin=None, rotary_interleaved=False, scale=None,
                 causal=True, window=(-1, -1), softcap=0.0, num_splits=1, out=None, lse=None,
-                workspace=None, alibi_slopes=None, stream=None):
+                workspace=None, alibi_slopes=None, stream=None, k_scale=None, v_scale=None):
     """One decode step: q (B,Sq,Hq,D); caches (num_pages, page_size, Hkv, D)
     with block_table int32 (B, max_pages), or block_table None and contiguous
     caches (B, capacity, Hkv, D); cache_seqlens int32 (B). Appends
     k_new/v_new (B,Sq,Hkv,D) in place, then attends. rotary_cos/rotary_sin:
     float32 (rows, rotary_dim/2) tables that rotate q and k_new at their
-    positions. Returns (out (B,Sq,Hq,D), lse (B,Hq,Sq))."""
+    positions. int8 caches (codes) take their float32 row scales k_scale,
+    v_scale (num_pages, Hkv, page_size) and run fa_fwd_kvcache_int8.
+    Returns (out (B,Sq,Hq,D), lse (B,Hq,Sq))."""
     _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new, rotary_cos,
-               rotary_sin)
+               rotary_sin, k_scale, v_scale)
+    q8 = k_cache.dtype == torch.int8
+    if q8 != (k_scale is not None) or (k_scale is None) != (v_scale is None):
+        raise FaError(FA_ERR_INVALID_ARG, "int8 caches take k_scale and v_scale; 16-bit caches take neither")
     B, Sq, Hq, D = q.shape
     num_pages, page_size, Hkv, _ = k_cache.shape
     max_pages = 1 if block_table is None else block_table.shape[1]
@@ -389,9 +421,26 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
     nbytes = fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits, rot_dim)
     if workspace is None and nbytes > 0:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, rotary_cos,
-                   rotary_sin, out, lse, B, Sq, Hq, Hkv, D, page_size, max_pages, num_pages,
-                   rot_rows, rot_dim, rotary_interleaved, _scale(scale, D), causal, window[0],
-                   window[1], softcap, *_alibi(alibi_slopes, Hq), num_splits, _dt(q), workspace,
-                   0 if workspace is None else workspace.numel(), stream)
+    args = (block_table, cache_seqlens, rotary_cos, rotary_sin, out, lse, B, Sq, Hq, Hkv, D,
+            page_size, max_pages, num_pages, rot_rows, rot_dim, rotary_interleaved,
+            _scale(scale, D), causal, window[0], window[1], softcap, *_alibi(alibi_slopes, Hq),
+            num_splits, _dt(q), workspace, 0 if workspace is None else workspace.numel(), stream)
+    if q8:
+        fa_fwd_kvcache_int8(q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, *args)
+    else:
+        fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, *args)
     return out, lse
+
+
+def kv_quantize_int8(cache, codes=None, scales=None, stream=None):
+    """A 16-bit cache (num_pages, page_size, Hkv, D) -> (int8 codes of the
+    same shape, float32 scales (num_pages, Hkv, page_size)) in the format of
+    fa_fwd_kvcache_int8."""
+    _need_cuda(cache, codes, scales)
+    num_pages, page_size, Hkv, D = cache.shape
+    if codes is None:
+        codes = torch.empty(cache.shape, dtype=torch.int8, device=cache.device)
+    if scales is None:
+        scales = torch.empty((num_pages, Hkv, page_size), dtype=torch.float32, device=cache.device)
+    fa_kv_quantize_int8(cache, codes, scales, num_pages, page_size, Hkv, D, _dt(cache), stream)
+    return codes, scales

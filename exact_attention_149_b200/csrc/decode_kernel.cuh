@@ -24,6 +24,14 @@
 //   O^T[16 d x 8 columns]     += V^T[16 d x 16 tokens] . P^T[16 tokens x 8 columns]
 // P^T's fragment is the transpose of S^T's accumulator fragment, done with
 // movmatrix.
+//
+// int8 cache: the chunks arrive as int8 codes plus one float32 scale per
+// (token, kv head) row; each consumer warp converts its 16 rows of codes to
+// exact 16-bit values in its own shared-memory tiles (K in the input type, V
+// in fp16) and the products above run on them: the K scale multiplies the
+// rows of S^T, and the V scale, divided by the largest V scale the warp has
+// seen, multiplies P (so the fp16 P keeps 11 bits without overflow); that
+// largest scale is folded into the accumulator's online rescale.
 #pragma once
 
 #include "ptx.cuh"
@@ -60,6 +68,10 @@ struct DecodeParams {
   int right;              // visible keys end at position + right (-1 = unbounded; causal = 0)
   const float* alibi;     // ALiBi slopes, nullable: slope of (b, hq) = alibi[b * alibi_bstride + hq]
   int alibi_bstride;
+  // int8 cache: k_cache / v_cache hold codes, these the per-row scales,
+  // (num_pages, Hkv, page_size) fp32; null for a 16-bit cache
+  float* k_scale;
+  float* v_scale;
 };
 
 // Keys visible to the query at position `qpos` of a sequence of Lk keys:
@@ -124,8 +136,35 @@ __device__ __forceinline__ uint4 rotate8(const uint16_t* row, int d0, const floa
   return pack8<kBF16>(y);
 }
 
-// grid B * Sq (one block per new token), block 128: 16 bytes per thread-step
-template <bool kBF16>
+// Symmetric int8 quantisation of one head row of D values held by 16 lanes
+// (8 consecutive values each; lanes at or past D / 8 hold zeros): scale =
+// max|x| / 127, code = round-half-even(x / scale), both in fp32 with IEEE
+// division; a zero row has scale 0 and codes 0. Returns the lane's 8 codes
+// packed little-endian into two words; *scale gets the row's scale.
+__device__ __forceinline__ uint2 quantize_row8(const float (&x)[8], float* scale) {
+  float am = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(x[j]));
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+  const float sc = __fdiv_rn(am, 127.f);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    int c = sc > 0.f ? __float2int_rn(__fdiv_rn(x[j], sc)) : 0;
+    c = max(-127, min(127, c));
+    w[j >> 2] |= (static_cast<uint32_t>(c) & 0xffu) << (8 * (j & 3));
+  }
+  *scale = sc;
+  return make_uint2(w[0], w[1]);
+}
+
+// grid B * Sq (one block per new token), block 128: 16 bytes per thread-step.
+// kQ8: the new rows are quantised into an int8 cache (keys after the rotary
+// rotation and the rounding to the 16-bit type, as the 16-bit cache stores
+// them); each warp takes heads warp, warp + 4, ..., lanes 0-15 the key row and
+// lanes 16-31 the value row.
+template <bool kBF16, bool kQ8>
 __global__ void kv_append_kernel(const DecodeParams p) {
   const int b = blockIdx.x / p.Sq, t = blockIdx.x % p.Sq;
   const int L = p.cache_seqlens[b];
@@ -165,6 +204,31 @@ __global__ void kv_append_kernel(const DecodeParams p) {
   const size_t src = (static_cast<size_t>(b) * p.Sq + t) * p.Hkv * p.D;
   const uint16_t* kn = static_cast<const uint16_t*>(p.k_new) + src;
   const uint16_t* vn = static_cast<const uint16_t*>(p.v_new) + src;
+  if constexpr (kQ8) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = lane >> 4, li = lane & 15;
+    const bool act = li < groups;
+    for (int h = warp; h < p.Hkv; h += blockDim.x >> 5) {
+      float x[8];
+      if (act) {
+        const uint4 raw = half == 0 ? rotate8<kBF16>(kn + h * p.D, li * 8, cs, sn, p)
+                                    : *reinterpret_cast<const uint4*>(vn + h * p.D + li * 8);
+        unpack8<kBF16>(raw, x);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = 0.f;
+      }
+      float sc;
+      const uint2 codes = quantize_row8(x, &sc);
+      uint8_t* cache = static_cast<uint8_t*>(half == 0 ? p.k_cache : p.v_cache);
+      if (act) *reinterpret_cast<uint2*>(cache + dst + h * p.D + li * 8) = codes;
+      if (li == 0) {
+        float* scales = half == 0 ? p.k_scale : p.v_scale;
+        scales[(static_cast<size_t>(page) * p.Hkv + h) * p.page_size + pos % p.page_size] = sc;
+      }
+    }
+    return;
+  }
   uint16_t* kc = static_cast<uint16_t*>(p.k_cache) + dst;
   uint16_t* vc = static_cast<uint16_t*>(p.v_cache) + dst;
   for (int i = threadIdx.x; i < p.Hkv * groups; i += blockDim.x) {
@@ -173,6 +237,79 @@ __global__ void kv_append_kernel(const DecodeParams p) {
     *reinterpret_cast<uint4*>(kc + e) = rotate8<kBF16>(kn + h * p.D, d0, cs, sn, p);
     *reinterpret_cast<uint4*>(vc + e) = *reinterpret_cast<const uint4*>(vn + e);
   }
+}
+
+// A 16-bit cache (rows, Hkv, D), rows = num_pages * page_size, into int8
+// codes of the same shape and scales (num_pages, Hkv, page_size): one
+// (row, head) unit per 16-lane half-warp, eight units per 128-thread block.
+template <bool kBF16>
+__global__ void kv_quantize_kernel(const uint16_t* src, uint8_t* codes, float* scales, long long units,
+                                   int Hkv, int D, int page_size) {
+  const int li = threadIdx.x & 15;
+  const long long u = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 4);
+  const bool act = u < units && li < (D >> 3);
+  float x[8];
+  if (act) {
+    unpack8<kBF16>(*reinterpret_cast<const uint4*>(src + u * D + li * 8), x);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = 0.f;
+  }
+  float sc;
+  const uint2 c = quantize_row8(x, &sc);
+  if (act) *reinterpret_cast<uint2*>(codes + u * D + li * 8) = c;
+  if (u < units && li == 0) {
+    const long long row = u / Hkv;
+    const int h = static_cast<int>(u % Hkv);
+    scales[((row / page_size) * Hkv + h) * page_size + row % page_size] = sc;
+  }
+}
+
+// Two biased codes (code + 128, bytes 0, 1 of w, or bytes 2, 3 with hi) ->
+// their exact fp16 pair: 0x64 above a biased byte is the fp16 value 1024 +
+// code + 128, and subtracting 1152 leaves the code.
+__device__ __forceinline__ uint32_t i8pair_to_f16(uint32_t w, bool hi) {
+  const uint32_t h = __byte_perm(w, 0x64646464u, hi ? 0x4342u : 0x4140u);
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h),
+                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// 16 int8 codes -> 16 exact 16-bit values (two uint4 of 8), without the
+// special-function unit. bf16: each biased byte (code + 128) becomes the low
+// mantissa byte of 2^23, so the fp32 value is 2^23 + code + 128; subtracting
+// 2^23 + 128 leaves the code, whose upper 16 bits are its exact bf16. fp16:
+// 0x64 above a biased byte is the fp16 value 1024 + code + 128; subtracting
+// 1152 leaves the code.
+template <bool kBF16>
+__device__ __forceinline__ void i8x16_to_16bit(const uint4& a, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t u = w[i] ^ 0x80808080u;
+    if constexpr (kBF16) {
+      const float2 bias = make_float2(-8388736.f, -8388736.f);
+      const float2 f01 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)),
+                                                __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541))),
+                                    bias);
+      const float2 f23 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)),
+                                                __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543))),
+                                    bias);
+      o[2 * i] = __byte_perm(__float_as_uint(f01.x), __float_as_uint(f01.y), 0x7632);
+      o[2 * i + 1] = __byte_perm(__float_as_uint(f23.x), __float_as_uint(f23.y), 0x7632);
+    } else {
+      const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152
+      const uint32_t h01 = __byte_perm(u, 0x64646464u, 0x4140);
+      const uint32_t h23 = __byte_perm(u, 0x64646464u, 0x4342);
+      const __half2 r01 = __hsub2(*reinterpret_cast<const __half2*>(&h01), bias);
+      const __half2 r23 = __hsub2(*reinterpret_cast<const __half2*>(&h23), bias);
+      o[2 * i] = *reinterpret_cast<const uint32_t*>(&r01);
+      o[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&r23);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // ---------------------------------------------------------------------------
@@ -219,20 +356,38 @@ __device__ __forceinline__ uint32_t sw128(uint32_t base, int r, int g) {
   return base + r * 128 + ((g ^ (r & 7)) << 4);
 }
 
-template <int kD>
+// kQ8: the ring holds int8 chunks (K codes, V codes, then the 64 K and 64 V
+// scales). D = 128: the code tiles arrive with the 128-byte swizzle and the
+// consumers build their fragments from them in registers. D = 64: unswizzled
+// tiles, and each consumer warp converts its 16 rows into 16-bit tiles in its
+// own scratch (K then V, 16 rows x 128 B in the 128-byte swizzle of the TMA
+// tiles) before the tensor-core steps.
+template <int kD, bool kQ8 = false>
 struct DecShape {
   static constexpr int kTok = 64;                      // tokens per chunk
   static constexpr int kChunks = kD / 64;              // 128-byte column chunks
   static constexpr int kBoxBytes = kTok * 128;         // 64 rows x 128 B
-  static constexpr int kKVBytes = kChunks * kBoxBytes; // K or V of one chunk
-  static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int kStages = kD == 128 ? 3 : 6;   // 2 CTAs per SM
-  static constexpr int kBarOffset = kStages * kStageBytes;
-  // cross-warp reduction scratch aliases the stage ring: it is written only
-  // after every issued chunk has been consumed
+  static constexpr int kKVBytes = kQ8 ? kTok * kD : kChunks * kBoxBytes;  // K or V of one chunk
+  static constexpr int kScaleOffset = 2 * kKVBytes;    // int8: 64 K scales, 64 V scales
+  // bytes the producer loads into a stage (the full barrier's transaction
+  // count); int8 stages are padded to 1 KB, which the 128-byte-swizzled TMA
+  // tiles need, so the stage stride can exceed the loaded bytes
+  static constexpr int kLoadBytes = 2 * kKVBytes + (kQ8 ? 2 * kTok * 4 : 0);
+  static constexpr int kStageBytes = kQ8 ? (kLoadBytes + 1023) / 1024 * 1024 : kLoadBytes;
+  static constexpr int kStages = kQ8 ? (kD == 128 ? 4 : 6) : (kD == 128 ? 3 : 6);  // 2 CTAs per SM
+  // int8 with D = 128 builds the tensor-core fragments straight from the
+  // swizzled int8 tiles in registers; D = 64 converts through a scratch
+  static constexpr bool kDirect = kQ8 && kD == 128;
+  static constexpr int kScrHalfBytes = kChunks * 16 * 128;   // 16 rows of K (or V), 16-bit
+  static constexpr int kScrOffset = kStages * kStageBytes;
+  static constexpr int kScrBytes = (kQ8 && !kDirect) ? 4 * 2 * kScrHalfBytes : 0;
+  static constexpr int kBarOffset = kScrOffset + kScrBytes;
+  // cross-warp reduction scratch aliases the stage ring (and the int8
+  // scratch): it is written only after every issued chunk has been consumed
   static constexpr int kRedOffset = 0;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
   static constexpr int kThreads = 160;                 // 4 consumer warps + 1 producer
+  static_assert(kScrOffset % 1024 == 0 && kStageBytes % 128 == 0, "scratch and stage alignment");
 };
 
 struct DecBars {
@@ -248,12 +403,13 @@ __device__ __forceinline__ float dec_logit(float s, const DecodeParams& p) {
 
 // kNT: number of 8-wide column tiles per CTA (a column block holds 8 * kNT
 // columns; column n is new token n / group, query head kvh * group + n % group)
-template <int kD, bool kBF16, int kNT>
+template <int kD, bool kBF16, int kNT, bool kQ8>
 __global__ void __launch_bounds__(160)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using Sh = DecShape<kD>;
+  using Sh = DecShape<kD, kQ8>;
   static_assert(sizeof(DecBars) <= 256, "barrier block exceeds its reservation");
+  static_assert((8 * 8 * kNT + 4 * 8 * kNT * kD) * 4 <= Sh::kBarOffset, "reduction scratch exceeds the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -335,12 +491,22 @@ __global__ void __launch_bounds__(160)
           page = 0;  // stay in bounds; the result is flagged as invalid
         }
         const int row = page * p.page_size + (pos % p.page_size);
-        mbar_arrive_expect_tx(&bars->full[slot], Sh::kStageBytes);
+        mbar_arrive_expect_tx(&bars->full[slot], Sh::kLoadBytes);
         uint8_t* dst = smem + slot * Sh::kStageBytes;
-        for (int c = 0; c < Sh::kChunks; ++c) {
-          tma_load_3d(&tm_k, &bars->full[slot], dst + c * Sh::kBoxBytes, c * 64, kvh, row);
-          tma_load_3d(&tm_v, &bars->full[slot], dst + Sh::kKVBytes + c * Sh::kBoxBytes, c * 64, kvh,
-                      row);
+        if constexpr (kQ8) {
+          // one box of 64 rows x kD bytes each, then the chunk's scales: 64
+          // contiguous floats of (page, kvh) (page_size is a multiple of 64)
+          tma_load_3d(&tm_k, &bars->full[slot], dst, 0, kvh, row);
+          tma_load_3d(&tm_v, &bars->full[slot], dst + Sh::kKVBytes, 0, kvh, row);
+          const size_t so = (static_cast<size_t>(page) * p.Hkv + kvh) * p.page_size + pos % p.page_size;
+          bulk_load(dst + Sh::kScaleOffset, p.k_scale + so, Sh::kTok * 4, &bars->full[slot]);
+          bulk_load(dst + Sh::kScaleOffset + Sh::kTok * 4, p.v_scale + so, Sh::kTok * 4, &bars->full[slot]);
+        } else {
+          for (int c = 0; c < Sh::kChunks; ++c) {
+            tma_load_3d(&tm_k, &bars->full[slot], dst + c * Sh::kBoxBytes, c * 64, kvh, row);
+            tma_load_3d(&tm_v, &bars->full[slot], dst + Sh::kKVBytes + c * Sh::kBoxBytes, c * 64, kvh,
+                        row);
+          }
         }
       }
       // drain the loads still in flight
@@ -355,7 +521,48 @@ __global__ void __launch_bounds__(160)
   // ======================= consumers (warps 0..3) =======================
   // Q^T fragments: B[k = d][n = column], n = lane / 4 within each 8-column tile
   uint32_t qf[kNT][kD / 16][2];
-  {
+  // int8, D = 128: the contraction index is permuted so that lane j = lane % 4
+  // owns d in [32 j, 32 j + 32): K-step kk, fragment k = 2j, 2j+1 <-> d =
+  // 32j + 4kk + {0, 1} and k = 2j+8, 2j+9 <-> d = 32j + 4kk + {2, 3}. The
+  // queries enter as fp16, each column scaled by an exact power of two 2^-e
+  // (its largest |q| lands in [2^14, 2^15)); qsc holds 2^e of this lane's two
+  // accumulator columns 2j, 2j+1.
+  float qsc[kNT][2];
+  if constexpr (Sh::kDirect) {
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      const int n = n0 + nt * 8 + (lane >> 2);
+      const bool real = n < p.n_cols;
+      const int t = real ? n / p.group : 0, hl = real ? n % p.group : 0;
+      const uint16_t* row = static_cast<const uint16_t*>(p.q) +
+                            ((static_cast<size_t>(b) * p.Sq + t) * p.Hq + kvh * p.group + hl) * kD +
+                            32 * (lane & 3);
+      float v[32];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint2 w = real ? *reinterpret_cast<const uint2*>(row + 4 * kk) : make_uint2(0u, 0u);
+        const float2 f0 = unpack2<kBF16>(w.x), f1 = unpack2<kBF16>(w.y);
+        v[4 * kk] = f0.x;
+        v[4 * kk + 1] = f0.y;
+        v[4 * kk + 2] = f1.x;
+        v[4 * kk + 3] = f1.y;
+      }
+      float am = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      const int e = am > 0.f ? ilogbf(am) - 14 : 0;
+      const float down = ldexpf(1.f, -e), up = ldexpf(1.f, e);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        qf[nt][kk][0] = pack2<false>(v[4 * kk] * down, v[4 * kk + 1] * down);
+        qf[nt][kk][1] = pack2<false>(v[4 * kk + 2] * down, v[4 * kk + 3] * down);
+      }
+      qsc[nt][0] = __shfl_sync(0xffffffffu, up, 8 * (lane & 3));
+      qsc[nt][1] = __shfl_sync(0xffffffffu, up, 8 * (lane & 3) + 4);
+    }
+  } else {
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
       const int n = n0 + nt * 8 + (lane >> 2);
@@ -369,6 +576,7 @@ __global__ void __launch_bounds__(160)
         qf[nt][kk][0] = real ? *reinterpret_cast<const uint32_t*>(row + d) : 0u;
         qf[nt][kk][1] = real ? *reinterpret_cast<const uint32_t*>(row + d + 8) : 0u;
       }
+      qsc[nt][0] = qsc[nt][1] = 1.f;
     }
   }
   // ALiBi: slope (exp2 domain) and query position of this lane's columns
@@ -386,6 +594,11 @@ __global__ void __launch_bounds__(160)
   }
   // running state per (column tile, column pair): columns nt*8 + 2*(lane&3) + {0,1}
   float m_run[kNT][2], l_part[kNT][2];
+  // int8: the PV product runs in fp16 on P * (V row scale / vC), vC the
+  // largest V scale this warp has seen, so every factor is <= 1 and keeps
+  // fp16's 11-bit precision; acc holds O / vC (vC only grows, and the change
+  // is folded into the online-softmax rescale of acc)
+  float vC = 1.17549435e-38f;
   float acc[kNT][kD / 16][4];
 #pragma unroll
   for (int nt = 0; nt < kNT; ++nt) {
@@ -415,29 +628,139 @@ __global__ void __launch_bounds__(160)
       }
       if (!ok) break;
     }
-    const uint32_t kbase = sbase + slot * Sh::kStageBytes;
-    const uint32_t vbase = kbase + Sh::kKVBytes;
     const int tok0 = warp * 16;  // this warp's 16 tokens of the chunk
+    // 16-bit tiles the tensor-core steps read: the TMA chunk itself, or (int8)
+    // this warp's converted rows, addressed by the row within the tile
+    uint32_t kbase = sbase + slot * Sh::kStageBytes;
+    uint32_t vbase = kbase + Sh::kKVBytes;
+    constexpr int kTileStride = kQ8 ? 16 * 128 : Sh::kBoxBytes;  // per 64-column chunk
+    const int trow0 = kQ8 ? tok0 : 0;                            // tile row = token - trow0
+    float ksc0 = 1.f, ksc1 = 1.f, vsc0 = 1.f, vsc1 = 1.f;
+    // direct int8 path: this lane's code words. K: rows tok0 + r and
+    // tok0 + r + 8 (r = lane / 4), bytes d = 32j .. 32j + 31 (j = lane % 4);
+    // V: tokens tok0 + 2j + {0, 1, 8, 9}, bytes d = 16r .. 16r + 15. Rows are
+    // 128 bytes with the 16-byte group g stored at g ^ (row & 7).
+    uint32_t kw[2][8], vw[4][4];
+    if constexpr (Sh::kDirect) {
+      const int r = lane >> 2, j = lane & 3;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t rb = kbase + (tok0 + r + 8 * h) * 128;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(smem + (rb - sbase) + (((2 * j + c) ^ r) << 4));
+          kw[h][4 * c] = w.x ^ 0x80808080u;
+          kw[h][4 * c + 1] = w.y ^ 0x80808080u;
+          kw[h][4 * c + 2] = w.z ^ 0x80808080u;
+          kw[h][4 * c + 3] = w.w ^ 0x80808080u;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int tk = tok0 + 2 * j + (u & 1) + 8 * (u >> 1);
+        const uint4 w = *reinterpret_cast<const uint4*>(smem + (vbase - sbase) + tk * 128 + ((r ^ (tk & 7)) << 4));
+        vw[u][0] = w.x ^ 0x80808080u;
+        vw[u][1] = w.y ^ 0x80808080u;
+        vw[u][2] = w.z ^ 0x80808080u;
+        vw[u][3] = w.w ^ 0x80808080u;
+      }
+      const float* sc = reinterpret_cast<const float*>(smem + slot * Sh::kStageBytes + Sh::kScaleOffset);
+      ksc0 = sc[tok0 + r];
+      ksc1 = sc[tok0 + r + 8];
+      vsc0 = sc[Sh::kTok + tok0 + r];
+      vsc1 = sc[Sh::kTok + tok0 + r + 8];
+      __syncwarp();
+      // everything this warp needs from the slot is in registers
+      if (lane == 0) mbar_arrive(&bars->empty[slot]);
+    } else if constexpr (kQ8) {
+      const uint8_t* kq = smem + slot * Sh::kStageBytes + tok0 * kD;
+      const uint8_t* vq = kq + Sh::kKVBytes;
+      uint8_t* ks = smem + Sh::kScrOffset + warp * 2 * Sh::kScrHalfBytes;
+      uint8_t* vs = ks + Sh::kScrHalfBytes;
+      // 16-byte pieces of the 16 rows: piece j = row (j / (kD/16)), values
+      // 16u .. 16u+15 (u = j % (kD/16)) -> column chunk u / 4, 16-byte
+      // groups 2 (u % 4) and 2 (u % 4) + 1 of the swizzled 128-byte row
+#pragma unroll
+      for (int j = lane; j < kD; j += 32) {
+        const int r = j / (kD / 16), u = j % (kD / 16);
+        const int c = u >> 2, g0 = (u & 3) * 2;
+        uint4 lo, hi;
+        i8x16_to_16bit<kBF16>(*reinterpret_cast<const uint4*>(kq + r * kD + u * 16), lo, hi);
+        *reinterpret_cast<uint4*>(ks + c * 2048 + r * 128 + ((g0 ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(ks + c * 2048 + r * 128 + (((g0 + 1) ^ (r & 7)) << 4)) = hi;
+        i8x16_to_16bit<false>(*reinterpret_cast<const uint4*>(vq + r * kD + u * 16), lo, hi);
+        *reinterpret_cast<uint4*>(vs + c * 2048 + r * 128 + ((g0 ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(vs + c * 2048 + r * 128 + (((g0 + 1) ^ (r & 7)) << 4)) = hi;
+      }
+      // the row scales of this lane's accumulator rows (tokens lane / 4, + 8)
+      const float* sc = reinterpret_cast<const float*>(smem + slot * Sh::kStageBytes + Sh::kScaleOffset);
+      ksc0 = sc[tok0 + (lane >> 2)];
+      ksc1 = sc[tok0 + (lane >> 2) + 8];
+      vsc0 = sc[Sh::kTok + tok0 + (lane >> 2)];
+      vsc1 = sc[Sh::kTok + tok0 + (lane >> 2) + 8];
+      __syncwarp();
+      // everything this warp needs from the slot is copied out
+      if (lane == 0) mbar_arrive(&bars->empty[slot]);
+      kbase = smem_u32(ks);
+      vbase = smem_u32(vs);
+    }
     // ---- S^T = K Q^T ----
     float s[kNT][4];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    if constexpr (Sh::kDirect) {
+      // A = K codes as exact fp16: word kk of a row holds d = 32j + 4kk + 0..3
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
-      const int mi = lane >> 3, r = lane & 7;
-      const int tok = tok0 + (mi & 1) * 8 + r;
-      const int c = kk >> 2;
-      const int g = (kk & 3) * 2 + (mi >> 1);
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(sw128(kbase + c * Sh::kBoxBytes, tok, g), a0, a1, a2, a3);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t a0 = i8pair_to_f16(kw[0][kk], false), a2 = i8pair_to_f16(kw[0][kk], true);
+        const uint32_t a1 = i8pair_to_f16(kw[1][kk], false), a3 = i8pair_to_f16(kw[1][kk], true);
 #pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) mma16816<kBF16>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+        for (int nt = 0; nt < kNT; ++nt) mma16816<false>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+      }
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const int mi = lane >> 3, r = lane & 7;
+        const int tok = tok0 + (mi & 1) * 8 + r;
+        const int c = kk >> 2;
+        const int g = (kk & 3) * 2 + (mi >> 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(sw128(kbase + c * kTileStride, tok - trow0, g), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) mma16816<kBF16>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+      }
     }
     // ---- logits, mask, online softmax ----
     const int wtok = (t_begin + i) * Sh::kTok + tok0;  // first token of this warp's 16
     const int pos0 = wtok + (lane >> 2);                // token of s[.][0], s[.][1]
     // every column sees all 16 tokens: no mask (warp-uniform)
     const bool all_visible = wtok >= lo_in && wtok + 16 <= hi_in;
+    float vr = 1.f;
+    if constexpr (kQ8) {
+      // S^T rows are tokens: the K scale multiplies each row (and, direct
+      // path, 2^e of the column undoes the query scaling)
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        s[nt][0] *= ksc0 * qsc[nt][0];
+        s[nt][1] *= ksc0 * qsc[nt][1];
+        s[nt][2] *= ksc1 * qsc[nt][0];
+        s[nt][3] *= ksc1 * qsc[nt][1];
+      }
+      // slots at positions >= Lk may hold any scale (NaN included): their P
+      // is 0 and must stay 0 after the V scale is folded in
+      if (wtok + 16 > Lk) {
+        if (pos0 >= Lk) vsc0 = 0.f;
+        if (pos0 + 8 >= Lk) vsc1 = 0.f;
+      }
+      float c = fmaxf(vsc0, vsc1);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, off));
+      const float c_new = fmaxf(vC, c);
+      vr = vC / c_new;  // acc (in units of vC) -> units of c_new
+      vC = c_new;
+      vsc0 = vsc0 / c_new;
+      vsc1 = vsc1 / c_new;
+    }
     uint32_t pb[kNT][2];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
@@ -480,48 +803,73 @@ __global__ void __launch_bounds__(160)
       const float e2 = ex2_approx(x2 - b0), e3 = ex2_approx(x3 - b1);
       l_part[nt][0] = l_part[nt][0] * al0 + e0 + e2;
       l_part[nt][1] = l_part[nt][1] * al1 + e1 + e3;
+      const float ar0 = al0 * vr, ar1 = al1 * vr;
 #pragma unroll
       for (int mt = 0; mt < kD / 16; ++mt) {
-        acc[nt][mt][0] *= al0;
-        acc[nt][mt][1] *= al1;
-        acc[nt][mt][2] *= al0;
-        acc[nt][mt][3] *= al1;
+        acc[nt][mt][0] *= ar0;
+        acc[nt][mt][1] *= ar1;
+        acc[nt][mt][2] *= ar0;
+        acc[nt][mt][3] *= ar1;
       }
       // P^T fragments: transpose the two 8x8 blocks of the 16x8 accumulator
-      pb[nt][0] = movmatrix_t(pack2<kBF16>(e0, e1));
-      pb[nt][1] = movmatrix_t(pack2<kBF16>(e2, e3));
+      // (int8: the V row scale folded into P, token by token)
+      if constexpr (kQ8) {
+        pb[nt][0] = movmatrix_t(pack2<false>(e0 * vsc0, e1 * vsc0));
+        pb[nt][1] = movmatrix_t(pack2<false>(e2 * vsc1, e3 * vsc1));
+      } else {
+        pb[nt][0] = movmatrix_t(pack2<kBF16>(e0, e1));
+        pb[nt][1] = movmatrix_t(pack2<kBF16>(e2, e3));
+      }
     }
     // ---- O^T += V^T P^T ----
-    // Slots at positions >= Lk (the rest of the last page, or the next
-    // sequence of a contiguous cache) may hold anything, NaN included; P is 0
-    // there but 0 * NaN is not, so those V elements are zeroed. Fragment
-    // registers a0, a1 hold tokens wtok + 2*(lane&3) + {0, 1} (low, high
-    // half), a2, a3 the same tokens + 8.
-    const bool tail = wtok + 16 > Lk;  // warp-uniform
-    uint32_t vm01 = 0xffffffffu, vm23 = 0xffffffffu;
-    if (tail) {
-      const int k0 = wtok + 2 * (lane & 3);
-      vm01 = (k0 < Lk ? 0x0000ffffu : 0u) | (k0 + 1 < Lk ? 0xffff0000u : 0u);
-      vm23 = (k0 + 8 < Lk ? 0x0000ffffu : 0u) | (k0 + 9 < Lk ? 0xffff0000u : 0u);
-    }
+    if constexpr (Sh::kDirect) {
+      // A = V^T codes as exact fp16; accumulator rows r, r + 8 of step mt are
+      // d = 16r + 2mt and 16r + 2mt + 1 (bytes 2mt, 2mt + 1 of this lane's V
+      // words); k = tokens 2j, 2j+1 (a0, a1) and 2j+8, 2j+9 (a2, a3)
 #pragma unroll
-    for (int mt = 0; mt < kD / 16; ++mt) {
-      const int mi = lane >> 3, r = lane & 7;
-      const int tok = tok0 + (mi >> 1) * 8 + r;
-      const int dcol = mt * 16 + (mi & 1) * 8;
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(sw128(vbase + (dcol >> 6) * Sh::kBoxBytes, tok, (dcol & 63) >> 3), a0, a1, a2, a3);
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t o = 2 * (mt & 1);
+        const uint32_t sel = o | ((o + 4) << 4) | ((o + 1) << 8) | ((o + 5) << 12);
+        const uint32_t x = __byte_perm(vw[0][mt >> 1], vw[1][mt >> 1], sel);
+        const uint32_t y = __byte_perm(vw[2][mt >> 1], vw[3][mt >> 1], sel);
+        const uint32_t a0 = i8pair_to_f16(x, false), a1 = i8pair_to_f16(x, true);
+        const uint32_t a2 = i8pair_to_f16(y, false), a3 = i8pair_to_f16(y, true);
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) mma16816<false>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      }
+    } else {
+      // Slots at positions >= Lk (the rest of the last page, or the next
+      // sequence of a contiguous cache) may hold anything, NaN included; P is 0
+      // there but 0 * NaN is not, so those V elements are zeroed. Fragment
+      // registers a0, a1 hold tokens wtok + 2*(lane&3) + {0, 1} (low, high
+      // half), a2, a3 the same tokens + 8.
+      const bool tail = wtok + 16 > Lk;  // warp-uniform
+      uint32_t vm01 = 0xffffffffu, vm23 = 0xffffffffu;
       if (tail) {
-        a0 &= vm01;
-        a1 &= vm01;
-        a2 &= vm23;
-        a3 &= vm23;
+        const int k0 = wtok + 2 * (lane & 3);
+        vm01 = (k0 < Lk ? 0x0000ffffu : 0u) | (k0 + 1 < Lk ? 0xffff0000u : 0u);
+        vm23 = (k0 + 8 < Lk ? 0x0000ffffu : 0u) | (k0 + 9 < Lk ? 0xffff0000u : 0u);
       }
 #pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) mma16816<kBF16>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      for (int mt = 0; mt < kD / 16; ++mt) {
+        const int mi = lane >> 3, r = lane & 7;
+        const int tok = tok0 + (mi >> 1) * 8 + r;
+        const int dcol = mt * 16 + (mi & 1) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(sw128(vbase + (dcol >> 6) * kTileStride, tok - trow0, (dcol & 63) >> 3), a0, a1, a2, a3);
+        if (tail) {
+          a0 &= vm01;
+          a1 &= vm01;
+          a2 &= vm23;
+          a3 &= vm23;
+        }
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+          mma16816<kBF16 && !kQ8>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars->empty[slot]);
+    if (!kQ8 && lane == 0) mbar_arrive(&bars->empty[slot]);
   }
 
   // ---- merge the four warps' states, then write the split's result ----
@@ -545,13 +893,16 @@ __global__ void __launch_bounds__(160)
       red_l[warp * kH + h0] = l0;
       red_l[warp * kH + h0 + 1] = l1;
     }
+    const float oc = kQ8 ? vC : 1.f;  // int8: acc holds O / vC
 #pragma unroll
     for (int mt = 0; mt < kD / 16; ++mt) {
-      const int d0 = mt * 16 + (lane >> 2);
-      red_o[(warp * kH + h0) * kD + d0] = acc[nt][mt][0];
-      red_o[(warp * kH + h0 + 1) * kD + d0] = acc[nt][mt][1];
-      red_o[(warp * kH + h0) * kD + d0 + 8] = acc[nt][mt][2];
-      red_o[(warp * kH + h0 + 1) * kD + d0 + 8] = acc[nt][mt][3];
+      // accumulator rows lane / 4 and lane / 4 + 8 of step mt
+      const int d0 = Sh::kDirect ? 16 * (lane >> 2) + 2 * mt : mt * 16 + (lane >> 2);
+      const int d1 = Sh::kDirect ? d0 + 1 : d0 + 8;
+      red_o[(warp * kH + h0) * kD + d0] = acc[nt][mt][0] * oc;
+      red_o[(warp * kH + h0 + 1) * kD + d0] = acc[nt][mt][1] * oc;
+      red_o[(warp * kH + h0) * kD + d1] = acc[nt][mt][2] * oc;
+      red_o[(warp * kH + h0 + 1) * kD + d1] = acc[nt][mt][3] * oc;
     }
   }
   named_bar_sync(1, 128);

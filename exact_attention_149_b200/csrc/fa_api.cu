@@ -109,6 +109,24 @@ fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, i
   return FA_OK;
 }
 
+// int8 cache (T, H, D) bytes: one box is `rows` tokens x the whole D-byte row
+// of one head; D = 128 rows arrive with the 128-byte swizzle (16-byte group g
+// of row r at g ^ (r & 7)), D = 64 rows unswizzled
+fa_status make_map_i8(CUtensorMap* map, const void* base, int D, int H, long long T, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H) * D};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), 1u, static_cast<cuuint32_t>(rows)};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
 // ---------------------------------------------------------------------------
 // optional per-kernel timing (events around each launch on the caller's stream)
 // ---------------------------------------------------------------------------

@@ -214,6 +214,55 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* k_new, const void* v_
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_fwd_kvcache against an int8 KV cache ("FlashAttention技术深度解析：重塑LLM
+ * 推理性能的新范式" §发展趋势 / 量化技术融合 names an INT8/INT4 quantised KV
+ * cache; the pages give no format, and this one is the plainest reading):
+ * every cached (token, kv head) row of D values is stored as int8 codes with
+ * one float32 scale and stands for code * scale. A row x is quantised as
+ * scale = max|x| / 127 and code = round-half-even(x / scale), both in
+ * float32 with IEEE division (a zero row: scale 0, codes 0); the new rows of
+ * an append are quantised that way on the device (keys after the rotary
+ * rotation and the rounding to the input dtype, i.e. what fa_fwd_kvcache
+ * would store). The attention is then fa_fwd_kvcache's on the values the
+ * codes stand for, with the same arguments, results, options and errors,
+ * and these differences:
+ *   k_cache, v_cache: DEVICE int8 (num_pages, page_size, Hkv, D) codes.
+ *   k_scale, v_scale: DEVICE float32 (num_pages, Hkv, page_size), the row
+ *     scales (per page, head-major so that a page's scales of one head are
+ *     contiguous); 16-byte aligned; written for the appended rows.
+ *   q, k_new, v_new, out stay in dtype (bf16 or fp16).
+ *   A contiguous cache (block_table NULL) needs a capacity (page_size) that
+ *     is a multiple of 64.
+ * Slots at positions >= Lk are never read into a result, whatever codes and
+ * scales (NaN included) they hold. Errors: as fa_fwd_kvcache, plus
+ * FA_ERR_INVALID_ARG for a NULL or misaligned k_scale / v_scale.
+ */
+FA_API fa_status fa_fwd_kvcache_int8(const void* q, const void* k_new, const void* v_new,
+                                     int8_t* k_cache, int8_t* v_cache, float* k_scale,
+                                     float* v_scale, const int32_t* block_table,
+                                     const int32_t* cache_seqlens, const float* rotary_cos,
+                                     const float* rotary_sin, void* out, float* lse, int B, int Sq,
+                                     int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                                     int num_pages, int rotary_rows, int rotary_dim,
+                                     int rotary_interleaved, float scale, int causal,
+                                     int window_left, int window_right, float softcap,
+                                     const float* alibi_slopes, int alibi_batch_stride,
+                                     int num_splits, fa_dtype dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
+ * Quantise a 16-bit KV cache into the int8 format of fa_fwd_kvcache_int8
+ * (e.g. a cache filled by a prefill): src (num_pages, page_size, Hkv, D) in
+ * dtype -> codes int8 of the same shape and scales float32 (num_pages, Hkv,
+ * page_size), every row by the rule above. All pointers are DEVICE memory;
+ * src 16-byte aligned, codes 8-byte aligned. Errors: FA_ERR_INVALID_ARG for
+ * NULL or misaligned pointers, sizes < 1 or a bad dtype; FA_ERR_UNSUPPORTED
+ * for D other than 64 or 128; FA_ERR_CUDA for launch failures.
+ */
+FA_API fa_status fa_kv_quantize_int8(const void* src, int8_t* codes, float* scales, int num_pages,
+                                     int page_size, int Hkv, int D, fa_dtype dtype, void* stream);
+
+/*
  * fa_fwd_kvcache without a workspace argument, for callers that cannot
  * allocate device memory on their decode path: a serving loop that has
  * handed all free device memory to its KV-cache pool up front (so a late

@@ -443,7 +443,7 @@ def kvcache_decode_int8(q, k_new, v_new, k_codes_logical, k_scales_logical, v_co
     rows already in the cache. Returns (O, LSE, appended k codes, k scales,
     v codes, v scales), the last four as lists of the B sequences' new rows.
     """
-    bsz, sq = np.asarray(q).shape[:2]
+    bsz, sq = tuple(q.shape)[:2]
     append = k_new is not None
     kd, vd, kc_new, ks_new, vc_new, vs_new = [], [], [], [], [], []
     lengths = []

@@ -137,3 +137,25 @@ def test_int8_decode_close_to_float_on_random_rows():
     o, lse, _, _ = kvcache_decode(q, None, None, kc, vc, lens, D ** -0.5)
     assert np.max(np.abs(o8 - o)) < 0.03
     assert np.max(np.abs(l8 - lse)) < 0.03
+
+
+def test_int8_decode_accepts_torch_16bit_inputs():
+    """q, k_new, v_new may be torch bf16 tensors (as the GPU tests pass them):
+    the result equals the one from the same values as float64 arrays."""
+    import torch
+
+    r = rng(37)
+    B, sq, hq, hkv, D = 2, 2, 4, 2, 16
+    lens = [3, 9]
+    kq = [quantize_int8(r.standard_normal((n, hkv, D))) for n in lens]
+    vq = [quantize_int8(r.standard_normal((n, hkv, D))) for n in lens]
+    t = [torch.randn(s, generator=torch.Generator().manual_seed(i)).to(torch.bfloat16)
+         for i, s in enumerate(((B, sq, hq, D), (B, sq, hkv, D), (B, sq, hkv, D)))]
+    args = ([c for c, _ in kq], [s for _, s in kq], [c for c, _ in vq], [s for _, s in vq], lens, 0.3)
+    a = kvcache_decode_int8(*t, *args)
+    b = kvcache_decode_int8(*(x.double().numpy() for x in t), *args)
+    for x, y in zip(a[:2], b[:2]):
+        np.testing.assert_array_equal(x, y)
+    for xs, ys in zip(a[2:], b[2:]):
+        for x, y in zip(xs, ys):
+            np.testing.assert_array_equal(x, y)
