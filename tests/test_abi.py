@@ -40,7 +40,8 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     names = declared_functions()
-    for n in ("fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_bwd_workspace_size",
+    for n in ("fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_fwd_kvcache_int8", "fa_kv_quantize_int8",
+              "fa_bwd_workspace_size",
               "fa_kvcache_workspace_size", "fa_get_device_status", "fa_last_error", "fa_version"):
         assert n in names
 
@@ -154,6 +155,40 @@ def test_kvcache_rejects_bad_arguments(fa):
     assert call(rd=64, **dict(rot, rrows=0)) == 1     # empty table
     assert call(rd=64, **dict(rot, sin=18)) == 1      # misaligned table
     assert call(rd=64, **dict(rot, ws=None, wsb=0)) == 1  # rotated queries need a workspace
+
+
+def test_kvcache_int8_rejects_bad_arguments(fa):
+    lib = fa.lib
+
+    def call(**kw):
+        a = dict(q=16, kn=16, vn=16, kc=16, vc=16, ks=256, vs=512, bt=16, cs=16, out=16, lse=16,
+                 B=2, Sq=1, Hkv=2, ps=256, mp=4, npg=8, ws=None, wsb=0)
+        a.update(kw)
+        return lib.fa_fwd_kvcache_int8(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["ks"], a["vs"],
+                                       a["bt"], a["cs"], None, None, a["out"], a["lse"], a["B"],
+                                       a["Sq"], 4, a["Hkv"], 128, a["ps"], a["mp"], a["npg"], 0, 0,
+                                       0, 0.1, 1, -1, -1, 0.0, None, 0, 1, 0, a["ws"], a["wsb"],
+                                       None)
+
+    assert call(ks=None) == 1                          # scales are required
+    assert call(vs=None) == 1
+    assert call(ks=260) == 1                           # scales 16-byte aligned
+    assert call(kc=None) == 1
+    assert call(ps=100) == 1
+    # a contiguous int8 cache needs a capacity that is a multiple of 64
+    assert call(bt=None, mp=1, npg=2, ps=300) == 1
+
+    def quant(**kw):
+        a = dict(src=16, codes=16, scales=16, npg=4, ps=64, Hkv=2, D=128, dtype=0)
+        a.update(kw)
+        return lib.fa_kv_quantize_int8(a["src"], a["codes"], a["scales"], a["npg"], a["ps"], a["Hkv"],
+                                       a["D"], a["dtype"], None)
+
+    assert quant(src=None) == 1
+    assert quant(src=24) == 1                          # misaligned source
+    assert quant(npg=0) == 1
+    assert quant(D=96) == 2
+    assert quant(dtype=7) == 1
 
 
 def test_valid_call_without_gpu_reports_cuda_error(fa):
