@@ -504,6 +504,12 @@ def run_ours(args, dist: Dist):
     best8 = max(dec8["splits"].values(), key=lambda d: d["gbs"])
     dec8["best_gbs"] = best8["gbs"]
     dec8["best_frac_of_hbm"] = best8["frac_of_hbm"]
+    trd8 = kernel_traffic("decode_split_int8")
+    k8 = best8.get("decode_split_kernel", best8)
+    dec8["roofline"] = {"kernel": "decode_split (int8 cache)", "bound": "hbm", "achieved": k8["gbs"],
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": k8["gbs"] / peaks["hbm_gbs"],
+                        "traffic": trd8["bytes_per_launch"] if trd8 else None,
+                        "peak_source": peaks["source"] + " HBM copy"}
     res["decode_int8"] = dec8
     del kq, vq, ksq, vsq
     torch.cuda.empty_cache()
