@@ -187,12 +187,14 @@ fa_status check_alibi(const float* slopes, int batch_stride, int Hq) {
   return FA_OK;
 }
 
+// fwd256: the forward also takes D = 256 (one Q tile per CTA)
 fa_status check_common(int B, int Hq, int Hkv, int S, int D, float scale, int wl, int wr,
-                       float softcap, fa_dtype dt, const int32_t* cu, int total) {
+                       float softcap, fa_dtype dt, const int32_t* cu, int total, bool fwd256 = false) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1)
     return fail(FA_ERR_INVALID_ARG, "B, Hq, Hkv and S must be >= 1 (got %d, %d, %d, %d)", B, Hq, Hkv, S);
   if (Hq % Hkv != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be an integer multiple of Hkv (%d)", Hq, Hkv);
-  if (D != 64 && D != 128) return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+  if (D != 64 && D != 128 && !(fwd256 && D == 256))
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128%s)", D, fwd256 ? ", or 256 forward" : "");
   if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
   if (wl < -1 || wr < -1) return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (got %d, %d)", wl, wr);
   if (!(softcap >= 0.f) || !std::isfinite(softcap))
@@ -246,7 +248,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, long long q_tok,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd: tensors must be 16-byte aligned");
   fa_status s = check_common(B, Hq, Hkv, S, D, scale, window_left, window_right, softcap, dtype,
-                             cu_seqlens, total_tokens);
+                             cu_seqlens, total_tokens, true);
   if (s != FA_OK) return s;
   if ((s = check_alibi(alibi_slopes, alibi_batch_stride, Hq)) != FA_OK) return s;
   if ((s = check_device()) != FA_OK) return s;
@@ -265,7 +267,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, long long q_tok,
   p.S = S;
   p.total = static_cast<int>(T);
   p.group = Hq / Hkv;
-  p.n_qblocks = (S + 255) / 256;
+  const int rows_per_cta = D == 256 ? fa::FwdShape<256>::kRows : fa::FwdShape<128>::kRows;
+  p.n_qblocks = (S + rows_per_cta - 1) / rows_per_cta;
   const float log2e = 1.4426950408889634f;
   p.scale_log2 = scale * log2e;
   p.softcap = softcap;
@@ -280,7 +283,12 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, long long q_tok,
   p.alibi_bstride = alibi_batch_stride;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool cap = softcap > 0.f;
-  if (D == 128) {
+  if (D == 256) {
+    if (dtype == FA_BF16)
+      s = cap ? launch_fwd<256, true, true>(tq, tk, tv, p, st) : launch_fwd<256, true, false>(tq, tk, tv, p, st);
+    else
+      s = cap ? launch_fwd<256, false, true>(tq, tk, tv, p, st) : launch_fwd<256, false, false>(tq, tk, tv, p, st);
+  } else if (D == 128) {
     if (dtype == FA_BF16)
       s = cap ? launch_fwd<128, true, true>(tq, tk, tv, p, st) : launch_fwd<128, true, false>(tq, tk, tv, p, st);
     else
@@ -369,9 +377,9 @@ fa_status fa_fwd_qkvpacked(const void* qkv, void* out, float* lse, int B, int H,
                            const int32_t* cu_seqlens, int total_tokens, fa_dtype dtype,
                            void* stream) {
   if (!qkv) return fail(FA_ERR_INVALID_ARG, "fa_fwd_qkvpacked: null qkv");
-  if (H < 1 || (D != 64 && D != 128))
-    return fail(D != 64 && D != 128 ? FA_ERR_UNSUPPORTED : FA_ERR_INVALID_ARG,
-                "fa_fwd_qkvpacked: H must be >= 1 and D 64 or 128");
+  if (H < 1 || (D != 64 && D != 128 && D != 256))
+    return fail(D != 64 && D != 128 && D != 256 ? FA_ERR_UNSUPPORTED : FA_ERR_INVALID_ARG,
+                "fa_fwd_qkvpacked: H must be >= 1 and D 64, 128 or 256");
   const long long hd = static_cast<long long>(H) * D;
   const uint16_t* base = static_cast<const uint16_t*>(qkv);
   return fwd_impl(base, base + hd, base + 2 * hd, 3 * hd, 3 * hd, out, lse, B, H, H, S, D, scale,

@@ -54,18 +54,23 @@ struct FwdParams {
   int alibi_bstride;
 };
 
+// D = 256: one Q tile per CTA (S 128 + O 256 TMEM columns; two tiles would
+// need 768) and one softmax warpgroup; Q (64 KB) and a two-slot K/V ring
+// (64 KB a tile) fill shared memory.
 template <int kD>
 struct FwdShape {
   static constexpr int kBM = 128;                    // rows per Q tile
   static constexpr int kBN = 128;                    // keys per KV tile
+  static constexpr int kQT = kD == 256 ? 1 : 2;      // Q tiles per CTA
+  static constexpr int kRows = kQT * kBM;            // query rows per CTA
   static constexpr int kChunks = kD / 64;            // 128-byte column chunks
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = kD == 128 ? 4 : 8;  // K/V ring slots
-  static constexpr int kBarOffset = (2 + kStages) * kTileBytes;
+  static constexpr int kStages = kD == 256 ? 2 : (kD == 128 ? 4 : 8);  // K/V ring slots
+  static constexpr int kBarOffset = (kQT + kStages) * kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;  // + barriers + align slack
-  static constexpr int kThreads = 384;
+  static constexpr int kThreads = 128 * (1 + kQT);
   static constexpr int kRegsLow = 88;   // warpgroup 0 after setmaxnreg.dec
   static constexpr int kRegsHigh = 208; // softmax warpgroups after setmaxnreg.inc
   static constexpr int kTmemCols = 512;
@@ -78,7 +83,7 @@ struct FwdShape {
   static constexpr int kPKeys = 128 / kPParts;
   static constexpr int kColS = 0;      // + 128 * t
   static constexpr int kColP = 64;     // + 128 * t
-  static constexpr int kColO = 256;    // + kD * t
+  static constexpr int kColO = 128 * kQT;  // + kD * t
 };
 
 // Barrier block in shared memory.
@@ -162,7 +167,7 @@ __device__ __forceinline__ float reduce128(const float (&x)[128]) {
 // kAlibi: the ALiBi bias is compiled in only where it is used, so the
 // common instantiations keep their register allocation
 template <int kD, bool kBF16, bool kCap, bool kAlibi>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Sh = FwdShape<kD>;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;                               // 2 tiles
-  uint8_t* sKV = smem + 2 * Sh::kTileBytes;         // kStages tiles
+  uint8_t* sKV = smem + Sh::kQT * Sh::kTileBytes;   // kStages tiles
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + Sh::kBarOffset);
 
   const int warp = threadIdx.x >> 5;
@@ -192,12 +197,12 @@ __global__ void __launch_bounds__(384, 1)
     seq_start = b * p.S;
     seq_len = p.S;
   }
-  const int q0 = qb * 256;
+  const int q0 = qb * Sh::kRows;
   if (q0 >= seq_len) return;  // uniform across the CTA, before any barrier
   const int kvh = h / p.group;
 
   // visible key range of the whole 256-row block (self-attention: Sk = Sq)
-  const int row_hi = min(q0 + 255, seq_len - 1);
+  const int row_hi = min(q0 + Sh::kRows - 1, seq_len - 1);
   int key_hi = seq_len - 1;
   if (p.wr >= 0) key_hi = min(key_hi, row_hi + p.wr);
   int key_lo = 0;
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < Sh::kQT; ++t) {
       mbar_init(&bars->s_full[t], 1);
       for (int h = 0; h < Sh::kPParts; ++h) mbar_init(p_ready_bar(bars, t, h), 4);
       mbar_init(&bars->o_final[t], 1);
@@ -232,12 +237,13 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   volatile int* abort = &bars->abort;
-  static_assert(Sh::kThreads * 168 >= 128 * Sh::kRegsLow + 256 * Sh::kRegsHigh,
+  static_assert(Sh::kQT == 1 || Sh::kThreads * 168 >= 128 * Sh::kRegsLow + 256 * Sh::kRegsHigh,
                 "register split exceeds the launch pool");
   // register reallocation sits inside each role's branch so the compiler
   // knows which limit every region runs under
   if (warp < 4) {
-    regs_dec<Sh::kRegsLow>();
+    // (one Q tile: 256 threads, every thread has the 255 registers it may use)
+    if constexpr (Sh::kQT == 2) regs_dec<Sh::kRegsLow>();
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (elect_one()) {
@@ -247,8 +253,8 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, 2 * Sh::kTileBytes);
-      for (int t = 0; t < 2; ++t)
+      mbar_arrive_expect_tx(&bars->q_full, Sh::kQT * Sh::kTileBytes);
+      for (int t = 0; t < Sh::kQT; ++t)
         for (int c = 0; c < Sh::kChunks; ++c)
           tma_load_3d(&tm_q, &bars->q_full, sQ + t * Sh::kTileBytes + c * Sh::kChunkBytes, c * 64,
                       h, seq_start + q0 + t * 128);
@@ -327,21 +333,22 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         if (it > 0) {
           const int fvp = fv - 2, svp = fvp % Sh::kStages;
-          // PV_0 of the previous tile, then QK_0 of this tile
+          // per Q tile: PV_t of the previous K/V tile, then QK_t of this one;
+          // the previous V slot is free after the last tile's PV
           const uint32_t ph = static_cast<uint32_t>(it - 1) & 1u;
-          if (!(ok = wait_issue_pv(0, svp, ph, it == 1))) break;
-          issue_qk(0, sk);
-          umma_commit(&bars->s_full[0]);
-          if (!(ok = wait_issue_pv(1, svp, ph, it == 1))) break;
-          umma_commit(&bars->kv_empty[svp]);
-          issue_qk(1, sk);
-          umma_commit(&bars->s_full[1]);
+          for (int t = 0; t < Sh::kQT && ok; ++t) {
+            if (!(ok = wait_issue_pv(t, svp, ph, it == 1))) break;
+            if (t == Sh::kQT - 1) umma_commit(&bars->kv_empty[svp]);
+            issue_qk(t, sk);
+            umma_commit(&bars->s_full[t]);
+          }
+          if (!ok) break;
           umma_commit(&bars->kv_empty[sk]);
         } else {
-          issue_qk(0, sk);
-          umma_commit(&bars->s_full[0]);
-          issue_qk(1, sk);
-          umma_commit(&bars->s_full[1]);
+          for (int t = 0; t < Sh::kQT; ++t) {
+            issue_qk(t, sk);
+            umma_commit(&bars->s_full[t]);
+          }
           umma_commit(&bars->kv_empty[sk]);
         }
         // V_it must be resident before next round's PV
@@ -351,7 +358,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (ok && n_tiles > 0) {
         const int fvl = 2 * (n_tiles - 1) + 1, svl = fvl % Sh::kStages;
-        for (int t = 0; t < 2 && ok; ++t) {
+        for (int t = 0; t < Sh::kQT && ok; ++t) {
           if (!(ok = wait_issue_pv(t, svl, static_cast<uint32_t>(n_tiles - 1) & 1u, n_tiles == 1)))
             break;
           umma_commit(&bars->o_final[t]);
@@ -365,7 +372,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   }
   } else {
-    regs_inc<Sh::kRegsHigh>();
+    if constexpr (Sh::kQT == 2) regs_inc<Sh::kRegsHigh>();
     const FwdItem w = load_item(bars);
     const uint32_t tmem = *static_cast<volatile uint32_t*>(&bars->tmem_base);
     const int seq_start = w.seq_start, seq_len = w.seq_len, q0 = w.q0, h = w.h, b = w.b;

@@ -94,7 +94,7 @@ def _fwd_status(fa, **kw):
     (dict(scale=float("nan")), 1),
     (dict(dtype=7), 1),
     (dict(D=96), 2),                # unsupported head dim
-    (dict(D=256), 2),
+    (dict(D=512), 2),
     (dict(cu=16, total=0), 1),
     (dict(al=18), 1),               # misaligned slopes
     (dict(al=16, als=1), 1),        # batch stride neither 0 nor >= Hq
@@ -155,6 +155,18 @@ def test_kvcache_rejects_bad_arguments(fa):
     assert call(rd=64, **dict(rot, rrows=0)) == 1     # empty table
     assert call(rd=64, **dict(rot, sin=18)) == 1      # misaligned table
     assert call(rd=64, **dict(rot, ws=None, wsb=0)) == 1  # rotated queries need a workspace
+
+
+def test_head_dim_256_is_forward_only(fa):
+    """D = 256 passes the forward's host checks (it then needs a device) and
+    is rejected by the backward and the kv-cache calls as unsupported."""
+    import torch
+
+    fwd_status = fa.lib.fa_fwd(16, 16, 16, 16, 16, 1, 2, 2, 64, 256, 0.1, 1, -1, -1, 0.0, None, 0,
+                               None, 0, 0, None)
+    assert fwd_status == (0 if torch.cuda.is_available() else 3)
+    a = [16] * 9 + [1, 2, 2, 64, 256, 0.1, 1, -1, -1, 0.0, None, 0, None, 0, 0]
+    assert fa.lib.fa_bwd(*a, 16, 1 << 20, None) == 2
 
 
 def test_kvcache_int8_rejects_bad_arguments(fa):

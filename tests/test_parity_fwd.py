@@ -34,6 +34,11 @@ SMALL = [
     (1, 384, 2, 2, 64, "fp16", True, (0, 0), 0.0),        # each row sees itself only
     (3, 1030, 4, 1, 128, "fp16", True, (-1, -1), 0.0),    # several Q blocks, B > 1
     (1, 260, 2, 2, 128, "bf16", False, (-1, -1), 0.0),    # non-causal ragged
+    # head dim 256: one 128-row Q tile per CTA
+    (1, 300, 2, 2, 256, "bf16", True, (-1, -1), 0.0),     # ragged, several Q tiles
+    (2, 513, 4, 2, 256, "fp16", False, (-1, -1), 0.0),    # GQA, non-causal, B > 1
+    (1, 640, 2, 1, 256, "bf16", True, (100, 0), 30.0),    # window + softcap, MQA
+    (1, 1, 2, 2, 256, "bf16", True, (-1, -1), 0.0),       # a single token
 ]
 
 
@@ -68,6 +73,7 @@ def test_fwd_deterministic(cuda_ok):
     ([1, 130, 257, 600, 33], 8, 2, 128, True, (200, 0), 30.0),
     ([128, 5, 384, 1], 4, 4, 64, False, (-1, -1), 0.0),
     ([513, 129], 4, 1, 128, True, (-1, -1), 0.0),
+    ([200, 1, 333], 4, 2, 256, True, (-1, -1), 0.0),
 ])
 def test_fwd_varlen(cuda_ok, lengths, Hq, Hkv, D, causal, window, softcap):
     inp = W.make_varlen_inputs(lengths, Hq, Hkv, D, "bf16", seed=len(lengths) * 13 + D)
