@@ -43,8 +43,10 @@
  *   default stream) and returns after the launch. Errors never abort: the
  *   call returns a status and fa_last_error() describes it. Invalid
  *   arguments are rejected on the host before anything is launched.
- * - Head dimension D must be 64 or 128. The device must be compute
- *   capability 10.0 (B200).
+ * - Head dimension D must be 64 or 128; the forward calls (fa_fwd,
+ *   fa_fwd_qkvpacked) also take 256 ("FlashAttention 实战指南" §版本怎么选:
+ *   head dims up to 256), the backward and kv-cache calls do not
+ *   (FA_ERR_UNSUPPORTED). The device must be compute capability 10.0 (B200).
  */
 #ifndef EXACT_ATTENTION_FA_H_
 #define EXACT_ATTENTION_FA_H_
