@@ -154,6 +154,7 @@ def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True
     (2, 8, 1, 128, "bf16", [1000, 1], 256),       # MQA, group 8
     (2, 32, 1, 64, "fp16", [129, 700], 64),       # group 32
     (5, 32, 8, 128, "bf16", [1024, 3000, 4095, 4096, 2047], 256),
+    (3, 8, 2, 128, "fp16", [5, 300, 1000], 128),  # fp16 queries on the register path
 ])
 def test_int8_decode_small(cuda_ok, B, Hq, Hkv, D, dtype, lengths, ps, splits):
     st = W.make_decode_structure(B, Hq, Hkv, D, 0, max(lengths), ps, dtype,

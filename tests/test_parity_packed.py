@@ -50,6 +50,27 @@ def test_qkvpacked_matches_unpacked_and_oracle(cuda_ok, B, S, H, D, dtype, causa
     check_bwd([dqkv[:, :, i].cpu() for i in range(3)], ref, "qkvpacked bwd")
 
 
+@pytest.mark.parametrize("alibi", [False, True])
+def test_qkvpacked_fwd_head_dim_256(cuda_ok, alibi):
+    """D = 256 (forward only): the packed forward equals the unpacked one
+    bitwise and the oracle within the usual tolerances, with and without
+    ALiBi slopes."""
+    dev = torch.device("cuda")
+    B, S, H, D = 2, 333, 2, 256
+    inp = W.make_fwd_inputs(B, S, H, H, D, "bf16", seed=256 + int(alibi))
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    qkv = torch.stack([q, k, v], dim=2).contiguous()
+    al = W.alibi_slopes(H, B, 0.2).to(dev) if alibi else None
+    o_p, l_p = fa.fwd_qkvpacked(qkv, causal=True, alibi_slopes=al)
+    o_u, l_u = fa.fwd(q, k, v, causal=True, alibi_slopes=al)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    assert torch.equal(o_p, o_u) and torch.equal(l_p, l_u)
+    o_ref, l_ref = attention_fwd(inp["q"], inp["k"], inp["v"], 1.0 / math.sqrt(D), True,
+                                 alibi_slopes=al.double().cpu().numpy() if alibi else None)
+    check_fwd(o_p, l_p, o_ref, l_ref, f"qkvpacked fwd D256 alibi={alibi}")
+
+
 def test_qkvpacked_varlen(cuda_ok):
     dev = torch.device("cuda")
     lengths = [130, 1, 400, 77]
