@@ -552,7 +552,10 @@ __global__ void __launch_bounds__(160)
       for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      const int e = am > 0.f ? ilogbf(am) - 14 : 0;
+      // e >= -100 keeps 2^-e finite when every |q| of the column is
+      // subnormal (such a column then scales to tiny fp16 values: its scores
+      // are 0 to within float32 anyway)
+      const int e = am > 0.f ? max(ilogbf(am) - 14, -100) : 0;
       const float down = ldexpf(1.f, -e), up = ldexpf(1.f, e);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {

@@ -241,3 +241,15 @@ def test_int8_decode_full_paged_b64(cuda_ok):
                                  c.dtype, seed=2000 + c.cid)
     for splits in (1, 16):
         _run_case(st, splits, heads=[0, 13, 31])
+
+
+def test_int8_decode_subnormal_query_column(cuda_ok):
+    """A query whose every element is subnormal (the register path scales each
+    query column by a power of two into fp16): the result stays finite and
+    matches the oracle; other columns of the same block are unaffected."""
+    st = W.make_decode_structure(2, 8, 2, 128, 0, 300, 64, "bf16", seed=97,
+                                 cache_seqlens=[300, 70])
+    st["q"][0, 0, 3] = (torch.randn(128, generator=torch.Generator().manual_seed(1)) * 1e-39).to(
+        torch.bfloat16)
+    assert st["q"][0, 0, 3].float().abs().max() < 1.2e-38
+    _run_case(st, 2)
