@@ -402,11 +402,19 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
     positions. int8 caches (codes) take their float32 row scales k_scale,
     v_scale (num_pages, Hkv, page_size) and run fa_fwd_kvcache_int8.
     Returns (out (B,Sq,Hq,D), lse (B,Hq,Sq))."""
-    _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new, rotary_cos,
-               rotary_sin, k_scale, v_scale)
     q8 = k_cache.dtype == torch.int8
     if q8 != (k_scale is not None) or (k_scale is None) != (v_scale is None):
         raise FaError(FA_ERR_INVALID_ARG, "int8 caches take k_scale and v_scale; 16-bit caches take neither")
+    if q8:
+        npg, ps, hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+        if v_cache.dtype != torch.int8 or v_cache.shape != k_cache.shape:
+            raise FaError(FA_ERR_INVALID_ARG, "k_cache and v_cache must both be int8 of one shape")
+        for sc in (k_scale, v_scale):
+            if sc.dtype != torch.float32 or tuple(sc.shape) != (npg, hkv, ps):
+                raise FaError(FA_ERR_INVALID_ARG,
+                              f"int8 cache scales must be float32 {(npg, hkv, ps)} (num_pages, Hkv, page_size)")
+    _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new, rotary_cos,
+               rotary_sin, k_scale, v_scale)
     B, Sq, Hq, D = q.shape
     num_pages, page_size, Hkv, _ = k_cache.shape
     max_pages = 1 if block_table is None else block_table.shape[1]
@@ -436,8 +444,13 @@ def kv_quantize_int8(cache, codes=None, scales=None, stream=None):
     """A 16-bit cache (num_pages, page_size, Hkv, D) -> (int8 codes of the
     same shape, float32 scales (num_pages, Hkv, page_size)) in the format of
     fa_fwd_kvcache_int8."""
-    _need_cuda(cache, codes, scales)
     num_pages, page_size, Hkv, D = cache.shape
+    if codes is not None and (codes.dtype != torch.int8 or codes.shape != cache.shape):
+        raise FaError(FA_ERR_INVALID_ARG, "codes must be int8 of the cache's shape")
+    if scales is not None and (scales.dtype != torch.float32 or
+                               tuple(scales.shape) != (num_pages, Hkv, page_size)):
+        raise FaError(FA_ERR_INVALID_ARG, "scales must be float32 (num_pages, Hkv, page_size)")
+    _need_cuda(cache, codes, scales)
     if codes is None:
         codes = torch.empty(cache.shape, dtype=torch.int8, device=cache.device)
     if scales is None:

@@ -203,6 +203,27 @@ def test_kvcache_int8_rejects_bad_arguments(fa):
     assert quant(dtype=7) == 1
 
 
+def test_binding_checks_int8_cache_shapes(fa):
+    """The binding checks what the C ABI cannot see: the dtype and shape of
+    the int8 cache's scale tensors (checked before any device access)."""
+    import torch
+
+    q = torch.zeros(2, 1, 4, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(3, 64, 2, 128, dtype=torch.int8)
+    good = torch.zeros(3, 2, 64)
+    cs = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(fa.FaError, match="scales must be float32"):
+        fa.fwd_kvcache(q, kc, kc.clone(), cs, None, k_scale=torch.zeros(3, 64, 2), v_scale=good)
+    with pytest.raises(fa.FaError, match="take k_scale and v_scale"):
+        fa.fwd_kvcache(q, kc, kc.clone(), cs, None, k_scale=good)
+    with pytest.raises(fa.FaError, match="take k_scale and v_scale"):
+        fa.fwd_kvcache(q, kc, kc.clone(), cs, None)
+    with pytest.raises(fa.FaError, match="both be int8"):
+        fa.fwd_kvcache(q, kc, kc.to(torch.bfloat16), cs, None, k_scale=good, v_scale=good)
+    with pytest.raises(fa.FaError, match="scales must be float32"):
+        fa.kv_quantize_int8(torch.zeros(3, 64, 2, 128, dtype=torch.bfloat16), scales=torch.zeros(3, 64, 2))
+
+
 def test_valid_call_without_gpu_reports_cuda_error(fa):
     import torch
 
