@@ -308,7 +308,8 @@ def round_to(x, dtype):
     if dtype is None:
         return x
     if dtype == "fp16":
-        return x.astype(np.float16).astype(np.float64)
+        with np.errstate(over="ignore"):  # beyond the fp16 range -> +-inf, as a cast gives
+            return x.astype(np.float16).astype(np.float64)
     if dtype == "bf16":
         b = x.astype(np.float32).view(np.uint32).astype(np.uint64)
         b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000

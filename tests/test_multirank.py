@@ -37,7 +37,7 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_max_and_aggregate():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of this (possibly threaded) process
     out = mgr.dict()
     mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
