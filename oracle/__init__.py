@@ -14,7 +14,10 @@ from .attention import (  # noqa: F401
     kvcache_decode,
     kvcache_decode_int8,
     lse_combine,
+    pack_int4,
+    quantize_int4,
     quantize_int8,
+    unpack_int4,
     rotary,
     round_to,
     scores,

@@ -43,13 +43,16 @@ notes of the repository):
   at position ``cache_seqlens[b]`` and attention covers ``cache_seqlens[b]+1``
   keys.
 * "FlashAttention技术深度解析：重塑LLM推理性能的新范式" §发展趋势 /
-  量化技术融合 mentions an INT8/INT4 quantised KV cache but gives no format; the int8 cache here is symmetric with one
-  float32 scale per (token, kv head) row: ``scale = max|x| / 127`` and
-  ``code = round-half-even(x / scale)``, both in float32 (the precision the
-  kernel takes the integer decision in), an all-zero row having scale 0 and
-  codes 0. A cached row stands for ``code * scale``; a new key is rotated (with
-  rotary) and rounded to the 16-bit input type first, as the 16-bit cache
-  stores it, then quantised.
+  量化技术融合 mentions an INT8/INT4 quantised KV cache but gives no format.
+  The int8 cache here is symmetric with one float32 scale per (token, kv
+  head) row: ``scale = max|x| / 127`` and ``code = round-half-even(x /
+  scale)``, both in float32 (the precision the kernel takes the integer
+  decision in), an all-zero row having scale 0 and codes 0. A cached row
+  stands for ``code * scale``; a new key is rotated (with rotary) and rounded
+  to the 16-bit input type first, as the 16-bit cache stores it, then
+  quantised. The int4 reading is the same with ``scale = max|x| / 7`` and
+  codes in [-7, 7], stored two per byte (the code of even d in the low
+  nibble, both biased by 8); no kernel uses it yet.
 
 Every array is float64. 16-bit inputs are converted exactly (every bf16 and
 fp16 value is representable in float64), so the oracle sees the same values
@@ -71,6 +74,9 @@ __all__ = [
     "kvcache_decode_int8",
     "quantize_int8",
     "dequantize_int8",
+    "quantize_int4",
+    "pack_int4",
+    "unpack_int4",
     "lse_combine",
     "rotary",
     "round_to",
@@ -422,6 +428,36 @@ def quantize_int8(x):
     codes = np.rint((x32 / div[..., None]).astype(np.float32))
     codes = np.where(scale[..., None] > 0, codes, np.float32(0.0))
     return np.clip(codes, -127, 127).astype(np.int8), scale
+
+
+def quantize_int4(x):
+    """Symmetric int4 quantisation of each row (the last axis) of ``x``: as
+    quantize_int8 with 7 in place of 127, codes in [-7, 7] (an int8 array,
+    one code per element; pack_int4 stores them two per byte). Returns
+    (codes, scales float32)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=-1)
+    scale = (amax / np.float32(7.0)).astype(np.float32)
+    div = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    codes = np.rint((x32 / div[..., None]).astype(np.float32))
+    codes = np.where(scale[..., None] > 0, codes, np.float32(0.0))
+    return np.clip(codes, -7, 7).astype(np.int8), scale
+
+
+def pack_int4(codes):
+    """int4 codes (..., D), D even -> bytes (..., D / 2): byte i holds code
+    2i + 8 in its low nibble and code 2i + 1 + 8 in its high nibble."""
+    c = np.asarray(codes, dtype=np.int16) + 8
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed):
+    """The inverse of pack_int4."""
+    b = np.asarray(packed, dtype=np.int16)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int8)
+    out[..., 0::2] = (b & 15) - 8
+    out[..., 1::2] = (b >> 4) - 8
+    return out
 
 
 def dequantize_int8(codes, scales):

@@ -159,3 +159,43 @@ def test_int8_decode_accepts_torch_16bit_inputs():
     for xs, ys in zip(a[2:], b[2:]):
         for x, y in zip(xs, ys):
             np.testing.assert_array_equal(x, y)
+
+
+# ---- int4 (the same reading with 7 levels per sign; no kernel yet) ----
+
+def test_quantize_int4_hand_rows():
+    from oracle import quantize_int4
+
+    # max |x| = 3.5 -> scale 0.5
+    codes, scale = quantize_int4(np.array([[3.5, -1.0, 0.25, 0.75, -3.5]]))
+    assert scale[0] == np.float32(0.5)
+    # 0.25 / 0.5 = 0.5 -> 0 (half to even); 0.75 / 0.5 = 1.5 -> 2
+    np.testing.assert_array_equal(codes[0], [7, -2, 0, 2, -7])
+    codes, scale = quantize_int4(np.zeros((1, 4)))
+    assert scale[0] == 0 and not codes.any()
+
+
+def test_int4_packing_round_trip_and_layout():
+    from oracle import pack_int4, unpack_int4
+
+    codes = np.array([[-7, 7, 0, -1, 3, -8 + 1]], dtype=np.int8)
+    packed = pack_int4(codes)
+    # byte 0: low nibble -7 + 8 = 1, high nibble 7 + 8 = 15
+    assert packed[0, 0] == (1 | (15 << 4))
+    assert packed[0, 1] == (8 | (7 << 4))
+    np.testing.assert_array_equal(unpack_int4(packed), codes)
+    r = rng(41)
+    c = r.integers(-7, 8, (5, 3, 64)).astype(np.int8)
+    np.testing.assert_array_equal(unpack_int4(pack_int4(c)), c)
+
+
+def test_quantize_int4_error_bound():
+    from oracle import quantize_int4
+
+    r = rng(43)
+    x = (r.standard_normal((64, 128)) * r.uniform(0.01, 30.0, (64, 1))).astype(np.float32)
+    codes, scale = quantize_int4(x)
+    assert np.all(np.abs(codes.astype(np.int32)) <= 7)
+    np.testing.assert_array_equal(np.max(np.abs(codes.astype(np.int32)), axis=1), 7)
+    err = np.abs(dequantize_int8(codes, scale) - x.astype(np.float64))
+    assert np.all(err <= scale.astype(np.float64)[:, None] * (0.5 + 7 * 2.0 ** -22))
