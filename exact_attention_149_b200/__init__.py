@@ -27,6 +27,7 @@ __all__ = [
     "fa_kernel_timing_enable", "fa_kernel_timing_read", "fa_kernel_timing_reset",
     "fwd", "bwd", "fwd_kvcache", "fwd_qkvpacked", "bwd_qkvpacked", "fa_fwd_qkvpacked",
     "fa_bwd_qkvpacked", "fa_fwd_kvcache_int8", "fa_kv_quantize_int8", "kv_quantize_int8",
+    "fa_fwd_kvcache_int4", "fa_kv_quantize_int4", "kv_quantize_int4",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -82,6 +83,10 @@ lib.fa_fwd_kvcache_int8.restype = _i
 lib.fa_fwd_kvcache_int8.argtypes = [_p] * 13 + _KV_ARGS[11:] + [_p, _z, _p]
 lib.fa_kv_quantize_int8.restype = _i
 lib.fa_kv_quantize_int8.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _p]
+lib.fa_fwd_kvcache_int4.restype = _i
+lib.fa_fwd_kvcache_int4.argtypes = [_p] * 13 + _KV_ARGS[11:] + [_p, _z, _p]
+lib.fa_kv_quantize_int4.restype = _i
+lib.fa_kv_quantize_int4.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.fa_bwd_workspace_size.restype = _z
 lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 lib.fa_kvcache_workspace_size.restype = _z
@@ -224,6 +229,28 @@ def fa_fwd_kvcache_int8(q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, blo
 
 def fa_kv_quantize_int8(src, codes, scales, num_pages, page_size, Hkv, D, dtype, stream=None):
     _check(lib.fa_kv_quantize_int8(_ptr(src), _ptr(codes), _ptr(scales), num_pages, page_size,
+                                   Hkv, D, dtype, _stream(stream)))
+
+
+def fa_fwd_kvcache_int4(q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_table,
+                        cache_seqlens, rotary_cos, rotary_sin, out, lse, B, Sq, Hq, Hkv, D,
+                        page_size, max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+                        rotary_interleaved, scale, causal, window_left, window_right, softcap,
+                        alibi_slopes, alibi_batch_stride, num_splits, dtype, workspace,
+                        workspace_bytes, stream=None):
+    _check(lib.fa_fwd_kvcache_int4(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_table),
+                                   _ptr(cache_seqlens), _ptr(rotary_cos), _ptr(rotary_sin),
+                                   _ptr(out), _ptr(lse), B, Sq, Hq, Hkv, D, page_size,
+                                   max_pages_per_seq, num_pages, rotary_rows, rotary_dim,
+                                   int(rotary_interleaved), scale, int(causal), window_left,
+                                   window_right, softcap, _ptr(alibi_slopes), alibi_batch_stride,
+                                   num_splits, dtype, _ptr(workspace), workspace_bytes,
+                                   _stream(stream)))
+
+
+def fa_kv_quantize_int4(src, codes, scales, num_pages, page_size, Hkv, D, dtype, stream=None):
+    _check(lib.fa_kv_quantize_int4(_ptr(src), _ptr(codes), _ptr(scales), num_pages, page_size,
                                    Hkv, D, dtype, _stream(stream)))
 
 
@@ -399,16 +426,21 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
     caches (B, capacity, Hkv, D); cache_seqlens int32 (B). Appends
     k_new/v_new (B,Sq,Hkv,D) in place, then attends. rotary_cos/rotary_sin:
     float32 (rows, rotary_dim/2) tables that rotate q and k_new at their
-    positions. int8 caches (codes) take their float32 row scales k_scale,
-    v_scale (num_pages, Hkv, page_size) and run fa_fwd_kvcache_int8.
+    positions. int8 caches (codes) and int4 caches (uint8, two codes per
+    byte: (num_pages, page_size, Hkv, D / 2)) take their float32 row scales
+    k_scale, v_scale (num_pages, Hkv, page_size) and run
+    fa_fwd_kvcache_int8 / _int4.
     Returns (out (B,Sq,Hq,D), lse (B,Hq,Sq))."""
-    q8 = k_cache.dtype == torch.int8
+    q4 = k_cache.dtype == torch.uint8
+    q8 = k_cache.dtype == torch.int8 or q4
     if q8 != (k_scale is not None) or (k_scale is None) != (v_scale is None):
         raise FaError(FA_ERR_INVALID_ARG, "int8 caches take k_scale and v_scale; 16-bit caches take neither")
     if q8:
         npg, ps, hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
-        if v_cache.dtype != torch.int8 or v_cache.shape != k_cache.shape:
+        if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
             raise FaError(FA_ERR_INVALID_ARG, "k_cache and v_cache must both be int8 of one shape")
+        if q4 and k_cache.shape[3] * 2 != q.shape[3]:
+            raise FaError(FA_ERR_INVALID_ARG, "an int4 cache's last dim is D / 2")
         for sc in (k_scale, v_scale):
             if sc.dtype != torch.float32 or tuple(sc.shape) != (npg, hkv, ps):
                 raise FaError(FA_ERR_INVALID_ARG,
@@ -416,7 +448,7 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
     _need_cuda(q, k_cache, v_cache, cache_seqlens, block_table, k_new, v_new, rotary_cos,
                rotary_sin, k_scale, v_scale)
     B, Sq, Hq, D = q.shape
-    num_pages, page_size, Hkv, _ = k_cache.shape
+    num_pages, page_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
     max_pages = 1 if block_table is None else block_table.shape[1]
     if (rotary_cos is None) != (rotary_sin is None):
         raise FaError(FA_ERR_INVALID_ARG, "rotary_cos and rotary_sin go together")
@@ -433,7 +465,9 @@ def fwd_kvcache(q, k_cache, v_cache, cache_seqlens, block_table, k_new=None, v_n
             page_size, max_pages, num_pages, rot_rows, rot_dim, rotary_interleaved,
             _scale(scale, D), causal, window[0], window[1], softcap, *_alibi(alibi_slopes, Hq),
             num_splits, _dt(q), workspace, 0 if workspace is None else workspace.numel(), stream)
-    if q8:
+    if q4:
+        fa_fwd_kvcache_int4(q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, *args)
+    elif q8:
         fa_fwd_kvcache_int8(q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, *args)
     else:
         fa_fwd_kvcache(q, k_new, v_new, k_cache, v_cache, *args)
@@ -456,4 +490,23 @@ def kv_quantize_int8(cache, codes=None, scales=None, stream=None):
     if scales is None:
         scales = torch.empty((num_pages, Hkv, page_size), dtype=torch.float32, device=cache.device)
     fa_kv_quantize_int8(cache, codes, scales, num_pages, page_size, Hkv, D, _dt(cache), stream)
+    return codes, scales
+
+
+def kv_quantize_int4(cache, codes=None, scales=None, stream=None):
+    """A 16-bit cache (num_pages, page_size, Hkv, D) -> (uint8 codes
+    (num_pages, page_size, Hkv, D / 2), two per byte, float32 scales
+    (num_pages, Hkv, page_size)) in the format of fa_fwd_kvcache_int4."""
+    num_pages, page_size, Hkv, D = cache.shape
+    if codes is not None and (codes.dtype != torch.uint8 or tuple(codes.shape) != (num_pages, page_size, Hkv, D // 2)):
+        raise FaError(FA_ERR_INVALID_ARG, "codes must be uint8 (num_pages, page_size, Hkv, D / 2)")
+    if scales is not None and (scales.dtype != torch.float32 or
+                               tuple(scales.shape) != (num_pages, Hkv, page_size)):
+        raise FaError(FA_ERR_INVALID_ARG, "scales must be float32 (num_pages, Hkv, page_size)")
+    _need_cuda(cache, codes, scales)
+    if codes is None:
+        codes = torch.empty((num_pages, page_size, Hkv, D // 2), dtype=torch.uint8, device=cache.device)
+    if scales is None:
+        scales = torch.empty((num_pages, Hkv, page_size), dtype=torch.float32, device=cache.device)
+    fa_kv_quantize_int4(cache, codes, scales, num_pages, page_size, Hkv, D, _dt(cache), stream)
     return codes, scales

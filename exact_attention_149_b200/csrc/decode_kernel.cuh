@@ -136,36 +136,44 @@ __device__ __forceinline__ uint4 rotate8(const uint16_t* row, int d0, const floa
   return pack8<kBF16>(y);
 }
 
-// Symmetric int8 quantisation of one head row of D values held by 16 lanes
-// (8 consecutive values each; lanes at or past D / 8 hold zeros): scale =
-// max|x| / 127, code = round-half-even(x / scale), both in fp32 with IEEE
-// division; a zero row has scale 0 and codes 0. Returns the lane's 8 codes
-// packed little-endian into two words; *scale gets the row's scale.
-__device__ __forceinline__ uint2 quantize_row8(const float (&x)[8], float* scale) {
+// Symmetric quantisation of one head row of D values held by 16 lanes (8
+// consecutive values each; lanes at or past D / 8 hold zeros): scale = max|x|
+// / qmax, code = round-half-even(x / scale), both in fp32 with IEEE
+// division; a zero row has scale 0 and codes 0. qmax is 127 (kQ = 8) or 7
+// (kQ = 4). Returns the lane's 8 codes: int8, little-endian in two words; int4,
+// biased by 8, two per byte (even d in the low nibble) in .x. *scale gets
+// the row's scale.
+template <int kQ>
+__device__ __forceinline__ uint2 quantize_row(const float (&x)[8], float* scale) {
+  constexpr int kMax = kQ == 8 ? 127 : 7;
   float am = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(x[j]));
 #pragma unroll
   for (int off = 1; off < 16; off <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-  const float sc = __fdiv_rn(am, 127.f);
+  const float sc = __fdiv_rn(am, static_cast<float>(kMax));
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     int c = sc > 0.f ? __float2int_rn(__fdiv_rn(x[j], sc)) : 0;
-    c = max(-127, min(127, c));
-    w[j >> 2] |= (static_cast<uint32_t>(c) & 0xffu) << (8 * (j & 3));
+    c = max(-kMax, min(kMax, c));
+    if constexpr (kQ == 8)
+      w[j >> 2] |= (static_cast<uint32_t>(c) & 0xffu) << (8 * (j & 3));
+    else
+      w[0] |= static_cast<uint32_t>(c + 8) << (4 * j);
   }
   *scale = sc;
   return make_uint2(w[0], w[1]);
 }
 
 // grid B * Sq (one block per new token), block 128: 16 bytes per thread-step.
-// kQ8: the new rows are quantised into an int8 cache (keys after the rotary
+// kQuant: the new rows are quantised into an int8 cache (keys after the rotary
 // rotation and the rounding to the 16-bit type, as the 16-bit cache stores
 // them); each warp takes heads warp, warp + 4, ..., lanes 0-15 the key row and
 // lanes 16-31 the value row.
-template <bool kBF16, bool kQ8>
+template <bool kBF16, int kQ>
 __global__ void kv_append_kernel(const DecodeParams p) {
+  constexpr bool kQuant = kQ != 0;
   const int b = blockIdx.x / p.Sq, t = blockIdx.x % p.Sq;
   const int L = p.cache_seqlens[b];
   const int Lk = L + (p.append ? p.Sq : 0);
@@ -204,7 +212,7 @@ __global__ void kv_append_kernel(const DecodeParams p) {
   const size_t src = (static_cast<size_t>(b) * p.Sq + t) * p.Hkv * p.D;
   const uint16_t* kn = static_cast<const uint16_t*>(p.k_new) + src;
   const uint16_t* vn = static_cast<const uint16_t*>(p.v_new) + src;
-  if constexpr (kQ8) {
+  if constexpr (kQuant) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int half = lane >> 4, li = lane & 15;
     const bool act = li < groups;
@@ -219,9 +227,14 @@ __global__ void kv_append_kernel(const DecodeParams p) {
         for (int j = 0; j < 8; ++j) x[j] = 0.f;
       }
       float sc;
-      const uint2 codes = quantize_row8(x, &sc);
+      const uint2 codes = quantize_row<kQ>(x, &sc);
       uint8_t* cache = static_cast<uint8_t*>(half == 0 ? p.k_cache : p.v_cache);
-      if (act) *reinterpret_cast<uint2*>(cache + dst + h * p.D + li * 8) = codes;
+      if (act) {
+        if constexpr (kQ == 8)
+          *reinterpret_cast<uint2*>(cache + dst + h * p.D + li * 8) = codes;
+        else  // two codes per byte
+          *reinterpret_cast<uint32_t*>(cache + (dst + h * p.D + li * 8) / 2) = codes.x;
+      }
       if (li == 0) {
         float* scales = half == 0 ? p.k_scale : p.v_scale;
         scales[(static_cast<size_t>(page) * p.Hkv + h) * p.page_size + pos % p.page_size] = sc;
@@ -240,9 +253,10 @@ __global__ void kv_append_kernel(const DecodeParams p) {
 }
 
 // A 16-bit cache (rows, Hkv, D), rows = num_pages * page_size, into int8
-// codes of the same shape and scales (num_pages, Hkv, page_size): one
-// (row, head) unit per 16-lane half-warp, eight units per 128-thread block.
-template <bool kBF16>
+// codes of the same shape (or int4 codes, two per byte: (rows, Hkv, D / 2))
+// and scales (num_pages, Hkv, page_size): one (row, head) unit per 16-lane
+// half-warp, eight units per 128-thread block.
+template <bool kBF16, int kQ>
 __global__ void kv_quantize_kernel(const uint16_t* src, uint8_t* codes, float* scales, long long units,
                                    int Hkv, int D, int page_size) {
   const int li = threadIdx.x & 15;
@@ -256,8 +270,13 @@ __global__ void kv_quantize_kernel(const uint16_t* src, uint8_t* codes, float* s
     for (int j = 0; j < 8; ++j) x[j] = 0.f;
   }
   float sc;
-  const uint2 c = quantize_row8(x, &sc);
-  if (act) *reinterpret_cast<uint2*>(codes + u * D + li * 8) = c;
+  const uint2 c = quantize_row<kQ>(x, &sc);
+  if (act) {
+    if constexpr (kQ == 8)
+      *reinterpret_cast<uint2*>(codes + u * D + li * 8) = c;
+    else
+      *reinterpret_cast<uint32_t*>(codes + (u * D + li * 8) / 2) = c.x;
+  }
   if (u < units && li == 0) {
     const long long row = u / Hkv;
     const int h = static_cast<int>(u % Hkv);
@@ -272,6 +291,16 @@ __device__ __forceinline__ uint32_t i8pair_to_f16(uint32_t w, bool hi) {
   const uint32_t h = __byte_perm(w, 0x64646464u, hi ? 0x4342u : 0x4140u);
   const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h),
                             __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// The biased int4 codes (code + 8) in bits 0-3 and 16-19 of w -> their exact
+// fp16 pair: 0x64 above the nibble is the fp16 value 1024 + code + 8, and
+// subtracting 1032 leaves the code.
+__device__ __forceinline__ uint32_t i4pair_to_f16(uint32_t w) {
+  const uint32_t h = (w & 0x000F000Fu) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h),
+                            __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408)));
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
@@ -356,31 +385,35 @@ __device__ __forceinline__ uint32_t sw128(uint32_t base, int r, int g) {
   return base + r * 128 + ((g ^ (r & 7)) << 4);
 }
 
-// kQ8: the ring holds int8 chunks (K codes, V codes, then the 64 K and 64 V
+// kQuant: the ring holds int8 chunks (K codes, V codes, then the 64 K and 64 V
 // scales). D = 128: the code tiles arrive with the 128-byte swizzle and the
 // consumers build their fragments from them in registers. D = 64: unswizzled
 // tiles, and each consumer warp converts its 16 rows into 16-bit tiles in its
 // own scratch (K then V, 16 rows x 128 B in the 128-byte swizzle of the TMA
 // tiles) before the tensor-core steps.
-template <int kD, bool kQ8 = false>
+template <int kD, int kQ = 0>
 struct DecShape {
+  static constexpr bool kQuant = kQ != 0;           // an int8 (kQ = 8) or int4 (kQ = 4) cache
+  static constexpr int kRowBytes = kD * (kQuant ? kQ : 16) / 8;  // one cached row of one head
   static constexpr int kTok = 64;                      // tokens per chunk
   static constexpr int kChunks = kD / 64;              // 128-byte column chunks
   static constexpr int kBoxBytes = kTok * 128;         // 64 rows x 128 B
-  static constexpr int kKVBytes = kQ8 ? kTok * kD : kChunks * kBoxBytes;  // K or V of one chunk
+  static constexpr int kKVBytes = kQuant ? kTok * kRowBytes : kChunks * kBoxBytes;  // K or V of one chunk
   static constexpr int kScaleOffset = 2 * kKVBytes;    // int8: 64 K scales, 64 V scales
   // bytes the producer loads into a stage (the full barrier's transaction
   // count); int8 stages are padded to 1 KB, which the 128-byte-swizzled TMA
   // tiles need, so the stage stride can exceed the loaded bytes
-  static constexpr int kLoadBytes = 2 * kKVBytes + (kQ8 ? 2 * kTok * 4 : 0);
-  static constexpr int kStageBytes = kQ8 ? (kLoadBytes + 1023) / 1024 * 1024 : kLoadBytes;
-  static constexpr int kStages = kQ8 ? (kD == 128 ? 4 : 6) : (kD == 128 ? 3 : 6);  // 2 CTAs per SM
+  static constexpr int kLoadBytes = 2 * kKVBytes + (kQuant ? 2 * kTok * 4 : 0);
+  static constexpr int kStageBytes = kQuant ? (kLoadBytes + 1023) / 1024 * 1024 : kLoadBytes;
+  // 2 (16-bit) or 3 CTAs per SM; int4 keeps 8 stages so that the cross-warp
+  // reduction scratch, which aliases the ring, fits
+  static constexpr int kStages = kQuant ? (kQ == 4 ? 8 : (kD == 128 ? 4 : 6)) : (kD == 128 ? 3 : 6);
   // int8 with D = 128 builds the tensor-core fragments straight from the
   // swizzled int8 tiles in registers; D = 64 converts through a scratch
-  static constexpr bool kDirect = kQ8 && kD == 128;
+  static constexpr bool kDirect = kQuant && kD == 128;
   static constexpr int kScrHalfBytes = kChunks * 16 * 128;   // 16 rows of K (or V), 16-bit
   static constexpr int kScrOffset = kStages * kStageBytes;
-  static constexpr int kScrBytes = (kQ8 && !kDirect) ? 4 * 2 * kScrHalfBytes : 0;
+  static constexpr int kScrBytes = (kQuant && !kDirect) ? 4 * 2 * kScrHalfBytes : 0;
   static constexpr int kBarOffset = kScrOffset + kScrBytes;
   // cross-warp reduction scratch aliases the stage ring (and the int8
   // scratch): it is written only after every issued chunk has been consumed
@@ -403,11 +436,13 @@ __device__ __forceinline__ float dec_logit(float s, const DecodeParams& p) {
 
 // kNT: number of 8-wide column tiles per CTA (a column block holds 8 * kNT
 // columns; column n is new token n / group, query head kvh * group + n % group)
-template <int kD, bool kBF16, int kNT, bool kQ8>
+template <int kD, bool kBF16, int kNT, int kQ>
 __global__ void __launch_bounds__(160)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using Sh = DecShape<kD, kQ8>;
+  using Sh = DecShape<kD, kQ>;
+  constexpr bool kQuant = Sh::kQuant;
+  constexpr bool kQ4 = kQ == 4;
   static_assert(sizeof(DecBars) <= 256, "barrier block exceeds its reservation");
   static_assert((8 * 8 * kNT + 4 * 8 * kNT * kD) * 4 <= Sh::kBarOffset, "reduction scratch exceeds the ring");
   extern __shared__ uint8_t smem_raw[];
@@ -493,7 +528,7 @@ __global__ void __launch_bounds__(160)
         const int row = page * p.page_size + (pos % p.page_size);
         mbar_arrive_expect_tx(&bars->full[slot], Sh::kLoadBytes);
         uint8_t* dst = smem + slot * Sh::kStageBytes;
-        if constexpr (kQ8) {
+        if constexpr (kQuant) {
           // one box of 64 rows x kD bytes each, then the chunk's scales: 64
           // contiguous floats of (page, kvh) (page_size is a multiple of 64)
           tma_load_3d(&tm_k, &bars->full[slot], dst, 0, kvh, row);
@@ -559,8 +594,17 @@ __global__ void __launch_bounds__(160)
       const float down = ldexpf(1.f, -e), up = ldexpf(1.f, e);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        qf[nt][kk][0] = pack2<false>(v[4 * kk] * down, v[4 * kk + 1] * down);
-        qf[nt][kk][1] = pack2<false>(v[4 * kk + 2] * down, v[4 * kk + 3] * down);
+        if constexpr (kQ4) {
+          // int4: K-step kk pairs nibbles (i, i + 4) and (i + 1, i + 5) of
+          // word kk / 2, i = 2 (kk % 2): d = 32j + 8 (kk / 2) + i + {0, 4}
+          // and + {1, 5}
+          const int i0 = 8 * (kk >> 1) + 2 * (kk & 1);
+          qf[nt][kk][0] = pack2<false>(v[i0] * down, v[i0 + 4] * down);
+          qf[nt][kk][1] = pack2<false>(v[i0 + 1] * down, v[i0 + 5] * down);
+        } else {
+          qf[nt][kk][0] = pack2<false>(v[4 * kk] * down, v[4 * kk + 1] * down);
+          qf[nt][kk][1] = pack2<false>(v[4 * kk + 2] * down, v[4 * kk + 3] * down);
+        }
       }
       qsc[nt][0] = __shfl_sync(0xffffffffu, up, 8 * (lane & 3));
       qsc[nt][1] = __shfl_sync(0xffffffffu, up, 8 * (lane & 3) + 4);
@@ -636,15 +680,43 @@ __global__ void __launch_bounds__(160)
     // this warp's converted rows, addressed by the row within the tile
     uint32_t kbase = sbase + slot * Sh::kStageBytes;
     uint32_t vbase = kbase + Sh::kKVBytes;
-    constexpr int kTileStride = kQ8 ? 16 * 128 : Sh::kBoxBytes;  // per 64-column chunk
-    const int trow0 = kQ8 ? tok0 : 0;                            // tile row = token - trow0
+    constexpr int kTileStride = kQuant ? 16 * 128 : Sh::kBoxBytes;  // per 64-column chunk
+    const int trow0 = kQuant ? tok0 : 0;                            // tile row = token - trow0
     float ksc0 = 1.f, ksc1 = 1.f, vsc0 = 1.f, vsc1 = 1.f;
     // direct int8 path: this lane's code words. K: rows tok0 + r and
     // tok0 + r + 8 (r = lane / 4), bytes d = 32j .. 32j + 31 (j = lane % 4);
     // V: tokens tok0 + 2j + {0, 1, 8, 9}, bytes d = 16r .. 16r + 15. Rows are
     // 128 bytes with the 16-byte group g stored at g ^ (row & 7).
     uint32_t kw[2][8], vw[4][4];
-    if constexpr (Sh::kDirect) {
+    if constexpr (kQ4) {
+      // int4 rows are 64 bytes, unswizzled: K, this lane's 16 bytes (d =
+      // 32j .. 32j + 31) of rows tok0 + r and tok0 + r + 8; V, its 8 bytes
+      // (d = 16r .. 16r + 15) of tokens tok0 + 2j + {0, 1, 8, 9}. Codes stay
+      // biased by 8.
+      const int r = lane >> 2, j = lane & 3;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4 w = *reinterpret_cast<const uint4*>(smem + (kbase - sbase) + (tok0 + r + 8 * h) * 64 + 16 * j);
+        kw[h][0] = w.x;
+        kw[h][1] = w.y;
+        kw[h][2] = w.z;
+        kw[h][3] = w.w;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int tk = tok0 + 2 * j + (u & 1) + 8 * (u >> 1);
+        const uint2 w = *reinterpret_cast<const uint2*>(smem + (vbase - sbase) + tk * 64 + 8 * r);
+        vw[u][0] = w.x;
+        vw[u][1] = w.y;
+      }
+      const float* sc = reinterpret_cast<const float*>(smem + slot * Sh::kStageBytes + Sh::kScaleOffset);
+      ksc0 = sc[tok0 + r];
+      ksc1 = sc[tok0 + r + 8];
+      vsc0 = sc[Sh::kTok + tok0 + r];
+      vsc1 = sc[Sh::kTok + tok0 + r + 8];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->empty[slot]);
+    } else if constexpr (Sh::kDirect) {
       const int r = lane >> 2, j = lane & 3;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -675,7 +747,7 @@ __global__ void __launch_bounds__(160)
       __syncwarp();
       // everything this warp needs from the slot is in registers
       if (lane == 0) mbar_arrive(&bars->empty[slot]);
-    } else if constexpr (kQ8) {
+    } else if constexpr (kQuant) {
       const uint8_t* kq = smem + slot * Sh::kStageBytes + tok0 * kD;
       const uint8_t* vq = kq + Sh::kKVBytes;
       uint8_t* ks = smem + Sh::kScrOffset + warp * 2 * Sh::kScrHalfBytes;
@@ -711,7 +783,18 @@ __global__ void __launch_bounds__(160)
     float s[kNT][4];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-    if constexpr (Sh::kDirect) {
+    if constexpr (kQ4) {
+      // A = K codes as exact fp16, nibbles (i, i + 4) and (i + 1, i + 5) of
+      // word kk / 2, i = 2 (kk % 2) (the permutation of the query fragments)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int sh = 8 * (kk & 1);
+        const uint32_t a0 = i4pair_to_f16(kw[0][kk >> 1] >> sh), a2 = i4pair_to_f16(kw[0][kk >> 1] >> (sh + 4));
+        const uint32_t a1 = i4pair_to_f16(kw[1][kk >> 1] >> sh), a3 = i4pair_to_f16(kw[1][kk >> 1] >> (sh + 4));
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) mma16816<false>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+      }
+    } else if constexpr (Sh::kDirect) {
       // A = K codes as exact fp16: word kk of a row holds d = 32j + 4kk + 0..3
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
@@ -739,7 +822,7 @@ __global__ void __launch_bounds__(160)
     // every column sees all 16 tokens: no mask (warp-uniform)
     const bool all_visible = wtok >= lo_in && wtok + 16 <= hi_in;
     float vr = 1.f;
-    if constexpr (kQ8) {
+    if constexpr (kQuant) {
       // S^T rows are tokens: the K scale multiplies each row (and, direct
       // path, 2^e of the column undoes the query scaling)
 #pragma unroll
@@ -816,7 +899,7 @@ __global__ void __launch_bounds__(160)
       }
       // P^T fragments: transpose the two 8x8 blocks of the 16x8 accumulator
       // (int8: the V row scale folded into P, token by token)
-      if constexpr (kQ8) {
+      if constexpr (kQuant) {
         pb[nt][0] = movmatrix_t(pack2<false>(e0 * vsc0, e1 * vsc0));
         pb[nt][1] = movmatrix_t(pack2<false>(e2 * vsc1, e3 * vsc1));
       } else {
@@ -825,7 +908,23 @@ __global__ void __launch_bounds__(160)
       }
     }
     // ---- O^T += V^T P^T ----
-    if constexpr (Sh::kDirect) {
+    if constexpr (kQ4) {
+      // A = V^T codes as exact fp16; accumulator rows r, r + 8 of step mt are
+      // d = 16r + 2mt and 16r + 2mt + 1, the low and high nibble of byte mt of
+      // this lane's V words; byte b of tokens 2j, 2j+1 (2j+8, 2j+9) is brought
+      // to bytes 0 and 2 first
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t bsel = static_cast<uint32_t>(mt & 3);
+        const uint32_t sel = bsel | ((bsel + 4) << 8);
+        const uint32_t x = __byte_perm(vw[0][mt >> 2], vw[1][mt >> 2], sel);
+        const uint32_t y = __byte_perm(vw[2][mt >> 2], vw[3][mt >> 2], sel);
+        const uint32_t a0 = i4pair_to_f16(x), a1 = i4pair_to_f16(x >> 4);
+        const uint32_t a2 = i4pair_to_f16(y), a3 = i4pair_to_f16(y >> 4);
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) mma16816<false>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      }
+    } else if constexpr (Sh::kDirect) {
       // A = V^T codes as exact fp16; accumulator rows r, r + 8 of step mt are
       // d = 16r + 2mt and 16r + 2mt + 1 (bytes 2mt, 2mt + 1 of this lane's V
       // words); k = tokens 2j, 2j+1 (a0, a1) and 2j+8, 2j+9 (a2, a3)
@@ -868,11 +967,11 @@ __global__ void __launch_bounds__(160)
         }
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt)
-          mma16816<kBF16 && !kQ8>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          mma16816<kBF16 && !kQuant>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
       }
     }
     __syncwarp();
-    if (!kQ8 && lane == 0) mbar_arrive(&bars->empty[slot]);
+    if (!kQuant && lane == 0) mbar_arrive(&bars->empty[slot]);
   }
 
   // ---- merge the four warps' states, then write the split's result ----
@@ -896,7 +995,7 @@ __global__ void __launch_bounds__(160)
       red_l[warp * kH + h0] = l0;
       red_l[warp * kH + h0 + 1] = l1;
     }
-    const float oc = kQ8 ? vC : 1.f;  // int8: acc holds O / vC
+    const float oc = kQuant ? vC : 1.f;  // int8: acc holds O / vC
 #pragma unroll
     for (int mt = 0; mt < kD / 16; ++mt) {
       // accumulator rows lane / 4 and lane / 4 + 8 of step mt

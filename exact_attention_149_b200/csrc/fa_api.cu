@@ -109,9 +109,10 @@ fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, i
   return FA_OK;
 }
 
-// int8 cache (T, H, D) bytes: one box is `rows` tokens x the whole D-byte row
-// of one head; D = 128 rows arrive with the 128-byte swizzle (16-byte group g
-// of row r at g ^ (r & 7)), D = 64 rows unswizzled
+// int8 / int4 cache (T, H, row_bytes) bytes, row_bytes = D (int8) or D / 2
+// (int4): one box is `rows` tokens x the whole row of one head; 128-byte rows
+// arrive with the 128-byte swizzle (16-byte group g of row r at g ^ (r & 7)),
+// shorter rows unswizzled
 fa_status make_map_i8(CUtensorMap* map, const void* base, int D, int H, long long T, int rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");

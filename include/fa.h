@@ -265,6 +265,37 @@ FA_API fa_status fa_kv_quantize_int8(const void* src, int8_t* codes, float* scal
                                      int page_size, int Hkv, int D, fa_dtype dtype, void* stream);
 
 /*
+ * fa_fwd_kvcache_int8 with an int4 cache (the same page; the other reading
+ * of its INT8/INT4 sentence): every cached row is int4 codes with one
+ * float32 scale, scale = max|x| / 7 and code = round-half-even(x / scale) in
+ * [-7, 7] (float32, IEEE division; a zero row: scale 0, codes 0), stored two
+ * per byte biased by 8, the code of even d in the low nibble.
+ *   k_cache, v_cache: DEVICE uint8 (num_pages, page_size, Hkv, D / 2).
+ *   k_scale, v_scale: as fa_fwd_kvcache_int8.
+ * Everything else as fa_fwd_kvcache_int8; D must be 128 (FA_ERR_UNSUPPORTED
+ * otherwise).
+ */
+FA_API fa_status fa_fwd_kvcache_int4(const void* q, const void* k_new, const void* v_new,
+                                     uint8_t* k_cache, uint8_t* v_cache, float* k_scale,
+                                     float* v_scale, const int32_t* block_table,
+                                     const int32_t* cache_seqlens, const float* rotary_cos,
+                                     const float* rotary_sin, void* out, float* lse, int B, int Sq,
+                                     int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                                     int num_pages, int rotary_rows, int rotary_dim,
+                                     int rotary_interleaved, float scale, int causal,
+                                     int window_left, int window_right, float softcap,
+                                     const float* alibi_slopes, int alibi_batch_stride,
+                                     int num_splits, fa_dtype dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
+ * fa_kv_quantize_int8 into the int4 format: codes uint8 (num_pages,
+ * page_size, Hkv, D / 2), 8-byte aligned; D 64 or 128.
+ */
+FA_API fa_status fa_kv_quantize_int4(const void* src, uint8_t* codes, float* scales, int num_pages,
+                                     int page_size, int Hkv, int D, fa_dtype dtype, void* stream);
+
+/*
  * fa_fwd_kvcache without a workspace argument, for callers that cannot
  * allocate device memory on their decode path: a serving loop that has
  * handed all free device memory to its KV-cache pool up front (so a late

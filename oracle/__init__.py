@@ -12,6 +12,7 @@ from .attention import (  # noqa: F401
     head_fwd,
     dequantize_int8,
     kvcache_decode,
+    kvcache_decode_int4,
     kvcache_decode_int8,
     lse_combine,
     pack_int4,

@@ -72,6 +72,7 @@ __all__ = [
     "attention_bwd",
     "kvcache_decode",
     "kvcache_decode_int8",
+    "kvcache_decode_int4",
     "quantize_int8",
     "dequantize_int8",
     "quantize_int4",
@@ -480,6 +481,31 @@ def kvcache_decode_int8(q, k_new, v_new, k_codes_logical, k_scales_logical, v_co
     rows already in the cache. Returns (O, LSE, appended k codes, k scales,
     v codes, v scales), the last four as lists of the B sequences' new rows.
     """
+    return _kvcache_decode_quant(quantize_int8, q, k_new, v_new, k_codes_logical,
+                                 k_scales_logical, v_codes_logical, v_scales_logical,
+                                 cache_seqlens, scale, causal, window, softcap, heads, rotary_cos,
+                                 rotary_sin, rotary_interleaved, rotated_dtype, alibi_slopes)
+
+
+def kvcache_decode_int4(q, k_new, v_new, k_codes_logical, k_scales_logical, v_codes_logical,
+                        v_scales_logical, cache_seqlens, scale: float, causal: bool = True,
+                        window=(-1, -1), softcap: float = 0.0, heads=None, rotary_cos=None,
+                        rotary_sin=None, rotary_interleaved=False, rotated_dtype=None,
+                        alibi_slopes=None):
+    """kvcache_decode_int8 with the int4 reading: codes in [-7, 7] (one per
+    element, unpacked; pack_int4 gives the stored bytes), appended rows
+    quantised by quantize_int4."""
+    return _kvcache_decode_quant(quantize_int4, q, k_new, v_new, k_codes_logical,
+                                 k_scales_logical, v_codes_logical, v_scales_logical,
+                                 cache_seqlens, scale, causal, window, softcap, heads, rotary_cos,
+                                 rotary_sin, rotary_interleaved, rotated_dtype, alibi_slopes)
+
+
+def _kvcache_decode_quant(quantize, q, k_new, v_new, k_codes_logical, k_scales_logical,
+                          v_codes_logical, v_scales_logical, cache_seqlens, scale, causal,
+                          window, softcap, heads, rotary_cos, rotary_sin, rotary_interleaved,
+                          rotated_dtype, alibi_slopes):
+    """The quantised-cache step shared by the int8 and int4 readings."""
     bsz, sq = tuple(q.shape)[:2]
     append = k_new is not None
     kd, vd, kc_new, ks_new, vc_new, vs_new = [], [], [], [], [], []
@@ -496,8 +522,8 @@ def kvcache_decode_int8(q, k_new, v_new, k_codes_logical, k_scales_logical, v_co
                 pos = np.arange(n, n + sq)
                 kn = round_to(rotary(kn, pos, rotary_cos, rotary_sin, rotary_interleaved),
                               rotated_dtype)
-            a_kc, a_ks = quantize_int8(kn)
-            a_vc, a_vs = quantize_int8(_f64(v_new[b]))
+            a_kc, a_ks = quantize(kn)
+            a_vc, a_vs = quantize(_f64(v_new[b]))
             kc_new.append(a_kc)
             ks_new.append(a_ks)
             vc_new.append(a_vc)

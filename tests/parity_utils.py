@@ -62,3 +62,29 @@ def check_bwd(grads_gpu, grads_ref, what=""):
             assert e <= BWD_REL_FRO, f"{what}: {name} rel-Frobenius {e:.3e}"
         out.append(e)
     return out
+
+
+# Quantised KV caches (int8 / int4): the forward bounds, with the mean-abs
+# bound widened by the output's own rounding. An output row mixes
+# dequantized rows (code * scale), which are not 16-bit values, so even a
+# one-key row is rounded once on output; that rounding averages a quarter of
+# an output ulp.
+MANTISSA_BITS = {"bf16": 7, "fp16": 10}
+
+
+def check_fwd_quant(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what):
+    o, lse = to64(o_gpu), to64(lse_gpu)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    lse_ref = np.asarray(lse_ref, dtype=np.float64)
+    assert o.shape == o_ref.shape and np.all(np.isfinite(o)), what
+    err = np.abs(o - o_ref)
+    assert err.max() <= FWD_MAX_ABS, f"{what}: max-abs {err.max():.3e}"
+    mag = np.abs(o_ref)
+    ulp = np.where(mag > 0, np.exp2(np.floor(np.log2(np.where(mag > 0, mag, 1.0))) - MANTISSA_BITS[dtype]), 0.0)
+    bound = FWD_MEAN_ABS + float(np.mean(ulp)) / 4
+    assert err.mean() <= bound, f"{what}: mean-abs {err.mean():.3e} > {bound:.3e}"
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse), fin), f"{what}: LSE finiteness differs"
+    if fin.any():
+        lerr = np.abs(lse[fin] - lse_ref[fin])
+        assert lerr.max() <= LSE_ABS, f"{what}: LSE max-abs {lerr.max():.3e}"

@@ -199,3 +199,42 @@ def test_quantize_int4_error_bound():
     np.testing.assert_array_equal(np.max(np.abs(codes.astype(np.int32)), axis=1), 7)
     err = np.abs(dequantize_int8(codes, scale) - x.astype(np.float64))
     assert np.all(err <= scale.astype(np.float64)[:, None] * (0.5 + 7 * 2.0 ** -22))
+
+
+def representable4(r, shape, exp_lo=-4, exp_hi=1):
+    """Rows of code * 2^e with |code| <= 7 and one +-7 per row: exact in the
+    int4 format (scale = 2^e) and in bf16 / fp16."""
+    codes = r.integers(-7, 8, shape)
+    idx = r.integers(0, shape[-1], shape[:-1])
+    np.put_along_axis(codes, idx[..., None], 7 * r.choice([-1, 1], shape[:-1])[..., None], -1)
+    e = r.integers(exp_lo, exp_hi + 1, shape[:-1])
+    return codes * np.exp2(e)[..., None].astype(np.float64)
+
+
+@pytest.mark.parametrize("sq,window,softcap,causal", [(1, (-1, -1), 0.0, True),
+                                                      (3, (5, 0), 1.3, True)])
+def test_int4_decode_reduces_to_plain_decode(sq, window, softcap, causal):
+    from oracle import kvcache_decode_int4, quantize_int4
+
+    r = rng(53 + sq)
+    B, hq, hkv, D = 2, 4, 2, 16
+    lens = [9, 2]
+    kc = [representable4(r, (n, hkv, D)) for n in lens]
+    vc = [representable4(r, (n, hkv, D)) for n in lens]
+    kn = representable4(r, (B, sq, hkv, D))
+    vn = representable4(r, (B, sq, hkv, D))
+    q = r.standard_normal((B, sq, hq, D))
+    kq = [quantize_int4(x) for x in kc]
+    vq = [quantize_int4(x) for x in vc]
+    for b in range(B):
+        np.testing.assert_array_equal(dequantize_int8(*kq[b]), kc[b])
+    o4, l4, akc, aks, avc, avs = kvcache_decode_int4(
+        q, kn, vn, [c for c, _ in kq], [s for _, s in kq], [c for c, _ in vq], [s for _, s in vq],
+        lens, 0.41, causal, window, softcap)
+    o, lse, _, _ = kvcache_decode(q, kn, vn, kc, vc, lens, 0.41, causal, window, softcap)
+    np.testing.assert_allclose(o4, o, atol=1e-13)
+    np.testing.assert_allclose(l4, lse, atol=1e-13)
+    for b in range(B):
+        np.testing.assert_array_equal(dequantize_int8(akc[b], aks[b]), kn[b])
+        np.testing.assert_array_equal(dequantize_int8(avc[b], avs[b]), vn[b])
+        assert np.all(np.abs(akc[b].astype(np.int32)) <= 7)

@@ -27,27 +27,7 @@ import torch
 
 import attn_workloads as W
 from oracle import dequantize_int8, kvcache_decode_int8, quantize_int8
-from parity_utils import FWD_MAX_ABS, FWD_MEAN_ABS, LSE_ABS, to64
-
-MANTISSA_BITS = {"bf16": 7, "fp16": 10}
-
-
-def check_fwd_int8(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what):
-    o, lse = to64(o_gpu), to64(lse_gpu)
-    o_ref = np.asarray(o_ref, dtype=np.float64)
-    lse_ref = np.asarray(lse_ref, dtype=np.float64)
-    assert o.shape == o_ref.shape and np.all(np.isfinite(o)), what
-    err = np.abs(o - o_ref)
-    assert err.max() <= FWD_MAX_ABS, f"{what}: max-abs {err.max():.3e}"
-    mag = np.abs(o_ref)
-    ulp = np.where(mag > 0, np.exp2(np.floor(np.log2(np.where(mag > 0, mag, 1.0))) - MANTISSA_BITS[dtype]), 0.0)
-    bound = FWD_MEAN_ABS + float(np.mean(ulp)) / 4
-    assert err.mean() <= bound, f"{what}: mean-abs {err.mean():.3e} > {bound:.3e}"
-    fin = np.isfinite(lse_ref)
-    assert np.array_equal(np.isfinite(lse), fin), f"{what}: LSE finiteness differs"
-    if fin.any():
-        lerr = np.abs(lse[fin] - lse_ref[fin])
-        assert lerr.max() <= LSE_ABS, f"{what}: LSE max-abs {lerr.max():.3e}"
+from parity_utils import check_fwd_quant as check_fwd_int8
 
 pytestmark = pytest.mark.gpu
 
