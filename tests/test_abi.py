@@ -41,6 +41,7 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_fwd_kvcache_int8", "fa_kv_quantize_int8",
+              "fa_fwd_kvcache_int4", "fa_kv_quantize_int4",
               "fa_bwd_workspace_size",
               "fa_kvcache_workspace_size", "fa_get_device_status", "fa_last_error", "fa_version"):
         assert n in names
@@ -222,6 +223,23 @@ def test_binding_checks_int8_cache_shapes(fa):
         fa.fwd_kvcache(q, kc, kc.to(torch.bfloat16), cs, None, k_scale=good, v_scale=good)
     with pytest.raises(fa.FaError, match="scales must be float32"):
         fa.kv_quantize_int8(torch.zeros(3, 64, 2, 128, dtype=torch.bfloat16), scales=torch.zeros(3, 64, 2))
+
+
+def test_kvcache_int4_rejects_bad_arguments(fa):
+    lib = fa.lib
+
+    def call(**kw):
+        a = dict(kc=16, ks=256, vs=512, D=128)
+        a.update(kw)
+        return lib.fa_fwd_kvcache_int4(16, 16, 16, a["kc"], 16, a["ks"], a["vs"], 16, 16, None, None,
+                                       16, 16, 2, 1, 4, 2, a["D"], 256, 4, 8, 0, 0, 0, 0.1, 1, -1,
+                                       -1, 0.0, None, 0, 1, 0, None, 0, None)
+
+    assert call(ks=None) == 1
+    assert call(kc=None) == 1
+    assert call(D=64) == 2          # int4 decode is D = 128 only
+    assert lib.fa_kv_quantize_int4(None, 16, 16, 1, 64, 1, 128, 0, None) == 1
+    assert lib.fa_kv_quantize_int4(16, 16, 16, 1, 64, 1, 96, 0, None) == 2
 
 
 def test_valid_call_without_gpu_reports_cuda_error(fa):
