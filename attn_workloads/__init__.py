@@ -313,6 +313,13 @@ def decode_kv_bytes(cache_seqlens, Hkv, D, elem_bytes=2):
     return 2 * n * Hkv * D * elem_bytes
 
 
+def decode_kv_bytes_int4(cache_seqlens, Hkv, D):
+    """The same for an int4 cache: per row D / 2 code bytes and a 4-byte
+    float32 scale."""
+    n = int(torch.as_tensor(cache_seqlens, dtype=torch.int64).sum().item()) + len(cache_seqlens)
+    return 2 * n * Hkv * (D // 2 + 4)
+
+
 def decode_kv_bytes_int8(cache_seqlens, Hkv, D):
     """The same for an int8 cache: per row D one-byte codes and a 4-byte
     float32 scale."""

@@ -475,6 +475,8 @@ def run_ours(args, dist: Dist):
     # then reads D + 4 bytes per cached row instead of 2 D
     kq, ksq = fa.kv_quantize_int8(kc)
     vq, vsq = fa.kv_quantize_int8(vc)
+    k4, ks4 = fa.kv_quantize_int4(kc)
+    v4, vs4 = fa.kv_quantize_int4(vc)
     del kc, vc
     torch.cuda.empty_cache()
     kv8 = W.decode_kv_bytes_int8(st["cache_seqlens"], cd.Hkv, cd.D)
@@ -512,6 +514,40 @@ def run_ours(args, dist: Dist):
                         "peak_source": peaks["source"] + " HBM copy"}
     res["decode_int8"] = dec8
     del kq, vq, ksq, vsq
+
+    # -------------------- and on an int4 cache (two codes per byte) --------------------
+    kv4 = W.decode_kv_bytes_int4(st["cache_seqlens"], cd.Hkv, cd.D)
+    dec4 = {"kv_bytes": kv4, "format": "int4 codes two per byte + one float32 scale per (token, kv head) row",
+            "splits": {}}
+    try:
+        for splits in cd.splits:
+            wsd = fa.fa_kvcache_workspace_size(cd.B, 1, cd.Hq, cd.D, splits)
+            wsb = torch.empty(max(wsd, 1), dtype=torch.uint8, device=dev)
+
+            def step_dec4(splits=splits, wsb=wsb):
+                fa.fwd_kvcache(dq_, k4, v4, cs, bt, k_new=kn, v_new=vn, scale=cd.scale, causal=True,
+                               num_splits=splits, out=dout, lse=dlse, workspace=wsb, k_scale=ks4,
+                               v_scale=vs4)
+
+            ms_d = timed(step_dec4, max(args.steps, 20), args.warmup, dist, fa_mod=fa)
+            ksplit, nsplit = fa.fa_kernel_timing_read("decode_split")
+            fa.fa_kernel_timing_reset()
+            gbs = kv4 / (ms_d * 1e-3) / 1e9
+            entry = {"ms": ms_d, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                     "speedup_vs_16bit": dec["splits"][str(splits)]["ms"] / ms_d}
+            if nsplit:
+                ks = ksplit / nsplit
+                entry["decode_split_kernel"] = {
+                    "ms_avg": ks, "gbs": kv4 / (ks * 1e-3) / 1e9,
+                    "frac_of_hbm": kv4 / (ks * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+            dec4["splits"][str(splits)] = entry
+        best4 = max(dec4["splits"].values(), key=lambda d: d["gbs"])
+        dec4["best_gbs"] = best4["gbs"]
+        dec4["best_frac_of_hbm"] = best4["frac_of_hbm"]
+    except Exception as e:  # recorded in the line; the headline measurement stands
+        dec4["error"] = f"{type(e).__name__}: {e}"
+    res["decode_int4"] = dec4
+    del k4, v4, ks4, vs4
     torch.cuda.empty_cache()
 
     # -------------------- roofline of the dominant kernel --------------------
