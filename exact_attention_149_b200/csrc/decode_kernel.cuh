@@ -25,13 +25,18 @@
 // P^T's fragment is the transpose of S^T's accumulator fragment, done with
 // movmatrix.
 //
-// int8 cache: the chunks arrive as int8 codes plus one float32 scale per
-// (token, kv head) row; each consumer warp converts its 16 rows of codes to
-// exact 16-bit values in its own shared-memory tiles (K in the input type, V
-// in fp16) and the products above run on them: the K scale multiplies the
-// rows of S^T, and the V scale, divided by the largest V scale the warp has
-// seen, multiplies P (so the fp16 P keeps 11 bits without overflow); that
-// largest scale is folded into the accumulator's online rescale.
+// int8 / int4 caches: the chunks arrive as codes plus one float32 scale per
+// (token, kv head) row. At D = 128 each consumer lane builds its mma
+// fragments straight from the code tiles in registers (codes become exact
+// fp16 by placing them under the exponent bits of 1024 and subtracting the
+// bias), with the head dimension permuted per lane so that its loads are
+// 16-byte reads; QK then runs in fp16 on queries scaled by a power of two.
+// At D = 64 (int8 only) each warp converts its 16 rows into 16-bit tiles in
+// its own shared memory and the products above run on them. Either way the K
+// scale multiplies the rows of S^T, and the V scale, divided by the largest
+// V scale the warp has seen, multiplies P (so the fp16 P keeps 11 bits
+// without overflow); that largest scale is folded into the accumulator's
+// online rescale.
 #pragma once
 
 #include "ptx.cuh"
