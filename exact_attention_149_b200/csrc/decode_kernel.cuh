@@ -172,7 +172,7 @@ __device__ __forceinline__ uint2 quantize_row(const float (&x)[8], float* scale)
 }
 
 // grid B * Sq (one block per new token), block 128: 16 bytes per thread-step.
-// kQuant: the new rows are quantised into an int8 cache (keys after the rotary
+// kQuant: the new rows are quantised into an int8 / int4 cache (keys after the rotary
 // rotation and the rounding to the 16-bit type, as the 16-bit cache stores
 // them); each warp takes heads warp, warp + 4, ..., lanes 0-15 the key row and
 // lanes 16-31 the value row.
@@ -390,7 +390,7 @@ __device__ __forceinline__ uint32_t sw128(uint32_t base, int r, int g) {
   return base + r * 128 + ((g ^ (r & 7)) << 4);
 }
 
-// kQuant: the ring holds int8 chunks (K codes, V codes, then the 64 K and 64 V
+// kQuant: the ring holds int8 / int4 chunks (K codes, V codes, then the 64 K and 64 V
 // scales). D = 128: the code tiles arrive with the 128-byte swizzle and the
 // consumers build their fragments from them in registers. D = 64: unswizzled
 // tiles, and each consumer warp converts its 16 rows into 16-bit tiles in its
@@ -1000,7 +1000,7 @@ __global__ void __launch_bounds__(160)
       red_l[warp * kH + h0] = l0;
       red_l[warp * kH + h0 + 1] = l1;
     }
-    const float oc = kQuant ? vC : 1.f;  // int8: acc holds O / vC
+    const float oc = kQuant ? vC : 1.f;  // int8 / int4: acc holds O / vC
 #pragma unroll
     for (int mt = 0; mt < kD / 16; ++mt) {
       // accumulator rows lane / 4 and lane / 4 + 8 of step mt
