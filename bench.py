@@ -277,10 +277,13 @@ def run_only(args, dist: Dist):
         kn, vn = st["k_new"].to(dev), st["v_new"].to(dev)
         cs, bt = st["cache_seqlens"].to(dev), st["block_table"].to(dev)
         kv_bytes = W.decode_kv_bytes(st["cache_seqlens"], cd.Hkv, cd.D)
-        if args.int8:
-            kc, ksc = fa.kv_quantize_int8(kc)
-            vc, vsc = fa.kv_quantize_int8(vc)
-            kv_bytes = W.decode_kv_bytes_int8(st["cache_seqlens"], cd.Hkv, cd.D)
+        if args.int8 or args.int4:
+            quant = fa.kv_quantize_int4 if args.int4 else fa.kv_quantize_int8
+            kc, ksc = quant(kc)
+            vc, vsc = quant(vc)
+            torch.cuda.empty_cache()
+            kv_bytes = (W.decode_kv_bytes_int4 if args.int4 else W.decode_kv_bytes_int8)(
+                st["cache_seqlens"], cd.Hkv, cd.D)
             fn = lambda: fa.fwd_kvcache(q, kc, vc, cs, bt, k_new=kn, v_new=vn, scale=cd.scale,  # noqa: E731
                                         causal=True, num_splits=args.splits, k_scale=ksc,
                                         v_scale=vsc)
@@ -290,7 +293,7 @@ def run_only(args, dist: Dist):
         ms = timed(fn, args.steps, args.warmup, dist)
         gbs = kv_bytes / (ms * 1e-3) / 1e9
         out.update(ms=ms, gbs=gbs, frac_of_hbm=gbs / peaks["hbm_gbs"], splits=args.splits, B=B,
-                   int8=bool(args.int8))
+                   cache="int4" if args.int4 else ("int8" if args.int8 else "16-bit"))
     return out
 
 
@@ -695,6 +698,7 @@ def main():
                     help="time one kernel family only (profiling runs)")
     ap.add_argument("--splits", type=int, default=16, help="num_splits for --only decode")
     ap.add_argument("--int8", action="store_true", help="--only decode on an int8 cache")
+    ap.add_argument("--int4", action="store_true", help="--only decode on an int4 cache")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="batch for --only decode (default: the B64 workload); smaller for ncu")
     args = ap.parse_args()
