@@ -44,9 +44,12 @@ __all__ = [
     "bwd_flops",
     "varlen_visible_pairs",
     "decode_kv_bytes",
+    "to_e4m3",
+    "make_fp8_inputs",
+    "make_fp8_varlen_inputs",
 ]
 
-DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
 
 
 @dataclass(frozen=True)
@@ -139,6 +142,39 @@ def make_fwd_inputs(B, S, Hq, Hkv, D, dtype="bf16", seed=0, with_do=False):
     out = {"q": q, "k": k, "v": v}
     if with_do:
         out["do"] = _randn(g, (B, S, Hq, D), dtype)
+    return out
+
+
+def to_e4m3(x: torch.Tensor):
+    """Per-tensor FP8 E4M3 encoding as a caller would prepare the FP8
+    forward's inputs: descale = max|x| / 448 (rounded to float32, the type the
+    library takes it in), codes = x / descale clamped to the finite range
+    and cast to torch.float8_e4m3fn (round to nearest even). Returns (codes
+    as a uint8 tensor of bit patterns, descale as a Python float)."""
+    amax = float(x.detach().abs().max().to(torch.float64))
+    descale = float(np.float32(amax / 448.0)) if amax > 0 else 1.0
+    y = (x.detach().to(torch.float64) / descale).clamp(-448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8), descale
+
+
+def make_fp8_inputs(B, S, Hq, Hkv, D, seed=0):
+    """FP8 forward inputs: q, k, v drawn as make_fwd_inputs draws them (fp32
+    N(0, 1), same generator order) and encoded per tensor by to_e4m3.
+    Returns {"q", "k", "v"} uint8 code tensors and {"q_descale", ...}."""
+    raw = make_fwd_inputs(B, S, Hq, Hkv, D, "fp32", seed)
+    out = {}
+    for n in ("q", "k", "v"):
+        out[n], out[n + "_descale"] = to_e4m3(raw[n])
+    return out
+
+
+def make_fp8_varlen_inputs(Hq, Hkv, D, seed=0, total=None, len_lo=None, len_hi=None,
+                           lengths=None):
+    """make_varlen_inputs in fp32, then every tensor encoded by to_e4m3."""
+    raw = make_varlen_inputs(lengths, Hq, Hkv, D, "fp32", seed, total, len_lo, len_hi)
+    out = {"lengths": raw["lengths"], "cu_seqlens": raw["cu_seqlens"]}
+    for n in ("q", "k", "v"):
+        out[n], out[n + "_descale"] = to_e4m3(raw[n])
     return out
 
 

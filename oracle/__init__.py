@@ -8,6 +8,9 @@ from .attention import (  # noqa: F401
     alibi_bias,
     attention_bwd,
     attention_fwd,
+    attention_fwd_fp8,
+    decode_e4m3,
+    head_probs,
     head_bwd,
     head_fwd,
     dequantize_int8,

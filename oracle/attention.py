@@ -52,7 +52,16 @@ notes of the repository):
   to the 16-bit input type first, as the 16-bit cache stores it, then
   quantised. The int4 reading is the same with ``scale = max|x| / 7`` and
   codes in [-7, 7], stored two per byte (the code of even d in the low
-  nibble, both biased by 8); no kernel uses it yet.
+  nibble, both biased by 8).
+* The guide (§版本怎么选) says FlashAttention-3 runs an FP8 forward and gives
+  no format. The reading here is the common one: Q, K and V are FP8 E4M3
+  tensors (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0
+  is subnormal, the all-ones pattern is NaN, no infinities; largest finite
+  value 448) with one float32 descale per tensor, so an element stands for
+  ``value(code) * descale``. The FP8 forward is then exact attention over
+  those values; its output is 16-bit. How close a kernel that feeds the
+  probabilities to the tensor cores in E4M3 comes to it is a tolerance,
+  derived in the tests (not emulated here).
 
 Every array is float64. 16-bit inputs are converted exactly (every bf16 and
 fp16 value is representable in float64), so the oracle sees the same values
@@ -73,6 +82,9 @@ __all__ = [
     "kvcache_decode",
     "kvcache_decode_int8",
     "kvcache_decode_int4",
+    "decode_e4m3",
+    "attention_fwd_fp8",
+    "head_probs",
     "quantize_int8",
     "dequantize_int8",
     "quantize_int4",
@@ -558,3 +570,52 @@ def lse_combine(o_parts, lse_parts):
     wn = np.where(has[None], w / np.where(has, s, 1.0)[None], 0.0)
     o = np.sum(wn[..., None] * o_parts, axis=0)
     return o, lse
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """Float64 values of FP8 E4M3 bit patterns (uint8 codes), from the
+    format's definition: bit 7 is the sign, bits 6..3 the exponent e (bias 7),
+    bits 2..0 the mantissa m. e = 0 gives the subnormal m * 2^-9; otherwise
+    (1 + m / 8) * 2^(e - 7); e = 15 with m = 7 is NaN (the format has no
+    infinities, and e = 15 with m < 7 are ordinary values up to 448)."""
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where((c & 0x80) != 0, -mag, mag)
+
+
+def attention_fwd_fp8(q_codes, k_codes, v_codes, q_descale: float, k_descale: float,
+                      v_descale: float, scale: float, causal: bool = False, window=(-1, -1),
+                      softcap: float = 0.0, cu_seqlens=None, alibi_slopes=None):
+    """The FP8 forward (reading in the module header): every E4M3 code times
+    its tensor's descale is the element it stands for, and the result is
+    attention_fwd over those values, in the layouts of attention_fwd."""
+    q = decode_e4m3(q_codes) * float(q_descale)
+    k = decode_e4m3(k_codes) * float(k_descale)
+    v = decode_e4m3(v_codes) * float(v_descale)
+    return attention_fwd(q, k, v, scale, causal, window, softcap, cu_seqlens, alibi_slopes)
+
+
+def head_probs(q_h, k_h, scale: float, causal: bool = False, window_left: int = -1,
+               window_right: int = -1, softcap: float = 0.0, rows=None,
+               alibi_slope: float = 0.0) -> np.ndarray:
+    """The attention probabilities of one head, [len(rows), Sk]: the softmax
+    step of the definition (logits, mask, row-normalised exponentials), zero
+    where masked and on rows with no visible key. O = head_probs @ V."""
+    q_h = _f64(q_h)
+    k_h = _f64(k_h)
+    sq, sk = q_h.shape[0], k_h.shape[0]
+    if rows is None:
+        rows = np.arange(sq)
+    rows = np.asarray(rows, dtype=np.int64)
+    x, _ = scores(q_h[rows], k_h, scale, softcap)
+    if alibi_slope != 0.0:
+        x = x + alibi_bias(sq, sk, alibi_slope, rows)
+    x = np.where(visible_mask(sq, sk, causal, window_left, window_right, rows), x, -np.inf)
+    m = np.max(x, axis=1, initial=-np.inf)
+    has = np.isfinite(m)
+    p = np.exp(x - np.where(has, m, 0.0)[:, None])
+    l = p.sum(axis=1)
+    return np.where(has[:, None], p / np.where(has, l, 1.0)[:, None], 0.0)
