@@ -28,6 +28,7 @@ __all__ = [
     "fwd", "bwd", "fwd_kvcache", "fwd_qkvpacked", "bwd_qkvpacked", "fa_fwd_qkvpacked",
     "fa_bwd_qkvpacked", "fa_fwd_kvcache_int8", "fa_kv_quantize_int8", "kv_quantize_int8",
     "fa_fwd_kvcache_int4", "fa_kv_quantize_int4", "kv_quantize_int4",
+    "fa_fwd_fp8", "fwd_fp8", "fa_selftest_poly",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -59,6 +60,11 @@ _z = ctypes.c_size_t
 lib.fa_fwd.restype = _i
 lib.fa_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _p, _i, _p, _i,
                        _i, _p]
+lib.fa_fwd_fp8.restype = _i
+lib.fa_fwd_fp8.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _f, _f, _i, _i, _i, _f,
+                           _p, _i, _p, _i, _i, _p]
+lib.fa_selftest_poly.restype = _i
+lib.fa_selftest_poly.argtypes = [_i, _p, _p, _p, _i, _p]
 lib.fa_bwd.restype = _i
 lib.fa_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f,
                        _p, _i, _p, _i, _i, _p, _z, _p]
@@ -157,6 +163,19 @@ def fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, scale, causal, window_left, wind
     _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, scale,
                       int(causal), window_left, window_right, softcap, _ptr(alibi_slopes),
                       alibi_batch_stride, _ptr(cu_seqlens), total_tokens, dtype, _stream(stream)))
+
+
+def fa_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, S, D, scale, q_descale, k_descale, v_descale,
+               causal, window_left, window_right, softcap, alibi_slopes, alibi_batch_stride,
+               cu_seqlens, total_tokens, out_dtype, stream=None):
+    _check(lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, scale,
+                          q_descale, k_descale, v_descale, int(causal), window_left, window_right,
+                          softcap, _ptr(alibi_slopes), alibi_batch_stride, _ptr(cu_seqlens),
+                          total_tokens, out_dtype, _stream(stream)))
+
+
+def fa_selftest_poly(which, x, out_poly, out_ref, n, stream=None):
+    _check(lib.fa_selftest_poly(which, _ptr(x), _ptr(out_poly), _ptr(out_ref), n, _stream(stream)))
 
 
 def fa_fwd_qkvpacked(qkv, out, lse, B, H, S, D, scale, causal, window_left, window_right, softcap,
@@ -343,6 +362,45 @@ def fwd(q, k, v, scale=None, causal=False, window=(-1, -1), softcap=0.0, cu_seql
     al, als = _alibi(alibi_slopes, Hq)
     fa_fwd(q, k, v, out, lse, B, Hq, Hkv, S, D, _scale(scale, D), causal, window[0], window[1],
            softcap, al, als, cu_seqlens, T, _dt(q), stream)
+    return out, lse
+
+
+_FP8_IN = (torch.uint8, torch.float8_e4m3fn)
+
+
+def fwd_fp8(q, k, v, q_descale, k_descale, v_descale, scale=None, causal=False, window=(-1, -1),
+            softcap=0.0, cu_seqlens=None, max_seqlen=None, out=None, lse=None, alibi_slopes=None,
+            out_dtype=torch.bfloat16, stream=None):
+    """FP8 forward: q, k, v are E4M3 codes (uint8 bit patterns or
+    torch.float8_e4m3fn) in fwd's layouts, each tensor with a float descale;
+    out in out_dtype (bf16 / fp16), lse float32 as in fwd."""
+    _need_cuda(q, k, v, cu_seqlens)
+    for t in (q, k, v):
+        if t.dtype not in _FP8_IN:
+            raise FaError(FA_ERR_INVALID_ARG, "fwd_fp8 takes uint8 or float8_e4m3fn q, k, v")
+    if cu_seqlens is None:
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+        T = 0
+        lse_shape = (B, Hq, S)
+    else:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise FaError(FA_ERR_INVALID_ARG, "max_seqlen is required with cu_seqlens")
+        S = int(max_seqlen)
+        lse_shape = (Hq, T)
+    if out_dtype not in _DTYPE:
+        raise FaError(FA_ERR_INVALID_ARG, f"out_dtype {out_dtype} not supported (bf16/fp16)")
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    al, als = _alibi(alibi_slopes, Hq)
+    fa_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, S, D, _scale(scale, D), float(q_descale),
+               float(k_descale), float(v_descale), causal, window[0], window[1], softcap, al, als,
+               cu_seqlens, T, _DTYPE[out.dtype], stream)
     return out, lse
 
 

@@ -384,6 +384,14 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
   }
 }
 
+// int4 slices: the token (0..15 within a warp's 16) that fragment row / k
+// index m stands for, m ^ ((m >> 1) & 1): rows m = r and r + 8 of the K
+// fragment and k = 2j + {0, 1, 8, 9} of the V fragment then fall, under the
+// 64-byte swizzle of the 64-byte int4 rows, on distinct banks. S^T row m and
+// P^T column m are the same token, so only the addressing and the token
+// positions change.
+__device__ __forceinline__ int i4_token(int m) { return m ^ ((m >> 1) & 1); }
+
 // address of the 16-byte group `g` (0..7 within a 128-byte row) of row `r`
 // of a TMA tile written with the 128-byte swizzle (tile base 1024-aligned)
 __device__ __forceinline__ uint32_t sw128(uint32_t base, int r, int g) {
@@ -652,6 +660,7 @@ __global__ void __launch_bounds__(160)
   // fp16's 11-bit precision; acc holds O / vC (vC only grows, and the change
   // is folded into the online-softmax rescale of acc)
   float vC = 1.17549435e-38f;
+  float vCinv = 1.f / 1.17549435e-38f;
   float acc[kNT][kD / 16][4];
 #pragma unroll
   for (int nt = 0; nt < kNT; ++nt) {
@@ -695,14 +704,19 @@ __global__ void __launch_bounds__(160)
     // 128 bytes with the 16-byte group g stored at g ^ (row & 7).
     uint32_t kw[2][8], vw[4][4];
     if constexpr (kQ4) {
-      // int4 rows are 64 bytes, unswizzled: K, this lane's 16 bytes (d =
-      // 32j .. 32j + 31) of rows tok0 + r and tok0 + r + 8; V, its 8 bytes
-      // (d = 16r .. 16r + 15) of tokens tok0 + 2j + {0, 1, 8, 9}. Codes stay
-      // biased by 8.
+      // int4 rows are 64 bytes, written by TMA with the 64-byte swizzle (the
+      // 16-byte group g of row t at g ^ ((t >> 1) & 3)). Fragment row / k
+      // index m of the warp's 16 tokens is token tok0 + i4_token(m), so that
+      // both reads below are free of bank conflicts. K: this lane's 16 bytes
+      // (d = 32j .. 32j + 31) of tokens i4_token(r), i4_token(r + 8); V, its
+      // 8 bytes (d = 16r .. 16r + 15) of tokens i4_token(2j + {0, 1, 8, 9}).
+      // Codes stay biased by 8.
       const int r = lane >> 2, j = lane & 3;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint4 w = *reinterpret_cast<const uint4*>(smem + (kbase - sbase) + (tok0 + r + 8 * h) * 64 + 16 * j);
+        const int tk = tok0 + i4_token(r + 8 * h);
+        const uint4 w = *reinterpret_cast<const uint4*>(smem + (kbase - sbase) + tk * 64 +
+                                                        ((j ^ ((tk >> 1) & 3)) << 4));
         kw[h][0] = w.x;
         kw[h][1] = w.y;
         kw[h][2] = w.z;
@@ -710,16 +724,18 @@ __global__ void __launch_bounds__(160)
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int tk = tok0 + 2 * j + (u & 1) + 8 * (u >> 1);
-        const uint2 w = *reinterpret_cast<const uint2*>(smem + (vbase - sbase) + tk * 64 + 8 * r);
+        const int tk = tok0 + i4_token(2 * j + (u & 1) + 8 * (u >> 1));
+        const uint2 w = *reinterpret_cast<const uint2*>(smem + (vbase - sbase) + tk * 64 +
+                                                        (((r >> 1) ^ ((tk >> 1) & 3)) << 4) + 8 * (r & 1));
         vw[u][0] = w.x;
         vw[u][1] = w.y;
       }
       const float* sc = reinterpret_cast<const float*>(smem + slot * Sh::kStageBytes + Sh::kScaleOffset);
-      ksc0 = sc[tok0 + r];
-      ksc1 = sc[tok0 + r + 8];
-      vsc0 = sc[Sh::kTok + tok0 + r];
-      vsc1 = sc[Sh::kTok + tok0 + r + 8];
+      const int tr = tok0 + i4_token(r);
+      ksc0 = sc[tr];
+      ksc1 = sc[tr + 8];
+      vsc0 = sc[Sh::kTok + tr];
+      vsc1 = sc[Sh::kTok + tr + 8];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->empty[slot]);
     } else if constexpr (Sh::kDirect) {
@@ -824,7 +840,8 @@ __global__ void __launch_bounds__(160)
     }
     // ---- logits, mask, online softmax ----
     const int wtok = (t_begin + i) * Sh::kTok + tok0;  // first token of this warp's 16
-    const int pos0 = wtok + (lane >> 2);                // token of s[.][0], s[.][1]
+    // token of s[.][0], s[.][1] (s[.][2], s[.][3]: + 8)
+    const int pos0 = wtok + (kQ4 ? i4_token(lane >> 2) : (lane >> 2));
     // every column sees all 16 tokens: no mask (warp-uniform)
     const bool all_visible = wtok >= lo_in && wtok + 16 <= hi_in;
     float vr = 1.f;
@@ -844,14 +861,19 @@ __global__ void __launch_bounds__(160)
         if (pos0 >= Lk) vsc0 = 0.f;
         if (pos0 + 8 >= Lk) vsc1 = 0.f;
       }
+      // the warp's largest V scale (the four lanes of a row hold the same
+      // two scales); vC and its reciprocal change only when it grows
       float c = fmaxf(vsc0, vsc1);
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, off));
-      const float c_new = fmaxf(vC, c);
-      vr = vC / c_new;  // acc (in units of vC) -> units of c_new
-      vC = c_new;
-      vsc0 = vsc0 / c_new;
-      vsc1 = vsc1 / c_new;
+      for (int off = 4; off < 32; off <<= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, off));
+      if (c > vC) {
+        const float inv = 1.f / c;
+        vr = vC * inv;  // acc (in units of vC) -> units of c
+        vC = c;
+        vCinv = inv;
+      }
+      vsc0 *= vCinv;
+      vsc1 *= vCinv;
     }
     uint32_t pb[kNT][2];
 #pragma unroll
@@ -896,12 +918,15 @@ __global__ void __launch_bounds__(160)
       l_part[nt][0] = l_part[nt][0] * al0 + e0 + e2;
       l_part[nt][1] = l_part[nt][1] * al1 + e1 + e3;
       const float ar0 = al0 * vr, ar1 = al1 * vr;
+      // (warp-uniform: most slices move neither the max nor vC)
+      if (__any_sync(0xffffffffu, ar0 != 1.f || ar1 != 1.f)) {
 #pragma unroll
-      for (int mt = 0; mt < kD / 16; ++mt) {
-        acc[nt][mt][0] *= ar0;
-        acc[nt][mt][1] *= ar1;
-        acc[nt][mt][2] *= ar0;
-        acc[nt][mt][3] *= ar1;
+        for (int mt = 0; mt < kD / 16; ++mt) {
+          acc[nt][mt][0] *= ar0;
+          acc[nt][mt][1] *= ar1;
+          acc[nt][mt][2] *= ar0;
+          acc[nt][mt][3] *= ar1;
+        }
       }
       // P^T fragments: transpose the two 8x8 blocks of the 16x8 accumulator
       // (int8: the V row scale folded into P, token by token)

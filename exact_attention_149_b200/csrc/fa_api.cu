@@ -109,11 +109,31 @@ fa_status make_map_thd(CUtensorMap* map, const void* base, fa_dtype dt, int D, i
   return FA_OK;
 }
 
+// 3-D map over a (tokens, heads, D) tensor of one-byte FP8 elements; box =
+// 128 columns (128 B, one swizzle row) x 1 head x `rows` tokens, 128-byte
+// swizzle; D a multiple of 128.
+fa_status make_map_thd8(CUtensorMap* map, const void* base, int D, int H, long long T, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H) * D};
+  cuuint32_t box[3] = {128u, 1u, static_cast<cuuint32_t>(rows)};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
 // int8 / int4 cache (T, H, row_bytes) bytes, row_bytes = D (int8) or D / 2
 // (int4): one box is `rows` tokens x the whole row of one head; 128-byte rows
 // arrive with the 128-byte swizzle (16-byte group g of row r at g ^ (r & 7)),
-// shorter rows unswizzled
-fa_status make_map_i8(CUtensorMap* map, const void* base, int D, int H, long long T, int rows) {
+// 64-byte rows with the 64-byte swizzle when swz64 is set (group g of row r
+// at g ^ ((r >> 1) & 3)), unswizzled otherwise
+fa_status make_map_i8(CUtensorMap* map, const void* base, int D, int H, long long T, int rows,
+                      bool swz64 = false) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
@@ -122,7 +142,9 @@ fa_status make_map_i8(CUtensorMap* map, const void* base, int D, int H, long lon
   cuuint32_t box[3] = {static_cast<cuuint32_t>(D), 1u, static_cast<cuuint32_t>(rows)};
   cuuint32_t es[3] = {1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                            : (swz64 && D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return FA_OK;
@@ -235,7 +257,60 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return FA_OK;
 }
 
+template <int kD, bool kBF16, bool kCap>
+fa_status launch_fwd8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const fa::FwdParams& p, cudaStream_t st) {
+  using Sh = fa::FwdShape<kD, true>;
+  auto kern = p.alibi ? fa::fwd_kernel<kD, kBF16, kCap, true, true>
+                      : fa::fwd_kernel<kD, kBF16, kCap, false, true>;
+  fa_status s = set_smem(kern, Sh::kSmemBytes);
+  if (s != FA_OK) return s;
+  const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "grid too large");
+  {
+    KernelTimer timer("fwd_fp8", st);
+    kern<<<static_cast<unsigned>(grid), Sh::kThreads, Sh::kSmemBytes, st>>>(tq, tk, tv, p);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "fwd_fp8 launch failed: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
 }  // namespace
+
+namespace fa {
+
+// Evaluates one of the FMA-pipe approximations the kernels use, and the CUDA
+// math function it stands in for, on the same inputs (two values per thread,
+// as the kernels evaluate them): 0 ex2_poly2 / exp2f, 1 tanh_poly2 / tanhf,
+// 2 the degree-2 folded tanh (tanh_fold2 with a = c = 1) / tanhf.
+__global__ void poly_selftest_kernel(int which, const float* x, float* out_poly, float* out_ref,
+                                     int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  float2 r, ref;
+  if (which == 0) {
+    r = ex2_poly2(v);
+    ref = make_float2(exp2f(v.x), exp2f(v.y));
+  } else if (which == 1) {
+    r = tanh_poly2(v);
+    ref = make_float2(tanhf(v.x), tanhf(v.y));
+  } else {
+    float pk[3];
+    fold_tanh(kTanhLo, 1.f, 1.f, pk);
+    r = tanh_fold2(v, pk);
+    ref = make_float2(tanhf(v.x), tanhf(v.y));
+  }
+  out_poly[i] = r.x;
+  out_ref[i] = ref.x;
+  if (i + 1 < n) {
+    out_poly[i + 1] = r.y;
+    out_ref[i + 1] = ref.y;
+  }
+}
+
+}  // namespace fa
 
 namespace {
 
@@ -370,6 +445,85 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   return fwd_impl(q, k, v, -1, -1, out, lse, B, Hq, Hkv, S, D, scale, causal, window_left,
                   window_right, softcap, alibi_slopes, alibi_batch_stride, cu_seqlens, total_tokens,
                   dtype, stream);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int Hq, int Hkv, int S, int D, float scale, float q_descale, float k_descale,
+                     float v_descale, int causal, int window_left, int window_right, float softcap,
+                     const float* alibi_slopes, int alibi_batch_stride, const int32_t* cu_seqlens,
+                     int total_tokens, fa_dtype out_dtype, void* stream) {
+  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd_fp8: null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd_fp8: tensors must be 16-byte aligned");
+  if (D != 128 && D != 256)
+    return fail(FA_ERR_UNSUPPORTED, "fa_fwd_fp8: head dim %d not supported (128 or 256)", D);
+  fa_status s = check_common(B, Hq, Hkv, S, D, scale, window_left, window_right, softcap, out_dtype,
+                             cu_seqlens, total_tokens, true);
+  if (s != FA_OK) return s;
+  for (float d : {q_descale, k_descale, v_descale})
+    if (!(d > 0.f) || !std::isfinite(d))
+      return fail(FA_ERR_INVALID_ARG, "fa_fwd_fp8: descales must be finite and > 0");
+  if ((s = check_alibi(alibi_slopes, alibi_batch_stride, Hq)) != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+
+  const long long T = cu_seqlens ? total_tokens : static_cast<long long>(B) * S;
+  CUtensorMap tq, tk, tv;
+  if ((s = make_map_thd8(&tq, q, D, Hq, T, 128)) != FA_OK) return s;
+  if ((s = make_map_thd8(&tk, k, D, Hkv, T, 128)) != FA_OK) return s;
+  if ((s = make_map_thd8(&tv, v, D, Hkv, T, 128)) != FA_OK) return s;
+
+  // the logits' scale carries both input descales; the output carries v's
+  const double eff = static_cast<double>(scale) * q_descale * k_descale;
+  if (!std::isfinite(eff)) return fail(FA_ERR_INVALID_ARG, "fa_fwd_fp8: scale * descales overflows");
+  fa::FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.total = static_cast<int>(T);
+  p.group = Hq / Hkv;
+  const int rows_per_cta = D == 256 ? fa::FwdShape<256, true>::kRows : fa::FwdShape<128, true>::kRows;
+  p.n_qblocks = (S + rows_per_cta - 1) / rows_per_cta;
+  p.scale_log2 = static_cast<float>(eff * 1.4426950408889634);
+  p.softcap = softcap;
+  p.cap_in = softcap > 0.f ? static_cast<float>(eff / softcap) : 0.f;
+  p.cap_out_log2 = static_cast<float>(static_cast<double>(softcap) * 1.4426950408889634);
+  p.wl = window_left;
+  p.wr = causal ? 0 : window_right;
+  p.o = out;
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.alibi = alibi_slopes;
+  p.alibi_bstride = alibi_batch_stride;
+  p.o_scale = v_descale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool cap = softcap > 0.f;
+  const bool bf = out_dtype == FA_BF16;
+  if (D == 256)
+    s = bf ? (cap ? launch_fwd8<256, true, true>(tq, tk, tv, p, st) : launch_fwd8<256, true, false>(tq, tk, tv, p, st))
+           : (cap ? launch_fwd8<256, false, true>(tq, tk, tv, p, st) : launch_fwd8<256, false, false>(tq, tk, tv, p, st));
+  else
+    s = bf ? (cap ? launch_fwd8<128, true, true>(tq, tk, tv, p, st) : launch_fwd8<128, true, false>(tq, tk, tv, p, st))
+           : (cap ? launch_fwd8<128, false, true>(tq, tk, tv, p, st) : launch_fwd8<128, false, false>(tq, tk, tv, p, st));
+  if (s != FA_OK) return s;
+  return ok();
+}
+
+fa_status fa_selftest_poly(int which, const float* x, float* out_poly, float* out_ref, int n,
+                           void* stream) {
+  if (which < 0 || which > 2) return fail(FA_ERR_INVALID_ARG, "fa_selftest_poly: which must be 0, 1 or 2");
+  if (n < 0 || (n > 0 && (!x || !out_poly || !out_ref)))
+    return fail(FA_ERR_INVALID_ARG, "fa_selftest_poly: bad arguments");
+  fa_status s = check_device();
+  if (s != FA_OK) return s;
+  if (n == 0) return ok();
+  const int pairs = (n + 1) / 2;
+  fa::poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      which, x, out_poly, out_ref, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "selftest launch failed: %s", cudaGetErrorString(e));
+  return ok();
 }
 
 fa_status fa_fwd_qkvpacked(const void* qkv, void* out, float* lse, int B, int H, int S, int D,

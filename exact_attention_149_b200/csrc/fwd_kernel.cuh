@@ -52,21 +52,38 @@ struct FwdParams {
   const int* cu_seqlens;     // nullable
   const float* alibi;        // ALiBi slopes, nullable: slope of (b, h) = alibi[b * alibi_bstride + h]
   int alibi_bstride;
+  float o_scale;             // FP8 inputs: the output's factor (v descale); unused otherwise
 };
 
 // D = 256: one Q tile per CTA (S 128 + O 256 TMEM columns; two tiles would
 // need 768) and one softmax warpgroup; Q (64 KB) and a two-slot K/V ring
 // (64 KB a tile) fill shared memory.
-template <int kD>
+//
+// kF8: Q, K, V are FP8 E4M3 (one byte per element; the guide's §版本怎么选
+// names an FP8 forward). A 128-byte swizzle row then holds 128 elements, a
+// QK^T K-step is 32 elements (still 32 bytes), a PV K-step 32 keys, and P
+// goes to the tensor core as E4M3, four per TMEM column. P is formed as
+// 2^(x - m + kPOff) with the row's running max m moved whenever the true max
+// exceeds it by more than kLazy, so the largest P of a row lies in
+// [2^kPOff, 2^(kPOff + kLazy)] = [16, 256]: inside E4M3's range (448), with
+// its 3-bit relative precision down to 2^-10 of the row's largest value.
+template <int kD, bool kF8 = false>
 struct FwdShape {
+  static constexpr int kElem = kF8 ? 1 : 2;          // bytes per Q/K/V element
   static constexpr int kBM = 128;                    // rows per Q tile
   static constexpr int kBN = 128;                    // keys per KV tile
   static constexpr int kQT = kD == 256 ? 1 : 2;      // Q tiles per CTA
   static constexpr int kRows = kQT * kBM;            // query rows per CTA
-  static constexpr int kChunks = kD / 64;            // 128-byte column chunks
+  static constexpr int kChunkElems = 128 / kElem;    // elements per 128-byte row
+  static constexpr int kChunks = kD / kChunkElems;   // 128-byte column chunks
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStages = kD == 256 ? 2 : (kD == 128 ? 4 : 8);  // K/V ring slots
+  static constexpr int kStages = kTileBytes >= 65536 ? 2 : (kTileBytes >= 32768 ? 4 : 8);  // K/V ring slots
+  static constexpr int kQKSteps = kD * kElem / 32;   // K-steps of QK^T (32 bytes each)
+  static constexpr int kPVKeys = 32 / kElem;         // keys per K-step of PV
+  static constexpr int kPVStepBytes = kPVKeys * 128; // V rows of one PV K-step
+  static constexpr float kLazy = kF8 ? 4.f : 8.f;    // max growth (log2) before a rescale
+  static constexpr float kPOff = kF8 ? 4.f : 0.f;    // P = 2^(x - m + kPOff)
   static constexpr int kBarOffset = (kQT + kStages) * kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;  // + barriers + align slack
@@ -77,10 +94,13 @@ struct FwdShape {
   // of every 8 pairs of exponentials, this many run as a cubic on the FMA
   // pipe instead of the special-function unit (which bounds the softmax)
   static constexpr int kPolyOf8 = 2;
+  // with softcap, whose tanh already loads the FMA pipe
+  static constexpr int kPolyOf8Cap = 1;
   // P_t is stored and signalled in this many parts, so that PV starts on
   // the first part while the rest of the row is exponentiated
   static constexpr int kPParts = 4;
   static constexpr int kPKeys = 128 / kPParts;
+  static constexpr int kPCols = kPKeys * kElem / 4;  // TMEM columns of one part of P
   static constexpr int kColS = 0;      // + 128 * t
   static constexpr int kColP = 64;     // + 128 * t
   static constexpr int kColO = 128 * kQT;  // + kD * t
@@ -104,6 +124,10 @@ struct FwdBars {
   // measured to move the forward's time by about 3 %; this order is the
   // fastest of those measured.
   uint64_t p_ready_hi[2][2];
+  // [t][0, 1]: the K/V tiles (indices into the CTA's n_tiles) Q tile t
+  // takes part in, [first, end): a tile that the mask hides from all of its
+  // rows is skipped
+  int tile_range[2][2];
 };
 
 __device__ __forceinline__ uint64_t* p_ready_bar(FwdBars* b, int t, int h) {
@@ -166,11 +190,12 @@ __device__ __forceinline__ float reduce128(const float (&x)[128]) {
 
 // kAlibi: the ALiBi bias is compiled in only where it is used, so the
 // common instantiations keep their register allocation
-template <int kD, bool kBF16, bool kCap, bool kAlibi>
-__global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
+// kBF16 is the output type (and, without kF8, the input type)
+template <int kD, bool kBF16, bool kCap, bool kAlibi, bool kF8 = false>
+__global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Sh = FwdShape<kD>;
+  using Sh = FwdShape<kD, kF8>;
   static_assert(sizeof(FwdBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -226,6 +251,23 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
     bars->abort = 0;
     const int item[8] = {seq_start, seq_len, q0, h, b, kvh, n_begin, n_tiles};
     for (int i = 0; i < 8; ++i) bars->item[i] = item[i];
+    // per Q tile: the sub-range of the CTA's K/V tiles its rows can see
+    for (int t = 0; t < Sh::kQT; ++t) {
+      const int r0 = q0 + t * Sh::kBM;
+      int first = 0, end = 0;
+      if (r0 < seq_len && n_tiles > 0) {
+        const int r1 = min(r0 + Sh::kBM - 1, seq_len - 1);
+        int hi = seq_len - 1;
+        if (p.wr >= 0) hi = min(hi, r1 + p.wr);
+        const int lo = p.wl >= 0 ? max(0, r0 - p.wl) : 0;
+        if (hi >= lo) {
+          first = lo / Sh::kBN - n_begin;
+          end = hi / Sh::kBN + 1 - n_begin;
+        }
+      }
+      bars->tile_range[t][0] = first;
+      bars->tile_range[t][1] = end;
+    }
     fence_mbar_init();
   }
   }
@@ -256,8 +298,8 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
       mbar_arrive_expect_tx(&bars->q_full, Sh::kQT * Sh::kTileBytes);
       for (int t = 0; t < Sh::kQT; ++t)
         for (int c = 0; c < Sh::kChunks; ++c)
-          tma_load_3d(&tm_q, &bars->q_full, sQ + t * Sh::kTileBytes + c * Sh::kChunkBytes, c * 64,
-                      h, seq_start + q0 + t * 128);
+          tma_load_3d(&tm_q, &bars->q_full, sQ + t * Sh::kTileBytes + c * Sh::kChunkBytes,
+                      c * Sh::kChunkElems, h, seq_start + q0 + t * 128);
       int fill = 0;
       for (int j = 0; j < n_tiles && !*abort; ++j) {
         const int tok = seq_start + (n_begin + j) * Sh::kBN;
@@ -269,7 +311,8 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
           uint8_t* dst = sKV + slot * Sh::kTileBytes;
           const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
           for (int c = 0; c < Sh::kChunks; ++c)
-            tma_load_3d(tm, &bars->kv_full[slot], dst + c * Sh::kChunkBytes, c * 64, kvh, tok);
+            tma_load_3d(tm, &bars->kv_full[slot], dst + c * Sh::kChunkBytes, c * Sh::kChunkElems,
+                        kvh, tok);
         }
       }
       // drain: every issued load must land before the CTA may exit
@@ -285,8 +328,10 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
     if (elect_one()) {
       const int n_tiles = load_item(bars).n_tiles;
       const uint32_t tmem = *static_cast<volatile uint32_t*>(&bars->tmem_base);
-      constexpr uint32_t id_qk = idesc_f16(kBF16, 128, 128, false, false);
-      constexpr uint32_t id_pv = idesc_f16(kBF16, 128, kD, false, true);
+      constexpr uint32_t id_qk = kF8 ? idesc_e4m3(128, 128, false, false)
+                                     : idesc_f16(kBF16, 128, 128, false, false);
+      constexpr uint32_t id_pv = kF8 ? idesc_e4m3(128, kD, false, true)
+                                     : idesc_f16(kBF16, 128, kD, false, true);
       // descriptors are built once; a tile or K-step offset is added to the
       // start-address field (bits 0..13, in 16-byte units; every address
       // stays below 256 KB, so the addition never carries out of the field)
@@ -295,26 +340,33 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
       const uint64_t dv_base = sdesc_sw128(smem_u32(sKV), Sh::kChunkBytes, 1024);
       bool ok = fwd_wait(&bars->q_full, 0, abort);
       tc_fence_after();
+      int t_first[2], t_end[2];
+      for (int t = 0; t < Sh::kQT; ++t) {
+        t_first[t] = static_cast<volatile int*>(bars->tile_range[t])[0];
+        t_end[t] = static_cast<volatile int*>(bars->tile_range[t])[1];
+      }
+      auto in_range = [&](int t, int j) { return j >= t_first[t] && j < t_end[t]; };
       auto issue_qk = [&](int t, int slot) {
         const uint64_t a0 = dq_base + static_cast<uint64_t>((t * Sh::kTileBytes) >> 4);
         const uint64_t b0 = dk_base + static_cast<uint64_t>((slot * Sh::kTileBytes) >> 4);
         const uint32_t d = tmem + Sh::kColS + 128 * t;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < Sh::kQKSteps; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32) >> 4);
-          umma_ss(d, a0 + off, b0 + off, id_qk, kk > 0 ? 1u : 0u);
+          umma_ss_k<kF8>(d, a0 + off, b0 + off, id_qk, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t V over the keys of part hf (K-steps of 16 keys)
+      // O_t += P_t V over the keys of part hf (K-steps of kPVKeys keys, each
+      // 8 TMEM columns of P)
       auto issue_pv = [&](int t, int slot, int hf, bool first) {
-        constexpr int kSteps = Sh::kPKeys / 16;
+        constexpr int kSteps = Sh::kPKeys / Sh::kPVKeys;
         const uint64_t b0 = dv_base + static_cast<uint64_t>((slot * Sh::kTileBytes) >> 4);
         const uint32_t d = tmem + Sh::kColO + kD * t;
         const uint32_t a = tmem + Sh::kColS + 128 * t + Sh::kColP;
 #pragma unroll
         for (int kk = kSteps * hf; kk < kSteps * (hf + 1); ++kk)
-          umma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), id_pv,
-                  (first && kk == 0) ? 0u : 1u);
+          umma_ts_k<kF8>(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * Sh::kPVStepBytes) >> 4),
+                         id_pv, (first && kk == 0) ? 0u : 1u);
       };
       // every part of PV_t, each as soon as its part of P is in TMEM
       auto wait_issue_pv = [&](int t, int slot, uint32_t ph, bool first) {
@@ -333,21 +385,31 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
         tc_fence_after();
         if (it > 0) {
           const int fvp = fv - 2, svp = fvp % Sh::kStages;
-          // per Q tile: PV_t of the previous K/V tile, then QK_t of this one;
-          // the previous V slot is free after the last tile's PV
-          const uint32_t ph = static_cast<uint32_t>(it - 1) & 1u;
+          // per Q tile: PV_t of the previous K/V tile, then QK_t of this one
+          // (each only inside the tile's range; a tile's output is final
+          // after its last PV); the previous V slot is free after the last
+          // tile's PV
+          const int j = it - 1;
           for (int t = 0; t < Sh::kQT && ok; ++t) {
-            if (!(ok = wait_issue_pv(t, svp, ph, it == 1))) break;
+            if (in_range(t, j)) {
+              const uint32_t ph = static_cast<uint32_t>(j - t_first[t]) & 1u;
+              if (!(ok = wait_issue_pv(t, svp, ph, j == t_first[t]))) break;
+              if (j == t_end[t] - 1) umma_commit(&bars->o_final[t]);
+            }
             if (t == Sh::kQT - 1) umma_commit(&bars->kv_empty[svp]);
-            issue_qk(t, sk);
-            umma_commit(&bars->s_full[t]);
+            if (in_range(t, it)) {
+              issue_qk(t, sk);
+              umma_commit(&bars->s_full[t]);
+            }
           }
           if (!ok) break;
           umma_commit(&bars->kv_empty[sk]);
         } else {
           for (int t = 0; t < Sh::kQT; ++t) {
-            issue_qk(t, sk);
-            umma_commit(&bars->s_full[t]);
+            if (in_range(t, 0)) {
+              issue_qk(t, sk);
+              umma_commit(&bars->s_full[t]);
+            }
           }
           umma_commit(&bars->kv_empty[sk]);
         }
@@ -357,10 +419,12 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
           break;
       }
       if (ok && n_tiles > 0) {
-        const int fvl = 2 * (n_tiles - 1) + 1, svl = fvl % Sh::kStages;
+        const int j = n_tiles - 1;
+        const int fvl = 2 * j + 1, svl = fvl % Sh::kStages;
         for (int t = 0; t < Sh::kQT && ok; ++t) {
-          if (!(ok = wait_issue_pv(t, svl, static_cast<uint32_t>(n_tiles - 1) & 1u, n_tiles == 1)))
-            break;
+          if (!in_range(t, j)) continue;
+          const uint32_t ph = static_cast<uint32_t>(j - t_first[t]) & 1u;
+          if (!(ok = wait_issue_pv(t, svl, ph, j == t_first[t]))) break;
           umma_commit(&bars->o_final[t]);
         }
         umma_commit(&bars->kv_empty[svl]);
@@ -376,9 +440,11 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
     const FwdItem w = load_item(bars);
     const uint32_t tmem = *static_cast<volatile uint32_t*>(&bars->tmem_base);
     const int seq_start = w.seq_start, seq_len = w.seq_len, q0 = w.q0, h = w.h, b = w.b;
-    const int n_begin = w.n_begin, n_tiles = w.n_tiles;
+    const int n_begin = w.n_begin;
     // ======================= softmax groups =======================
     const int t = (warp - 4) >> 2;            // Q tile of this group
+    const int it_first = static_cast<volatile int*>(bars->tile_range[t])[0];
+    const int it_end = static_cast<volatile int*>(bars->tile_range[t])[1];
     const int lane_base = 32 * (warp & 3);    // TMEM lanes this warp may touch
     const int row = lane_base + lane;         // row within the Q tile
     const int qrow = q0 + t * 128 + row;      // row within the sequence
@@ -394,8 +460,8 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
     constexpr bool alibi = kAlibi;
     const float sl2 = alibi ? p.alibi[static_cast<size_t>(b) * p.alibi_bstride + h] * 1.4426950408889634f : 0.f;
     bool ok = true;
-    for (int it = 0; it < n_tiles; ++it) {
-      if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it) & 1u, abort))) break;
+    for (int it = it_first; it < it_end; ++it) {
+      if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it - it_first) & 1u, abort))) break;
       tc_fence_after();
       // ---- the row of S_t: 128 raw scores ----
       float x[128];
@@ -415,18 +481,28 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
       if constexpr (kCap) {
         // logits in the exp2 domain: softcap * tanh(scale * s / softcap) * log2(e).
         // When every |scale * s / softcap| of the warp's rows is small, tanh
-        // is the FMA-pipe polynomial (two values per instruction); otherwise
-        // the exp-based identity.
+        // is an FMA-pipe polynomial with the scale and softcap folded into
+        // its coefficients (two values per instruction; degree 2 below 1/4,
+        // degree 4 below 1/2); otherwise the exp-based identity.
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < 128; i += 2) amax = max3(amax, fabsf(x[i]), fabsf(x[i + 1]));
-        if (__all_sync(0xffffffffu, amax * fabsf(p.cap_in) <= kTanhPolyMax)) {
-          const float2 ci = make_float2(p.cap_in, p.cap_in);
-          const float2 co = make_float2(p.cap_out_log2, p.cap_out_log2);
+        const float ya = amax * fabsf(p.cap_in);
+        if (__all_sync(0xffffffffu, ya <= kTanhPolyMaxLo)) {
+          float pk[3];
+          fold_tanh(kTanhLo, p.cap_in, p.cap_out_log2, pk);
 #pragma unroll
           for (int i = 0; i < 128; i += 2) {
-            const float2 t = tanh_poly2(__fmul2_rn(make_float2(x[i], x[i + 1]), ci));
-            const float2 v = __fmul2_rn(t, co);
+            const float2 v = tanh_fold2(make_float2(x[i], x[i + 1]), pk);
+            x[i] = v.x;
+            x[i + 1] = v.y;
+          }
+        } else if (__all_sync(0xffffffffu, ya <= kTanhPolyMax)) {
+          float pk[5];
+          fold_tanh(kTanhHi, p.cap_in, p.cap_out_log2, pk);
+#pragma unroll
+          for (int i = 0; i < 128; i += 2) {
+            const float2 v = tanh_fold2(make_float2(x[i], x[i + 1]), pk);
             x[i] = v.x;
             x[i + 1] = v.y;
           }
@@ -437,9 +513,27 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
       }
       if constexpr (alibi) {
         // ALiBi: -slope * |query - key| added to the logit, in the exp2
-        // domain (after softcap); x then holds exp2-domain logits
+        // domain (after softcap); x then holds exp2-domain logits. When every
+        // key of the tile lies on one side of every row of the warp (always,
+        // for the visible keys of a causal tile), the bias is affine in the
+        // key index i, c + d * i, and costs one packed FMA per pair; a tile
+        // that straddles the warp's rows takes the absolute value per key.
         const float dq = static_cast<float>(qrow - k0);
-        if constexpr (kCap) {
+        const bool left = p.wr == 0 || k0 + 127 <= r_lo;  // keys at or before the rows
+        const bool right = k0 >= r_hi;                     // keys at or after the rows
+        if (__all_sync(0xffffffffu, left || right)) {
+          const float c = left ? -sl2 * dq : sl2 * dq;
+          const float d = left ? sl2 : -sl2;
+          const float2 c2 = make_float2(c, c), d2 = make_float2(d, d);
+          const float2 sc2 = make_float2(kCap ? 1.f : p.scale_log2, kCap ? 1.f : p.scale_log2);
+#pragma unroll
+          for (int i = 0; i < 128; i += 2) {
+            const float2 bias = __ffma2_rn(make_float2(static_cast<float>(i), static_cast<float>(i + 1)), d2, c2);
+            const float2 v = __ffma2_rn(make_float2(x[i], x[i + 1]), sc2, bias);
+            x[i] = v.x;
+            x[i + 1] = v.y;
+          }
+        } else if constexpr (kCap) {
 #pragma unroll
           for (int i = 0; i < 128; ++i) x[i] = fmaf(-sl2, fabsf(dq - static_cast<float>(i)), x[i]);
         } else {
@@ -469,12 +563,12 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
         if (mt != mt) mt = -INFINITY;
       }
       const float m_new = fmaxf(m_run, mt);
-      const bool grow = m_new > m_run + 8.0f;
+      const bool grow = m_new > m_run + Sh::kLazy;
       if (__any_sync(0xffffffffu, grow)) {
         const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_run - m_new);
         if (m_new != -INFINITY) m_run = m_new;
         l_run *= alpha;
-        if (it > 0) {
+        if (it > it_first) {
           // O_t holds the previous PV results (complete: s_full commit
           // follows them); rescale it in place
 #pragma unroll 1
@@ -488,7 +582,7 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
           }
         }
       }
-      const float base = (m_run == -INFINITY) ? 0.f : m_run;
+      const float base = (m_run == -INFINITY) ? 0.f : m_run - Sh::kPOff;
       // P = 2^(x - base): one packed FMA (or add) per pair, then the
       // exponentials, 64 at a time, all issued before any of their results is
       // used so that they pipeline through the special-function unit
@@ -511,7 +605,7 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
         float* xh = x + Sh::kPKeys * hf;
 #pragma unroll
         for (int i = 0; i < Sh::kPKeys; i += 2) {
-          if (((i >> 1) & 7) < Sh::kPolyOf8) {
+          if (((i >> 1) & 7) < (kCap ? Sh::kPolyOf8Cap : Sh::kPolyOf8)) {
             const float2 e = ex2_poly2(make_float2(xh[i], xh[i + 1]));
             xh[i] = e.x;
             xh[i + 1] = e.y;
@@ -520,16 +614,28 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
             xh[i + 1] = ex2_approx(xh[i + 1]);
           }
         }
-        uint32_t r[Sh::kPKeys / 2];
+        uint32_t r[Sh::kPCols];
+        if constexpr (kF8) {
 #pragma unroll
-        for (int i = 0; i < Sh::kPKeys / 2; ++i) {
-          r[i] = pack2_alu<kBF16>(xh[2 * i], xh[2 * i + 1]);
-          sum2[i & 3] = __fadd2_rn(sum2[i & 3], make_float2(xh[2 * i], xh[2 * i + 1]));
+          for (int i = 0; i < Sh::kPCols; ++i) {
+            r[i] = pack4_e4m3(xh[4 * i], xh[4 * i + 1], xh[4 * i + 2], xh[4 * i + 3]);
+            sum2[(2 * i) & 3] = __fadd2_rn(sum2[(2 * i) & 3], make_float2(xh[4 * i], xh[4 * i + 1]));
+            sum2[(2 * i + 1) & 3] =
+                __fadd2_rn(sum2[(2 * i + 1) & 3], make_float2(xh[4 * i + 2], xh[4 * i + 3]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < Sh::kPCols; ++i) {
+            r[i] = pack2_alu<kBF16>(xh[2 * i], xh[2 * i + 1]);
+            sum2[i & 3] = __fadd2_rn(sum2[i & 3], make_float2(xh[2 * i], xh[2 * i + 1]));
+          }
         }
-        if constexpr (Sh::kPKeys == 64)
+        if constexpr (Sh::kPCols == 32)
           tmem_st32(t_p + hf * 32, r);
-        else
+        else if constexpr (Sh::kPCols == 16)
           tmem_st16(t_p + hf * 16, r);
+        else
+          tmem_st8(t_p + hf * 8, r);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -540,17 +646,18 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
       l_run += s4.x + s4.y;
     }
     // ---- epilogue: O / l and LSE ----
-    if (ok && n_tiles > 0) ok = fwd_wait(&bars->o_final[t], 0, abort);
+    const bool any = it_end > it_first;
+    if (ok && any) ok = fwd_wait(&bars->o_final[t], 0, abort);
     tc_fence_after();
     const bool valid_row = qrow < seq_len;
-    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+    const float inv_l = l_run > 0.f ? (kF8 ? p.o_scale : 1.f) / l_run : 0.f;
     typedef uint4 Vec;
     uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
                     (static_cast<size_t>(seq_start + qrow) * p.Hq + h) * kD * 2;
 #pragma unroll 1
     for (int c = 0; c < kD / 32; ++c) {
       uint32_t r[32];
-      if (ok && n_tiles > 0) {
+      if (ok && any) {
         tmem_ld32(t_o + c * 32, r);
         tmem_ld_wait();
       } else {
@@ -568,7 +675,8 @@ __global__ void __launch_bounds__(FwdShape<kD>::kThreads, 1)
       }
     }
     if (valid_row) {
-      const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      const float lse =
+          l_run > 0.f ? (m_run - Sh::kPOff + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       const size_t li = p.cu_seqlens != nullptr
                             ? static_cast<size_t>(h) * p.total + seq_start + qrow
                             : (static_cast<size_t>(b) * p.Hq + h) * p.S + qrow;

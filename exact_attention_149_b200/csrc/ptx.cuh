@@ -218,6 +218,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -269,6 +276,37 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       : "memory");
 }
 
+// kind::f8f6f4 forms of the two above (both operands 8-bit, here E4M3; the
+// instruction descriptor names the formats)
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <bool kF8>
+__device__ __forceinline__ void umma_ss_k(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  if constexpr (kF8) umma_ss_f8(d, a, b, id, acc); else umma_ss(d, a, b, id, acc);
+}
+template <bool kF8>
+__device__ __forceinline__ void umma_ts_k(uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  if constexpr (kF8) umma_ts_f8(d, a, b, id, acc); else umma_ts(d, a, b, id, acc);
+}
+
 // Arrive once on *bar when every tcgen05 async op issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -295,6 +333,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
   return d;
+}
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0
+// in both fields) and fp32 accumulation; the other fields as idesc_f16.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16 with fp32 accumulation.
@@ -366,6 +411,38 @@ __device__ __forceinline__ float2 tanh_poly2(float2 y) {
   return __fmul2_rn(y, q);
 }
 
+// c * tanh(a * x) for a pair of values, as x * P(x^2) with the fitted
+// coefficients q_k of tanh(y) = y Q(y^2) folded into P_k = c a^(2k+1) q_k
+// (fold_tanh), so that the scale, the softcap division and multiplication
+// and the tanh together cost one multiply and kN FMAs per pair.
+// kTanhLo: degree 2 for |a x| <= kTanhPolyMaxLo (Remez, fit_polynomials.py;
+// float64 relative error 4.0e-7, float32 evaluation within 1.1e-7 absolute).
+// kTanhHi: the degree-4 coefficients of tanh_poly2, |a x| <= kTanhPolyMax.
+constexpr float kTanhPolyMaxLo = 0.25f;
+__device__ constexpr float kTanhLo[3] = {9.999996043e-01f, -3.332190823e-01f, 1.284161343e-01f};
+__device__ constexpr float kTanhHi[5] = {9.999999869e-01f, -3.333306939e-01f, 1.332477932e-01f,
+                                         -5.298607529e-02f, 1.713500663e-02f};
+
+template <int kN>
+__device__ __forceinline__ void fold_tanh(const float (&q)[kN], float a, float c, float (&pk)[kN]) {
+  float f = c * a;
+  const float a2 = a * a;
+#pragma unroll
+  for (int k = 0; k < kN; ++k) {
+    pk[k] = f * q[k];
+    f *= a2;
+  }
+}
+
+template <int kN>
+__device__ __forceinline__ float2 tanh_fold2(float2 x, const float (&pk)[kN]) {
+  const float2 u = __fmul2_rn(x, x);
+  float2 r = make_float2(pk[kN - 1], pk[kN - 1]);
+#pragma unroll
+  for (int k = kN - 2; k >= 0; --k) r = __ffma2_rn(r, u, make_float2(pk[k], pk[k]));
+  return __fmul2_rn(x, r);
+}
+
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   if constexpr (kBF16) {
@@ -394,6 +471,20 @@ __device__ __forceinline__ uint32_t pack2_alu(float lo, float hi) {
   } else {
     return pack2<false>(lo, hi);
   }
+}
+
+// Four non-negative floats -> four FP8 E4M3 bytes, x0 in the lowest byte
+// (round to nearest even, saturating at 448). The conversion instruction
+// takes two floats and writes its first source into the upper byte.
+__device__ __forceinline__ uint32_t pack4_e4m3(float x0, float x1, float x2, float x3) {
+  uint32_t lo, hi;
+  asm("{\n\t.reg .b16 t;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u16 %0, t;\n\t}" : "=r"(lo) : "f"(x1), "f"(x0));
+  asm("{\n\t.reg .b16 t;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u16 %0, t;\n\t}" : "=r"(hi) : "f"(x3), "f"(x2));
+  return lo | (hi << 16);
 }
 
 template <bool kBF16>

@@ -106,6 +106,33 @@ FA_API fa_status fa_fwd_qkvpacked(const void* qkv, void* out, float* lse, int B,
                                   int total_tokens, fa_dtype dtype, void* stream);
 
 /*
+ * FP8 forward ("FlashAttention 实战指南" §版本怎么选: FlashAttention-3 runs
+ * the forward pass in FP8; the page gives no format, and this one is the
+ * common reading): q, k, v are FP8 E4M3 codes (one byte each: sign, 4
+ * exponent bits with bias 7, 3 mantissa bits; exponent 0 subnormal; 0x7F and
+ * 0xFF NaN; largest finite 448) in the layouts of fa_fwd, and element x of
+ * q stands for value(x) * q_descale (likewise k, v). The result is fa_fwd's
+ * on those values: out = softmax(scale * Q K^T [softcap, bias, mask]) V in
+ * out_dtype (bf16 or fp16), lse float32 as in fa_fwd. Q K^T runs on the
+ * tensor cores in E4M3 with float32 accumulation (exact products); the
+ * probabilities are rounded to E4M3 for the P V product (relative error at
+ * most 2^-4 each, the largest of a row kept in [16, 256] so that none leaves
+ * the format's normal range above 2^-10 of it) and the row sums and LSE are
+ * taken from the unrounded values.
+ *   q_descale, k_descale, v_descale: finite and > 0.
+ * D must be 128 or 256 (FA_ERR_UNSUPPORTED otherwise). Every other option
+ * (causal, window, softcap, ALiBi, GQA, varlen) as in fa_fwd.
+ * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for a descale that is not
+ *   finite and positive.
+ */
+FA_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int Hq, int Hkv, int S, int D, float scale, float q_descale,
+                            float k_descale, float v_descale, int causal, int window_left,
+                            int window_right, float softcap, const float* alibi_slopes,
+                            int alibi_batch_stride, const int32_t* cu_seqlens, int total_tokens,
+                            fa_dtype out_dtype, void* stream);
+
+/*
  * Workspace bytes needed by fa_bwd for these sizes: two float32 values per
  * token and query head (the row's dot(dO, O) and its LSE in the exp2
  * domain), each sequence's rows padded to a multiple of 128, i.e.
@@ -347,8 +374,8 @@ FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const 
  *   fa_kernel_timing_enable(1/0) switches recording on or off (host-wide).
  *   fa_kernel_timing_read(name, &total_ms, &launches) waits for the recorded
  *     events and returns the summed duration and count of the launches of
- *     the kernel `name` ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq", "kv_append",
- *     "decode_split", "lse_combine") since the last reset.
+ *     the kernel `name` ("fwd", "fwd_fp8", "bwd_pre", "bwd_dkdv", "bwd_dq", "kv_append",
+ *     "decode_split", "lse_combine", "fwd_fp8") since the last reset.
  *   fa_kernel_timing_reset() drops all records.
  * Errors: FA_ERR_INVALID_ARG for null arguments, FA_ERR_CUDA if an event
  * call fails.
@@ -356,6 +383,24 @@ FA_API fa_status fa_fwd_kvcache_noalloc(const void* q, const void* k_new, const 
 FA_API fa_status fa_kernel_timing_enable(int enable);
 FA_API fa_status fa_kernel_timing_read(const char* name, float* total_ms, int* launches);
 FA_API fa_status fa_kernel_timing_reset(void);
+
+/*
+ * Self-test of the approximations the kernels evaluate on the FMA pipe
+ * instead of the special-function unit (the pages have no counterpart; this
+ * exists so that their error can be checked against CUDA's own functions on
+ * the device): for the n DEVICE floats x, out_poly receives the library's
+ * approximation and out_ref the CUDA math function on the same input, with
+ *   which = 0: 2^x by the cubic of the forward's softmax (x >= -126;
+ *              relative error 7.5e-5), reference exp2f;
+ *   which = 1: tanh(x) by the degree-4 odd polynomial (|x| <= 0.5; absolute
+ *              error 4e-8), reference tanhf;
+ *   which = 2: tanh(x) by the degree-2 polynomial with folded scales
+ *              (|x| <= 0.25; absolute error 1.1e-7), reference tanhf.
+ * Asynchronous on `stream`. Errors: FA_ERR_INVALID_ARG for another `which`,
+ * n < 0 or null pointers with n > 0; FA_ERR_CUDA on launch failure.
+ */
+FA_API fa_status fa_selftest_poly(int which, const float* x, float* out_poly, float* out_ref, int n,
+                                  void* stream);
 
 /*
  * Reads and clears the library's device status word on the current device
