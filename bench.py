@@ -386,9 +386,16 @@ def run_ours(args, dist: Dist):
             fa.bwd(q, k, v, out, lse, do, scale=c.scale, causal=True, dq=dq, dk=dk, dv=dv,
                    workspace=ws, alibi_slopes=slopes)
 
-        ms_al = timed(step_alibi, args.steps, args.warmup, dist)
+        ms_al = timed(step_alibi, args.steps, args.warmup, dist, fa_mod=fa)
         res["alibi_fwd_bwd"] = {"ms": ms_al, "tflops": flop_step / (ms_al * 1e-3) / 1e12,
-                                "slopes": "2^(-8(h+1)/Hq)"}
+                                "slopes": "2^(-8(h+1)/Hq)", "kernels": {}}
+        for name in ("fwd", "bwd_dkdv", "bwd_dq"):
+            tot, n = fa.fa_kernel_timing_read(name)
+            if n:
+                res["alibi_fwd_bwd"]["kernels"][name] = {
+                    "ms_avg": tot / n,
+                    "vs_without_alibi": (tot / n) / kern[name]["ms_avg"] if name in kern else None}
+        fa.fa_kernel_timing_reset()
         res["alibi_fwd_bwd"]["frac_of_bf16_peak"] = res["alibi_fwd_bwd"]["tflops"] / peaks["bf16_tflops"]
 
     # -------------------- end to end through the public API --------------------

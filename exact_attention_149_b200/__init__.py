@@ -28,7 +28,7 @@ __all__ = [
     "fwd", "bwd", "fwd_kvcache", "fwd_qkvpacked", "bwd_qkvpacked", "fa_fwd_qkvpacked",
     "fa_bwd_qkvpacked", "fa_fwd_kvcache_int8", "fa_kv_quantize_int8", "kv_quantize_int8",
     "fa_fwd_kvcache_int4", "fa_kv_quantize_int4", "kv_quantize_int4",
-    "fa_fwd_fp8", "fwd_fp8", "fa_selftest_poly",
+    "fa_fwd_fp8", "fwd_fp8", "fa_selftest_poly", "fa_selftest_fwd_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -63,6 +63,8 @@ lib.fa_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _i, _
 lib.fa_fwd_fp8.restype = _i
 lib.fa_fwd_fp8.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _f, _f, _i, _i, _i, _f,
                            _p, _i, _p, _i, _i, _p]
+lib.fa_selftest_fwd_timeout.restype = _i
+lib.fa_selftest_fwd_timeout.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _f, ctypes.c_ulonglong, _i, _p]
 lib.fa_selftest_poly.restype = _i
 lib.fa_selftest_poly.argtypes = [_i, _p, _p, _p, _i, _p]
 lib.fa_bwd.restype = _i
@@ -172,6 +174,11 @@ def fa_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, S, D, scale, q_descale, k_descale,
                           q_descale, k_descale, v_descale, int(causal), window_left, window_right,
                           softcap, _ptr(alibi_slopes), alibi_batch_stride, _ptr(cu_seqlens),
                           total_tokens, out_dtype, _stream(stream)))
+
+
+def fa_selftest_fwd_timeout(q, k, v, out, lse, B, H, S, scale, wait_limit_ns, dtype, stream=None):
+    _check(lib.fa_selftest_fwd_timeout(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S,
+                                       scale, wait_limit_ns, dtype, _stream(stream)))
 
 
 def fa_selftest_poly(which, x, out_poly, out_ref, n, stream=None):

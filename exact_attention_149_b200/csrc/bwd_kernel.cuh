@@ -103,7 +103,16 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
   const uint16_t* o = static_cast<const uint16_t*>(p.o) + gw * kD + lane * kPer;
   const uint16_t* d = static_cast<const uint16_t*>(p.dout) + gw * kD + lane * kPer;
   float acc = 0.f;
-  if constexpr (kPer == 4) {
+  if constexpr (kPer == 8) {
+    const uint4 ov = *reinterpret_cast<const uint4*>(o);
+    const uint4 dv = *reinterpret_cast<const uint4*>(d);
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 o2 = unpack2<kBF16>(ow[i]), d2 = unpack2<kBF16>(dw[i]);
+      acc = fmaf(o2.x, d2.x, fmaf(o2.y, d2.y, acc));
+    }
+  } else if constexpr (kPer == 4) {
     const uint2 ov = *reinterpret_cast<const uint2*>(o);
     const uint2 dv = *reinterpret_cast<const uint2*>(d);
     const float2 o0 = unpack2<kBF16>(ov.x), o1 = unpack2<kBF16>(ov.y);
@@ -192,6 +201,31 @@ __device__ __forceinline__ bool poly_ok(const uint32_t (&sr)[32], float cap_in) 
   return __all_sync(0xffffffffu, amax * fabsf(cap_in) <= kTanhPolyMax);
 }
 
+// ALiBi for 32 entries: w[i] -= sl2 * |d0 + sgn * i| (sl2: slope in the exp2
+// domain). When the sign of d0 + sgn * i is the same for all 32 entries in
+// every lane of the warp (`one_side`: always, for the visible pairs of a
+// causal mask), |.| is affine in i and one packed FMA per pair adds it.
+__device__ __forceinline__ void alibi32(float (&w)[32], float sl2, float d0, float sgn,
+                                        bool one_side) {
+  const float last = d0 + sgn * 31.f;
+  const bool pos = d0 >= 0.f && last >= 0.f, neg = d0 <= 0.f && last <= 0.f;
+  if (__all_sync(0xffffffffu, one_side || pos || neg)) {
+    // one_side: the visible pairs have d0 + sgn i >= 0 (masked ones are zeroed later)
+    const float s = (one_side || pos) ? -sl2 : sl2;
+    const float2 c2 = make_float2(s * d0, s * d0), d2 = make_float2(s * sgn, s * sgn);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float2 b = __ffma2_rn(make_float2(static_cast<float>(i), static_cast<float>(i + 1)), d2, c2);
+      const float2 v = __fadd2_rn(make_float2(w[i], w[i + 1]), b);
+      w[i] = v.x;
+      w[i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = fmaf(-sl2, fabsf(d0 + sgn * static_cast<float>(i)), w[i]);
+  }
+}
+
 // P (or P * (1 - tanh^2) under softcap) of 32 raw scores sharing one -LSE
 // (nl2, in the exp2 domain): all exponentials are issued before any result
 // is consumed, so they pipeline through the special-function unit. With
@@ -199,7 +233,8 @@ __device__ __forceinline__ bool poly_ok(const uint32_t (&sr)[32], float cap_in) 
 // the exp2 domain, d0: query position minus the first key's).
 template <bool kCap>
 __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, const BwdParams& p,
-                                            bool alibi, float sl2, float d0, float (&w)[32]) {
+                                            bool alibi, float sl2, float d0, float (&w)[32],
+                                            bool causal_side) {
   const bool poly = kCap ? poly_ok(sr, p.cap_in) : false;
 #pragma unroll
   for (int j2 = 0; j2 < 16; ++j2) {
@@ -213,10 +248,7 @@ __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, cons
       sr[2 * j2 + 1] = __float_as_uint(fac.y);
     }
   }
-  if (alibi) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) w[i] = fmaf(-sl2, fabsf(d0 - static_cast<float>(i)), w[i]);
-  }
+  if (alibi) alibi32(w, sl2, d0, -1.f, causal_side);
 #pragma unroll
   for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
   if constexpr (kCap) {
@@ -228,33 +260,48 @@ __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, cons
 // ===========================================================================
 // dK, dV
 // ===========================================================================
-template <int kD>
+// kPass: which gradients one launch computes. D <= 128: both (kDkdvBoth),
+// their accumulators side by side in TMEM. D = 256: dV and dK alone take all
+// 512 TMEM columns ("FlashAttention 实战指南" §版本怎么选 allows head dims up
+// to 256), so the host runs a dV pass (S^T, P^T, dV += P^T dO; K resident, no
+// V) and then a dK pass (S^T, dP^T, dS^T, dK += dS^T Q; P stays in
+// registers). Each pass recomputes S^T; the two cost 10 D per pair against 8 D
+// for the fused kernel. At D = 256 an item is 32 query rows (one compute
+// group per team), so that K and V (64 KB each) and three Q/dO slots fit in
+// shared memory.
+enum : int { kDkdvBoth = 0, kDvOnly = 1, kDkOnly = 2 };
+
+template <int kD, int kPass = kDkdvBoth>
 struct DkdvShape {
+  static_assert((kPass == kDkdvBoth) == (kD <= 128), "D <= 128 fuses dK and dV; D = 256 splits them");
   static constexpr int kChunks = kD / 64;
   static constexpr int kChunkBytes = 128 * 128;        // K/V: 128 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kQRows = 64;                    // query rows per item
+  static constexpr int kQRows = kD == 256 ? 32 : 64;   // query rows per item
+  static constexpr int kGroups = kQRows / 32;          // compute groups per team
   static constexpr int kQChunkBytes = kQRows * 128;
   static constexpr int kQTileBytes = kChunks * kQChunkBytes;
-  static constexpr int kSlots = 4;                     // Q/dO ring
+  static constexpr bool kNeedV = kPass != kDvOnly;
+  static constexpr int kSlots = kD == 256 ? (kNeedV ? 3 : 5) : 4;  // Q/dO ring
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;         // + slot * 2 * kQTileBytes (Q, dO)
-  // per slot: -LSE (exp2 domain)[64], Drow[64] of the slot's query rows
+  static constexpr int kOffQ = (kNeedV ? 2 : 1) * kTileBytes;  // + slot * 2 * kQTileBytes (Q, dO)
+  // per slot: -LSE (exp2 domain)[kQRows], Drow[kQRows] of the slot's query rows
   static constexpr int kOffVec = kOffQ + kSlots * 2 * kQTileBytes;
-  static constexpr int kVecBytes = 512;
+  static constexpr int kVecBytes = 2 * kQRows * 4;
   static constexpr int kOffBar = kOffVec + kSlots * kVecBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
-  // warp 0 TMA, warp 1 MMA, then two teams of two compute groups (4 warps
-  // each); team t takes the items it with it % 2 == t, group g of a team the
-  // 32 query columns [32g, 32g + 32) of the item
-  static constexpr int kThreads = 64 + 4 * 128;
+  // warp 0 TMA, warp 1 MMA, then two teams of kGroups compute groups (4
+  // warps each); team t takes the items it with it % 2 == t, group g of a
+  // team the 32 query columns [32g, 32g + 32) of the item
+  static constexpr int kThreads = 64 + 2 * kGroups * 128;
   static constexpr int kTmemCols = 512;
-  static constexpr int kColA = 0;    // + 64 t: team t's S^T, then P^T
-  static constexpr int kColB = 128;  // + 64 t: team t's dP^T, then dS^T
-  static constexpr int kColDV = 256;
-  static constexpr int kColDK = 256 + kD;
+  static constexpr int kColA = 0;             // + kQRows t: team t's S^T, then P^T
+  static constexpr int kColB = 2 * kQRows;    // + kQRows t: team t's dP^T, then dS^T
+  static constexpr int kColDV = kPass == kDkdvBoth ? 256 : 256;
+  static constexpr int kColDK = kPass == kDkdvBoth ? 256 + kD : 256;
+  static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB a CTA may use");
 };
 
 struct DkdvBars {
@@ -271,12 +318,14 @@ struct DkdvBars {
   int abort;
 };
 
-template <int kD, bool kBF16, bool kCap, bool kAlibi>
-__global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
+template <int kD, bool kBF16, bool kCap, bool kAlibi, int kPass = kDkdvBoth>
+__global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
-  using Sh = DkdvShape<kD>;
+  using Sh = DkdvShape<kD, kPass>;
+  constexpr bool kDoDV = kPass != kDkOnly;  // this launch accumulates dV
+  constexpr bool kDoDK = kPass != kDvOnly;  // and dK
   static_assert(sizeof(DkdvBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -320,8 +369,8 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_ready[t], 1);
       mbar_init(&bars->dp_ready[t], 1);
-      mbar_init(&bars->p_ready[t], 8);
-      mbar_init(&bars->ds_ready[t], 8);
+      mbar_init(&bars->p_ready[t], 4 * Sh::kGroups);
+      mbar_init(&bars->ds_ready[t], 4 * Sh::kGroups);
     }
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
@@ -345,12 +394,13 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * Sh::kTileBytes);
+      mbar_arrive_expect_tx(&bars->kv_full, (Sh::kNeedV ? 2 : 1) * Sh::kTileBytes);
       for (int c = 0; c < Sh::kChunks; ++c) {
         tma_load_3d(&tm_k, &bars->kv_full, smem + Sh::kOffK + c * Sh::kChunkBytes, c * 64, kvh,
                     seq_start + k0);
-        tma_load_3d(&tm_v, &bars->kv_full, smem + Sh::kOffV + c * Sh::kChunkBytes, c * 64, kvh,
-                    seq_start + k0);
+        if constexpr (Sh::kNeedV)
+          tma_load_3d(&tm_v, &bars->kv_full, smem + Sh::kOffV + c * Sh::kChunkBytes, c * 64, kvh,
+                      seq_start + k0);
       }
       int it = 0;
       for (; it < n_items && !*abort; ++it) {
@@ -416,7 +466,7 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       };
       auto issue_s = [&](int it) {  // S^T = K Q^T -> region A of the item's team
         const uint32_t sQ = q_addr(it);
-        const uint32_t d = tmem + Sh::kColA + 64 * (it & 1);
+        const uint32_t d = tmem + Sh::kColA + Sh::kQRows * (it & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           umma_ss(d, kmajor_kv(sK, kk), kmajor_q(sQ, kk), id_s, kk > 0 ? 1u : 0u);
@@ -424,7 +474,7 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       };
       auto issue_dp = [&](int it) {  // dP^T = V dO^T -> region B of the item's team
         const uint32_t sDO = q_addr(it) + Sh::kQTileBytes;
-        const uint32_t d = tmem + Sh::kColB + 64 * (it & 1);
+        const uint32_t d = tmem + Sh::kColB + Sh::kQRows * (it & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           umma_ss(d, kmajor_kv(sV, kk), kmajor_q(sDO, kk), id_s, kk > 0 ? 1u : 0u);
@@ -433,7 +483,7 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       for (int it = 0; it < 2 && it < n_items && ok; ++it) {
         if ((ok = wait_q(it))) {
           issue_s(it);
-          issue_dp(it);
+          if constexpr (kDoDK) issue_dp(it);
         }
       }
       for (int it = 0; it < n_items && ok; ++it) {
@@ -442,28 +492,36 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
         const uint32_t sQ = q_addr(it);
         const uint32_t sDO = sQ + Sh::kQTileBytes;
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
-        // dV += P^T dO: A = P^T of the team's region (queries [32c, 32c+32)
-        // packed into columns [32c, 32c+16), 16 queries = 8 columns per step)
+        // the team's P pass of item it: P^T in region A (dV's operand), or,
+        // in the dK pass, S^T read out of region A into registers
         if (!(ok = bwd_wait(&bars->p_ready[t], ph, abort))) break;
         tc_fence_after();
+        if constexpr (kDoDV) {
+          // dV += P^T dO: A = P^T of the team's region (queries [32c, 32c+32)
+          // packed into columns [32c, 32c+16), 16 queries = 8 columns per step)
 #pragma unroll
-        for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
-          umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + 64 * t + (kk >> 1) * 32 + (kk & 1) * 8,
-                  mnmajor_q(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
+          for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
+            umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + Sh::kQRows * t + (kk >> 1) * 32 + (kk & 1) * 8,
+                    mnmajor_q(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
+        }
         const bool more = it + 2 < n_items;
         if (more) {
           if (!(ok = wait_q(it + 2))) break;
           issue_s(it + 2);
         }
-        // dK += dS^T Q: A = dS^T of the team's region B, packed like P^T
-        if (!(ok = bwd_wait(&bars->ds_ready[t], ph, abort))) break;
-        tc_fence_after();
+        if constexpr (kDoDK) {
+          // dK += dS^T Q: A = dS^T of the team's region B, packed like P^T
+          if (!(ok = bwd_wait(&bars->ds_ready[t], ph, abort))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
-          umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + 64 * t + (kk >> 1) * 32 + (kk & 1) * 8,
-                  mnmajor_q(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
+          for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
+            umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + Sh::kQRows * t + (kk >> 1) * 32 + (kk & 1) * 8,
+                    mnmajor_q(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
+        }
         umma_commit(&bars->qd_empty[it % Sh::kSlots]);
-        if (more) issue_dp(it + 2);
+        if constexpr (kDoDK) {
+          if (more) issue_dp(it + 2);
+        }
       }
       umma_commit(&bars->final_done);
       umma_commit(&bars->drain);
@@ -472,8 +530,8 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     __syncwarp();
   } else {
     // ======================= compute teams =======================
-    const int team = (warp - 2) >> 3;
-    const int g = ((warp - 2) >> 2) & 1;       // group within the team
+    const int team = (warp - 2) / (4 * Sh::kGroups);
+    const int g = ((warp - 2) >> 2) % Sh::kGroups;  // group within the team
     const int lane_base = 32 * (warp & 3);
     const int r = lane_base + lane;             // key row within the tile
     const int key = k0 + r;
@@ -481,8 +539,8 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     // this group's 32 query columns of the team's S^T / dP^T, and the 16
     // columns its P^T / dS^T (16-bit pairs) overwrite: only columns it has
     // read itself
-    const uint32_t t_a = tmem + lane_off + Sh::kColA + 64 * team + 32 * g;
-    const uint32_t t_b = tmem + lane_off + Sh::kColB + 64 * team + 32 * g;
+    const uint32_t t_a = tmem + lane_off + Sh::kColA + Sh::kQRows * team + 32 * g;
+    const uint32_t t_b = tmem + lane_off + Sh::kColB + Sh::kQRows * team + 32 * g;
     constexpr bool alibi = kAlibi;  // compiled in only where used
     bool ok = true;
     for (int it = team; it < n_items; it += 2) {
@@ -537,11 +595,8 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
             sr[2 * j2 + 1] = __float_as_uint(fac.y);
           }
         }
-        if constexpr (alibi) {  // -slope * |query - key| in the exp2 domain
-          const float d0 = static_cast<float>(qg_lo - key);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = fmaf(-sl2, fabsf(d0 + static_cast<float>(i)), w[i]);
-        }
+        if constexpr (alibi)  // -slope * |query - key| in the exp2 domain
+          alibi32(w, sl2, static_cast<float>(qg_lo - key), 1.f, p.wr == 0);
 #pragma unroll
         for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
         if (need_mask) {
@@ -554,10 +609,12 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
             w[i] = v ? w[i] : 0.f;
           }
         }
-        uint32_t pk[16];
+        if constexpr (kDoDV) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int j2 = 0; j2 < 16; ++j2) pk[j2] = pack2_alu<kBF16>(w[2 * j2], w[2 * j2 + 1]);
-        tmem_st16(t_a, pk);
+          for (int j2 = 0; j2 < 16; ++j2) pk[j2] = pack2_alu<kBF16>(w[2 * j2], w[2 * j2 + 1]);
+          tmem_st16(t_a, pk);
+        }
         if constexpr (kCap) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) w[i] *= __uint_as_float(sr[i]);
@@ -566,7 +623,8 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_ready[team]);  // dV may start
+      if (lane == 0) mbar_arrive(&bars->p_ready[team]);  // dV may start (or S may be overwritten)
+      if constexpr (!kDoDK) continue;
       // pass 2: dS^T = w * (dP^T - Drow) -> TMEM region B (the dK operand),
       // once dP^T is in TMEM (dK two items back, the last reader of these
       // columns, precedes the dP^T MMA in issue order)
@@ -610,13 +668,15 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
     // rows (warps 2-9) and of the dK rows (warps 10-17) ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
+    // (both: warps 2-9 write dV, 10-17 dK, each group half of a row; one
+    // accumulator: each of the 2 kGroups groups its share of the row)
     const int e = (warp - 2) >> 2;
-    const bool is_dk = e >= 2;
+    const bool is_dk = kPass == kDkdvBoth ? e >= 2 : kPass == kDkOnly;
     void* outp = is_dk ? p.dk : p.dv;
     const uint32_t col = is_dk ? Sh::kColDK : Sh::kColDV;
     const float osc = is_dk ? p.scale : 1.f;  // dK = scale * dS^T Q
-    constexpr int kHalfChunks = kD / 64;      // 32-column chunks per half row
-    const int c_begin = (e & 1) * kHalfChunks;
+    constexpr int kHalfChunks = kPass == kDkdvBoth ? kD / 64 : kD / 32 / (2 * Sh::kGroups);
+    const int c_begin = (kPass == kDkdvBoth ? (e & 1) : e) * kHalfChunks;
     uint8_t* dst = static_cast<uint8_t*>(outp) +
                    (static_cast<size_t>(seq_start + key) * p.dkv_tok + static_cast<size_t>(kvh) * kD) * 2;
     if (ok && n_items > 0) {
@@ -670,30 +730,40 @@ __global__ void __launch_bounds__(DkdvShape<kD>::kThreads, 1)
 // MMA order per item j (team t): dQ_j (after the dS pass of j), S_{j+2} -> S_t,
 // dP_{j+2} -> dP_t. While one team computes, the tensor core runs the other
 // team's products; the order is fixed, so dQ is deterministic.
+//
+// D = 256: Q (128 columns) and dQ (256) fill TMEM with S and dP, so dO stays
+// in shared memory (loaded once by TMA, the A operand of dP = dO V^T), an
+// item is 32 keys and each team has one compute group.
 template <int kD>
 struct DqShape {
   static constexpr int kChunks = kD / 64;
-  static constexpr int kKRows = 64;                    // keys per item
-  static constexpr int kChunkBytes = kKRows * 128;     // 64 rows x 128 B
+  static constexpr int kKRows = kD == 256 ? 32 : 64;   // keys per item
+  static constexpr int kGroups = kKRows / 32;          // compute groups per team
+  static constexpr bool kDOSmem = kD == 256;           // dO in shared memory
+  static constexpr int kChunkBytes = kKRows * 128;     // kKRows rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   // K/V ring slots (one tile each): six items in flight hide the L2 -> shared
   // latency of the next blocks behind about 1.3k cycles per item
-  static constexpr int kStages = kD == 128 ? 12 : 24;
+  static constexpr int kStages = kD == 256 ? 8 : (kD == 128 ? 12 : 24);
   static constexpr int kOffKV = 0;
-  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffDO = kOffKV + kStages * kTileBytes;     // D = 256: dO, 128 rows
+  static constexpr int kDOBytes = kDOSmem ? kChunks * 128 * 128 : 0;
+  static constexpr int kOffBar = kOffDO + kDOBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
-  static constexpr int kThreads = 64 + 4 * 128;
+  static constexpr int kThreads = 64 + 2 * kGroups * 128;
   static constexpr int kTmemCols = 512;
   static constexpr int kColQ = 0;
-  static constexpr int kColDO = kD / 2;
-  static constexpr int kColS = 128;    // + 64 t
-  static constexpr int kColDP = 256;   // + 64 t
-  static constexpr int kColDQ = 384;
+  static constexpr int kColDO = kD / 2;                // (D <= 128)
+  static constexpr int kColS = 128;                    // + kKRows t
+  static constexpr int kColDP = kDOSmem ? 128 + 2 * kKRows : 256;  // + kKRows t
+  static constexpr int kColDQ = kDOSmem ? 256 : 384;
+  static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB a CTA may use");
 };
 
 struct DqBars {
-  uint64_t qd_tmem;      // Q and dO written to TMEM (8 warps)
+  uint64_t qd_tmem;      // Q (and dO, D <= 128) written to TMEM (4 kGroups warps)
+  uint64_t do_full;      // D = 256: the dO tile in shared memory
   uint64_t kv_full[24];
   uint64_t kv_empty[24];
   uint64_t s_ready[2];
@@ -708,7 +778,7 @@ struct DqBars {
 template <int kD, bool kBF16, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
   using Sh = DqShape<kD>;
   static_assert(sizeof(DqBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
@@ -745,7 +815,8 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
   const int n_tiles = key_hi >= key_lo ? key_hi / Sh::kKRows + 1 - n_begin : 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->qd_tmem, 8);
+    mbar_init(&bars->qd_tmem, 4 * Sh::kGroups);
+    mbar_init(&bars->do_full, 1);
     for (int i = 0; i < Sh::kStages; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
@@ -753,7 +824,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_ready[t], 1);
       mbar_init(&bars->dp_ready[t], 1);
-      mbar_init(&bars->ds_ready[t], 8);
+      mbar_init(&bars->ds_ready[t], 4 * Sh::kGroups);
     }
     mbar_init(&bars->final_done, 1);
     mbar_init(&bars->drain, 1);
@@ -775,6 +846,12 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     if (elect_one()) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      if constexpr (Sh::kDOSmem) {
+        mbar_arrive_expect_tx(&bars->do_full, Sh::kDOBytes);
+        for (int c = 0; c < Sh::kChunks; ++c)
+          tma_load_3d(&tm_do, &bars->do_full, smem + Sh::kOffDO + c * 128 * 128, c * 64, h,
+                      seq_start + q0);
+      }
       int fill = 0;
       for (int j = 0; j < n_tiles && !*abort; ++j) {
         const int tok = seq_start + (n_begin + j) * Sh::kKRows;
@@ -791,6 +868,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       }
       for (int f = max(0, fill - Sh::kStages); f < fill; ++f)
         mbar_wait(&bars->kv_full[f % Sh::kStages], static_cast<uint32_t>(f / Sh::kStages) & 1u);
+      if constexpr (Sh::kDOSmem) mbar_wait(&bars->do_full, 0);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -799,7 +877,9 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       constexpr uint32_t id_s = idesc_f16(kBF16, 128, Sh::kKRows, false, false);  // S, dP
       constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, false, true);          // dS (tmem) x K
       const uint32_t sKV = smem_u32(smem + Sh::kOffKV);
+      const uint32_t sDO = smem_u32(smem + Sh::kOffDO);
       bool ok = bwd_wait(&bars->qd_tmem, 0, abort);
+      if (ok && Sh::kDOSmem) ok = bwd_wait(&bars->do_full, 0, abort);
       tc_fence_after();
       auto kmajor = [](uint32_t base, int kk) {
         return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
@@ -813,7 +893,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       auto slot_addr = [&](int fill) { return sKV + (fill % Sh::kStages) * Sh::kTileBytes; };
       auto issue_s = [&](int j) {  // S_j = Q K_j^T -> S_{j%2}
         const uint32_t sK = slot_addr(2 * j);
-        const uint32_t d = tmem + Sh::kColS + 64 * (j & 1);
+        const uint32_t d = tmem + Sh::kColS + Sh::kKRows * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           umma_ts(d, tmem + Sh::kColQ + 8 * kk, kmajor(sK, kk), id_s, kk > 0 ? 1u : 0u);
@@ -821,10 +901,15 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       };
       auto issue_dp = [&](int j) {  // dP_j = dO V_j^T -> dP_{j%2}
         const uint32_t sV = slot_addr(2 * j + 1);
-        const uint32_t d = tmem + Sh::kColDP + 64 * (j & 1);
+        const uint32_t d = tmem + Sh::kColDP + Sh::kKRows * (j & 1);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ts(d, tmem + Sh::kColDO + 8 * kk, kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          if constexpr (Sh::kDOSmem)  // A = the dO tile, K-major, 128-row chunks
+            umma_ss(d, sdesc_sw128(sDO + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                    kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+          else
+            umma_ts(d, tmem + Sh::kColDO + 8 * kk, kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+        }
         umma_commit(&bars->dp_ready[j & 1]);
       };
       for (int j = 0; j < 2 && j < n_tiles && ok; ++j) {
@@ -841,7 +926,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         // columns [32c, 32c+16)), B = K_j with N = D (MN-major)
         {
           const uint32_t sK = slot_addr(2 * j);
-          const uint32_t a = tmem + Sh::kColS + 64 * t;
+          const uint32_t a = tmem + Sh::kColS + Sh::kKRows * t;
 #pragma unroll
           for (int kk = 0; kk < Sh::kKRows / 16; ++kk)
             umma_ts(tmem + Sh::kColDQ, a + (kk >> 1) * 32 + (kk & 1) * 8,
@@ -866,13 +951,13 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     __syncwarp();
   } else {
     // ======================= compute teams =======================
-    const int team = (warp - 2) >> 3;
-    const int g = ((warp - 2) >> 2) & 1;     // group within the team
+    const int team = (warp - 2) / (4 * Sh::kGroups);
+    const int g = ((warp - 2) >> 2) % Sh::kGroups;  // group within the team
     const int lane_base = 32 * (warp & 3);
     const int r = lane_base + lane;          // query row within the tile
     const int qrow = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
-    if (team == 0) {
+    if (team == 0) {  // (D = 256: group 0 only, Q; dO arrives by TMA)
       // Q (group 0) or dO (group 1) row -> TMEM, two 16-bit values per column
       // (the A-operand layout: K-step kk of 16 values at columns 8kk..8kk+7);
       // rows past the sequence end are zero
@@ -917,8 +1002,8 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort))) break;
       tc_fence_after();
       const int k0 = (n_begin + j) * Sh::kKRows + 32 * g;  // first key of this group's columns
-      const uint32_t t_s = tmem + lane_off + Sh::kColS + 64 * team + 32 * g;
-      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 64 * team + 32 * g;
+      const uint32_t t_s = tmem + lane_off + Sh::kColS + Sh::kKRows * team + 32 * g;
+      const uint32_t t_dp = tmem + lane_off + Sh::kColDP + Sh::kKRows * team + 32 * g;
       // mask needed for this warp's 32 rows x the group's 32 keys?
       const int r_lo = q0 + lane_base, r_hi = r_lo + 31;
       bool need_mask = (k0 + 31 >= seq_len) || (r_hi >= seq_len);
@@ -931,7 +1016,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         uint32_t sr[32];
         tmem_ld32(t_s, sr);
         tmem_ld_wait();
-        bwd_probs32<kCap>(sr, nl2, p, alibi, sl2, static_cast<float>(qrow - k0), w);
+        bwd_probs32<kCap>(sr, nl2, p, alibi, sl2, static_cast<float>(qrow - k0), w, p.wr == 0);
         if (need_mask) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -966,29 +1051,32 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_ready[team]);
     }
-    // ---- epilogue: dQ row -> dq; warps 2-5, 6-9, 10-13, 14-17 write the
-    // 32-column chunks 0..3 (D = 64: the first two) ----
+    // ---- epilogue: dQ row -> dq; the 2 kGroups warp groups write the
+    // 32-column chunks e * kPer .. (e + 1) * kPer - 1 of their rows (D = 64:
+    // groups 2, 3 have none) ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
     tc_fence_after();
     const int e = (warp - 2) >> 2;
+    constexpr int kPer = (kD / 32 + 2 * Sh::kGroups - 1) / (2 * Sh::kGroups);
     uint8_t* dst = static_cast<uint8_t*>(p.dq) +
                    (static_cast<size_t>(seq_start + qrow) * p.dq_tok + static_cast<size_t>(h) * kD) * 2;
-    if (e < kD / 32) {
+#pragma unroll 1
+    for (int c = e * kPer; c < (e + 1) * kPer && c < kD / 32; ++c) {
       if (ok && n_tiles > 0) {
         uint32_t rr[32];
-        tmem_ld32(tmem + lane_off + Sh::kColDQ + e * 32, rr);
+        tmem_ld32(tmem + lane_off + Sh::kColDQ + c * 32, rr);
         tmem_ld_wait();
         uint32_t wv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]) * p.scale, __uint_as_float(rr[2 * i + 1]) * p.scale);
         if (qrow < seq_len) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + e * 64);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
 #pragma unroll
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
         }
       } else if (ok && qrow < seq_len) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + e * 64);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
         for (int i = 0; i < 4; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
       }
     }

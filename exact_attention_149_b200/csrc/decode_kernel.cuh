@@ -309,6 +309,16 @@ __device__ __forceinline__ uint32_t i4pair_to_f16(uint32_t w) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// The same for the codes in bits 4-7 and 20-23, left in place: 0x64 above
+// them is 1024 + 16 (code + 8), and subtracting 1152 leaves 16 * code (exact;
+// the caller undoes the factor 16 elsewhere, saving the shift).
+__device__ __forceinline__ uint32_t i4pair_hi_to_f16x16(uint32_t w) {
+  const uint32_t h = (w & 0x00F000F0u) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h),
+                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // 16 int8 codes -> 16 exact 16-bit values (two uint4 of 8), without the
 // special-function unit. bf16: each biased byte (code + 128) becomes the low
 // mantissa byte of 2^23, so the fp32 value is 2^23 + code + 128; subtracting
@@ -421,7 +431,9 @@ struct DecShape {
   static constexpr int kStageBytes = kQuant ? (kLoadBytes + 1023) / 1024 * 1024 : kLoadBytes;
   // 2 (16-bit) or 3 CTAs per SM; int4 keeps 8 stages so that the cross-warp
   // reduction scratch, which aliases the ring, fits
-  static constexpr int kStages = kQuant ? (kQ == 4 ? 8 : (kD == 128 ? 4 : 6)) : (kD == 128 ? 3 : 6);
+  // (16-bit D = 256: 64 KB stages, three of them, one CTA per SM)
+  static constexpr int kStages =
+      kQuant ? (kQ == 4 ? 8 : (kD == 128 ? 4 : 6)) : (kD == 256 ? 3 : (kD == 128 ? 3 : 6));
   // int8 with D = 128 builds the tensor-core fragments straight from the
   // swizzled int8 tiles in registers; D = 64 converts through a scratch
   static constexpr bool kDirect = kQuant && kD == 128;
@@ -611,10 +623,12 @@ __global__ void __launch_bounds__(160)
         if constexpr (kQ4) {
           // int4: K-step kk pairs nibbles (i, i + 4) and (i + 1, i + 5) of
           // word kk / 2, i = 2 (kk % 2): d = 32j + 8 (kk / 2) + i + {0, 4}
-          // and + {1, 5}
+          // and + {1, 5}. The K values of the second pair arrive as 16 x
+          // code (i4pair_hi_to_f16x16), so their queries carry 1 / 16.
           const int i0 = 8 * (kk >> 1) + 2 * (kk & 1);
+          const float down16 = down * 0.0625f;
           qf[nt][kk][0] = pack2<false>(v[i0] * down, v[i0 + 4] * down);
-          qf[nt][kk][1] = pack2<false>(v[i0 + 1] * down, v[i0 + 5] * down);
+          qf[nt][kk][1] = pack2<false>(v[i0 + 1] * down16, v[i0 + 5] * down16);
         } else {
           qf[nt][kk][0] = pack2<false>(v[4 * kk] * down, v[4 * kk + 1] * down);
           qf[nt][kk][1] = pack2<false>(v[4 * kk + 2] * down, v[4 * kk + 3] * down);
@@ -810,9 +824,11 @@ __global__ void __launch_bounds__(160)
       // word kk / 2, i = 2 (kk % 2) (the permutation of the query fragments)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
+        // (a2, a3: 16 x code, matched by the queries' 1 / 16)
         const int sh = 8 * (kk & 1);
-        const uint32_t a0 = i4pair_to_f16(kw[0][kk >> 1] >> sh), a2 = i4pair_to_f16(kw[0][kk >> 1] >> (sh + 4));
-        const uint32_t a1 = i4pair_to_f16(kw[1][kk >> 1] >> sh), a3 = i4pair_to_f16(kw[1][kk >> 1] >> (sh + 4));
+        const uint32_t w0 = kw[0][kk >> 1] >> sh, w1 = kw[1][kk >> 1] >> sh;
+        const uint32_t a0 = i4pair_to_f16(w0), a2 = i4pair_hi_to_f16x16(w0);
+        const uint32_t a1 = i4pair_to_f16(w1), a3 = i4pair_hi_to_f16x16(w1);
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) mma16816<false>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
       }
@@ -950,8 +966,9 @@ __global__ void __launch_bounds__(160)
         const uint32_t sel = bsel | ((bsel + 4) << 8);
         const uint32_t x = __byte_perm(vw[0][mt >> 2], vw[1][mt >> 2], sel);
         const uint32_t y = __byte_perm(vw[2][mt >> 2], vw[3][mt >> 2], sel);
-        const uint32_t a0 = i4pair_to_f16(x), a1 = i4pair_to_f16(x >> 4);
-        const uint32_t a2 = i4pair_to_f16(y), a3 = i4pair_to_f16(y >> 4);
+        // rows r + 8 (odd d) as 16 x code: the epilogue divides them by 16
+        const uint32_t a0 = i4pair_to_f16(x), a1 = i4pair_hi_to_f16x16(x);
+        const uint32_t a2 = i4pair_to_f16(y), a3 = i4pair_hi_to_f16x16(y);
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) mma16816<false>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
       }
@@ -1027,6 +1044,7 @@ __global__ void __launch_bounds__(160)
       red_l[warp * kH + h0 + 1] = l1;
     }
     const float oc = kQuant ? vC : 1.f;  // int8 / int4: acc holds O / vC
+    const float oc1 = kQ4 ? oc * 0.0625f : oc;  // int4: rows d1 hold 16 O / vC
 #pragma unroll
     for (int mt = 0; mt < kD / 16; ++mt) {
       // accumulator rows lane / 4 and lane / 4 + 8 of step mt
@@ -1034,8 +1052,8 @@ __global__ void __launch_bounds__(160)
       const int d1 = Sh::kDirect ? d0 + 1 : d0 + 8;
       red_o[(warp * kH + h0) * kD + d0] = acc[nt][mt][0] * oc;
       red_o[(warp * kH + h0 + 1) * kD + d0] = acc[nt][mt][1] * oc;
-      red_o[(warp * kH + h0) * kD + d1] = acc[nt][mt][2] * oc;
-      red_o[(warp * kH + h0 + 1) * kD + d1] = acc[nt][mt][3] * oc;
+      red_o[(warp * kH + h0) * kD + d1] = acc[nt][mt][2] * oc1;
+      red_o[(warp * kH + h0 + 1) * kD + d1] = acc[nt][mt][3] * oc1;
     }
   }
   named_bar_sync(1, 128);

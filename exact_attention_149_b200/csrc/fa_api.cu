@@ -210,14 +210,14 @@ fa_status check_alibi(const float* slopes, int batch_stride, int Hq) {
   return FA_OK;
 }
 
-// fwd256: the forward also takes D = 256 (one Q tile per CTA)
+// allow256: the call also takes D = 256 (forward and backward)
 fa_status check_common(int B, int Hq, int Hkv, int S, int D, float scale, int wl, int wr,
-                       float softcap, fa_dtype dt, const int32_t* cu, int total, bool fwd256 = false) {
+                       float softcap, fa_dtype dt, const int32_t* cu, int total, bool allow256 = false) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1)
     return fail(FA_ERR_INVALID_ARG, "B, Hq, Hkv and S must be >= 1 (got %d, %d, %d, %d)", B, Hq, Hkv, S);
   if (Hq % Hkv != 0) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be an integer multiple of Hkv (%d)", Hq, Hkv);
-  if (D != 64 && D != 128 && !(fwd256 && D == 256))
-    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128%s)", D, fwd256 ? ", or 256 forward" : "");
+  if (D != 64 && D != 128 && !(allow256 && D == 256))
+    return fail(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128%s)", D, allow256 ? " or 256" : "");
   if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
   if (wl < -1 || wr < -1) return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (got %d, %d)", wl, wr);
   if (!(softcap >= 0.f) || !std::isfinite(softcap))
@@ -357,6 +357,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, long long q_tok,
   p.cu_seqlens = cu_seqlens;
   p.alibi = alibi_slopes;
   p.alibi_bstride = alibi_batch_stride;
+  p.wait_ns = fa::kWaitTimeoutNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool cap = softcap > 0.f;
   if (D == 256) {
@@ -497,6 +498,7 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
   p.alibi = alibi_slopes;
   p.alibi_bstride = alibi_batch_stride;
   p.o_scale = v_descale;
+  p.wait_ns = fa::kWaitTimeoutNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool cap = softcap > 0.f;
   const bool bf = out_dtype == FA_BF16;
@@ -507,6 +509,48 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
     s = bf ? (cap ? launch_fwd8<128, true, true>(tq, tk, tv, p, st) : launch_fwd8<128, true, false>(tq, tk, tv, p, st))
            : (cap ? launch_fwd8<128, false, true>(tq, tk, tv, p, st) : launch_fwd8<128, false, false>(tq, tk, tv, p, st));
   if (s != FA_OK) return s;
+  return ok();
+}
+
+fa_status fa_selftest_fwd_timeout(const void* q, const void* k, const void* v, void* out, float* lse,
+                                  int B, int H, int S, float scale, unsigned long long wait_limit_ns,
+                                  fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_selftest_fwd_timeout: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_selftest_fwd_timeout: tensors must be 16-byte aligned");
+  if (wait_limit_ns < 1000000ull || wait_limit_ns > fa::kWaitTimeoutNs)
+    return fail(FA_ERR_INVALID_ARG, "fa_selftest_fwd_timeout: the wait limit must lie in [1 ms, 4 s]");
+  fa_status s = check_common(B, H, H, S, 128, scale, -1, -1, 0.f, dtype, nullptr, 0);
+  if (s != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+  const long long T = static_cast<long long>(B) * S;
+  CUtensorMap tq, tk, tv;
+  if ((s = make_map_thd(&tq, q, dtype, 128, H, T, 128)) != FA_OK) return s;
+  if ((s = make_map_thd(&tk, k, dtype, 128, H, T, 128)) != FA_OK) return s;
+  if ((s = make_map_thd(&tv, v, dtype, 128, H, T, 128)) != FA_OK) return s;
+  fa::FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.Hq = p.Hkv = H;
+  p.S = S;
+  p.total = static_cast<int>(T);
+  p.group = 1;
+  p.n_qblocks = (S + fa::FwdShape<128>::kRows - 1) / fa::FwdShape<128>::kRows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wl = p.wr = -1;
+  p.o = out;
+  p.lse = lse;
+  p.wait_ns = wait_limit_ns;
+  using Sh = fa::FwdShape<128>;
+  auto kern = dtype == FA_BF16 ? fa::fwd_kernel<128, true, false, false, false, true>
+                               : fa::fwd_kernel<128, false, false, false, false, true>;
+  if ((s = set_smem(kern, Sh::kSmemBytes)) != FA_OK) return s;
+  const long long grid = static_cast<long long>(p.n_qblocks) * B * H;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "grid too large");
+  kern<<<static_cast<unsigned>(grid), Sh::kThreads, Sh::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "selftest launch failed: %s", cudaGetErrorString(e));
   return ok();
 }
 

@@ -53,6 +53,7 @@ struct FwdParams {
   const float* alibi;        // ALiBi slopes, nullable: slope of (b, h) = alibi[b * alibi_bstride + h]
   int alibi_bstride;
   float o_scale;             // FP8 inputs: the output's factor (v descale); unused otherwise
+  unsigned long long wait_ns;  // limit of every bounded wait (4 s; shorter in the failure test)
 };
 
 // D = 256: one Q tile per CTA (S 128 + O 256 TMEM columns; two tiles would
@@ -143,14 +144,15 @@ __device__ __forceinline__ FwdItem load_item(const FwdBars* bars) {
   return FwdItem{v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]};
 }
 
-__device__ __forceinline__ bool fwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool fwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                         uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         atomicExch(&g_device_status, kDevTimeout);
         *abort = 1;
         return false;
@@ -190,8 +192,12 @@ __device__ __forceinline__ float reduce128(const float (&x)[128]) {
 
 // kAlibi: the ALiBi bias is compiled in only where it is used, so the
 // common instantiations keep their register allocation
-// kBF16 is the output type (and, without kF8, the input type)
-template <int kD, bool kBF16, bool kCap, bool kAlibi, bool kF8 = false>
+// kBF16 is the output type (and, without kF8, the input type).
+// kWithhold (only the failure-path test instantiates it): the producer never
+// issues the first K tile's load, so every wait on it runs out after
+// p.wait_ns and the CTA unwinds (FA_ERR_TIMEOUT in the status word) with no
+// copy or MMA left in flight.
+template <int kD, bool kBF16, bool kCap, bool kAlibi, bool kF8 = false, bool kWithhold = false>
 __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -306,7 +312,8 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % Sh::kStages;
           const uint32_t ph = static_cast<uint32_t>(fill / Sh::kStages) & 1u;
-          if (!fwd_wait(&bars->kv_empty[slot], ph ^ 1u, abort)) break;
+          if (!fwd_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.wait_ns)) break;
+          if (kWithhold && fill == 0) continue;  // neither the transaction count nor the copy
           mbar_arrive_expect_tx(&bars->kv_full[slot], Sh::kTileBytes);
           uint8_t* dst = sKV + slot * Sh::kTileBytes;
           const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
@@ -318,9 +325,9 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       // drain: every issued load must land before the CTA may exit
       for (int f = max(0, fill - Sh::kStages); f < fill; ++f) {
         const int slot = f % Sh::kStages;
-        mbar_wait(&bars->kv_full[slot], static_cast<uint32_t>(f / Sh::kStages) & 1u);
+        mbar_wait(&bars->kv_full[slot], static_cast<uint32_t>(f / Sh::kStages) & 1u, p.wait_ns);
       }
-      mbar_wait(&bars->q_full, 0);
+      mbar_wait(&bars->q_full, 0, p.wait_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       const uint64_t dq_base = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dk_base = sdesc_sw128(smem_u32(sKV), 16, 1024);
       const uint64_t dv_base = sdesc_sw128(smem_u32(sKV), Sh::kChunkBytes, 1024);
-      bool ok = fwd_wait(&bars->q_full, 0, abort);
+      bool ok = fwd_wait(&bars->q_full, 0, abort, p.wait_ns);
       tc_fence_after();
       int t_first[2], t_end[2];
       for (int t = 0; t < Sh::kQT; ++t) {
@@ -371,7 +378,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       // every part of PV_t, each as soon as its part of P is in TMEM
       auto wait_issue_pv = [&](int t, int slot, uint32_t ph, bool first) {
         for (int hf = 0; hf < Sh::kPParts; ++hf) {
-          if (!fwd_wait(p_ready_bar(bars, t, hf), ph, abort)) return false;
+          if (!fwd_wait(p_ready_bar(bars, t, hf), ph, abort, p.wait_ns)) return false;
           tc_fence_after();
           issue_pv(t, slot, hf, first);
         }
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       for (int it = 0; it < n_tiles && ok; ++it) {
         const int fk = 2 * it, fv = 2 * it + 1;
         const int sk = fk % Sh::kStages;
-        if (!(ok = fwd_wait(&bars->kv_full[sk], static_cast<uint32_t>(fk / Sh::kStages) & 1u, abort)))
+        if (!(ok = fwd_wait(&bars->kv_full[sk], static_cast<uint32_t>(fk / Sh::kStages) & 1u, abort, p.wait_ns)))
           break;
         tc_fence_after();
         if (it > 0) {
@@ -415,7 +422,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
         }
         // V_it must be resident before next round's PV
         const int sv = fv % Sh::kStages;
-        if (!(ok = fwd_wait(&bars->kv_full[sv], static_cast<uint32_t>(fv / Sh::kStages) & 1u, abort)))
+        if (!(ok = fwd_wait(&bars->kv_full[sv], static_cast<uint32_t>(fv / Sh::kStages) & 1u, abort, p.wait_ns)))
           break;
       }
       if (ok && n_tiles > 0) {
@@ -431,7 +438,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       }
       // wait for everything this thread issued before TMEM is released
       umma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0);
+      mbar_wait(&bars->drain, 0, p.wait_ns);
     }
     __syncwarp();
   }
@@ -461,7 +468,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
     const float sl2 = alibi ? p.alibi[static_cast<size_t>(b) * p.alibi_bstride + h] * 1.4426950408889634f : 0.f;
     bool ok = true;
     for (int it = it_first; it < it_end; ++it) {
-      if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it - it_first) & 1u, abort))) break;
+      if (!(ok = fwd_wait(&bars->s_full[t], static_cast<uint32_t>(it - it_first) & 1u, abort, p.wait_ns))) break;
       tc_fence_after();
       // ---- the row of S_t: 128 raw scores ----
       float x[128];
@@ -647,7 +654,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
     }
     // ---- epilogue: O / l and LSE ----
     const bool any = it_end > it_first;
-    if (ok && any) ok = fwd_wait(&bars->o_final[t], 0, abort);
+    if (ok && any) ok = fwd_wait(&bars->o_final[t], 0, abort, p.wait_ns);
     tc_fence_after();
     const bool valid_row = qrow < seq_len;
     const float inv_l = l_run > 0.f ? (kF8 ? p.o_scale : 1.f) / l_run : 0.f;

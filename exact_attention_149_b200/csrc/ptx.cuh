@@ -92,12 +92,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Returns false (and
 // records kDevTimeout in the library's device status word) if it has not
 // completed within kWaitTimeoutNs; the caller then unwinds instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if ((it & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) {
       atomicExch(&g_device_status, kDevTimeout);
       return false;
     }

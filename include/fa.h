@@ -345,8 +345,11 @@ FA_API fa_status fa_kv_quantize_int4(const void* src, uint8_t* codes, float* sca
  * routine.
  *
  * - The first call on a device looks up the array's device address on that
- *   device (cudaGetSymbolAddress, with that device current) and caches it;
- *   make that first call outside any stream capture.
+ *   device (cudaGetSymbolAddress, with that device current) and caches it
+ *   with the device's current context; make that first call outside any
+ *   stream capture. After a cudaDeviceReset the context, and with it the
+ *   array's address, is new: the next call looks the address up again (so
+ *   it too belongs outside a capture).
  * - Every call on a device shares the one array and leaves its contents
  *   behind. Nothing in it needs to start at zero: each call writes every
  *   partial it later reads. Calls whose kernels overlap on the GPU (other
@@ -401,6 +404,24 @@ FA_API fa_status fa_kernel_timing_reset(void);
  */
 FA_API fa_status fa_selftest_poly(int which, const float* x, float* out_poly, float* out_ref, int n,
                                   void* stream);
+
+/*
+ * Self-test of the failure path (the pages have no counterpart): runs the
+ * forward kernel (non-causal, D = 128, Hq = Hkv = H, layouts of fa_fwd) in
+ * a test build of it whose producer never issues the first K tile's load,
+ * with every bounded wait limited to wait_limit_ns (1 ms .. 4 s; the
+ * library's own calls use 4 s). Each CTA's waits on that tile run out; the
+ * CTA then records FA_ERR_TIMEOUT in the device status word, lets the copies
+ * and tensor-core operations it did issue finish, releases its tensor memory
+ * and returns, so the context stays usable and fa_get_device_status reports
+ * FA_ERR_TIMEOUT. out and lse are not valid afterwards. Asynchronous on
+ * `stream`. Errors: FA_ERR_INVALID_ARG for null or misaligned pointers, bad
+ * sizes or a limit outside the range; FA_ERR_CUDA on launch failure.
+ */
+FA_API fa_status fa_selftest_fwd_timeout(const void* q, const void* k, const void* v, void* out,
+                                         float* lse, int B, int H, int S, float scale,
+                                         unsigned long long wait_limit_ns, fa_dtype dtype,
+                                         void* stream);
 
 /*
  * Reads and clears the library's device status word on the current device

@@ -43,6 +43,14 @@ SMALL = [
     (2, 512, 16, 16, 64, "fp16", True, (-1, -1), 0.0),    # B2 H16 S512 D64 fp16
     (1, 1, 2, 1, 128, "bf16", True, (-1, -1), 0.0),       # a single token
     (1, 1030, 4, 1, 128, "fp16", True, (-1, -1), 0.0),    # many Q tiles per key tile
+    # head dim 256: a dV pass and a dK pass of 32-row items, dQ with dO in
+    # shared memory and 32-key blocks
+    (1, 300, 2, 2, 256, "bf16", True, (-1, -1), 0.0),     # causal, ragged
+    (2, 513, 4, 2, 256, "fp16", False, (-1, -1), 0.0),    # GQA, non-causal, B > 1
+    (1, 640, 2, 1, 256, "bf16", True, (100, 0), 30.0),    # window + softcap, MQA
+    (1, 256, 4, 4, 256, "bf16", True, (-1, -1), 2.0),     # softcap that bites
+    (1, 1, 2, 2, 256, "bf16", True, (-1, -1), 0.0),       # a single token
+    (1, 700, 2, 2, 256, "fp16", False, (64, 32), 0.0),    # two-sided window
 ]
 
 
@@ -58,6 +66,8 @@ def test_bwd_small(cuda_ok, B, S, Hq, Hkv, D, dtype, causal, window, softcap):
 @pytest.mark.parametrize("lengths,Hq,Hkv,D,causal,window,softcap", [
     ([1, 130, 257, 600, 33], 8, 2, 128, True, (200, 0), 30.0),
     ([128, 5, 384, 1], 4, 4, 64, False, (-1, -1), 0.0),
+    ([200, 1, 333, 97], 4, 2, 256, True, (-1, -1), 0.0),
+    ([1, 130, 257, 600, 33], 4, 1, 256, True, (200, 0), 30.0),
 ])
 def test_bwd_varlen(cuda_ok, lengths, Hq, Hkv, D, causal, window, softcap):
     inp = W.make_varlen_inputs(lengths, Hq, Hkv, D, "bf16", seed=len(lengths) * 31 + D, with_do=True)
@@ -67,6 +77,14 @@ def test_bwd_varlen(cuda_ok, lengths, Hq, Hkv, D, causal, window, softcap):
     ref = attention_bwd(inp["q"], inp["k"], inp["v"], inp["do"], scale, causal, window, softcap,
                         cu_seqlens=inp["cu_seqlens"].numpy())
     check_bwd(got, ref, f"varlen {lengths}")
+
+
+def test_bwd_d256_is_deterministic(cuda_ok):
+    inp = W.make_fwd_inputs(1, 400, 4, 2, 256, "bf16", seed=19, with_do=True)
+    a = _gpu_fwd_bwd(inp, 0.06, True, (-1, -1), 0.0)
+    b = _gpu_fwd_bwd(inp, 0.06, True, (-1, -1), 0.0)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
 
 
 def test_bwd_is_deterministic(cuda_ok):

@@ -257,3 +257,26 @@ def test_decode_full_paged_b64(cuda_ok):
                                  c.dtype, seed=1000 + c.cid)
     for splits in c.splits:
         _run_case(st, splits, heads=[0, 13, 31], check_pool=(splits == 1))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,dtype,lengths,ps,rd,splits", [
+    (3, 8, 2, 1, "bf16", [5, 64, 700], 64, 0, 1),          # head dim 256, one column tile
+    (3, 8, 2, 1, "fp16", [0, 129, 1000], 128, 0, 4),
+    (2, 8, 1, 3, "bf16", [300, 77], 64, 128, 3),           # 24 columns: two tiles, two blocks
+    (2, 32, 8, 1, "bf16", [2047, 4096], 256, 256, 16),     # rotary over the whole head
+])
+def test_decode_head_dim_256(cuda_ok, B, Hq, Hkv, Sq, dtype, lengths, ps, rd, splits):
+    """Head dim 256 on a 16-bit cache (the guide's §版本怎么选: head dims up to
+    256): three 64 KB stages, at most two 8-column tiles per CTA."""
+    st = W.make_decode_structure(B, Hq, Hkv, 256, 0, max(lengths), ps, dtype,
+                                 seed=sum(lengths) + Sq + splits, cache_seqlens=lengths, sq=Sq)
+    _run_case(st, splits, rotary_dim=rd)
+
+
+def test_decode_head_dim_256_options(cuda_ok):
+    st = W.make_decode_structure(2, 8, 2, 256, 0, 500, 64, "bf16", seed=61,
+                                 cache_seqlens=[500, 33], sq=2)
+    nan = float("nan")
+    _run_case(st, 2, window=(100, 0), softcap=20.0, fill=(nan, nan))
+    _run_case(st, 1, causal=False, append=False)
+    _run_case(st, 3, contiguous_capacity=600)

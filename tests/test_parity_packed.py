@@ -22,6 +22,7 @@ fa = pytest.importorskip("exact_attention_149_b200")
     (2, 300, 4, 128, "bf16", True, (-1, -1), 0.0, False),
     (1, 513, 2, 64, "fp16", False, (64, 32), 0.0, False),
     (2, 200, 4, 128, "bf16", True, (-1, -1), 10.0, True),
+    (1, 300, 2, 256, "bf16", True, (-1, -1), 0.0, True),   # head dim 256
 ])
 def test_qkvpacked_matches_unpacked_and_oracle(cuda_ok, B, S, H, D, dtype, causal, window, softcap,
                                                alibi):
