@@ -93,41 +93,33 @@ __device__ __forceinline__ size_t vec_index(const BwdParams& p, int h, int b, in
 // ---------------------------------------------------------------------------
 template <int kD, bool kBF16>
 __global__ void bwd_pre_kernel(const BwdParams p) {
+  // kLanes lanes per (token, head) row, 16 bytes of O and of dO each: D = 128
+  // puts two rows in a warp, so every load is a 16-byte one
+  constexpr int kLanes = kD / 8;
+  constexpr int kRowsPerWarp = 32 / kLanes;
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(p.total) * p.Hq;
-  if (gw >= rows) return;
-  const int tok = static_cast<int>(gw / p.Hq);
-  const int h = static_cast<int>(gw % p.Hq);
-  constexpr int kPer = kD / 32;  // elements per lane
-  const uint16_t* o = static_cast<const uint16_t*>(p.o) + gw * kD + lane * kPer;
-  const uint16_t* d = static_cast<const uint16_t*>(p.dout) + gw * kD + lane * kPer;
+  if (gw * kRowsPerWarp >= rows) return;  // uniform across the warp
+  const long long row = gw * kRowsPerWarp + lane / kLanes;
+  const int li = lane % kLanes;
   float acc = 0.f;
-  if constexpr (kPer == 8) {
-    const uint4 ov = *reinterpret_cast<const uint4*>(o);
-    const uint4 dv = *reinterpret_cast<const uint4*>(d);
+  if (row < rows) {
+    const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + row * kD + li * 8);
+    const uint4 dv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + row * kD + li * 8);
     const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 o2 = unpack2<kBF16>(ow[i]), d2 = unpack2<kBF16>(dw[i]);
       acc = fmaf(o2.x, d2.x, fmaf(o2.y, d2.y, acc));
     }
-  } else if constexpr (kPer == 4) {
-    const uint2 ov = *reinterpret_cast<const uint2*>(o);
-    const uint2 dv = *reinterpret_cast<const uint2*>(d);
-    const float2 o0 = unpack2<kBF16>(ov.x), o1 = unpack2<kBF16>(ov.y);
-    const float2 d0 = unpack2<kBF16>(dv.x), d1 = unpack2<kBF16>(dv.y);
-    acc = o0.x * d0.x + o0.y * d0.y + o1.x * d1.x + o1.y * d1.y;
-  } else {
-    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o);
-    const uint32_t dv = *reinterpret_cast<const uint32_t*>(d);
-    const float2 o0 = unpack2<kBF16>(ov), d0 = unpack2<kBF16>(dv);
-    acc = o0.x * d0.x + o0.y * d0.y;
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    size_t li;
+  for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  const int tok = static_cast<int>(row / p.Hq);
+  const int h = static_cast<int>(row % p.Hq);
+  if (li == 0 && row < rows) {
+    size_t lidx;
     int b, seq_start;
     if (p.cu_seqlens != nullptr) {
       // the sequence holding tok: the largest b with cu_seqlens[b] <= tok
@@ -141,20 +133,23 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
       }
       b = lo;
       seq_start = p.cu_seqlens[b];
-      li = static_cast<size_t>(h) * p.total + tok;
+      lidx = static_cast<size_t>(h) * p.total + tok;
     } else {
       b = tok / p.S;
       seq_start = b * p.S;
-      li = (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
+      lidx = (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
     }
-    const float l = p.lse[li];
+    const float l = p.lse[lidx];
     const size_t vi = vec_index(p, h, b, seq_start, tok - seq_start);
     p.vec_nlse[vi] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
     p.vec_drow[vi] = acc;
   }
 }
 
-__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// site: 100 * kernel (1 dK/dV, 2 dV pass, 3 dK pass, 4 dQ) + wait, recorded
+// when this wait is the one that gives up
+__device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                         int site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -162,7 +157,7 @@ __device__ __forceinline__ bool bwd_wait(uint64_t* bar, uint32_t parity, volatil
     if ((it & 63u) == 0u) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-        atomicExch(&g_device_status, kDevTimeout);
+        record_timeout(site);
         *abort = 1;
         return false;
       }
@@ -302,12 +297,13 @@ struct DkdvShape {
   static constexpr int kColDV = kPass == kDkdvBoth ? 256 : 256;
   static constexpr int kColDK = kPass == kDkdvBoth ? 256 + kD : 256;
   static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB a CTA may use");
+  static_assert(kSlots <= 8, "more ring slots than the barrier block holds");
 };
 
 struct DkdvBars {
   uint64_t kv_full;
-  uint64_t qd_full[4];
-  uint64_t qd_empty[4];
+  uint64_t qd_full[8];   // one per ring slot (DkdvShape::kSlots <= 8)
+  uint64_t qd_empty[8];
   uint64_t s_ready[2];   // per team
   uint64_t dp_ready[2];
   uint64_t p_ready[2];
@@ -324,6 +320,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using Sh = DkdvShape<kD, kPass>;
+  constexpr int kSite = 100 * (1 + kPass);  // wait sites of this kernel (bwd_wait)
   constexpr bool kDoDV = kPass != kDkOnly;  // this launch accumulates dV
   constexpr bool kDoDK = kPass != kDvOnly;  // and dK
   static_assert(sizeof(DkdvBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
@@ -406,7 +403,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       for (; it < n_items && !*abort; ++it) {
         const int slot = it % Sh::kSlots;
         const uint32_t ph = static_cast<uint32_t>(it / Sh::kSlots) & 1u;
-        if (!bwd_wait(&bars->qd_empty[slot], ph ^ 1u, abort)) break;
+        if (!bwd_wait(&bars->qd_empty[slot], ph ^ 1u, abort, kSite + 1)) break;
         const int h = kvh * p.group + it / i_cnt;
         const int q0 = (i_begin + it % i_cnt) * Sh::kQRows;
         const int tok = seq_start + q0;
@@ -425,8 +422,8 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
         bulk_load(vdst + Sh::kVecBytes / 2, p.vec_drow + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
       }
       for (int f = max(0, it - Sh::kSlots); f < it; ++f)
-        mbar_wait(&bars->qd_full[f % Sh::kSlots], static_cast<uint32_t>(f / Sh::kSlots) & 1u);
-      mbar_wait(&bars->kv_full, 0);
+        mbar_wait(&bars->qd_full[f % Sh::kSlots], static_cast<uint32_t>(f / Sh::kSlots) & 1u, kWaitTimeoutNs, kSite + 10);
+      mbar_wait(&bars->kv_full, 0, kWaitTimeoutNs, kSite + 11);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -444,7 +441,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       constexpr uint32_t id_dk = idesc_f16(kBF16, 128, kD, false, true);          // dS^T (tmem) x Q
       const uint32_t sK = smem_u32(smem + Sh::kOffK);
       const uint32_t sV = smem_u32(smem + Sh::kOffV);
-      bool ok = bwd_wait(&bars->kv_full, 0, abort);
+      bool ok = bwd_wait(&bars->kv_full, 0, abort, kSite + 2);
       tc_fence_after();
       auto kmajor_kv = [](uint32_t base, int kk) {
         return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
@@ -460,7 +457,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       };
       auto wait_q = [&](int it) {
         const bool r = bwd_wait(&bars->qd_full[it % Sh::kSlots],
-                                static_cast<uint32_t>(it / Sh::kSlots) & 1u, abort);
+                                static_cast<uint32_t>(it / Sh::kSlots) & 1u, abort, kSite + 3);
         tc_fence_after();
         return r;
       };
@@ -494,7 +491,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
         // the team's P pass of item it: P^T in region A (dV's operand), or,
         // in the dK pass, S^T read out of region A into registers
-        if (!(ok = bwd_wait(&bars->p_ready[t], ph, abort))) break;
+        if (!(ok = bwd_wait(&bars->p_ready[t], ph, abort, kSite + 4))) break;
         tc_fence_after();
         if constexpr (kDoDV) {
           // dV += P^T dO: A = P^T of the team's region (queries [32c, 32c+32)
@@ -511,7 +508,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
         }
         if constexpr (kDoDK) {
           // dK += dS^T Q: A = dS^T of the team's region B, packed like P^T
-          if (!(ok = bwd_wait(&bars->ds_ready[t], ph, abort))) break;
+          if (!(ok = bwd_wait(&bars->ds_ready[t], ph, abort, kSite + 5))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
@@ -525,7 +522,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       }
       umma_commit(&bars->final_done);
       umma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0);
+      mbar_wait(&bars->drain, 0, kWaitTimeoutNs, kSite + 12);
     }
     __syncwarp();
   } else {
@@ -557,7 +554,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       // (shared-memory loads are slow while the tensor core reads its
       // operands), then P (* (1 - tanh^2)) for the dS pass
       float w[32];
-      if (!(ok = bwd_wait(&bars->qd_full[slot], static_cast<uint32_t>(it / Sh::kSlots) & 1u, abort))) break;
+      if (!(ok = bwd_wait(&bars->qd_full[slot], static_cast<uint32_t>(it / Sh::kSlots) & 1u, abort, kSite + 6))) break;
 #pragma unroll
       for (int j4 = 0; j4 < 8; ++j4) {
         const float4 l4 = *reinterpret_cast<const float4*>(glse + 4 * j4);
@@ -566,7 +563,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
         w[4 * j4 + 2] = l4.z;
         w[4 * j4 + 3] = l4.w;
       }
-      if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort))) break;
+      if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort, kSite + 7))) break;
       tc_fence_after();
       // does any (key, query) of this warp's 32 keys x the group's 32 queries need masking?
       const int kw_lo = k0 + lane_base, kw_hi = kw_lo + 31;
@@ -628,7 +625,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       // pass 2: dS^T = w * (dP^T - Drow) -> TMEM region B (the dK operand),
       // once dP^T is in TMEM (dK two items back, the last reader of these
       // columns, precedes the dP^T MMA in issue order)
-      if (!(ok = bwd_wait(&bars->dp_ready[team], ph, abort))) break;
+      if (!(ok = bwd_wait(&bars->dp_ready[team], ph, abort, kSite + 8))) break;
       tc_fence_after();
       {
         uint32_t dr[32];
@@ -666,7 +663,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
 
     // ---- epilogue: the four groups write the two column halves of the dV
     // rows (warps 2-9) and of the dK rows (warps 10-17) ----
-    if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
+    if (ok) ok = bwd_wait(&bars->final_done, 0, abort, kSite + 9);
     tc_fence_after();
     // (both: warps 2-9 write dV, 10-17 dK, each group half of a row; one
     // accumulator: each of the 2 kGroups groups its share of the row)
@@ -759,6 +756,7 @@ struct DqShape {
   static constexpr int kColDP = kDOSmem ? 128 + 2 * kKRows : 256;  // + kKRows t
   static constexpr int kColDQ = kDOSmem ? 256 : 384;
   static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB a CTA may use");
+  static_assert(kStages <= 24, "more ring slots than the barrier block holds");
 };
 
 struct DqBars {
@@ -858,7 +856,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % Sh::kStages;
           const uint32_t ph = static_cast<uint32_t>(fill / Sh::kStages) & 1u;
-          if (!bwd_wait(&bars->kv_empty[slot], ph ^ 1u, abort)) break;
+          if (!bwd_wait(&bars->kv_empty[slot], ph ^ 1u, abort, 401)) break;
           mbar_arrive_expect_tx(&bars->kv_full[slot], Sh::kTileBytes);
           uint8_t* dst = smem + Sh::kOffKV + slot * Sh::kTileBytes;
           const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
@@ -867,8 +865,8 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         }
       }
       for (int f = max(0, fill - Sh::kStages); f < fill; ++f)
-        mbar_wait(&bars->kv_full[f % Sh::kStages], static_cast<uint32_t>(f / Sh::kStages) & 1u);
-      if constexpr (Sh::kDOSmem) mbar_wait(&bars->do_full, 0);
+        mbar_wait(&bars->kv_full[f % Sh::kStages], static_cast<uint32_t>(f / Sh::kStages) & 1u, kWaitTimeoutNs, 409);
+      if constexpr (Sh::kDOSmem) mbar_wait(&bars->do_full, 0, kWaitTimeoutNs, 410);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -878,15 +876,15 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, false, true);          // dS (tmem) x K
       const uint32_t sKV = smem_u32(smem + Sh::kOffKV);
       const uint32_t sDO = smem_u32(smem + Sh::kOffDO);
-      bool ok = bwd_wait(&bars->qd_tmem, 0, abort);
-      if (ok && Sh::kDOSmem) ok = bwd_wait(&bars->do_full, 0, abort);
+      bool ok = bwd_wait(&bars->qd_tmem, 0, abort, 402);
+      if (ok && Sh::kDOSmem) ok = bwd_wait(&bars->do_full, 0, abort, 403);
       tc_fence_after();
       auto kmajor = [](uint32_t base, int kk) {
         return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
       };
       auto wait_slot = [&](int fill) {
         const bool r = bwd_wait(&bars->kv_full[fill % Sh::kStages],
-                                static_cast<uint32_t>(fill / Sh::kStages) & 1u, abort);
+                                static_cast<uint32_t>(fill / Sh::kStages) & 1u, abort, 404);
         tc_fence_after();
         return r;
       };
@@ -920,7 +918,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       }
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int t = j & 1;
-        if (!(ok = bwd_wait(&bars->ds_ready[t], static_cast<uint32_t>(j >> 1) & 1u, abort))) break;
+        if (!(ok = bwd_wait(&bars->ds_ready[t], static_cast<uint32_t>(j >> 1) & 1u, abort, 405))) break;
         tc_fence_after();
         // dQ += dS_j K_j: A = dS_j from S_t (keys [32c, 32c+32) packed into
         // columns [32c, 32c+16)), B = K_j with N = D (MN-major)
@@ -946,7 +944,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
       }
       umma_commit(&bars->final_done);
       umma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0);
+      mbar_wait(&bars->drain, 0, kWaitTimeoutNs, 411);
     }
     __syncwarp();
   } else {
@@ -999,7 +997,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     bool ok = true;
     for (int j = team; j < n_tiles; j += 2) {
       const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
-      if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort))) break;
+      if (!(ok = bwd_wait(&bars->s_ready[team], ph, abort, 406))) break;
       tc_fence_after();
       const int k0 = (n_begin + j) * Sh::kKRows + 32 * g;  // first key of this group's columns
       const uint32_t t_s = tmem + lane_off + Sh::kColS + Sh::kKRows * team + 32 * g;
@@ -1029,7 +1027,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         }
       }
       // pass 2 (needs dP_j): dS = w * (dP - Drow) -> the S columns already read
-      if (!(ok = bwd_wait(&bars->dp_ready[team], ph, abort))) break;
+      if (!(ok = bwd_wait(&bars->dp_ready[team], ph, abort, 407))) break;
       tc_fence_after();
       {
         uint32_t dr[32];
@@ -1054,7 +1052,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
     // ---- epilogue: dQ row -> dq; the 2 kGroups warp groups write the
     // 32-column chunks e * kPer .. (e + 1) * kPer - 1 of their rows (D = 64:
     // groups 2, 3 have none) ----
-    if (ok) ok = bwd_wait(&bars->final_done, 0, abort);
+    if (ok) ok = bwd_wait(&bars->final_done, 0, abort, 408);
     tc_fence_after();
     const int e = (warp - 2) >> 2;
     constexpr int kPer = (kD / 32 + 2 * Sh::kGroups - 1) / (2 * Sh::kGroups);

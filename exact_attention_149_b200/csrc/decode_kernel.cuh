@@ -447,6 +447,7 @@ struct DecShape {
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
   static constexpr int kThreads = 160;                 // 4 consumer warps + 1 producer
   static_assert(kScrOffset % 1024 == 0 && kStageBytes % 128 == 0, "scratch and stage alignment");
+  static_assert(kStages <= 8, "more ring slots than the barrier block holds");
 };
 
 struct DecBars {

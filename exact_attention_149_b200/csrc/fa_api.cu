@@ -426,13 +426,21 @@ fa_status fa_kernel_timing_read(const char* name, float* total_ms, int* launches
 
 fa_status fa_get_device_status(int* status_out) {
   if (status_out == nullptr) return fail(FA_ERR_INVALID_ARG, "status_out is NULL");
-  int v = 0;
+  int v = 0, site = 0;
   const int zero = 0;
   FA_CUDA_CHECK(cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(int)));
+  FA_CUDA_CHECK(cudaMemcpyFromSymbol(&site, fa::g_wait_site, sizeof(int)));
   FA_CUDA_CHECK(cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(int)));
-  if (v == fa::kDevTimeout)
+  FA_CUDA_CHECK(cudaMemcpyToSymbol(fa::g_wait_site, &zero, sizeof(int)));
+  if (v == fa::kDevTimeout) {
     *status_out = static_cast<int>(FA_ERR_TIMEOUT);
-  else if (v == fa::kDevBadIndex)
+    // the message names the wait that gave up first (when the kernel
+    // recorded one: 100 * kernel + wait, see bwd_wait)
+    g_last_error = "a kernel gave up on a bounded wait";
+    if (site != 0) g_last_error += " (wait site " + std::to_string(site) + ")";
+    return FA_OK;
+  }
+  if (v == fa::kDevBadIndex)
     *status_out = static_cast<int>(FA_ERR_INVALID_ARG);
   else
     *status_out = 0;

@@ -24,6 +24,14 @@ enum : int {
 // The library is built as one translation unit, so a file-scope variable is
 // shared by every kernel and by the host code that reads it back.
 static __device__ int g_device_status = 0;
+// which bounded wait gave up first (0 = none): 100 * kernel + wait, for the
+// error message of fa_get_device_status
+static __device__ int g_wait_site = 0;
+
+__device__ __forceinline__ void record_timeout(int site) {
+  atomicExch(&g_device_status, 1 /* kDevTimeout */);
+  if (site != 0) atomicCAS(&g_wait_site, 0, site);
+}
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;  // 4 s
@@ -93,13 +101,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // records kDevTimeout in the library's device status word) if it has not
 // completed within kWaitTimeoutNs; the caller then unwinds instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          uint64_t limit_ns = kWaitTimeoutNs) {
+                                          uint64_t limit_ns = kWaitTimeoutNs, int site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) {
-      atomicExch(&g_device_status, kDevTimeout);
+      record_timeout(site);
       return false;
     }
   }
@@ -371,11 +379,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // algorithm (fit_polynomials.py next to this file; float32 relative error
 // 7.5e-5), and n is added into the exponent field: the low 9 bits of the
 // rounded value's bit pattern, shifted by 23, are n << 23 modulo 2^32.
-// x is clamped at -126 so that the exponent cannot underflow: smaller inputs
-// (masked logits, -inf) give a value below 2^-125 rather than 0.
+// x is clamped at -125 so that the result's exponent field stays >= 1 (at
+// n = -126 a cubic below 1 would land on the subnormal encoding, which the
+// bit addition does not produce correctly): smaller inputs (masked logits,
+// -inf) give a value near 2^-125 rather than 0.
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
   const float2 j = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
   const float2 n = __fadd2_rn(j, make_float2(-12582912.f, -12582912.f));
   const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);

@@ -393,12 +393,13 @@ FA_API fa_status fa_kernel_timing_reset(void);
  * exists so that their error can be checked against CUDA's own functions on
  * the device): for the n DEVICE floats x, out_poly receives the library's
  * approximation and out_ref the CUDA math function on the same input, with
- *   which = 0: 2^x by the cubic of the forward's softmax (x >= -126;
- *              relative error 7.5e-5), reference exp2f;
- *   which = 1: tanh(x) by the degree-4 odd polynomial (|x| <= 0.5; absolute
- *              error 4e-8), reference tanhf;
+ *   which = 0: 2^x by the cubic of the forward's softmax (x >= -125;
+ *              relative error 7.5e-5 plus float32 rounding), reference exp2f;
+ *   which = 1: tanh(x) by the degree-4 odd polynomial (|x| <= 0.5; about
+ *              4e-8 absolute plus float32 rounding), reference tanhf;
  *   which = 2: tanh(x) by the degree-2 polynomial with folded scales
- *              (|x| <= 0.25; absolute error 1.1e-7), reference tanhf.
+ *              (|x| <= 0.25; about 1e-7 absolute plus float32 rounding),
+ *              reference tanhf.
  * Asynchronous on `stream`. Errors: FA_ERR_INVALID_ARG for another `which`,
  * n < 0 or null pointers with n > 0; FA_ERR_CUDA on launch failure.
  */
@@ -429,7 +430,9 @@ FA_API fa_status fa_selftest_fwd_timeout(const void* q, const void* k, const voi
  * last call, FA_ERR_TIMEOUT if one gave up on a bounded wait, and
  * FA_ERR_INVALID_ARG if a decode kernel met a cache length or page-table
  * entry out of range (it then skipped the out-of-range access and its output
- * is not valid). Returns FA_ERR_CUDA if the word cannot be read.
+ * is not valid). With FA_ERR_TIMEOUT, fa_last_error() names the wait that
+ * gave up when the kernel recorded it. Returns FA_ERR_CUDA if the word cannot
+ * be read.
  */
 FA_API fa_status fa_get_device_status(int* status_out);
 

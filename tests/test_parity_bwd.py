@@ -27,7 +27,8 @@ def _gpu_fwd_bwd(inp, scale, causal, window, softcap, cu=None, max_seqlen=None):
     dq, dk, dv = fa.bwd(q, k, v, o, lse, do, scale=scale, causal=causal, window=window,
                         softcap=softcap, cu_seqlens=cud, max_seqlen=max_seqlen)
     torch.cuda.synchronize()
-    assert fa.fa_get_device_status() == 0
+    st = fa.fa_get_device_status()
+    assert st == 0, fa.fa_last_error()
     return dq.cpu(), dk.cpu(), dv.cpu()
 
 
