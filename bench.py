@@ -595,6 +595,13 @@ def run_ours(args, dist: Dist):
         best4 = max(dec4["splits"].values(), key=lambda d: d["gbs"])
         dec4["best_gbs"] = best4["gbs"]
         dec4["best_frac_of_hbm"] = best4["frac_of_hbm"]
+        trd4 = kernel_traffic("decode_split_int4")
+        k4 = best4.get("decode_split_kernel", best4)
+        dec4["roofline"] = {"kernel": "decode_split (int4 cache)", "bound": "hbm",
+                            "achieved": k4["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": k4["gbs"] / peaks["hbm_gbs"],
+                            "traffic": trd4["bytes_per_launch"] if trd4 else None,
+                            "peak_source": peaks["source"] + " HBM copy"}
     except Exception as e:  # recorded in the line; the headline measurement stands
         dec4["error"] = f"{type(e).__name__}: {e}"
     res["decode_int4"] = dec4

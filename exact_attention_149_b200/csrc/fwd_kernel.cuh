@@ -493,37 +493,15 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       bool need_mask = (k0 + 127 >= seq_len);
       if (p.wr >= 0) need_mask |= (k0 + 127 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
-      // softcap on a tile with no masked key and no bias ("fused"): the capped
-      // logit is monotone in the raw score, so the raw row max and min give
-      // both the polynomial's range check and the row max, and the max is
-      // subtracted inside the polynomial's last FMA further down; x stays raw
-      // until then
-      bool fused = false;
-      float raw_ext = 0.f;
-      float pkf[3] = {0.f, 0.f, 0.f};
-      float amax = -1.f;  // (>= 0 once known)
-      if constexpr (kCap && !alibi) {
-        if (!need_mask) {
-          const float mx = reduce128<true>(x), mn = reduce128<false>(x);
-          amax = fmaxf(fabsf(mx), fabsf(mn));
-          if (__all_sync(0xffffffffu, amax * fabsf(p.cap_in) <= kTanhPolyMaxLo)) {
-            fused = true;
-            raw_ext = p.cap_in >= 0.f ? mx : mn;
-            fold_tanh(kTanhLo, p.cap_in, p.cap_out_log2, pkf);
-          }
-        }
-      }
-      if (kCap && !fused) {
+      if constexpr (kCap) {
         // logits in the exp2 domain: softcap * tanh(scale * s / softcap) * log2(e).
         // When every |scale * s / softcap| of the warp's rows is small, tanh
         // is an FMA-pipe polynomial with the scale and softcap folded into
         // its coefficients (two values per instruction; degree 2 below 1/4,
         // degree 4 below 1/2); otherwise the exp-based identity.
-        if (amax < 0.f) {
-          amax = 0.f;
+        float amax = 0.f;
 #pragma unroll
-          for (int i = 0; i < 128; i += 2) amax = max3(amax, fabsf(x[i]), fabsf(x[i + 1]));
-        }
+        for (int i = 0; i < 128; i += 2) amax = max3(amax, fabsf(x[i]), fabsf(x[i + 1]));
         const float ya = amax * fabsf(p.cap_in);
         if (__all_sync(0xffffffffu, ya <= kTanhPolyMaxLo)) {
           float pk[3];
@@ -592,11 +570,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
         for (int i = 0; i < 128; ++i) x[i] = (i > jmax || i < jmin) ? hide : x[i];
       }
       float mt;
-      if (fused) {
-        // the capped logit of the raw extreme, by the same polynomial
-        const float u = raw_ext * raw_ext;
-        mt = raw_ext * fmaf(fmaf(pkf[2], u, pkf[1]), u, pkf[0]);
-      } else if constexpr (lg) {
+      if constexpr (lg) {
         mt = reduce128<true>(x);
       } else {
         mt = pos ? reduce128<true>(x) : reduce128<false>(x);
@@ -629,27 +603,12 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       // used so that they pipeline through the special-function unit
       const float2 nb2 = make_float2(-base, -base);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-      if (kCap && fused) {
-        // x * P(x^2) - base: the folded degree-2 tanh and the max in one pass
-        const float2 p0 = make_float2(pkf[0], pkf[0]), p1 = make_float2(pkf[1], pkf[1]),
-                     p2 = make_float2(pkf[2], pkf[2]);
 #pragma unroll
-        for (int i = 0; i < 128; i += 2) {
-          const float2 xv = make_float2(x[i], x[i + 1]);
-          const float2 u = __fmul2_rn(xv, xv);
-          const float2 q = __ffma2_rn(__ffma2_rn(p2, u, p1), u, p0);
-          const float2 d = __ffma2_rn(xv, q, nb2);
-          x[i] = d.x;
-          x[i + 1] = d.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; i += 2) {
-          const float2 xv = make_float2(x[i], x[i + 1]);
-          const float2 d = lg ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
-          x[i] = d.x;
-          x[i + 1] = d.y;
-        }
+      for (int i = 0; i < 128; i += 2) {
+        const float2 xv = make_float2(x[i], x[i + 1]);
+        const float2 d = lg ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
+        x[i] = d.x;
+        x[i + 1] = d.y;
       }
       // the parts of the row in turn: their exponentials, then their 16-bit
       // P into TMEM and a signal, so that the tensor core starts on the first
