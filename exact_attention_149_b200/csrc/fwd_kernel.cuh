@@ -90,8 +90,15 @@ struct FwdShape {
   static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;  // + barriers + align slack
   static_assert(kStages <= 8, "more ring slots than the barrier block holds");
   static constexpr int kThreads = 128 * (1 + kQT);
-  static constexpr int kRegsLow = 88;   // warpgroup 0 after setmaxnreg.dec
-  static constexpr int kRegsHigh = 208; // softmax warpgroups after setmaxnreg.inc
+  // registers of warpgroup 0 (producer, MMA issuer) after setmaxnreg.dec
+  // and of the softmax warpgroups after setmaxnreg.inc. With softcap or FP8
+  // the producer/MMA code spills at 88, so those variants move 16 registers
+  // to it (measured: varlen softcap 3% and FP8 1.4% faster; the plain
+  // causal forward 0.5% slower, so it keeps the first split).
+  static constexpr int kRegsLow = 88;
+  static constexpr int kRegsHigh = 208;
+  static constexpr int kRegsLowWide = 104;
+  static constexpr int kRegsHighWide = 200;
   static constexpr int kTmemCols = 512;
   // of every 8 pairs of exponentials, this many run as a cubic on the FMA
   // pipe instead of the special-function unit (which bounds the softmax)
@@ -293,13 +300,17 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   volatile int* abort = &bars->abort;
-  static_assert(Sh::kQT == 1 || Sh::kThreads * 168 >= 128 * Sh::kRegsLow + 256 * Sh::kRegsHigh,
+  constexpr bool kWide = kCap || kF8;
+  constexpr int kRegsLow = kWide ? Sh::kRegsLowWide : Sh::kRegsLow;
+  constexpr int kRegsHigh = kWide ? Sh::kRegsHighWide : Sh::kRegsHigh;
+  static_assert(Sh::kQT == 1 || Sh::kThreads * 168 >= 128 * kRegsLow + 256 * kRegsHigh,
                 "register split exceeds the launch pool");
+  static_assert(kRegsLow % 8 == 0 && kRegsHigh % 8 == 0, "setmaxnreg takes multiples of 8");
   // register reallocation sits inside each role's branch so the compiler
   // knows which limit every region runs under
   if (warp < 4) {
     // (one Q tile: 256 threads, every thread has the 255 registers it may use)
-    if constexpr (Sh::kQT == 2) regs_dec<Sh::kRegsLow>();
+    if constexpr (Sh::kQT == 2) regs_dec<kRegsLow>();
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (elect_one()) {
@@ -451,7 +462,7 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
     __syncwarp();
   }
   } else {
-    if constexpr (Sh::kQT == 2) regs_inc<Sh::kRegsHigh>();
+    if constexpr (Sh::kQT == 2) regs_inc<kRegsHigh>();
     const FwdItem w = load_item(bars);
     const uint32_t tmem = *static_cast<volatile uint32_t*>(&bars->tmem_base);
     const int seq_start = w.seq_start, seq_len = w.seq_len, q0 = w.q0, h = w.h, b = w.b;
