@@ -226,7 +226,9 @@ __device__ __forceinline__ void alibi32(float (&w)[32], float sl2, float d0, flo
 // is consumed, so they pipeline through the special-function unit. With
 // ALiBi, entry i gets -sl2 * |d0 - i| added to its exponent (sl2: slope in
 // the exp2 domain, d0: query position minus the first key's).
-template <bool kCap>
+// kPolyOf8: of every 8 pairs of exponentials, this many run as an FMA-pipe
+// cubic instead of on the special-function unit.
+template <bool kCap, int kPolyOf8 = 0>
 __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, const BwdParams& p,
                                             bool alibi, float sl2, float d0, float (&w)[32],
                                             bool causal_side) {
@@ -245,7 +247,16 @@ __device__ __forceinline__ void bwd_probs32(uint32_t (&sr)[32], float2 nl2, cons
   }
   if (alibi) alibi32(w, sl2, d0, -1.f, causal_side);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) w[i] = ex2_approx(w[i]);
+  for (int j2 = 0; j2 < 16; ++j2) {
+    if ((j2 & 7) < kPolyOf8) {
+      const float2 e = ex2_poly2(make_float2(w[2 * j2], w[2 * j2 + 1]));
+      w[2 * j2] = e.x;
+      w[2 * j2 + 1] = e.y;
+    } else {
+      w[2 * j2] = ex2_approx(w[2 * j2]);
+      w[2 * j2 + 1] = ex2_approx(w[2 * j2 + 1]);
+    }
+  }
   if constexpr (kCap) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) w[i] *= __uint_as_float(sr[i]);
@@ -732,7 +743,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
 // in shared memory (loaded once by TMA, the A operand of dP = dO V^T), an
 // item is 32 keys and each team has one compute group.
 template <int kD>
-struct DqShape {
+struct Dq256Shape {
   static constexpr int kChunks = kD / 64;
   static constexpr int kKRows = kD == 256 ? 32 : 64;   // keys per item
   static constexpr int kGroups = kKRows / 32;          // compute groups per team
@@ -759,7 +770,7 @@ struct DqShape {
   static_assert(kStages <= 24, "more ring slots than the barrier block holds");
 };
 
-struct DqBars {
+struct Dq256Bars {
   uint64_t qd_tmem;      // Q (and dO, D <= 128) written to TMEM (4 kGroups warps)
   uint64_t do_full;      // D = 256: the dO tile in shared memory
   uint64_t kv_full[24];
@@ -774,15 +785,15 @@ struct DqBars {
 };
 
 template <int kD, bool kBF16, bool kCap, bool kAlibi>
-__global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+__global__ void __launch_bounds__(Dq256Shape<kD>::kThreads, 1)
+    bwd_dq256_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
-  using Sh = DqShape<kD>;
-  static_assert(sizeof(DqBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
+  using Sh = Dq256Shape<kD>;
+  static_assert(sizeof(Dq256Bars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  DqBars* bars = reinterpret_cast<DqBars*>(smem + Sh::kOffBar);
+  Dq256Bars* bars = reinterpret_cast<Dq256Bars*>(smem + Sh::kOffBar);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1060,6 +1071,355 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
                    (static_cast<size_t>(seq_start + qrow) * p.dq_tok + static_cast<size_t>(h) * kD) * 2;
 #pragma unroll 1
     for (int c = e * kPer; c < (e + 1) * kPer && c < kD / 32; ++c) {
+      if (ok && n_tiles > 0) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_off + Sh::kColDQ + c * 32, rr);
+        tmem_ld_wait();
+        uint32_t wv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          wv[i] = pack2<kBF16>(__uint_as_float(rr[2 * i]) * p.scale, __uint_as_float(rr[2 * i + 1]) * p.scale);
+        if (qrow < seq_len) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+        }
+      } else if (ok && qrow < seq_len) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 64);
+        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Sh::kTmemCols);
+  }
+}
+
+// ===========================================================================
+// dQ (D = 64, 128)
+// ===========================================================================
+// One CTA per (sequence, query head, 128-row Q tile); an item is one 128-key
+// block, so every product has N = 128 (N = D for dQ += dS K):
+//   warp 0      TMA producer: the Q and dO tiles once, then K_j and V_j
+//               (128 rows each) into two rings: V_j is free once dP_j has
+//               run, K_j only after dQ_j.
+//   warp 1      MMA issuer and TMEM owner.
+//   warps 2-17  four compute groups of four warps, one thread per query row;
+//               group g takes the key columns [32g, 32g + 32) of each block:
+//               P = exp(S - LSE) into registers, then dS = P * (dP - Drow)
+//               (16-bit pairs) over the first half of the dP columns it has
+//               read.
+// TMEM columns: S [0, 128), dP_t [128 + 128t, +128) for t = j % 2, dQ
+// [384, 384 + D). Q and dO stay in shared memory as the A operands of
+// S = Q K^T and dP = dO V^T, which leaves tensor memory room for two dP
+// buffers: the P pass frees S as soon as it has read it, and dP_{j+1} needs
+// only dQ_{j-1} (the last reader of its buffer) to be issued, so S_{j+1} and
+// dP_{j+1} run while the groups form P_j and dS_j. MMA order: S_{j+1},
+// dP_{j+1}, dQ_j; the order is fixed, so dQ is deterministic.
+template <int kD>
+struct DqShape {
+  static_assert(kD == 64 || kD == 128, "this dQ kernel takes D = 64 or 128");
+  static constexpr int kChunks = kD / 64;
+  static constexpr int kKRows = 128;                   // keys per item
+  static constexpr int kGroups = 4;                    // 32 key columns each
+  static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 B
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kTileBytes;
+  static constexpr int kKStages = kD == 128 ? 3 : 6;   // K ring slots
+  static constexpr int kVStages = kD == 128 ? 2 : 4;   // V ring slots
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
+  static constexpr int kThreads = 64 + kGroups * 128;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kColS = 0;
+  static constexpr int kColDP = 128;                   // + 128 t
+  static constexpr int kColDQ = 384;
+  static constexpr int kPolyOf8 = 2;  // FMA-pipe share of the exponentials
+  static_assert(kSmemBytes <= 232448, "shared memory exceeds the 227 KB a CTA may use");
+  static_assert(kKStages <= 8 && kVStages <= 8, "more ring slots than the barrier block holds");
+};
+
+struct DqBars {
+  uint64_t qdo_full;     // the Q and dO tiles
+  uint64_t k_full[8];
+  uint64_t k_empty[8];
+  uint64_t v_full[8];
+  uint64_t v_empty[8];
+  uint64_t s_ready;
+  uint64_t s_free;       // every group has read S
+  uint64_t dp_ready[2];  // per dP buffer
+  uint64_t ds_ready[2];
+  uint64_t final_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int kD, bool kBF16, bool kCap, bool kAlibi>
+__global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+  using Sh = DqShape<kD>;
+  static_assert(sizeof(DqBars) <= Sh::kBarBytes, "barrier block exceeds its reservation");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + Sh::kOffBar);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (sequence, head) major; Q tiles with most keys first
+  const int nq = p.n_ktiles;  // 128-row tiles per sequence
+  const int bh = static_cast<int>(blockIdx.x) / nq;
+  const int qt = nq - 1 - static_cast<int>(blockIdx.x) % nq;
+  const int h = bh % p.Hq;
+  const int b = bh / p.Hq;
+  int seq_start, seq_len;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    seq_len = p.cu_seqlens[b + 1] - seq_start;
+  } else {
+    seq_start = b * p.S;
+    seq_len = p.S;
+  }
+  const int q0 = qt * 128;
+  if (q0 >= seq_len) return;
+  const int kvh = h / p.group;
+  const int row_hi = min(q0 + 127, seq_len - 1);
+  int key_hi = seq_len - 1;
+  if (p.wr >= 0) key_hi = min(key_hi, row_hi + p.wr);
+  int key_lo = 0;
+  if (p.wl >= 0) key_lo = max(0, q0 - p.wl);
+  const int n_begin = key_lo / Sh::kKRows;
+  const int n_tiles = key_hi >= key_lo ? key_hi / Sh::kKRows + 1 - n_begin : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->qdo_full, 1);
+    for (int i = 0; i < Sh::kKStages; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < Sh::kVStages; ++i) {
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
+    }
+    mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->s_free, 4 * Sh::kGroups);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->dp_ready[t], 1);
+      mbar_init(&bars->ds_ready[t], 4 * Sh::kGroups);
+    }
+    mbar_init(&bars->final_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, Sh::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      // (rows past the end of the tensor read as zero; rows of the next
+      // sequence are masked out of P)
+      mbar_arrive_expect_tx(&bars->qdo_full, 2 * Sh::kTileBytes);
+      for (int c = 0; c < Sh::kChunks; ++c) {
+        tma_load_3d(&tm_q, &bars->qdo_full, smem + Sh::kOffQ + c * Sh::kChunkBytes, c * 64, h, seq_start + q0);
+        tma_load_3d(&tm_do, &bars->qdo_full, smem + Sh::kOffDO + c * Sh::kChunkBytes, c * 64, h, seq_start + q0);
+      }
+      int nk = 0, nv = 0;  // K and V tiles issued
+      while (nv < n_tiles && !*abort) {
+        const int tok = seq_start + (n_begin + nv) * Sh::kKRows;
+        if (nk == nv) {
+          const int slot = nk % Sh::kKStages;
+          if (!bwd_wait(&bars->k_empty[slot], (static_cast<uint32_t>(nk / Sh::kKStages) & 1u) ^ 1u, abort, 401)) break;
+          mbar_arrive_expect_tx(&bars->k_full[slot], Sh::kTileBytes);
+          for (int c = 0; c < Sh::kChunks; ++c)
+            tma_load_3d(&tm_k, &bars->k_full[slot], smem + Sh::kOffK + slot * Sh::kTileBytes + c * Sh::kChunkBytes,
+                        c * 64, kvh, tok);
+          ++nk;
+        }
+        const int slot = nv % Sh::kVStages;
+        if (!bwd_wait(&bars->v_empty[slot], (static_cast<uint32_t>(nv / Sh::kVStages) & 1u) ^ 1u, abort, 409)) break;
+        mbar_arrive_expect_tx(&bars->v_full[slot], Sh::kTileBytes);
+        for (int c = 0; c < Sh::kChunks; ++c)
+          tma_load_3d(&tm_v, &bars->v_full[slot], smem + Sh::kOffV + slot * Sh::kTileBytes + c * Sh::kChunkBytes,
+                      c * 64, kvh, tok);
+        ++nv;
+      }
+      // the copies still in flight finish before the CTA may exit
+      for (int f = max(0, nk - Sh::kKStages); f < nk; ++f)
+        mbar_wait(&bars->k_full[f % Sh::kKStages], static_cast<uint32_t>(f / Sh::kKStages) & 1u, kWaitTimeoutNs, 410);
+      for (int f = max(0, nv - Sh::kVStages); f < nv; ++f)
+        mbar_wait(&bars->v_full[f % Sh::kVStages], static_cast<uint32_t>(f / Sh::kVStages) & 1u, kWaitTimeoutNs, 410);
+      mbar_wait(&bars->qdo_full, 0, kWaitTimeoutNs, 410);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (elect_one()) {
+      constexpr uint32_t id_s = idesc_f16(kBF16, 128, Sh::kKRows, false, false);  // S, dP
+      constexpr uint32_t id_dq = idesc_f16(kBF16, 128, kD, false, true);          // dS (tmem) x K
+      const uint32_t sQ = smem_u32(smem + Sh::kOffQ);
+      const uint32_t sDO = smem_u32(smem + Sh::kOffDO);
+      const uint32_t sK0 = smem_u32(smem + Sh::kOffK);
+      const uint32_t sV0 = smem_u32(smem + Sh::kOffV);
+      bool ok = bwd_wait(&bars->qdo_full, 0, abort, 402);
+      tc_fence_after();
+      // 128 rows, K-major, 64-element chunks
+      auto kmajor = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + (kk >> 2) * Sh::kChunkBytes + (kk & 3) * 32, 16, 1024);
+      };
+      auto k_addr = [&](int j) { return sK0 + (j % Sh::kKStages) * Sh::kTileBytes; };
+      auto issue_s = [&](int j) {  // S_j = Q K_j^T
+        if (!bwd_wait(&bars->k_full[j % Sh::kKStages], static_cast<uint32_t>(j / Sh::kKStages) & 1u, abort, 404))
+          return false;
+        tc_fence_after();
+        const uint32_t sK = k_addr(j);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColS, kmajor(sQ, kk), kmajor(sK, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_ready);
+        return true;
+      };
+      auto issue_dp = [&](int j) {  // dP_j = dO V_j^T -> buffer j % 2; V_j is then free
+        if (!bwd_wait(&bars->v_full[j % Sh::kVStages], static_cast<uint32_t>(j / Sh::kVStages) & 1u, abort, 412))
+          return false;
+        tc_fence_after();
+        const uint32_t sV = sV0 + (j % Sh::kVStages) * Sh::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          umma_ss(tmem + Sh::kColDP + 128 * (j & 1), kmajor(sDO, kk), kmajor(sV, kk), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->dp_ready[j & 1]);
+        umma_commit(&bars->v_empty[j % Sh::kVStages]);
+        return true;
+      };
+      if (ok && n_tiles > 0) ok = issue_s(0) && issue_dp(0);
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const bool more = j + 1 < n_tiles;
+        // S_{j+1} once every group has read S_j; dP_{j+1} into the buffer
+        // that dQ_{j-1}, issued before, read
+        if (!(ok = bwd_wait(&bars->s_free, static_cast<uint32_t>(j) & 1u, abort, 403))) break;
+        if (more && !(ok = issue_s(j + 1) && issue_dp(j + 1))) break;
+        // dQ += dS_j K_j: A = dS_j over dP buffer j % 2 (keys [32c, 32c + 32)
+        // packed into columns [32c, 32c + 16)), B = K_j with N = D (MN-major)
+        if (!(ok = bwd_wait(&bars->ds_ready[j & 1], static_cast<uint32_t>(j >> 1) & 1u, abort, 405))) break;
+        tc_fence_after();
+        const uint32_t sK = k_addr(j);
+        const uint32_t a = tmem + Sh::kColDP + 128 * (j & 1);
+#pragma unroll
+        for (int kk = 0; kk < Sh::kKRows / 16; ++kk)
+          umma_ts(tmem + Sh::kColDQ, a + (kk >> 1) * 32 + (kk & 1) * 8,
+                  sdesc_sw128(sK + kk * 2048, Sh::kChunkBytes, 1024), id_dq, (j == 0 && kk == 0) ? 0u : 1u);
+        umma_commit(&bars->k_empty[j % Sh::kKStages]);
+      }
+      umma_commit(&bars->final_done);
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, kWaitTimeoutNs, 411);
+    }
+    __syncwarp();
+  } else {
+    // ======================= compute groups =======================
+    const int g = (warp - 2) >> 2;           // key columns [32g, 32g + 32)
+    const int lane_base = 32 * (warp & 3);
+    const int r = lane_base + lane;          // query row within the tile
+    const int qrow = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(lane_base) << 16;
+    // the row's -LSE (exp2 domain) and Drow
+    float nlse = -INFINITY, drow = 0.f;
+    if (qrow < seq_len) {
+      const size_t vi = vec_index(p, h, b, seq_start, qrow);
+      nlse = p.vec_nlse[vi];
+      drow = p.vec_drow[vi];
+    }
+    const float2 nl2 = make_float2(nlse, nlse);
+    const float2 nd2 = make_float2(-drow, -drow);
+    constexpr bool alibi = kAlibi;  // compiled in only where used
+    const float sl2 = alibi_slope2(p, b, h);
+    const uint32_t t_s = tmem + lane_off + Sh::kColS + 32 * g;
+    const int r_lo = q0 + lane_base, r_hi = r_lo + 31;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!(ok = bwd_wait(&bars->s_ready, static_cast<uint32_t>(j) & 1u, abort, 406))) break;
+      tc_fence_after();
+      const int k0 = (n_begin + j) * Sh::kKRows + 32 * g;  // first key of this group's columns
+      // mask needed for this warp's 32 rows x the group's 32 keys?
+      bool need_mask = (k0 + 31 >= seq_len) || (r_hi >= seq_len);
+      if (p.wr >= 0) need_mask |= (k0 + 31 > r_lo + p.wr);
+      if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
+      // P pass (needs S_j only): w = P (* (1 - tanh^2)) for the group's 32
+      // keys, kept in registers; S is free once every group has read it
+      float w[32];
+      {
+        uint32_t sr[32];
+        tmem_ld32(t_s, sr);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+        bwd_probs32<kCap, Sh::kPolyOf8>(sr, nl2, p, alibi, sl2, static_cast<float>(qrow - k0), w, p.wr == 0);
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int kj = k0 + i;
+            bool v = qrow < seq_len && kj < seq_len;
+            if (p.wr >= 0) v = v && kj <= qrow + p.wr;
+            if (p.wl >= 0) v = v && kj >= qrow - p.wl;
+            w[i] = v ? w[i] : 0.f;
+          }
+        }
+      }
+      // dS pass (needs dP_j): dS = w * (dP - Drow) -> the dP columns already read
+      if (!(ok = bwd_wait(&bars->dp_ready[j & 1], static_cast<uint32_t>(j >> 1) & 1u, abort, 407))) break;
+      tc_fence_after();
+      {
+        const uint32_t t_dp = tmem + lane_off + Sh::kColDP + 128 * (j & 1) + 32 * g;
+        uint32_t dr[32];
+        tmem_ld32(t_dp, dr);
+        tmem_ld_wait();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
+          const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2), make_float2(w[2 * j2], w[2 * j2 + 1]));
+          dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
+        }
+        // dS of keys [k0, k0 + 32) -> columns [32g, 32g + 16) of the buffer
+        tmem_st16(t_dp, dsk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ds_ready[j & 1]);
+    }
+    // ---- epilogue: dQ row -> dq; group g writes the 32-column chunk g of
+    // its rows (D = 64: groups 0, 1) ----
+    if (ok) ok = bwd_wait(&bars->final_done, 0, abort, 408);
+    tc_fence_after();
+    uint8_t* dst = static_cast<uint8_t*>(p.dq) +
+                   (static_cast<size_t>(seq_start + qrow) * p.dq_tok + static_cast<size_t>(h) * kD) * 2;
+    const int c = g;
+    if (c < kD / 32) {
       if (ok && n_tiles > 0) {
         uint32_t rr[32];
         tmem_ld32(tmem + lane_off + Sh::kColDQ + c * 32, rr);
