@@ -23,19 +23,20 @@
 // for no dQ reduction across CTAs and a pipeline with no write-back on the
 // critical path.
 //
-// bwd_dkdv warp roles (576 threads); an item is one (query head, 64-row
+// bwd_dkdv warp roles (608 threads); an item is one (query head, 64-row
 // query block) against the CTA's 128 keys:
 //   warp 0      TMA producer: K, V once; Q_i, dO_i and the rows' -LSE and Drow
 //               into a 4-slot ring.
-//   warp 1      MMA issuer (one lane), TMEM owner.
-//   warps 2-17  two teams of two compute groups; team t takes the items with
+//   warp 1      MMA issuer of S^T and dV (one lane), TMEM owner.
+//   warp 2      MMA issuer of dP^T and dK (one lane).
+//   warps 3-18  two teams of two compute groups; team t takes the items with
 //               i % 2 == t, group g of a team the item's query columns
 //               [32g, 32g+32): one thread per key row computes
 //               P^T = exp(S^T - LSE) and then dS^T = P^T * (dP^T - Drow), each
 //               written back to TMEM as 16-bit pairs over the first half of
 //               the columns it came from, where the dV and dK MMAs read their
 //               A operand. While one team computes, the tensor core runs the
-//               other team's MMAs. At the end warps 2-9 write dV, 10-17 dK.
+//               other team's MMAs. At the end warps 3-10 write dV, 11-18 dK.
 // TMEM columns: A_t [64t, 64t+64) S^T then P^T; B_t [128+64t, +64) dP^T then
 // dS^T (queries [32g, 32g+32) packed into [32g, 32g+16) of each);
 // dV [256, 256+D); dK [256+D, 256+2D).
@@ -298,10 +299,15 @@ struct DkdvShape {
   static constexpr int kOffBar = kOffVec + kSlots * kVecBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
-  // warp 0 TMA, warp 1 MMA, then two teams of kGroups compute groups (4
-  // warps each); team t takes the items it with it % 2 == t, group g of a
-  // team the 32 query columns [32g, 32g + 32) of the item
-  static constexpr int kThreads = 64 + 2 * kGroups * 128;
+  // warp 0 TMA, warps 1 .. kIssuers MMA, then two teams of kGroups compute
+  // groups (4 warps each); team t takes the items it with it % 2 == t, group
+  // g of a team the 32 query columns [32g, 32g + 32) of the item. The fused
+  // kernel issues from two threads (one tcgen05.mma with N = 64 takes about
+  // as long to issue as to run): warp 1 the S^T and dV products, warp 2 the
+  // dP^T and dK ones.
+  static constexpr int kIssuers = kPass == kDkdvBoth ? 2 : 1;
+  static constexpr int kFirst = 1 + kIssuers;  // first compute warp
+  static constexpr int kThreads = 32 * kFirst + 2 * kGroups * 128;
   static constexpr int kTmemCols = 512;
   static constexpr int kColA = 0;             // + kQRows t: team t's S^T, then P^T
   static constexpr int kColB = 2 * kQRows;    // + kQRows t: team t's dP^T, then dS^T
@@ -319,8 +325,8 @@ struct DkdvBars {
   uint64_t dp_ready[2];
   uint64_t p_ready[2];
   uint64_t ds_ready[2];
-  uint64_t final_done;
-  uint64_t drain;
+  uint64_t final_done;   // one commit per issuer
+  uint64_t drain[2];     // per issuer
   uint32_t tmem_base;
   int abort;
 };
@@ -372,16 +378,16 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < Sh::kSlots; ++s) {
       mbar_init(&bars->qd_full[s], 1);
-      mbar_init(&bars->qd_empty[s], 1);
+      mbar_init(&bars->qd_empty[s], Sh::kIssuers);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_ready[t], 1);
       mbar_init(&bars->dp_ready[t], 1);
       mbar_init(&bars->p_ready[t], 4 * Sh::kGroups);
       mbar_init(&bars->ds_ready[t], 4 * Sh::kGroups);
+      mbar_init(&bars->drain[t], 1);
     }
-    mbar_init(&bars->final_done, 1);
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->final_done, Sh::kIssuers);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -437,15 +443,22 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       mbar_wait(&bars->kv_full, 0, kWaitTimeoutNs, kSite + 11);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ======================= MMA issuer =======================
+  } else if (warp <= Sh::kIssuers) {
+    // ======================= MMA issuers =======================
     // Issue order per item i (team t = i % 2, regions A_t, B_t):
     //   dV_i (after the P pass of i), S_{i+2} -> A_t, dK_i (after the dS pass
     //   of i), dP_{i+2} -> B_t.
     // S_{i+2} overwrites A_t only after dV_i, its last reader, in issue
-    // order; dP_{i+2} overwrites B_t after dK_i. The other team's item i+1
-    // is in its P or dS pass meanwhile, so the tensor core has work while
-    // each team computes. The order is fixed, so the sums are deterministic.
+    // order; dP_{i+2} overwrites B_t after dK_i. With two issuers the first
+    // runs the A chain (S, dV) and the second the B chain (dP, dK): each
+    // region is written and read by one thread, whose products run in issue
+    // order, and no product reads the other chain's region. The other
+    // team's item i+1 is in its P or dS pass meanwhile, so the tensor core
+    // has work while each team computes. Each accumulator is summed in a
+    // fixed order, so the sums are deterministic.
+    constexpr bool kSplit = Sh::kIssuers == 2;
+    const bool do_a = !kSplit || warp == 1;  // S^T and dV
+    const bool do_b = !kSplit || warp == 2;  // dP^T and dK
     if (elect_one()) {
       constexpr uint32_t id_s = idesc_f16(kBF16, 128, Sh::kQRows, false, false);  // S^T, dP^T
       constexpr uint32_t id_dv = idesc_f16(kBF16, 128, kD, false, true);          // P^T (tmem) x dO
@@ -490,8 +503,8 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       };
       for (int it = 0; it < 2 && it < n_items && ok; ++it) {
         if ((ok = wait_q(it))) {
-          issue_s(it);
-          if constexpr (kDoDK) issue_dp(it);
+          if (do_a) issue_s(it);
+          if (kDoDK && do_b) issue_dp(it);
         }
       }
       for (int it = 0; it < n_items && ok; ++it) {
@@ -500,24 +513,26 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
         const uint32_t sQ = q_addr(it);
         const uint32_t sDO = sQ + Sh::kQTileBytes;
         const uint32_t acc_first = (it == 0) ? 0u : 1u;
-        // the team's P pass of item it: P^T in region A (dV's operand), or,
-        // in the dK pass, S^T read out of region A into registers
-        if (!(ok = bwd_wait(&bars->p_ready[t], ph, abort, kSite + 4))) break;
-        tc_fence_after();
-        if constexpr (kDoDV) {
-          // dV += P^T dO: A = P^T of the team's region (queries [32c, 32c+32)
-          // packed into columns [32c, 32c+16), 16 queries = 8 columns per step)
-#pragma unroll
-          for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
-            umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + Sh::kQRows * t + (kk >> 1) * 32 + (kk & 1) * 8,
-                    mnmajor_q(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
-        }
         const bool more = it + 2 < n_items;
-        if (more) {
-          if (!(ok = wait_q(it + 2))) break;
-          issue_s(it + 2);
+        if (do_a) {
+          // the team's P pass of item it: P^T in region A (dV's operand), or,
+          // in the dK pass, S^T read out of region A into registers
+          if (!(ok = bwd_wait(&bars->p_ready[t], ph, abort, kSite + 4))) break;
+          tc_fence_after();
+          if constexpr (kDoDV) {
+            // dV += P^T dO: A = P^T of the team's region (queries [32c, 32c+32)
+            // packed into columns [32c, 32c+16), 16 queries = 8 columns per step)
+#pragma unroll
+            for (int kk = 0; kk < Sh::kQRows / 16; ++kk)
+              umma_ts(tmem + Sh::kColDV, tmem + Sh::kColA + Sh::kQRows * t + (kk >> 1) * 32 + (kk & 1) * 8,
+                      mnmajor_q(sDO, kk), id_dv, (kk == 0) ? acc_first : 1u);
+          }
+          if (more) {
+            if (!(ok = wait_q(it + 2))) break;
+            issue_s(it + 2);
+          }
         }
-        if constexpr (kDoDK) {
+        if (kDoDK && do_b) {
           // dK += dS^T Q: A = dS^T of the team's region B, packed like P^T
           if (!(ok = bwd_wait(&bars->ds_ready[t], ph, abort, kSite + 5))) break;
           tc_fence_after();
@@ -526,20 +541,24 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
             umma_ts(tmem + Sh::kColDK, tmem + Sh::kColB + Sh::kQRows * t + (kk >> 1) * 32 + (kk & 1) * 8,
                     mnmajor_q(sQ, kk), id_dk, (kk == 0) ? acc_first : 1u);
         }
+        // the slot is free once the readers of it that this thread issued
+        // have run (each issuer commits once)
         umma_commit(&bars->qd_empty[it % Sh::kSlots]);
-        if constexpr (kDoDK) {
-          if (more) issue_dp(it + 2);
+        if (kDoDK && do_b && more) {
+          if (kSplit && !(ok = wait_q(it + 2))) break;
+          issue_dp(it + 2);
         }
       }
       umma_commit(&bars->final_done);
-      umma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, kWaitTimeoutNs, kSite + 12);
+      const int di = kSplit ? warp - 1 : 0;
+      umma_commit(&bars->drain[di]);
+      mbar_wait(&bars->drain[di], 0, kWaitTimeoutNs, kSite + 12);
     }
     __syncwarp();
   } else {
     // ======================= compute teams =======================
-    const int team = (warp - 2) / (4 * Sh::kGroups);
-    const int g = ((warp - 2) >> 2) % Sh::kGroups;  // group within the team
+    const int team = (warp - Sh::kFirst) / (4 * Sh::kGroups);
+    const int g = ((warp - Sh::kFirst) >> 2) % Sh::kGroups;  // group within the team
     const int lane_base = 32 * (warp & 3);
     const int r = lane_base + lane;             // key row within the tile
     const int key = k0 + r;
@@ -672,13 +691,13 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
       if (lane == 0) mbar_arrive(&bars->ds_ready[team]);
     }
 
-    // ---- epilogue: the four groups write the two column halves of the dV
-    // rows (warps 2-9) and of the dK rows (warps 10-17) ----
+    // ---- epilogue: compute group e (four warps from kFirst + 4e) writes
+    // its share of the rows: both accumulators, groups 0-1 the two column
+    // halves of dV and 2-3 those of dK; one accumulator, each of the
+    // 2 kGroups groups its share of the row ----
     if (ok) ok = bwd_wait(&bars->final_done, 0, abort, kSite + 9);
     tc_fence_after();
-    // (both: warps 2-9 write dV, 10-17 dK, each group half of a row; one
-    // accumulator: each of the 2 kGroups groups its share of the row)
-    const int e = (warp - 2) >> 2;
+    const int e = (warp - Sh::kFirst) >> 2;
     const bool is_dk = kPass == kDkdvBoth ? e >= 2 : kPass == kDkOnly;
     void* outp = is_dk ? p.dk : p.dv;
     const uint32_t col = is_dk ? Sh::kColDK : Sh::kColDV;
