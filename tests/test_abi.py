@@ -249,6 +249,7 @@ def test_kvcache_int4_rejects_bad_arguments(fa):
     assert call(D=64) == 2          # int4 decode is D = 128 only
     assert lib.fa_kv_quantize_int4(None, 16, 16, 1, 64, 1, 128, 0, None) == 1
     assert lib.fa_kv_quantize_int4(16, 16, 16, 1, 64, 1, 96, 0, None) == 2
+    assert lib.fa_kv_quantize_int4(16, 16, 16, 1, 64, 1, 64, 0, None) == 2  # nothing reads D = 64
 
 
 def test_valid_call_without_gpu_reports_cuda_error(fa):
