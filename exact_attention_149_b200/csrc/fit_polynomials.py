@@ -2,8 +2,8 @@
 
 A minimax fit (Remez exchange algorithm, minimal maximum *relative* error)
 written for this library: tanh(y) = y * Q(y^2) for |y| <= 0.5, Q of degree 4
-on t = y^2 in [0, 0.25], and of degree 2 for |y| <= 0.25, used for softcap
-when every |y| of a warp's rows is small. The same routine also gives the degree-3 fit of 2^f on [-0.5, 0.5]
+on t = y^2 in [0, 0.25], of degree 2 for |y| <= 0.25 and of degree 1 for
+|y| <= 0.125, used for softcap when every |y| of a warp's rows is small. The same routine also gives the degree-3 fit of 2^f on [-0.5, 0.5]
 (relative error 7.5e-5) that the forward kernel evaluates for a quarter of
 its exponentials (ex2_poly2), moving that share of the work from the
 special-function unit, which bounds the softmax, to the FMA pipe.
@@ -72,6 +72,14 @@ if __name__ == "__main__":
     for k, v in enumerate(c):
         print(f"  q{k} = {v:.9e}f")
     y = np.linspace(-0.25, 0.25, 400001).astype(np.float32)
+    th = (y * horner32(c, (y * y).astype(np.float32))).astype(np.float32)
+    print("  float32 max abs error:", float(np.max(np.abs(th - np.tanh(y.astype(np.float64))))))
+
+    c, e = remez(tanh_ratio, 1, 0.0, 0.015625)
+    print("tanh: Q(t), t = y^2 in [0, 1/64] (|y| <= 1/8); max relative error (float64):", e)
+    for k, v in enumerate(c):
+        print(f"  q{k} = {v:.9e}f")
+    y = np.linspace(-0.125, 0.125, 400001).astype(np.float32)
     th = (y * horner32(c, (y * y).astype(np.float32))).astype(np.float32)
     print("  float32 max abs error:", float(np.max(np.abs(th - np.tanh(y.astype(np.float64))))))
 

@@ -504,16 +504,55 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       bool need_mask = (k0 + 127 >= seq_len);
       if (p.wr >= 0) need_mask |= (k0 + 127 > r_lo + p.wr);
       if (p.wl >= 0) need_mask |= (k0 < r_hi - p.wl);
-      if constexpr (kCap) {
+      // softcap on an unmasked tile whose |scale * s / softcap| are all below
+      // kTanhCubicMax (the common case): tanh is the odd cubic s (b0 + b1 s^2)
+      // with the scale and softcap folded into b0, b1, and its subtraction
+      // of the row's running max fuses into the last FMA below, after the
+      // tile's max, which the cubic, being monotone, takes at the raw max or
+      // min. x keeps the raw scores until then.
+      bool cubic = false;
+      float cb[2];       // folded cubic coefficients
+      float mt_cubic = 0.f;
+      if constexpr (kCap && !alibi) {
+        if (!need_mask) {
+          float hi[4], lo[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) hi[c] = lo[c] = x[c];
+#pragma unroll
+          for (int i = 4; i + 8 <= 128; i += 8) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              hi[c] = max3(hi[c], x[i + c], x[i + 4 + c]);
+              lo[c] = min3(lo[c], x[i + c], x[i + 4 + c]);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            hi[c] = fmaxf(hi[c], x[124 + c]);
+            lo[c] = fminf(lo[c], x[124 + c]);
+          }
+          const float smax = max3(fmaxf(hi[0], hi[1]), hi[2], hi[3]);
+          const float smin = min3(fminf(lo[0], lo[1]), lo[2], lo[3]);
+          cubic = __all_sync(0xffffffffu, fmaxf(smax, -smin) * fabsf(p.cap_in) <= kTanhCubicMax);
+          if (cubic) {
+            fold_tanh(kTanhCubic, p.cap_in, p.cap_out_log2, cb);
+            mt_cubic = fmaxf(smax * fmaf(cb[1], smax * smax, cb[0]), smin * fmaf(cb[1], smin * smin, cb[0]));
+          }
+        }
+      }
+      if (kCap && !cubic) {
         // logits in the exp2 domain: softcap * tanh(scale * s / softcap) * log2(e).
         // When every |scale * s / softcap| of the warp's rows is small, tanh
         // is an FMA-pipe polynomial with the scale and softcap folded into
         // its coefficients (two values per instruction; degree 2 below 1/4,
         // degree 4 below 1/2); otherwise the exp-based identity.
-        float amax = 0.f;
+        float am[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 128; i += 2) amax = max3(amax, fabsf(x[i]), fabsf(x[i + 1]));
-        const float ya = amax * fabsf(p.cap_in);
+        for (int i = 0; i < 128; i += 8) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) am[c] = max3(am[c], fabsf(x[i + c]), fabsf(x[i + 4 + c]));
+        }
+        const float ya = max3(fmaxf(am[0], am[1]), am[2], am[3]) * fabsf(p.cap_in);
         if (__all_sync(0xffffffffu, ya <= kTanhPolyMaxLo)) {
           float pk[3];
           fold_tanh(kTanhLo, p.cap_in, p.cap_out_log2, pk);
@@ -581,7 +620,9 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
         for (int i = 0; i < 128; ++i) x[i] = (i > jmax || i < jmin) ? hide : x[i];
       }
       float mt;
-      if constexpr (lg) {
+      if (cubic) {
+        mt = mt_cubic;
+      } else if constexpr (lg) {
         mt = reduce128<true>(x);
       } else {
         mt = pos ? reduce128<true>(x) : reduce128<false>(x);
@@ -614,12 +655,25 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
       // used so that they pipeline through the special-function unit
       const float2 nb2 = make_float2(-base, -base);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      if (kCap && cubic) {
+        // raw scores: s (b0 + b1 s^2) - base, three packed operations a pair
+        const float2 b0 = make_float2(cb[0], cb[0]), b1 = make_float2(cb[1], cb[1]);
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        const float2 xv = make_float2(x[i], x[i + 1]);
-        const float2 d = lg ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
-        x[i] = d.x;
-        x[i + 1] = d.y;
+        for (int i = 0; i < 128; i += 2) {
+          const float2 xv = make_float2(x[i], x[i + 1]);
+          const float2 q = __ffma2_rn(__fmul2_rn(xv, xv), b1, b0);
+          const float2 d = __ffma2_rn(q, xv, nb2);
+          x[i] = d.x;
+          x[i + 1] = d.y;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; i += 2) {
+          const float2 xv = make_float2(x[i], x[i + 1]);
+          const float2 d = lg ? __fadd2_rn(xv, nb2) : __ffma2_rn(xv, sc2, nb2);
+          x[i] = d.x;
+          x[i + 1] = d.y;
+        }
       }
       // the parts of the row in turn: their exponentials, then their 16-bit
       // P into TMEM and a signal, so that the tensor core starts on the first

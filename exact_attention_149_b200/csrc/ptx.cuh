@@ -429,7 +429,12 @@ __device__ __forceinline__ float2 tanh_poly2(float2 y) {
 // kTanhLo: degree 2 for |a x| <= kTanhPolyMaxLo (Remez, fit_polynomials.py;
 // float64 relative error 4.0e-7, float32 evaluation within 1.1e-7 absolute).
 // kTanhHi: the degree-4 coefficients of tanh_poly2, |a x| <= kTanhPolyMax.
+// kTanhCubic: degree 1 (tanh as an odd cubic) for |a x| <= kTanhCubicMax
+// (Remez, fit_polynomials.py; float64 relative error 4.0e-6, float32
+// evaluation within 5.1e-7 absolute).
 constexpr float kTanhPolyMaxLo = 0.25f;
+constexpr float kTanhCubicMax = 0.125f;
+__device__ constexpr float kTanhCubic[2] = {9.999959588e-01f, -3.312617543e-01f};
 __device__ constexpr float kTanhLo[3] = {9.999996043e-01f, -3.332190823e-01f, 1.284161343e-01f};
 __device__ constexpr float kTanhHi[5] = {9.999999869e-01f, -3.333306939e-01f, 1.332477932e-01f,
                                          -5.298607529e-02f, 1.713500663e-02f};

@@ -62,6 +62,26 @@ def test_fwd_small(cuda_ok, B, S, Hq, Hkv, D, dtype, causal, window, softcap):
     check_fwd(o, lse, o_ref, lse_ref, f"B{B} S{S} H{Hq}/{Hkv} D{D} {dtype}")
 
 
+@pytest.mark.parametrize("q_mult,softcap", [
+    (0.25, 50.0),   # every |scale * s / softcap| below 1/8: the cubic tanh on every tile
+    (1.0, 50.0),    # mostly the cubic, a few tiles on the degree-2 polynomial
+    (1.0, 25.0),    # the degree-2 polynomial (|y| <= 1/4)
+    (1.0, 12.0),    # the degree-4 polynomial (|y| <= 1/2)
+    (1.0, 3.0),     # the exp-based tanh
+])
+def test_fwd_softcap_paths(cuda_ok, q_mult, softcap):
+    """Each way the forward evaluates tanh for softcap (chosen per tile from
+    the largest |scale * s / softcap| of a warp's rows) against the oracle;
+    non-causal S = 512, so no tile is masked and every tile may take the
+    cubic."""
+    inp = W.make_fwd_inputs(1, 512, 4, 4, 128, "bf16", seed=int(softcap * 10 + q_mult * 3))
+    q = (inp["q"].float() * q_mult).to(inp["q"].dtype)
+    scale = 1.0 / math.sqrt(128)
+    o, lse = _run_fwd(q, inp["k"], inp["v"], scale, False, (-1, -1), softcap)
+    o_ref, lse_ref = attention_fwd(q, inp["k"], inp["v"], scale, False, (-1, -1), softcap)
+    check_fwd(o, lse, o_ref, lse_ref, f"softcap {softcap} q x {q_mult}")
+
+
 def test_fwd_deterministic(cuda_ok):
     inp = W.make_fwd_inputs(2, 700, 8, 2, 128, "bf16", seed=5)
     a = _run_fwd(inp["q"], inp["k"], inp["v"], 0.09, True, (-1, -1), 0.0)
