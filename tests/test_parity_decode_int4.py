@@ -167,7 +167,7 @@ def test_int4_decode_alibi(cuda_ok):
     _run_case(st, 3, alibi=W.alibi_slopes(8))
 
 
-@pytest.mark.parametrize("D,dtype,ps", [(128, "bf16", 64), (64, "fp16", 128)])
+@pytest.mark.parametrize("D,dtype,ps", [(128, "bf16", 64), (128, "fp16", 128)])
 def test_kv_quantize_int4_matches_oracle(cuda_ok, D, dtype, ps):
     g = torch.Generator().manual_seed(D + ps + 4)
     x = (torch.randn(5, ps, 3, D, generator=g) * torch.rand(5, ps, 3, 1, generator=g) * 10).to(
@@ -178,6 +178,12 @@ def test_kv_quantize_int4_matches_oracle(cuda_ok, D, dtype, ps):
     rc, rs = quantize_int4(x.double().numpy())
     np.testing.assert_array_equal(codes.cpu().numpy(), pack_int4(rc))
     np.testing.assert_array_equal(scales.cpu().numpy(), np.transpose(rs, (0, 2, 1)))
+
+
+def test_kv_quantize_int4_rejects_head_dim_64(cuda_ok):
+    """The int4 decode reads D = 128 only, so its quantiser takes nothing else."""
+    with pytest.raises(fa.FaError, match="FA_ERR_UNSUPPORTED"):
+        fa.kv_quantize_int4(torch.zeros(2, 64, 2, 64, dtype=torch.bfloat16, device="cuda"))
 
 
 def test_int4_decode_rejects_head_dim_64(cuda_ok):
