@@ -444,6 +444,7 @@ def run_ours(args, dist: Dist):
     res["varlen_fwd"] = {"ms": ms_var, "tflops": vflop / (ms_var * 1e-3) / 1e12, "flop": vflop,
                          "lengths": vin["lengths"]}
     res["varlen_fwd"]["frac_of_bf16_peak"] = res["varlen_fwd"]["tflops"] / peaks["bf16_tflops"]
+    res["varlen_fwd"]["traffic"] = kernel_traffic("fwd_varlen")
     del vq, vk, vv, vout, vlse
 
     # -------------------- FP8 forward on the headline shape --------------------
@@ -471,6 +472,7 @@ def run_ours(args, dist: Dist):
         res["fp8_fwd"]["frac_of_fp8_peak"] = res["fp8_fwd"]["tflops"] / fp8_peak
         if kn:
             res["fp8_fwd"]["kernel_ms_avg"] = kt / kn
+        res["fp8_fwd"]["traffic"] = kernel_traffic("fwd_fp8")
         del q8, k8, v8, o8, l8
     except Exception as e:  # recorded in the line; the headline measurement stands
         res["fp8_fwd"] = {"error": f"{type(e).__name__}: {e}"}
