@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
             const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
             const float2 d2 = h2 == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
             const float2 ds = __fmul2_rn(__fadd2_rn(dp2, d2), make_float2(w[jl + 2 * h2], w[jl + 2 * h2 + 1]));
-            dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
+            dsk[j2] = pack2<kBF16>(ds.x, ds.y);  // one conversion a pair (no ex2 in this pass)
           }
         }
         tmem_st16(t_b, dsk);
@@ -1068,7 +1068,7 @@ __global__ void __launch_bounds__(Dq256Shape<kD>::kThreads, 1)
         for (int j2 = 0; j2 < 16; ++j2) {
           const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
           const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2), make_float2(w[2 * j2], w[2 * j2 + 1]));
-          dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
+          dsk[j2] = pack2<kBF16>(ds.x, ds.y);  // one conversion a pair (no ex2 in this pass)
         }
         // dS of keys [k0, k0 + 32) -> columns [32g, 32g + 16) of S_t
         // (columns this group has already read)
@@ -1421,7 +1421,7 @@ __global__ void __launch_bounds__(DqShape<kD>::kThreads, 1)
         for (int j2 = 0; j2 < 16; ++j2) {
           const float2 dp2 = make_float2(__uint_as_float(dr[2 * j2]), __uint_as_float(dr[2 * j2 + 1]));
           const float2 ds = __fmul2_rn(__fadd2_rn(dp2, nd2), make_float2(w[2 * j2], w[2 * j2 + 1]));
-          dsk[j2] = pack2_alu<kBF16>(ds.x, ds.y);
+          dsk[j2] = pack2<kBF16>(ds.x, ds.y);  // one conversion a pair (no ex2 in this pass)
         }
         // dS of keys [k0, k0 + 32) -> columns [32g, 32g + 16) of the buffer
         tmem_st16(t_dp, dsk);
