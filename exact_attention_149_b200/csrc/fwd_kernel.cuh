@@ -92,13 +92,17 @@ struct FwdShape {
   static constexpr int kThreads = 128 * (1 + kQT);
   // registers of warpgroup 0 (producer, MMA issuer) after setmaxnreg.dec
   // and of the softmax warpgroups after setmaxnreg.inc. With softcap or FP8
-  // the producer/MMA code spills at 88, so those variants move 16 registers
-  // to it (measured: varlen softcap 3% and FP8 1.4% faster; the plain
-  // causal forward 0.5% slower, so it keeps the first split).
+  // the producer/MMA code spills at 88, so those variants move registers to
+  // it (measured against 88/208: FP8 1.4 % faster at 104/200; softcap 3 %
+  // faster at 104/200 and another 1 % at 112/192, where FP8 is 2.7 % slower;
+  // the plain causal forward is 0.5 % slower with either, so it keeps the
+  // first split).
   static constexpr int kRegsLow = 88;
   static constexpr int kRegsHigh = 208;
-  static constexpr int kRegsLowWide = 104;
-  static constexpr int kRegsHighWide = 200;
+  static constexpr int kRegsLowF8 = 104;
+  static constexpr int kRegsHighF8 = 200;
+  static constexpr int kRegsLowCap = 112;
+  static constexpr int kRegsHighCap = 192;
   static constexpr int kTmemCols = 512;
   // of every 8 pairs of exponentials, this many run as a cubic on the FMA
   // pipe instead of the special-function unit (which bounds the softmax)
@@ -300,9 +304,8 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   volatile int* abort = &bars->abort;
-  constexpr bool kWide = kCap || kF8;
-  constexpr int kRegsLow = kWide ? Sh::kRegsLowWide : Sh::kRegsLow;
-  constexpr int kRegsHigh = kWide ? Sh::kRegsHighWide : Sh::kRegsHigh;
+  constexpr int kRegsLow = kCap ? Sh::kRegsLowCap : (kF8 ? Sh::kRegsLowF8 : Sh::kRegsLow);
+  constexpr int kRegsHigh = kCap ? Sh::kRegsHighCap : (kF8 ? Sh::kRegsHighF8 : Sh::kRegsHigh);
   static_assert(Sh::kQT == 1 || Sh::kThreads * 168 >= 128 * kRegsLow + 256 * kRegsHigh,
                 "register split exceeds the launch pool");
   static_assert(kRegsLow % 8 == 0 && kRegsHigh % 8 == 0, "setmaxnreg takes multiples of 8");
