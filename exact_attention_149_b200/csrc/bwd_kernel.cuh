@@ -12,12 +12,15 @@
 //                    (token, query head), into a padded per-row layout.
 //   bwd_dkdv_kernel  one CTA per (sequence, kv head, 128-key tile): K and V
 //                    stay resident while the CTA walks every query head of the
-//                    GQA group and every 128-row Q tile that can see the keys;
-//                    dK and dV accumulate in tensor memory (no atomics).
+//                    GQA group and every 64-row query block that can see the
+//                    keys; dK and dV accumulate in tensor memory (no atomics).
 //   bwd_dq_kernel    one CTA per (sequence, query head, 128-row Q tile): Q and
-//                    dO stay resident while the CTA walks the visible K/V
-//                    tiles; dQ accumulates in tensor memory and is written
-//                    once (no atomics, so the whole backward is deterministic).
+//                    dO stay resident in shared memory while the CTA walks the
+//                    visible 128-key K/V blocks; dQ accumulates in tensor
+//                    memory and is written once (no atomics, so the whole
+//                    backward is deterministic).
+//   bwd_dkdv_pass_kernel, bwd_dq256_kernel: the same two halves at D = 256,
+//                    where the accumulators leave less tensor memory.
 // dS is computed in both kernels (S and dP are recomputed twice): seven
 // 128x128xD products per (query tile, key tile) instead of five, in exchange
 // for no dQ reduction across CTAs and a pipeline with no write-back on the
@@ -738,8 +741,10 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
 }
 
 // ===========================================================================
-// dQ
+// dQ, D = 256 (bwd_dq256_kernel; D = 64 and 128 use bwd_dq_kernel below)
 // ===========================================================================
+// The template keeps the general form of this design (D <= 128 first used
+// it); only D = 256 is instantiated.
 // One CTA per (sequence, query head, 128-row Q tile). Q and dO stay in tensor
 // memory as the A operands of S = Q K^T and dP = dO V^T, so shared memory
 // carries only the streamed K/V blocks; an item is one 64-key block:
@@ -763,6 +768,7 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
 // item is 32 keys and each team has one compute group.
 template <int kD>
 struct Dq256Shape {
+  static_assert(kD == 256, "D <= 128 takes bwd_dq_kernel");
   static constexpr int kChunks = kD / 64;
   static constexpr int kKRows = kD == 256 ? 32 : 64;   // keys per item
   static constexpr int kGroups = kKRows / 32;          // compute groups per team
