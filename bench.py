@@ -220,6 +220,85 @@ def timed(fn, steps, warmup, dist: Dist, sampler: ClockSampler | None = None, fa
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
+def e2e_pipeline(fa, c, inp, have_bwd, steps, dist: Dist):
+    """Milliseconds per step of fwd (+ bwd) through the public API with the
+    inputs copied in from pinned host memory and o, dq, dk, dv copied back,
+    every step, pipelined over two buffer sets (see the caller)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    names = ("q", "k", "v", "do")
+    host_in = {n: inp[n].pin_memory() for n in names}
+    bufs = []
+    for _ in range(2):
+        b = {n: torch.empty_like(inp[n], device=dev) for n in names}
+        b["out"] = torch.empty_like(b["q"])
+        b["lse"] = torch.empty((c.B, c.Hq, c.S), dtype=torch.float32, device=dev)
+        b["dq"], b["dk"], b["dv"] = torch.empty_like(b["q"]), torch.empty_like(b["k"]), torch.empty_like(b["v"])
+        b["ws"] = torch.empty(fa.fa_bwd_workspace_size(c.B, c.Hq, c.S, c.D), dtype=torch.uint8, device=dev)
+        b["h_out"] = torch.empty(b["q"].shape, dtype=b["q"].dtype).pin_memory()
+        b["h_dq"] = torch.empty(b["q"].shape, dtype=b["q"].dtype).pin_memory()
+        b["h_dk"] = torch.empty(b["k"].shape, dtype=b["k"].dtype).pin_memory()
+        b["h_dv"] = torch.empty(b["v"].shape, dtype=b["v"].dtype).pin_memory()
+        for e in ("in_ready", "fwd_done", "done", "out_copied"):
+            b[e] = torch.cuda.Event()
+        bufs.append(b)
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def copy_in(b):
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(b["done"])        # the step that last read these buffers
+            for n in names:
+                b[n].copy_(host_in[n], non_blocking=True)
+            b["in_ready"].record(s_in)
+
+    def run(n_steps):
+        for b in bufs:                        # nothing outstanding on either set
+            b["done"].record(comp)
+            b["out_copied"].record(comp)
+        copy_in(bufs[0])
+        for i in range(n_steps):
+            b = bufs[i % 2]
+            if i + 1 < n_steps:
+                copy_in(bufs[(i + 1) % 2])
+            comp.wait_event(b["in_ready"])
+            comp.wait_event(b["out_copied"])  # its outputs of two steps ago are home
+            fa.fwd(b["q"], b["k"], b["v"], scale=c.scale, causal=True, out=b["out"], lse=b["lse"])
+            b["fwd_done"].record(comp)
+            if have_bwd:
+                fa.bwd(b["q"], b["k"], b["v"], b["out"], b["lse"], b["do"], scale=c.scale, causal=True,
+                       dq=b["dq"], dk=b["dk"], dv=b["dv"], workspace=b["ws"])
+            b["done"].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(b["fwd_done"])
+                b["h_out"].copy_(b["out"], non_blocking=True)
+                if have_bwd:
+                    s_out.wait_event(b["done"])
+                    b["h_dq"].copy_(b["dq"], non_blocking=True)
+                    b["h_dk"].copy_(b["dk"], non_blocking=True)
+                    b["h_dv"].copy_(b["dv"], non_blocking=True)
+                b["out_copied"].record(s_out)
+        for b in bufs:                        # the timed region ends with every copy home
+            comp.wait_event(b["out_copied"])
+
+    run(2)                                    # warm-up
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(comp)
+    run(steps)
+    end.record(comp)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(start.elapsed_time(end) / steps)
+    h2d = sum(host_in[n].numel() * host_in[n].element_size() for n in names)
+    d2h = bufs[0]["h_out"].numel() * 2 + ((bufs[0]["h_dq"].numel() + bufs[0]["h_dk"].numel() +
+                                           bufs[0]["h_dv"].numel()) * 2 if have_bwd else 0)
+    del bufs, host_in
+    return {"unit": "TFLOP/s", "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipeline": "two buffer sets; H2D and D2H on their own streams, overlapping the compute"}
+
+
 def prefill_inputs(dev):
     c = W.CONFIGS[3]
     inp = W.make_fwd_inputs(c.B, c.S, c.Hq, c.Hkv, c.D, c.dtype, seed=1000 + c.cid, with_do=True)
@@ -399,31 +478,16 @@ def run_ours(args, dist: Dist):
         res["alibi_fwd_bwd"]["frac_of_bf16_peak"] = res["alibi_fwd_bwd"]["tflops"] / peaks["bf16_tflops"]
 
     # -------------------- end to end through the public API --------------------
-    hq_, hk_, hv_, hdo_ = (inp[n].pin_memory() for n in ("q", "k", "v", "do"))
-    h_out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    h_dq = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    h_dk = torch.empty(k.shape, dtype=k.dtype).pin_memory()
-    h_dv = torch.empty(v.shape, dtype=v.dtype).pin_memory()
-
-    def step_e2e():
-        q.copy_(hq_, non_blocking=True)
-        k.copy_(hk_, non_blocking=True)
-        v.copy_(hv_, non_blocking=True)
-        do.copy_(hdo_, non_blocking=True)
-        step_fwd()
-        h_out.copy_(out, non_blocking=True)
-        if have_bwd:
-            step_bwd()
-            h_dq.copy_(dq, non_blocking=True)
-            h_dk.copy_(dk, non_blocking=True)
-            h_dv.copy_(dv, non_blocking=True)
-
-    ms_e2e = timed(step_e2e, max(2, args.steps // 2), 1, dist)
-    h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hdo_))
-    d2h = h_out.numel() * 2 + ((h_dq.numel() + h_dk.numel() + h_dv.numel()) * 2 if have_bwd else 0)
-    e2e = {"value": dist.world * flop_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-           "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del hq_, hk_, hv_, hdo_, h_out, h_dq, h_dk, h_dv
+    # A user's training loop: every step copies its inputs in from pinned host
+    # memory and its outputs (o, dq, dk, dv) back, all inside the timed
+    # region. The copies run on their own streams with two sets of device
+    # buffers, so step i+1's inputs and step i's outputs cross PCIe (both
+    # directions at once) while step i computes; the compute stream waits
+    # only for its own step's inputs and for the copy-out of the buffers it
+    # reuses.
+    e2e = e2e_pipeline(fa, c, inp, have_bwd, max(4, args.steps // 2), dist)
+    h2d, d2h = e2e["h2d_bytes_per_step"], e2e["d2h_bytes_per_step"]
+    e2e["value"] = dist.world * flop_step / (e2e["ms_per_step"] * 1e-3) / 1e12
 
     # -------------------- varlen forward (GQA, window, softcap) --------------------
     cv = W.CONFIGS[4]
