@@ -356,6 +356,37 @@ __device__ __forceinline__ void i8x16_to_16bit(const uint4& a, uint4& lo, uint4&
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// 32 int4 codes (16 bytes; byte i holds code 2i + 8 in its low nibble and
+// code 2i + 1 + 8 in its high one) -> 32 exact 16-bit values in d order. For
+// each byte one permute puts it in bytes 0 and 2, one AND/OR against
+// 0x64006400 makes the fp16 pair (1024 + low, 1024 + 16 high), and one
+// packed FMA by (1, 1/16) minus (1032, 72) leaves the two codes (exact).
+// bf16 takes the exact fp16 values through float.
+template <bool kBF16>
+__device__ __forceinline__ void i4x32_to_16bit(const uint4& a, uint4 (&o)[4]) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  const __half2 mul = __halves2half2(__float2half_rn(1.f), __float2half_rn(0.0625f));
+  const __half2 sub = __halves2half2(__float2half_rn(-1032.f), __float2half_rn(-72.f));
+  uint32_t r[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t t = __byte_perm(w[i], 0u, static_cast<uint32_t>(k | (4 << 4) | (k << 8) | (4 << 12)));
+      const uint32_t h = (t & 0x00F0000Fu) | 0x64006400u;
+      const __half2 c = __hfma2(*reinterpret_cast<const __half2*>(&h), mul, sub);
+      if constexpr (kBF16) {
+        const float2 f = __half22float2(c);
+        r[4 * i + k] = pack2<true>(f.x, f.y);
+      } else {
+        r[4 * i + k] = *reinterpret_cast<const uint32_t*>(&c);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) o[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+}
+
 // ---------------------------------------------------------------------------
 // warp-level tensor-core helpers (legacy mma.sync path)
 // ---------------------------------------------------------------------------
@@ -718,7 +749,7 @@ __global__ void __launch_bounds__(160)
     // V: tokens tok0 + 2j + {0, 1, 8, 9}, bytes d = 16r .. 16r + 15. Rows are
     // 128 bytes with the 16-byte group g stored at g ^ (row & 7).
     uint32_t kw[2][8], vw[4][4];
-    if constexpr (kQ4) {
+    if constexpr (kQ4 && Sh::kDirect) {
       // int4 rows are 64 bytes, written by TMA with the 64-byte swizzle (the
       // 16-byte group g of row t at g ^ ((t >> 1) & 3)). Fragment row / k
       // index m of the warp's 16 tokens is token tok0 + i4_token(m), so that
@@ -784,6 +815,38 @@ __global__ void __launch_bounds__(160)
       __syncwarp();
       // everything this warp needs from the slot is in registers
       if (lane == 0) mbar_arrive(&bars->empty[slot]);
+    } else if constexpr (kQ4) {
+      // int4 at D = 64: 32-byte rows, unswizzled; lane = (row r, half u)
+      // converts values 32u .. 32u + 31 of its row into the 16-bit groups
+      // 4u .. 4u + 3 of the swizzled 128-byte scratch row
+      static_assert(kD == 64, "the int4 scratch path is written for D = 64");
+      const uint8_t* kq = smem + slot * Sh::kStageBytes + tok0 * Sh::kRowBytes;
+      const uint8_t* vq = kq + Sh::kKVBytes;
+      uint8_t* ks = smem + Sh::kScrOffset + warp * 2 * Sh::kScrHalfBytes;
+      uint8_t* vs = ks + Sh::kScrHalfBytes;
+      {
+        const int r = lane >> 1, u = lane & 1;
+        uint4 o[4];
+        i4x32_to_16bit<kBF16>(*reinterpret_cast<const uint4*>(kq + r * Sh::kRowBytes + u * 16), o);
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          *reinterpret_cast<uint4*>(ks + r * 128 + (((4 * u + g) ^ (r & 7)) << 4)) = o[g];
+        i4x32_to_16bit<false>(*reinterpret_cast<const uint4*>(vq + r * Sh::kRowBytes + u * 16), o);
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          *reinterpret_cast<uint4*>(vs + r * 128 + (((4 * u + g) ^ (r & 7)) << 4)) = o[g];
+      }
+      // the row scales of this lane's accumulator rows (tokens lane / 4, + 8)
+      const float* sc = reinterpret_cast<const float*>(smem + slot * Sh::kStageBytes + Sh::kScaleOffset);
+      ksc0 = sc[tok0 + (lane >> 2)];
+      ksc1 = sc[tok0 + (lane >> 2) + 8];
+      vsc0 = sc[Sh::kTok + tok0 + (lane >> 2)];
+      vsc1 = sc[Sh::kTok + tok0 + (lane >> 2) + 8];
+      __syncwarp();
+      // everything this warp needs from the slot is copied out
+      if (lane == 0) mbar_arrive(&bars->empty[slot]);
+      kbase = smem_u32(ks);
+      vbase = smem_u32(vs);
     } else if constexpr (kQuant) {
       const uint8_t* kq = smem + slot * Sh::kStageBytes + tok0 * kD;
       const uint8_t* vq = kq + Sh::kKVBytes;
@@ -820,7 +883,7 @@ __global__ void __launch_bounds__(160)
     float s[kNT][4];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-    if constexpr (kQ4) {
+    if constexpr (kQ4 && Sh::kDirect) {
       // A = K codes as exact fp16, nibbles (i, i + 4) and (i + 1, i + 5) of
       // word kk / 2, i = 2 (kk % 2) (the permutation of the query fragments)
 #pragma unroll
@@ -858,7 +921,7 @@ __global__ void __launch_bounds__(160)
     // ---- logits, mask, online softmax ----
     const int wtok = (t_begin + i) * Sh::kTok + tok0;  // first token of this warp's 16
     // token of s[.][0], s[.][1] (s[.][2], s[.][3]: + 8)
-    const int pos0 = wtok + (kQ4 ? i4_token(lane >> 2) : (lane >> 2));
+    const int pos0 = wtok + ((kQ4 && Sh::kDirect) ? i4_token(lane >> 2) : (lane >> 2));
     // every column sees all 16 tokens: no mask (warp-uniform)
     const bool all_visible = wtok >= lo_in && wtok + 16 <= hi_in;
     float vr = 1.f;
@@ -956,7 +1019,7 @@ __global__ void __launch_bounds__(160)
       }
     }
     // ---- O^T += V^T P^T ----
-    if constexpr (kQ4) {
+    if constexpr (kQ4 && Sh::kDirect) {
       // A = V^T codes as exact fp16; accumulator rows r, r + 8 of step mt are
       // d = 16r + 2mt and 16r + 2mt + 1, the low and high nibble of byte mt of
       // this lane's V words; byte b of tokens 2j, 2j+1 (2j+8, 2j+9) is brought
@@ -1045,7 +1108,7 @@ __global__ void __launch_bounds__(160)
       red_l[warp * kH + h0 + 1] = l1;
     }
     const float oc = kQuant ? vC : 1.f;  // int8 / int4: acc holds O / vC
-    const float oc1 = kQ4 ? oc * 0.0625f : oc;  // int4: rows d1 hold 16 O / vC
+    const float oc1 = (kQ4 && Sh::kDirect) ? oc * 0.0625f : oc;  // int4, D = 128: rows d1 hold 16 O / vC
 #pragma unroll
     for (int mt = 0; mt < kD / 16; ++mt) {
       // accumulator rows lane / 4 and lane / 4 + 8 of step mt

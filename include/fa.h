@@ -299,8 +299,8 @@ FA_API fa_status fa_kv_quantize_int8(const void* src, int8_t* codes, float* scal
  * per byte biased by 8, the code of even d in the low nibble.
  *   k_cache, v_cache: DEVICE uint8 (num_pages, page_size, Hkv, D / 2).
  *   k_scale, v_scale: as fa_fwd_kvcache_int8.
- * Everything else as fa_fwd_kvcache_int8; D must be 128 (FA_ERR_UNSUPPORTED
- * otherwise).
+ * Everything else as fa_fwd_kvcache_int8; D must be 64 or 128
+ * (FA_ERR_UNSUPPORTED otherwise).
  */
 FA_API fa_status fa_fwd_kvcache_int4(const void* q, const void* k_new, const void* v_new,
                                      uint8_t* k_cache, uint8_t* v_cache, float* k_scale,

@@ -246,10 +246,11 @@ def test_kvcache_int4_rejects_bad_arguments(fa):
 
     assert call(ks=None) == 1
     assert call(kc=None) == 1
-    assert call(D=64) == 2          # int4 decode is D = 128 only
+    assert call(D=256) == 2         # int4 decode is D = 64 or 128
+    assert call(D=96) == 2
     assert lib.fa_kv_quantize_int4(None, 16, 16, 1, 64, 1, 128, 0, None) == 1
     assert lib.fa_kv_quantize_int4(16, 16, 16, 1, 64, 1, 96, 0, None) == 2
-    assert lib.fa_kv_quantize_int4(16, 16, 16, 1, 64, 1, 64, 0, None) == 2  # nothing reads D = 64
+    assert lib.fa_kv_quantize_int4(16, 16, 16, 1, 64, 1, 256, 0, None) == 2
 
 
 def test_valid_call_without_gpu_reports_cuda_error(fa):

@@ -115,6 +115,9 @@ def _run_case(st, splits, causal=True, window=(-1, -1), softcap=0.0, append=True
     (2, 8, 1, 128, "bf16", [1000, 1], 256),       # MQA, group 8
     (5, 32, 8, 128, "bf16", [1024, 3000, 4095, 4096, 2047], 256),
     (3, 8, 2, 128, "fp16", [0, 300, 1000], 128),
+    (3, 8, 2, 64, "bf16", [5, 64, 200], 64),      # D = 64: the shared-memory scratch path
+    (2, 8, 1, 64, "fp16", [1000, 1], 256),
+    (5, 32, 8, 64, "bf16", [1024, 3000, 4095, 4096, 2047], 256),
 ])
 def test_int4_decode_small(cuda_ok, B, Hq, Hkv, D, dtype, lengths, ps, splits):
     st = W.make_decode_structure(B, Hq, Hkv, D, 0, max(lengths), ps, dtype,
@@ -167,7 +170,7 @@ def test_int4_decode_alibi(cuda_ok):
     _run_case(st, 3, alibi=W.alibi_slopes(8))
 
 
-@pytest.mark.parametrize("D,dtype,ps", [(128, "bf16", 64), (128, "fp16", 128)])
+@pytest.mark.parametrize("D,dtype,ps", [(128, "bf16", 64), (64, "fp16", 128)])
 def test_kv_quantize_int4_matches_oracle(cuda_ok, D, dtype, ps):
     g = torch.Generator().manual_seed(D + ps + 4)
     x = (torch.randn(5, ps, 3, D, generator=g) * torch.rand(5, ps, 3, 1, generator=g) * 10).to(
@@ -180,16 +183,23 @@ def test_kv_quantize_int4_matches_oracle(cuda_ok, D, dtype, ps):
     np.testing.assert_array_equal(scales.cpu().numpy(), np.transpose(rs, (0, 2, 1)))
 
 
-def test_kv_quantize_int4_rejects_head_dim_64(cuda_ok):
-    """The int4 decode reads D = 128 only, so its quantiser takes nothing else."""
-    with pytest.raises(fa.FaError, match="FA_ERR_UNSUPPORTED"):
-        fa.kv_quantize_int4(torch.zeros(2, 64, 2, 64, dtype=torch.bfloat16, device="cuda"))
+@pytest.mark.parametrize("D,opts", [(64, dict(window=(30, 0), softcap=20.0)), (64, dict(causal=False))])
+def test_int4_decode_head_dim_64_options(cuda_ok, D, opts):
+    st = W.make_decode_structure(3, 8, 2, D, 0, 700, 64, "bf16", seed=191 + D,
+                                 cache_seqlens=[700, 65, 130], sq=2)
+    _run_case(st, 3, **opts)
 
 
-def test_int4_decode_rejects_head_dim_64(cuda_ok):
+def test_int4_decode_head_dim_64_rotary_alibi(cuda_ok):
+    st = W.make_decode_structure(2, 8, 2, 64, 0, 400, 64, "bf16", seed=197,
+                                 cache_seqlens=[400, 33], sq=2)
+    _run_case(st, 2, rotary_dim=64, alibi=W.alibi_slopes(8))
+
+
+def test_int4_decode_rejects_head_dim_256(cuda_ok):
     dev = torch.device("cuda")
-    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16, device=dev)
-    kc = torch.zeros(2, 64, 2, 32, dtype=torch.uint8, device=dev)
+    q = torch.zeros(1, 1, 4, 256, dtype=torch.bfloat16, device=dev)
+    kc = torch.zeros(2, 64, 2, 128, dtype=torch.uint8, device=dev)
     sc = torch.zeros(2, 2, 64, device=dev)
     with pytest.raises(fa.FaError, match="FA_ERR_UNSUPPORTED"):
         fa.fwd_kvcache(q, kc, kc.clone(), torch.zeros(1, dtype=torch.int32, device=dev),
