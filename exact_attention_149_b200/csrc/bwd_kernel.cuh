@@ -93,60 +93,79 @@ __device__ __forceinline__ size_t vec_index(const BwdParams& p, int h, int b, in
 
 // ---------------------------------------------------------------------------
 // pre: Drow = rowsum(dO * O) and -LSE in the exp2 domain, both into the padded
-// layout. One warp per (token, head) row.
+// layout. kLanes lanes per (token, head) row, 16 bytes of O and of dO each
+// (D = 128: two rows per warp at a time); each lane group takes two rows,
+// whose loads are issued together. Index arithmetic is 32-bit: the host
+// keeps total * Hq below 2^31.
 // ---------------------------------------------------------------------------
+template <int kD>
+struct PreShape {
+  static constexpr int kLanes = kD / 8;
+  static constexpr int kRowsPerWarp = 32 / kLanes;
+  static constexpr int kIter = 2;                        // rows per lane group
+  static constexpr int kRowsPerWarpAll = kRowsPerWarp * kIter;
+};
+
 template <int kD, bool kBF16>
 __global__ void bwd_pre_kernel(const BwdParams p) {
-  // kLanes lanes per (token, head) row, 16 bytes of O and of dO each: D = 128
-  // puts two rows in a warp, so every load is a 16-byte one
-  constexpr int kLanes = kD / 8;
-  constexpr int kRowsPerWarp = 32 / kLanes;
-  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  using Sh = PreShape<kD>;
+  const uint32_t rows = static_cast<uint32_t>(p.total) * static_cast<uint32_t>(p.Hq);
+  const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (gw * Sh::kRowsPerWarpAll >= rows) return;  // uniform across the warp
   const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(p.total) * p.Hq;
-  if (gw * kRowsPerWarp >= rows) return;  // uniform across the warp
-  const long long row = gw * kRowsPerWarp + lane / kLanes;
-  const int li = lane % kLanes;
-  float acc = 0.f;
-  if (row < rows) {
-    const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + row * kD + li * 8);
-    const uint4 dv = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + row * kD + li * 8);
-    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+  const int li = lane % Sh::kLanes;
+  const uint32_t row0 = gw * Sh::kRowsPerWarpAll + lane / Sh::kLanes;
+  uint4 ov[Sh::kIter], dv[Sh::kIter];
+#pragma unroll
+  for (int k = 0; k < Sh::kIter; ++k) {
+    const uint32_t row = row0 + k * Sh::kRowsPerWarp;
+    ov[k] = dv[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (row < rows) {
+      const size_t e = static_cast<size_t>(row) * kD + li * 8;
+      ov[k] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + e);
+      dv[k] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + e);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < Sh::kIter; ++k) {
+    const uint32_t ow[4] = {ov[k].x, ov[k].y, ov[k].z, ov[k].w}, dw[4] = {dv[k].x, dv[k].y, dv[k].z, dv[k].w};
+    float acc = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 o2 = unpack2<kBF16>(ow[i]), d2 = unpack2<kBF16>(dw[i]);
       acc = fmaf(o2.x, d2.x, fmaf(o2.y, d2.y, acc));
     }
-  }
 #pragma unroll
-  for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  const int tok = static_cast<int>(row / p.Hq);
-  const int h = static_cast<int>(row % p.Hq);
-  if (li == 0 && row < rows) {
-    size_t lidx;
-    int b, seq_start;
-    if (p.cu_seqlens != nullptr) {
-      // the sequence holding tok: the largest b with cu_seqlens[b] <= tok
-      int lo = 0, hi = p.B - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.cu_seqlens[mid] <= tok)
-          lo = mid;
-        else
-          hi = mid - 1;
+    for (int off = Sh::kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    const uint32_t row = row0 + k * Sh::kRowsPerWarp;
+    if (li == 0 && row < rows) {
+      const int tok = static_cast<int>(row / static_cast<uint32_t>(p.Hq));
+      const int h = static_cast<int>(row - static_cast<uint32_t>(tok) * static_cast<uint32_t>(p.Hq));
+      size_t lidx;
+      int b, seq_start;
+      if (p.cu_seqlens != nullptr) {
+        // the sequence holding tok: the largest b with cu_seqlens[b] <= tok
+        int lo = 0, hi = p.B - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (p.cu_seqlens[mid] <= tok)
+            lo = mid;
+          else
+            hi = mid - 1;
+        }
+        b = lo;
+        seq_start = p.cu_seqlens[b];
+        lidx = static_cast<size_t>(h) * p.total + tok;
+      } else {
+        b = tok / p.S;
+        seq_start = b * p.S;
+        lidx = (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
       }
-      b = lo;
-      seq_start = p.cu_seqlens[b];
-      lidx = static_cast<size_t>(h) * p.total + tok;
-    } else {
-      b = tok / p.S;
-      seq_start = b * p.S;
-      lidx = (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
+      const float l = p.lse[lidx];
+      const size_t vi = vec_index(p, h, b, seq_start, tok - seq_start);
+      p.vec_nlse[vi] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+      p.vec_drow[vi] = acc;
     }
-    const float l = p.lse[lidx];
-    const size_t vi = vec_index(p, h, b, seq_start, tok - seq_start);
-    p.vec_nlse[vi] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
-    p.vec_drow[vi] = acc;
   }
 }
 
