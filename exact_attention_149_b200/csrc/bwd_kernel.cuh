@@ -95,8 +95,8 @@ __device__ __forceinline__ size_t vec_index(const BwdParams& p, int h, int b, in
 // pre: Drow = rowsum(dO * O) and -LSE in the exp2 domain, both into the padded
 // layout. kLanes lanes per (token, head) row, 16 bytes of O and of dO each
 // (D = 128: two rows per warp at a time); each lane group takes two rows,
-// whose loads are issued together. Index arithmetic is 32-bit: the host
-// keeps total * Hq below 2^31.
+// whose loads are issued together. Rows are numbered head-major. Index
+// arithmetic is 32-bit: the host keeps total * Hq below 2^31.
 // ---------------------------------------------------------------------------
 template <int kD>
 struct PreShape {
@@ -121,7 +121,9 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
     const uint32_t row = row0 + k * Sh::kRowsPerWarp;
     ov[k] = dv[k] = make_uint4(0u, 0u, 0u, 0u);
     if (row < rows) {
-      const size_t e = static_cast<size_t>(row) * kD + li * 8;
+      const uint32_t h = row / static_cast<uint32_t>(p.total);
+      const uint32_t tok = row - h * static_cast<uint32_t>(p.total);
+      const size_t e = (static_cast<size_t>(tok) * p.Hq + h) * kD + li * 8;
       ov[k] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + e);
       dv[k] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + e);
     }
@@ -139,8 +141,11 @@ __global__ void bwd_pre_kernel(const BwdParams p) {
     for (int off = Sh::kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     const uint32_t row = row0 + k * Sh::kRowsPerWarp;
     if (li == 0 && row < rows) {
-      const int tok = static_cast<int>(row / static_cast<uint32_t>(p.Hq));
-      const int h = static_cast<int>(row - static_cast<uint32_t>(tok) * static_cast<uint32_t>(p.Hq));
+      // rows run head-major (row = h * total + tok), so that consecutive
+      // rows write consecutive entries of the padded vectors and read
+      // consecutive LSE values
+      const int h = static_cast<int>(row / static_cast<uint32_t>(p.total));
+      const int tok = static_cast<int>(row - static_cast<uint32_t>(h) * static_cast<uint32_t>(p.total));
       size_t lidx;
       int b, seq_start;
       if (p.cu_seqlens != nullptr) {
