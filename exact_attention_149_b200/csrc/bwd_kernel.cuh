@@ -400,6 +400,26 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
   const int i_begin = q_lo / Sh::kQRows;
   const int i_cnt = q_hi >= q_lo ? q_hi / Sh::kQRows + 1 - i_begin : 0;
   const int n_items = i_cnt * p.group;  // (head, 64-row query block) pairs
+  // item it's Q and dO tiles and row vectors into ring slot it % kSlots
+  auto load_qd = [&](int it) {
+    const int slot = it % Sh::kSlots;
+    const int h = kvh * p.group + it / i_cnt;
+    const int q0 = (i_begin + it % i_cnt) * Sh::kQRows;
+    const int tok = seq_start + q0;
+    uint8_t* dst = smem + Sh::kOffQ + slot * 2 * Sh::kQTileBytes;
+    uint8_t* vdst = smem + Sh::kOffVec + slot * Sh::kVecBytes;
+    const size_t vi = vec_index(p, h, b, seq_start, q0);
+    mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kQTileBytes + Sh::kVecBytes);
+    for (int c = 0; c < Sh::kChunks; ++c) {
+      tma_load_3d(&tm_q, &bars->qd_full[slot], dst + c * Sh::kQChunkBytes, c * 64, h, tok);
+      tma_load_3d(&tm_do, &bars->qd_full[slot], dst + Sh::kQTileBytes + c * Sh::kQChunkBytes, c * 64,
+                  h, tok);
+    }
+    // the rows' vectors (rows past the sequence end hold stale values; the
+    // compute groups mask those columns)
+    bulk_load(vdst, p.vec_nlse + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
+    bulk_load(vdst + Sh::kVecBytes / 2, p.vec_drow + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -417,6 +437,21 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
     mbar_init(&bars->final_done, Sh::kIssuers);
     bars->abort = 0;
     fence_mbar_init();
+    // the key block and the first item are requested here, so that their
+    // latency overlaps the TMEM allocation and the block sync below
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+    mbar_arrive_expect_tx(&bars->kv_full, (Sh::kNeedV ? 2 : 1) * Sh::kTileBytes);
+    for (int c = 0; c < Sh::kChunks; ++c) {
+      tma_load_3d(&tm_k, &bars->kv_full, smem + Sh::kOffK + c * Sh::kChunkBytes, c * 64, kvh,
+                  seq_start + k0);
+      if constexpr (Sh::kNeedV)
+        tma_load_3d(&tm_v, &bars->kv_full, smem + Sh::kOffV + c * Sh::kChunkBytes, c * 64, kvh,
+                    seq_start + k0);
+    }
+    if (n_items > 0) load_qd(0);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, Sh::kTmemCols);
@@ -431,39 +466,13 @@ __global__ void __launch_bounds__(DkdvShape<kD, kPass>::kThreads, 1)
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (elect_one()) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&bars->kv_full, (Sh::kNeedV ? 2 : 1) * Sh::kTileBytes);
-      for (int c = 0; c < Sh::kChunks; ++c) {
-        tma_load_3d(&tm_k, &bars->kv_full, smem + Sh::kOffK + c * Sh::kChunkBytes, c * 64, kvh,
-                    seq_start + k0);
-        if constexpr (Sh::kNeedV)
-          tma_load_3d(&tm_v, &bars->kv_full, smem + Sh::kOffV + c * Sh::kChunkBytes, c * 64, kvh,
-                      seq_start + k0);
-      }
-      int it = 0;
+      // (the key block and item 0 were requested at setup)
+      int it = n_items > 0 ? 1 : 0;
       for (; it < n_items && !*abort; ++it) {
         const int slot = it % Sh::kSlots;
         const uint32_t ph = static_cast<uint32_t>(it / Sh::kSlots) & 1u;
         if (!bwd_wait(&bars->qd_empty[slot], ph ^ 1u, abort, kSite + 1)) break;
-        const int h = kvh * p.group + it / i_cnt;
-        const int q0 = (i_begin + it % i_cnt) * Sh::kQRows;
-        const int tok = seq_start + q0;
-        uint8_t* dst = smem + Sh::kOffQ + slot * 2 * Sh::kQTileBytes;
-        uint8_t* vdst = smem + Sh::kOffVec + slot * Sh::kVecBytes;
-        const size_t vi = vec_index(p, h, b, seq_start, q0);
-        mbar_arrive_expect_tx(&bars->qd_full[slot], 2 * Sh::kQTileBytes + Sh::kVecBytes);
-        for (int c = 0; c < Sh::kChunks; ++c) {
-          tma_load_3d(&tm_q, &bars->qd_full[slot], dst + c * Sh::kQChunkBytes, c * 64, h, tok);
-          tma_load_3d(&tm_do, &bars->qd_full[slot], dst + Sh::kQTileBytes + c * Sh::kQChunkBytes,
-                      c * 64, h, tok);
-        }
-        // the rows' vectors (rows past the sequence end hold stale values;
-        // the compute groups mask those columns)
-        bulk_load(vdst, p.vec_nlse + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
-        bulk_load(vdst + Sh::kVecBytes / 2, p.vec_drow + vi, Sh::kVecBytes / 2, &bars->qd_full[slot]);
+        load_qd(it);
       }
       for (int f = max(0, it - Sh::kSlots); f < it; ++f)
         mbar_wait(&bars->qd_full[f % Sh::kSlots], static_cast<uint32_t>(f / Sh::kSlots) & 1u, kWaitTimeoutNs, kSite + 10);
