@@ -93,84 +93,110 @@ __device__ __forceinline__ size_t vec_index(const BwdParams& p, int h, int b, in
 
 // ---------------------------------------------------------------------------
 // pre: Drow = rowsum(dO * O) and -LSE in the exp2 domain, both into the padded
-// layout. kLanes lanes per (token, head) row, 16 bytes of O and of dO each
-// (D = 128: two rows per warp at a time); each lane group takes two rows,
-// whose loads are issued together. Rows are numbered head-major. Index
-// arithmetic is 32-bit: the host keeps total * Hq below 2^31.
+// layout. A block takes tpb consecutive tokens with all their heads
+// (tpb * Hq rows of the (token, head)-major O and dO, one contiguous range) and
+// reads them in order: kLanes lanes per row, 16 bytes of O and of dO each,
+// kIter rows per lane group with their loads issued together. The row sums go
+// to shared memory; the block then writes both vectors head by head, tpb
+// consecutive entries each. Index arithmetic is 32-bit within a block.
 // ---------------------------------------------------------------------------
 template <int kD>
 struct PreShape {
+  static constexpr int kThreads = 256;
   static constexpr int kLanes = kD / 8;
-  static constexpr int kRowsPerWarp = 32 / kLanes;
-  static constexpr int kIter = 2;                        // rows per lane group
-  static constexpr int kRowsPerWarpAll = kRowsPerWarp * kIter;
+  static constexpr int kRowsPerWarp = 32 / kLanes;  // rows a warp reads at a time
+  static constexpr int kIter = 4;                   // of those, per lane group in flight
 };
+constexpr int kPreRowsPerBlock = 512;  // rows a block covers (at least one token)
+constexpr int kPreMaxHeads = 8192;     // keeps one token's row sums within 48 KB of shared memory
+
+// tokens per block, and the dynamic shared memory that takes
+inline int pre_tokens_per_block(int Hq) { return Hq >= kPreRowsPerBlock ? 1 : kPreRowsPerBlock / Hq; }
+inline size_t pre_smem_bytes(int Hq) {
+  const int tpb = pre_tokens_per_block(Hq);
+  return (static_cast<size_t>(tpb) * Hq + 2 * static_cast<size_t>(tpb)) * sizeof(float);
+}
 
 template <int kD, bool kBF16>
-__global__ void bwd_pre_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(PreShape<kD>::kThreads) bwd_pre_kernel(const BwdParams p, int tpb) {
   using Sh = PreShape<kD>;
-  const uint32_t rows = static_cast<uint32_t>(p.total) * static_cast<uint32_t>(p.Hq);
-  const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (gw * Sh::kRowsPerWarpAll >= rows) return;  // uniform across the warp
-  const int lane = threadIdx.x & 31;
+  extern __shared__ float pre_smem[];
+  const int tok0 = static_cast<int>(blockIdx.x) * tpb;
+  const int ntok = min(tpb, p.total - tok0);
+  const uint32_t nrows = static_cast<uint32_t>(ntok) * static_cast<uint32_t>(p.Hq);
+  float* s_acc = pre_smem;                                    // [ntok][Hq]
+  int* s_b = reinterpret_cast<int*>(pre_smem + static_cast<size_t>(tpb) * p.Hq);  // sequence of a token
+  int* s_start = s_b + tpb;                                   // and its first token
+  for (int tl = threadIdx.x; tl < ntok; tl += Sh::kThreads) {
+    const int tok = tok0 + tl;
+    int b;
+    if (p.cu_seqlens != nullptr) {
+      // the largest b with cu_seqlens[b] <= tok
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cu_seqlens[mid] <= tok)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      b = lo;
+      s_start[tl] = p.cu_seqlens[b];
+    } else {
+      b = tok / p.S;
+      s_start[tl] = b * p.S;
+    }
+    s_b[tl] = b;
+  }
+  // ---- row sums, reading the block's range in order ----
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int li = lane % Sh::kLanes;
-  const uint32_t row0 = gw * Sh::kRowsPerWarpAll + lane / Sh::kLanes;
-  uint4 ov[Sh::kIter], dv[Sh::kIter];
+  constexpr uint32_t kWarpRows = Sh::kRowsPerWarp * Sh::kIter;
+  constexpr uint32_t kStride = kWarpRows * (Sh::kThreads / 32);
+  const uint16_t* o_blk = static_cast<const uint16_t*>(p.o) + static_cast<size_t>(tok0) * p.Hq * kD;
+  const uint16_t* d_blk = static_cast<const uint16_t*>(p.dout) + static_cast<size_t>(tok0) * p.Hq * kD;
+  // (the loop bound depends on the warp only, so every lane takes part in
+  // the shuffles)
+  for (uint32_t rb = warp * kWarpRows; rb < nrows; rb += kStride) {
+    uint4 ov[Sh::kIter], dv[Sh::kIter];
 #pragma unroll
-  for (int k = 0; k < Sh::kIter; ++k) {
-    const uint32_t row = row0 + k * Sh::kRowsPerWarp;
-    ov[k] = dv[k] = make_uint4(0u, 0u, 0u, 0u);
-    if (row < rows) {
-      const uint32_t h = row / static_cast<uint32_t>(p.total);
-      const uint32_t tok = row - h * static_cast<uint32_t>(p.total);
-      const size_t e = (static_cast<size_t>(tok) * p.Hq + h) * kD + li * 8;
-      ov[k] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.o) + e);
-      dv[k] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.dout) + e);
+    for (int k = 0; k < Sh::kIter; ++k) {
+      const uint32_t r = rb + k * Sh::kRowsPerWarp + lane / Sh::kLanes;
+      ov[k] = dv[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < nrows) {
+        ov[k] = *reinterpret_cast<const uint4*>(o_blk + r * kD + li * 8);
+        dv[k] = *reinterpret_cast<const uint4*>(d_blk + r * kD + li * 8);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < Sh::kIter; ++k) {
+      const uint32_t ow[4] = {ov[k].x, ov[k].y, ov[k].z, ov[k].w}, dw[4] = {dv[k].x, dv[k].y, dv[k].z, dv[k].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 o2 = unpack2<kBF16>(ow[i]), d2 = unpack2<kBF16>(dw[i]);
+        acc = fmaf(o2.x, d2.x, fmaf(o2.y, d2.y, acc));
+      }
+#pragma unroll
+      for (int off = Sh::kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const uint32_t r = rb + k * Sh::kRowsPerWarp + lane / Sh::kLanes;
+      if (li == 0 && r < nrows) s_acc[r] = acc;
     }
   }
-#pragma unroll
-  for (int k = 0; k < Sh::kIter; ++k) {
-    const uint32_t ow[4] = {ov[k].x, ov[k].y, ov[k].z, ov[k].w}, dw[4] = {dv[k].x, dv[k].y, dv[k].z, dv[k].w};
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 o2 = unpack2<kBF16>(ow[i]), d2 = unpack2<kBF16>(dw[i]);
-      acc = fmaf(o2.x, d2.x, fmaf(o2.y, d2.y, acc));
-    }
-#pragma unroll
-    for (int off = Sh::kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    const uint32_t row = row0 + k * Sh::kRowsPerWarp;
-    if (li == 0 && row < rows) {
-      // rows run head-major (row = h * total + tok), so that consecutive
-      // rows write consecutive entries of the padded vectors and read
-      // consecutive LSE values
-      const int h = static_cast<int>(row / static_cast<uint32_t>(p.total));
-      const int tok = static_cast<int>(row - static_cast<uint32_t>(h) * static_cast<uint32_t>(p.total));
-      size_t lidx;
-      int b, seq_start;
-      if (p.cu_seqlens != nullptr) {
-        // the sequence holding tok: the largest b with cu_seqlens[b] <= tok
-        int lo = 0, hi = p.B - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (p.cu_seqlens[mid] <= tok)
-            lo = mid;
-          else
-            hi = mid - 1;
-        }
-        b = lo;
-        seq_start = p.cu_seqlens[b];
-        lidx = static_cast<size_t>(h) * p.total + tok;
-      } else {
-        b = tok / p.S;
-        seq_start = b * p.S;
-        lidx = (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
-      }
-      const float l = p.lse[lidx];
-      const size_t vi = vec_index(p, h, b, seq_start, tok - seq_start);
-      p.vec_nlse[vi] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
-      p.vec_drow[vi] = acc;
-    }
+  __syncthreads();
+  // ---- both vectors, head by head: consecutive threads take consecutive
+  // tokens of one head ----
+  for (uint32_t i = threadIdx.x; i < nrows; i += Sh::kThreads) {
+    const int h = static_cast<int>(i / static_cast<uint32_t>(ntok));
+    const int tl = static_cast<int>(i - static_cast<uint32_t>(h) * static_cast<uint32_t>(ntok));
+    const int tok = tok0 + tl, b = s_b[tl], seq_start = s_start[tl];
+    const size_t lidx = p.cu_seqlens != nullptr
+                            ? static_cast<size_t>(h) * p.total + tok
+                            : (static_cast<size_t>(b) * p.Hq + h) * p.S + (tok - seq_start);
+    const float l = p.lse[lidx];
+    const size_t vi = vec_index(p, h, b, seq_start, tok - seq_start);
+    p.vec_nlse[vi] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+    p.vec_drow[vi] = s_acc[static_cast<uint32_t>(tl) * static_cast<uint32_t>(p.Hq) + h];
   }
 }
 
