@@ -44,6 +44,10 @@ SMALL = [
     (2, 512, 16, 16, 64, "fp16", True, (-1, -1), 0.0),    # B2 H16 S512 D64 fp16
     (1, 1, 2, 1, 128, "bf16", True, (-1, -1), 0.0),       # a single token
     (1, 1030, 4, 1, 128, "fp16", True, (-1, -1), 0.0),    # many Q tiles per key tile
+    # the pre pass takes 512 / Hq whole tokens a block: 85 tokens at Hq = 6
+    # (blocks of 85, 85, 85, 45), one token at Hq = 520 (GQA group 65)
+    (1, 300, 6, 2, 64, "bf16", True, (-1, -1), 0.0),
+    (1, 40, 520, 8, 64, "bf16", False, (-1, -1), 0.0),
     # head dim 256: a dV pass and a dK pass of 32-row items, dQ with dO in
     # shared memory and 32-key blocks
     (1, 300, 2, 2, 256, "bf16", True, (-1, -1), 0.0),     # causal, ragged
