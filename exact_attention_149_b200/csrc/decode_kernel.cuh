@@ -441,11 +441,11 @@ __device__ __forceinline__ uint32_t sw128(uint32_t base, int r, int g) {
 
 // kQuant: the ring holds int8 / int4 chunks (K codes, V codes, then the 64 K and 64 V
 // scales). D = 128: int8 code tiles arrive with the 128-byte swizzle, int4
-// tiles (64-byte rows) unswizzled, and the consumers build their fragments
-// from them in registers. int8 at D = 64: unswizzled
-// tiles, and each consumer warp converts its 16 rows into 16-bit tiles in its
-// own scratch (K then V, 16 rows x 128 B in the 128-byte swizzle of the TMA
-// tiles) before the tensor-core steps.
+// tiles (64-byte rows) with the 64-byte swizzle, and the consumers build their
+// fragments from them in registers. D = 64 (int8 64-byte rows, int4 32-byte
+// rows): unswizzled tiles, and each consumer warp converts its 16 rows into
+// 16-bit tiles in its own scratch (K then V, 16 rows x 128 B in the 128-byte
+// swizzle of the TMA tiles) before the tensor-core steps.
 template <int kD, int kQ = 0>
 struct DecShape {
   static constexpr bool kQuant = kQ != 0;           // an int8 (kQ = 8) or int4 (kQ = 4) cache
