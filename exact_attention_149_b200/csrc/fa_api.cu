@@ -239,6 +239,17 @@ fa_status set_smem(K kernel, int bytes) {
   return FA_OK;
 }
 
+// blocks of a forward launch: n_qblocks per (sequence, head), or, with
+// seq_blocks (varlen), the bound Hq * (ceil(total / rows) + B) on the blocks
+// that sequences of those lengths need
+inline long long fwd_grid(const fa::FwdParams& p, int rows) {
+  if (p.seq_blocks) return static_cast<long long>(p.Hq) * ((p.total + rows - 1) / rows + p.B);
+  return static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
+}
+// varlen launches with at most this many sequences number their blocks
+// sequence by sequence (one warp's two lanes a sequence find each block's)
+constexpr int kSeqBlocksMaxB = 64;
+
 template <int kD, bool kBF16, bool kCap>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const fa::FwdParams& p, cudaStream_t st) {
@@ -246,7 +257,7 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   auto kern = p.alibi ? fa::fwd_kernel<kD, kBF16, kCap, true> : fa::fwd_kernel<kD, kBF16, kCap, false>;
   fa_status s = set_smem(kern, Sh::kSmemBytes);
   if (s != FA_OK) return s;
-  const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
+  const long long grid = fwd_grid(p, Sh::kRows);
   if (grid > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "grid too large");
   {
     KernelTimer timer("fwd", st);
@@ -265,7 +276,7 @@ fa_status launch_fwd8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
                       : fa::fwd_kernel<kD, kBF16, kCap, false, true>;
   fa_status s = set_smem(kern, Sh::kSmemBytes);
   if (s != FA_OK) return s;
-  const long long grid = static_cast<long long>(p.n_qblocks) * p.B * p.Hq;
+  const long long grid = fwd_grid(p, Sh::kRows);
   if (grid > 0x7fffffffll) return fail(FA_ERR_INVALID_ARG, "grid too large");
   {
     KernelTimer timer("fwd_fp8", st);
@@ -355,6 +366,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, long long q_tok,
   p.o = out;
   p.lse = lse;
   p.cu_seqlens = cu_seqlens;
+  p.seq_blocks = cu_seqlens != nullptr && B <= kSeqBlocksMaxB;
   p.alibi = alibi_slopes;
   p.alibi_bstride = alibi_batch_stride;
   p.wait_ns = fa::kWaitTimeoutNs;
@@ -503,6 +515,7 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
   p.o = out;
   p.lse = lse;
   p.cu_seqlens = cu_seqlens;
+  p.seq_blocks = cu_seqlens != nullptr && B <= kSeqBlocksMaxB;
   p.alibi = alibi_slopes;
   p.alibi_bstride = alibi_batch_stride;
   p.o_scale = v_descale;

@@ -42,6 +42,7 @@ struct FwdParams {
   int B, Hq, Hkv, S, total;  // S: sequence length (max length when varlen)
   int group;                 // Hq / Hkv
   int n_qblocks;             // ceil(S / 256)
+  int seq_blocks;            // varlen, B <= 64: blocks numbered sequence by sequence
   float scale_log2;          // scale * log2(e)
   float softcap;             // 0 = off
   float cap_in;              // scale / softcap
@@ -237,17 +238,61 @@ __global__ void __launch_bounds__(FwdShape<kD, kF8>::kThreads, 1)
   {
   // ---- work item: (sequence, head) major so the CTAs in flight share the
   // K/V of a few heads in L2; heaviest query blocks first within a head
-  const int bh = static_cast<int>(blockIdx.x) / p.n_qblocks;
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) % p.n_qblocks;
-  const int h = bh % p.Hq;
-  const int b = bh / p.Hq;
-  int seq_start, seq_len;
-  if (p.cu_seqlens != nullptr) {
-    seq_start = p.cu_seqlens[b];
-    seq_len = p.cu_seqlens[b + 1] - seq_start;
+  int b, h, qb, seq_start, seq_len;
+  if (p.seq_blocks) {
+    // varlen, B <= 64: sequence b owns Hq * ceil(len_b / kRows) consecutive
+    // blocks, so that no block starts past its sequence's end (the grid is
+    // the bound Hq * (ceil(total / kRows) + B)). Every warp finds its block's
+    // sequence: lanes take sequences lane and lane + 32, and an inclusive
+    // prefix sum of their block counts over the warp locates blockIdx.x.
+    const unsigned full = 0xffffffffu;
+    const int ln = threadIdx.x & 31;
+    const int blk = static_cast<int>(blockIdx.x);
+    int st[2] = {0, 0}, en[2] = {0, 0}, cnt[2] = {0, 0};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int sq = ln + 32 * u;
+      if (sq < p.B) {
+        st[u] = p.cu_seqlens[sq];
+        en[u] = p.cu_seqlens[sq + 1];
+        cnt[u] = (en[u] - st[u] + Sh::kRows - 1) / Sh::kRows * p.Hq;
+      }
+    }
+    int inc[2] = {cnt[0], cnt[1]};
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int t = __shfl_up_sync(full, inc[u], off);
+        if (ln >= off) inc[u] += t;
+      }
+    }
+    inc[1] += __shfl_sync(full, inc[0], 31);
+    const unsigned m0 = __ballot_sync(full, ln < p.B && inc[0] > blk);
+    const unsigned m1 = __ballot_sync(full, ln + 32 < p.B && inc[1] > blk);
+    if (m0 == 0u && m1 == 0u) return;  // past the last sequence's blocks (uniform, before any barrier)
+    const int u = m0 != 0u ? 0 : 1;
+    const int src = __ffs(static_cast<int>(m0 != 0u ? m0 : m1)) - 1;
+    b = src + 32 * u;
+    const int first = __shfl_sync(full, u == 0 ? inc[0] - cnt[0] : inc[1] - cnt[1], src);
+    seq_start = __shfl_sync(full, u == 0 ? st[0] : st[1], src);
+    seq_len = __shfl_sync(full, u == 0 ? en[0] : en[1], src) - seq_start;
+    const int nq = (seq_len + Sh::kRows - 1) / Sh::kRows;
+    const int rem = blk - first;
+    h = rem / nq;
+    qb = nq - 1 - rem % nq;
   } else {
-    seq_start = b * p.S;
-    seq_len = p.S;
+    const int bh = static_cast<int>(blockIdx.x) / p.n_qblocks;
+    qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) % p.n_qblocks;
+    h = bh % p.Hq;
+    b = bh / p.Hq;
+    if (p.cu_seqlens != nullptr) {
+      seq_start = p.cu_seqlens[b];
+      seq_len = p.cu_seqlens[b + 1] - seq_start;
+    } else {
+      seq_start = b * p.S;
+      seq_len = p.S;
+    }
   }
   const int q0 = qb * Sh::kRows;
   if (q0 >= seq_len) return;  // uniform across the CTA, before any barrier
