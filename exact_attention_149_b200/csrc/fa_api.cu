@@ -51,22 +51,22 @@ fa_status ok() {
 // ---------------------------------------------------------------------------
 fa_status check_device() {
   static std::mutex mu;
-  static int verdict[128] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  static int arch_state[128] = {0};  // 0 unknown, 1 ok, 2 unsupported
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= 128) return fail(FA_ERR_UNSUPPORTED, "device index %d out of range", dev);
   std::lock_guard<std::mutex> lock(mu);
-  if (verdict[dev] == 0) {
+  if (arch_state[dev] == 0) {
     int major = 0, minor = 0;
     FA_CUDA_CHECK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
     FA_CUDA_CHECK(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
-    verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
-    if (verdict[dev] == 2)
+    arch_state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    if (arch_state[dev] == 2)
       return fail(FA_ERR_UNSUPPORTED, "device %d has compute capability %d.%d; this library is built for sm_100a (10.0)",
                   dev, major, minor);
   }
-  if (verdict[dev] != 1) return fail(FA_ERR_UNSUPPORTED, "device %d is not compute capability 10.0", dev);
+  if (arch_state[dev] != 1) return fail(FA_ERR_UNSUPPORTED, "device %d is not compute capability 10.0", dev);
   return FA_OK;
 }
 
