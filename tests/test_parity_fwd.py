@@ -94,6 +94,11 @@ def test_fwd_deterministic(cuda_ok):
     ([128, 5, 384, 1], 4, 4, 64, False, (-1, -1), 0.0),
     ([513, 129], 4, 1, 128, True, (-1, -1), 0.0),
     ([200, 1, 333], 4, 2, 256, True, (-1, -1), 0.0),
+    # empty sequences; at most 64 sequences number the blocks sequence by
+    # sequence, more take the padded grid
+    ([0, 300, 0, 1, 513, 0], 4, 2, 128, True, (-1, -1), 0.0),
+    ([(5 * i) % 29 for i in range(64)], 4, 2, 64, True, (-1, -1), 0.0),
+    ([(7 * i) % 37 + 1 for i in range(70)], 4, 2, 64, False, (-1, -1), 0.0),
 ])
 def test_fwd_varlen(cuda_ok, lengths, Hq, Hkv, D, causal, window, softcap):
     inp = W.make_varlen_inputs(lengths, Hq, Hkv, D, "bf16", seed=len(lengths) * 13 + D)
