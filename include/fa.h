@@ -154,7 +154,8 @@ FA_API size_t fa_bwd_workspace_size(int B, int Hq, int S, int D, int total_token
  *   The result is deterministic: no atomics; dK, dV come from one CTA per key
  *   tile and dQ from one CTA per query tile.
  * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG for null dout/dq/dk/dv or a
- *   workspace that is null or too small.
+ *   workspace that is null or too small, and FA_ERR_UNSUPPORTED for more than
+ *   8192 query heads.
  */
 FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                  const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S,

@@ -175,6 +175,12 @@ def test_head_dim_256_forward_and_backward(fa):
     assert fa.lib.fa_bwd(*a, 256, 1 << 20, None) == want
     a512 = [16] * 9 + [1, 2, 2, 64, 512, 0.1, 1, -1, -1, 0.0, None, 0, None, 0, 0]
     assert fa.lib.fa_bwd(*a512, 256, 1 << 20, None) == 2
+    # more query heads than the backward's pre pass takes (8192): unsupported,
+    # before the workspace check
+    heads = [16] * 9 + [1, 8200, 8200, 64, 128, 0.1, 1, -1, -1, 0.0, None, 0, None, 0, 0]
+    assert fa.lib.fa_bwd(*heads, 256, 1 << 20, None) == 2
+    heads[10] = heads[11] = 8192
+    assert fa.lib.fa_bwd(*heads, 256, 1 << 30, None) == want
     assert fa.lib.fa_fwd(16, 16, 16, 16, 16, 1, 2, 2, 64, 512, 0.1, 1, -1, -1, 0.0, None, 0,
                          None, 0, 0, None) == 2
 
